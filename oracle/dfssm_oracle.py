@@ -1,0 +1,336 @@
+"""CPU oracle for the DF-SSM decode step -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, obviously-correct numpy restatement of what one DF-SSM Mamba-2
+decode step computes.  Only the tests, the package's smoke check and the
+benchmark's CPU-baseline leg may import this module; the product path never
+does.  It shares no code with the CUDA library and imports nothing from it.
+
+Arithmetic is fp64 except where the method fixes a storage format or where a
+floating-point value decides an integer:
+  * activations entering a projection are stored as fp16;
+  * SSM state, conv state and the residual stream are stored as fp32;
+  * the int8 activation quantiser takes its decision in fp32 (scale = amax/127
+    as an IEEE fp32 divide, code = round-half-even of x/scale in fp32), the
+    precision the kernel uses, so both sides take the same integer decision;
+  * the low-rank stage-1 product A_q . x_q is exact integer arithmetic.
+
+Sources ("Density Field State Space Models", C. Shinde):
+  Eq. 3 (Section 3.2)   y = W_scaffold x + W_A (W_B x): frozen scaffold plus low-rank correction
+  Section 3.3           LoRA matrices int8 with per-channel scales
+  Table 1               scaffold stored 1-bit packed
+  Section 4.1           bits expanded on the fly; conv step is a stateful shift register;
+                        SSM step is a stateful recurrence; preallocated persistent state
+  Appendix B, Table 12  h = A h + (x dt) (x) B; d_state = 128 at 1.3B; norm(y * silu(z))
+Where the pages are silent (the [z|x|B|C|dt] split, softplus, eps, conv tap order,
+activation quantiser, the per-row scaffold scale alpha) the standard Mamba-2
+block and the decode-step description this package implements fix the reading;
+every such reading is listed in the design notes.
+
+Parity pins: every function here is checked by tests/test_oracle_pins.py
+against brute force, closed forms, library routines and the pages' own numbers.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+EPS = 1e-5          # RMSNorm epsilon (pages silent; Mamba-2 default)
+TILE_ROWS = 16      # tiled sign-word layout: 16 rows ...
+TILE_COLS = 256     # ... by 256 columns per 512-byte tile
+
+
+# --------------------------------------------------------------------------
+# 1-bit scaffold storage (Table 1: "1-bit packed"; Section 4.1: expanded on the fly)
+# --------------------------------------------------------------------------
+
+def pack_signs(w: np.ndarray) -> np.ndarray:
+    """Dense [rows, cols] -> uint32 [rows, cols/32]; bit j of word k is column 32k+j.
+
+    bit = 1 encodes +1 and is taken where w >= 0 (so -0.0 packs to +1); any
+    other value (negative, NaN) packs to 0, which encodes -1.
+    """
+    w = np.asarray(w)
+    rows, cols = w.shape
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    b = (w >= 0).astype(np.uint64).reshape(rows, cols // 32, 32)
+    weights = np.uint64(1) << np.arange(32, dtype=np.uint64)
+    return (b * weights).sum(axis=-1).astype(np.uint32)
+
+
+def unpack_signs(bits: np.ndarray, cols: int) -> np.ndarray:
+    """uint32 [rows, cols/32] -> int8 [rows, cols] of +1 (bit set) / -1 (bit clear)."""
+    bits = np.asarray(bits, dtype=np.uint32)
+    rows = bits.shape[0]
+    shifts = np.arange(32, dtype=np.uint32)
+    b = ((bits[:, :, None] >> shifts) & np.uint32(1)).reshape(rows, cols)
+    return (2 * b.astype(np.int8) - 1).astype(np.int8)
+
+
+def tiled_bit_position(row, col, cols: int):
+    """(word index, bit index) of weight (row, col) in the tiled sign-word layout.
+
+    Works elementwise on integers or integer arrays.  The tiled layout is a
+    bijective permutation of the row-major bits, chosen so that each of the 32
+    lanes of a warp reads one 16-byte vector per 16x256 tile and obtains its
+    tensor-core A-fragment signs for an m16n8k16 product with one shift and one
+    mask per fp16 pair.  Within a tile:
+      row r16 = row % 16, column c = col % 256, k-subtile kt = c // 64,
+      16-column chunk ch = (c % 64) // 16, column in chunk c16 = c % 16,
+      lane = (r16 % 8) * 4 + (c16 % 8) // 2,
+      q = (r16 // 8) + 2 * (c16 // 8),  s = 4 * ch + q,
+      bit = 15 - s for even c16, 31 - s for odd c16,
+      word = ((row // 16) * (cols // 256) + col // 256) * 128 + lane * 4 + kt.
+    """
+    row = np.asarray(row, dtype=np.int64)
+    col = np.asarray(col, dtype=np.int64)
+    r16 = row % TILE_ROWS
+    c = col % TILE_COLS
+    kt = c // 64
+    ch = (c % 64) // 16
+    c16 = c % 16
+    lane = (r16 % 8) * 4 + (c16 % 8) // 2
+    q = (r16 // 8) + 2 * (c16 // 8)
+    s = 4 * ch + q
+    bit = np.where(c16 % 2 == 0, 15 - s, 31 - s)
+    word = ((row // TILE_ROWS) * (cols // TILE_COLS) + col // TILE_COLS) * 128 + lane * 4 + kt
+    return word, bit
+
+
+def padded_rows(rows: int) -> int:
+    return -(-rows // TILE_ROWS) * TILE_ROWS
+
+
+def tile_signs(bits_rowmajor: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Row-major sign words -> tiled sign words (rows padded to 16 with clear bits)."""
+    if cols % TILE_COLS:
+        raise ValueError("cols must be a multiple of 256 for the tiled layout")
+    s = unpack_signs(bits_rowmajor, cols)
+    out = np.zeros(padded_rows(rows) * cols // 32, dtype=np.uint64)
+    r_idx, c_idx = np.nonzero(s > 0)
+    wd, bt = tiled_bit_position(r_idx, c_idx, cols)
+    np.bitwise_or.at(out, wd, np.uint64(1) << bt.astype(np.uint64))
+    return out.astype(np.uint32)
+
+
+# --------------------------------------------------------------------------
+# int8 low-rank correction (Eq. 3; Section 3.3 "int8 with per-channel scaling")
+# --------------------------------------------------------------------------
+
+def quantize_act(x16: np.ndarray):
+    """Per-row symmetric int8 quantisation of fp16 activations, decided in fp32.
+
+    amax = max|x| (exact in fp32); scale sx = amax / 127 (IEEE fp32 divide);
+    code = clamp(round_half_even(x / sx), -127, 127) with x / sx an fp32 divide.
+    A zero row gives codes 0 and sx = 1.  Returns (int8 codes, fp32 scales [rows]).
+    """
+    xf = np.asarray(x16, dtype=np.float16).astype(np.float32)
+    amax = np.max(np.abs(xf), axis=-1)
+    safe = np.where(amax > 0, amax, np.float32(127.0)).astype(np.float32)
+    sx = (safe / np.float32(127.0)).astype(np.float32)
+    q = np.rint((xf / sx[..., None]).astype(np.float32))
+    q = np.clip(q, -127, 127)
+    q = np.where(amax[..., None] > 0, q, 0)
+    return q.astype(np.int8), sx
+
+
+def lora_stage1(A: np.ndarray, xq: np.ndarray) -> np.ndarray:
+    """acc[b, j] = sum_k A[j, k] * xq[b, k], exact in int64, checked to fit int32."""
+    acc = xq.astype(np.int64) @ A.astype(np.int64).T
+    if acc.size and (acc.max() >= 2 ** 31 or acc.min() < -(2 ** 31)):
+        raise OverflowError("int8 x int8 partial exceeds int32")
+    return acc
+
+
+@dataclass
+class ProjTrace:
+    y: np.ndarray                       # fp64 [B, rows]
+    xq: Optional[np.ndarray] = None     # int8 [B, cols]
+    sx: Optional[np.ndarray] = None     # fp32 [B]
+    acc: Optional[np.ndarray] = None    # int64 [B, rank]
+    u: Optional[np.ndarray] = None      # fp64 [B, rank]
+
+
+def project(x16: np.ndarray, p) -> ProjTrace:
+    """One DF-SSM projection (Eq. 3 with the per-row scaffold scale alpha):
+
+        y[o] = alpha[o] * sum_k s[o,k] x[k]  +  sB[o] * sum_j B_q[o,j] u[j],
+        u[j] = acc[j] * sA[j] * sx,  acc = A_q . x_q.
+
+    The LoRA multiplier of Eq. 3 is folded into the scales (taken as 1).
+    """
+    x = np.asarray(x16, dtype=np.float16).astype(np.float64)
+    S = unpack_signs(p.bits, p.cols).astype(np.float64)
+    y = p.alpha.astype(np.float64) * (x @ S.T)
+    if p.A is None or p.A.shape[0] == 0:
+        return ProjTrace(y=y)
+    xq, sx = quantize_act(x16)
+    acc = lora_stage1(p.A, xq)
+    u = acc.astype(np.float64) * p.sA.astype(np.float64) * sx.astype(np.float64)[:, None]
+    y = y + p.sB.astype(np.float64) * (u @ p.B.astype(np.float64).T)
+    return ProjTrace(y=y, xq=xq, sx=sx, acc=acc, u=u)
+
+
+# --------------------------------------------------------------------------
+# Mamba-2 block pieces
+# --------------------------------------------------------------------------
+
+def rmsnorm(v: np.ndarray, w: np.ndarray, eps: float = EPS) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float64)
+    r = 1.0 / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+    return v * r * np.asarray(w, dtype=np.float64)
+
+
+def silu(v: np.ndarray) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float64)
+    return v / (1.0 + np.exp(-v))
+
+
+def softplus(v: np.ndarray) -> np.ndarray:
+    """log(1 + e^v), returned as v itself above 20."""
+    v = np.asarray(v, dtype=np.float64)
+    return np.where(v > 20.0, v, np.log1p(np.exp(np.minimum(v, 20.0))))
+
+
+def conv_step(conv_state: np.ndarray, xBC: np.ndarray, w: np.ndarray, b: np.ndarray):
+    """Causal depthwise conv1d step as a shift register (Section 4.1).
+
+    conv_state [B, W-1, C] holds the previous W-1 inputs, oldest first; the window
+    is [state..., xBC]; tap j multiplies window entry j (tap W-1 the newest input).
+    Output silu(bias + sum_j w[:, j] * window[j]); the state shifts by one.
+    Returns (xc fp64 [B, C], new state fp32).
+    """
+    cs = np.asarray(conv_state, dtype=np.float64)
+    xBC = np.asarray(xBC, dtype=np.float64)
+    win = np.concatenate([cs, xBC[:, None, :]], axis=1)           # [B, W, C]
+    wt = np.asarray(w, dtype=np.float64).T                         # [W, C]
+    pre = np.asarray(b, dtype=np.float64) + np.sum(wt[None] * win, axis=1)
+    new_state = win[:, 1:, :].astype(np.float32)
+    return silu(pre), new_state
+
+
+def ssm_step(h: np.ndarray, x: np.ndarray, Bv: np.ndarray, Cv: np.ndarray,
+             dt_raw: np.ndarray, dt_bias: np.ndarray, A_log: np.ndarray, D: np.ndarray):
+    """Selective-SSM state update for one token (Appendix B, corrected form).
+
+    h [B, H, P, N], x [B, H, P], Bv/Cv [B, N] (one group), dt_raw [B, H].
+      dt = softplus(dt_raw + dt_bias),  A = -exp(A_log),  dA = exp(dt * A)
+      h' = dA * h + (x * dt) (outer) B
+      y  = sum_n C[n] h'[.., n] + D * x
+    Returns (y fp64 [B, H, P], h' fp32).
+    """
+    h = np.asarray(h, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    dt = softplus(np.asarray(dt_raw, dtype=np.float64) + np.asarray(dt_bias, dtype=np.float64))
+    A = -np.exp(np.asarray(A_log, dtype=np.float64))
+    dA = np.exp(dt * A)                                            # [B, H]
+    xdt = x * dt[:, :, None]                                       # [B, H, P]
+    hn = dA[:, :, None, None] * h + xdt[:, :, :, None] * np.asarray(Bv, dtype=np.float64)[:, None, None, :]
+    y = np.einsum("bhpn,bn->bhp", hn, np.asarray(Cv, dtype=np.float64))
+    y = y + np.asarray(D, dtype=np.float64)[None, :, None] * x
+    return y, hn.astype(np.float32)
+
+
+def gated_rmsnorm(y: np.ndarray, z: np.ndarray, w: np.ndarray, eps: float = EPS) -> np.ndarray:
+    """norm(y * silu(z)) -- gate first, then RMSNorm over the whole d_inner (Appendix B)."""
+    g = np.asarray(y, dtype=np.float64) * silu(z)
+    return rmsnorm(g, w, eps)
+
+
+@dataclass
+class LayerTrace:
+    res: np.ndarray          # fp32 [B, D] residual after the layer
+    conv: np.ndarray         # fp32 new conv state
+    ssm: np.ndarray          # fp32 new SSM state
+    x_in: np.ndarray         # fp16 [B, D] pre-norm output (in_proj activation)
+    proj_in: ProjTrace
+    zxbcdt: np.ndarray       # fp64 [B, in_rows]
+    xc: np.ndarray           # fp64 [B, conv_dim] conv output
+    y: np.ndarray            # fp64 [B, d_inner] SSM output (before gate)
+    g: np.ndarray            # fp64 [B, d_inner] gated value y * silu(z)
+    x_out: np.ndarray        # fp16 [B, d_inner] gated-norm output (out_proj activation)
+    proj_out: ProjTrace
+
+
+def check_layer_shapes(d, lw, st) -> None:
+    """Argument validation; a d_state or head mismatch is an error (Appendix B, Table 12)."""
+    conv_dim = d.d_inner + 2 * d.ngroups * d.d_state
+    in_rows = 2 * d.d_inner + 2 * d.ngroups * d.d_state + d.nheads
+    if d.nheads * d.headdim != d.d_inner:
+        raise ValueError("d_inner must equal nheads * headdim")
+    if lw.inp.rows != in_rows or lw.inp.cols != d.d_model:
+        raise ValueError(f"in_proj shape {lw.inp.rows}x{lw.inp.cols} does not match dims ({in_rows}x{d.d_model})")
+    if lw.out.rows != d.d_model or lw.out.cols != d.d_inner:
+        raise ValueError("out_proj shape does not match dims")
+    if st.ssm.shape != (d.batch, d.nheads, d.headdim, d.d_state):
+        raise ValueError(f"ssm state shape {st.ssm.shape} does not match dims")
+    if st.conv.shape != (d.batch, d.d_conv - 1, conv_dim):
+        raise ValueError("conv state shape does not match dims")
+    if lw.conv_w.shape != (conv_dim, d.d_conv):
+        raise ValueError("conv weight shape does not match dims")
+
+
+def layer_step(res: np.ndarray, lw, st, d) -> LayerTrace:
+    """One decode token through one DF-SSM Mamba-2 layer (residual add included)."""
+    check_layer_shapes(d, lw, st)
+    E, N, G, H, P = d.d_inner, d.d_state, d.ngroups, d.nheads, d.headdim
+    C = E + 2 * G * N
+    res = np.asarray(res, dtype=np.float32)
+    x_in = rmsnorm(res, lw.prenorm_w).astype(np.float16)
+    pin = project(x_in, lw.inp)
+    zxbcdt = pin.y
+    z = zxbcdt[:, :E]
+    xBC = zxbcdt[:, E:E + C]
+    dt_raw = zxbcdt[:, E + C:]
+    xc, conv_new = conv_step(st.conv, xBC, lw.conv_w, lw.conv_b)
+    xs = xc[:, :E].reshape(d.batch, H, P)
+    Bg = xc[:, E:E + G * N].reshape(d.batch, G, N)
+    Cg = xc[:, E + G * N:].reshape(d.batch, G, N)
+    heads_per_group = H // G
+    y = np.zeros((d.batch, H, P))
+    ssm_new = np.zeros_like(st.ssm)
+    for gi in range(G):
+        hs = slice(gi * heads_per_group, (gi + 1) * heads_per_group)
+        y[:, hs], ssm_new[:, hs] = ssm_step(st.ssm[:, hs], xs[:, hs], Bg[:, gi], Cg[:, gi],
+                                            dt_raw[:, hs], lw.dt_bias[hs], lw.A_log[hs], lw.D[hs])
+    y = y.reshape(d.batch, E)
+    g = y * silu(z)
+    gw = g.reshape(d.batch, G, E // G)
+    xo = rmsnorm(gw, lw.gnorm_w.reshape(G, E // G)).reshape(d.batch, E)
+    x_out = xo.astype(np.float16)
+    pout = project(x_out, lw.out)
+    res_new = (res.astype(np.float64) + pout.y).astype(np.float32)
+    return LayerTrace(res_new, conv_new, ssm_new, x_in, pin, zxbcdt, xc, y, g, x_out, pout)
+
+
+@dataclass
+class State:
+    conv: np.ndarray         # fp32 [B, W-1, conv_dim]
+    ssm: np.ndarray          # fp32 [B, H, P, N]
+
+
+@dataclass
+class ModelTrace:
+    logits: np.ndarray       # fp64 [B, vocab]
+    tokens: np.ndarray       # int32 [B]
+    res: np.ndarray          # fp32 [B, D] residual entering the final norm
+    states: list             # [State] per layer, fp32
+
+
+def model_step(tokens: np.ndarray, m, states) -> ModelTrace:
+    """One greedy decode token for the whole model: embedding gather, all layers,
+    final RMSNorm, tied LM head (logits = E . norm(res)), argmax with the lowest
+    token id winning ties."""
+    d = m.dims
+    res = m.embed[np.asarray(tokens, dtype=np.int64)].astype(np.float32)
+    new_states = []
+    for lw, st in zip(m.layers, states):
+        t = layer_step(res, lw, st, d)
+        res = t.res
+        new_states.append(State(t.conv, t.ssm))
+    xf = rmsnorm(res, m.normf_w)
+    logits = xf @ m.embed.astype(np.float64).T
+    toks = np.argmax(logits, axis=-1).astype(np.int32)
+    return ModelTrace(logits, toks, res, new_states)

@@ -1,0 +1,472 @@
+"""Pins for the CPU oracle: each check ties an oracle function to something other
+than itself -- brute force on tiny inputs, closed forms, invariants, library
+routines (np.convolve, np.logaddexp) and numbers printed in "Density Field State
+Space Models" (Table 1, Appendix B).  A plausible slip anywhere in the oracle
+(a dropped term, a wrong sign or index, a transposed operand) fails one of these.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import dfssm_oracle as O
+from bit_scaffold_quantized_b200 import synth as S
+from bit_scaffold_quantized_b200 import roofline as R
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _proj_from_dense(rng, S0, rank, alpha=None):
+    rows, cols = S0.shape
+    p = S.gen_proj(rng, rows, cols, rank)
+    p.bits = O.pack_signs(S0.astype(np.float32))
+    if alpha is not None:
+        p.alpha = alpha.astype(np.float16)
+    return p
+
+
+# ---------------------------------------------------------------- packing
+
+def test_pack_single_bit_position():
+    # bit j of word k <-> column 32k + j; +1 <-> bit set
+    w = -np.ones((3, 96), dtype=np.float32)
+    w[1, 37] = 1.0
+    bits = O.pack_signs(w)
+    expect = np.zeros((3, 3), dtype=np.uint32)
+    expect[1, 1] = 1 << 5
+    assert np.array_equal(bits, expect)
+
+
+def test_pack_zero_negzero_nan():
+    w = np.array([[0.0, -0.0, np.nan, -1e-30] + [1.0] * 28], dtype=np.float32)
+    b = int(O.pack_signs(w)[0, 0])
+    assert b & 1 == 1 and (b >> 1) & 1 == 1      # 0.0 and -0.0 -> +1
+    assert (b >> 2) & 1 == 0 and (b >> 3) & 1 == 0  # NaN, negative -> -1
+
+
+def test_pack_unpack_roundtrip_bruteforce():
+    rng = np.random.default_rng(10)
+    w = rng.normal(size=(7, 64)).astype(np.float32)
+    bits = O.pack_signs(w)
+    s = O.unpack_signs(bits, 64)
+    for r in range(7):
+        for c in range(64):
+            assert s[r, c] == (1 if w[r, c] >= 0 else -1)
+    assert np.array_equal(O.pack_signs(s.astype(np.float32)), bits)
+
+
+def test_tiled_layout_is_bijection():
+    rows, cols = 32, 512
+    r, c = np.meshgrid(np.arange(rows), np.arange(cols), indexing="ij")
+    wd, bt = O.tiled_bit_position(r.ravel(), c.ravel(), cols)
+    flat = wd * 32 + bt
+    assert flat.min() == 0 and flat.max() == rows * cols - 1
+    assert len(np.unique(flat)) == rows * cols
+
+
+def test_tiled_layout_matches_mma_fragment_table():
+    """Independent check against the m16n8k16 fp16 A-fragment table of the PTX ISA:
+    lane = 4*groupID + threadID_in_group; a0,a1 -> (g, 2t..2t+1); a2,a3 -> (g+8, 2t..);
+    a4,a5 -> (g, 2t+8..); a6,a7 -> (g+8, 2t+8..).  Register q of chunk ch comes from
+    the lane's word with shift s = 4ch+q: its low half sign is bit 15-s, high half 31-s."""
+    rng = np.random.default_rng(11)
+    rows, cols = 16, 256
+    dense = rng.choice([-1.0, 1.0], size=(rows, cols)).astype(np.float32)
+    tiled = O.tile_signs(O.pack_signs(dense), rows, cols)
+    frag_pos = {0: (0, 0), 1: (8, 0), 2: (0, 8), 3: (8, 8)}   # reg q -> (row offset, col offset)
+    for lane in range(32):
+        g, t = lane // 4, lane % 4
+        for kt in range(4):
+            word = int(tiled[lane * 4 + kt])
+            for ch in range(4):
+                for q in range(4):
+                    s = 4 * ch + q
+                    ro, co = frag_pos[q]
+                    row = g + ro
+                    col = kt * 64 + ch * 16 + 2 * t + co
+                    lo = 1.0 if (word >> (15 - s)) & 1 else -1.0
+                    hi = 1.0 if (word >> (31 - s)) & 1 else -1.0
+                    assert lo == dense[row, col] and hi == dense[row, col + 1]
+
+
+def test_tiled_rows_padded():
+    rows, cols = 24, 256
+    dense = np.ones((rows, cols), dtype=np.float32)
+    tiled = O.tile_signs(O.pack_signs(dense), rows, cols)
+    assert tiled.size == 32 * cols // 32
+    # padded rows 24..31 are clear
+    r, c = np.meshgrid(np.arange(24, 32), np.arange(cols), indexing="ij")
+    wd, bt = O.tiled_bit_position(r.ravel(), c.ravel(), cols)
+    assert all(((int(tiled[w]) >> int(b)) & 1) == 0 for w, b in zip(wd, bt))
+
+
+# ---------------------------------------------------------------- scaffold
+
+def test_scaffold_matches_dense_source_matrix():
+    """Pack a known dense +/-1 matrix; the oracle projection must equal alpha * (S0 x)
+    computed from the original dense matrix (not from the unpacked bits)."""
+    rng = np.random.default_rng(12)
+    for rows, cols, batch in [(40, 64, 1), (33, 96, 3), (17, 32, 2)]:
+        S0 = rng.choice([-1, 1], size=(rows, cols))
+        alpha = rng.uniform(0.01, 0.05, size=rows).astype(np.float16)
+        p = _proj_from_dense(rng, S0, 0, alpha)
+        x = rng.normal(size=(batch, cols)).astype(np.float16)
+        y = O.project(x, p).y
+        ref = np.zeros((batch, rows))
+        for b in range(batch):
+            for o in range(rows):
+                acc = 0.0
+                for k in range(cols):
+                    acc += float(S0[o, k]) * float(x[b, k])
+                ref[b, o] = float(alpha[o]) * acc
+        np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("sign", [1, -1])
+def test_all_same_sign_gives_alpha_sum(sign):
+    rng = np.random.default_rng(13)
+    rows, cols = 24, 128
+    p = _proj_from_dense(rng, np.full((rows, cols), sign), 0)
+    x = rng.normal(size=(2, cols)).astype(np.float16)
+    y = O.project(x, p).y
+    closed = sign * p.alpha.astype(np.float64)[None, :] * x.astype(np.float64).sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(y, closed, rtol=1e-13)
+
+
+# ---------------------------------------------------------------- low-rank correction
+
+def test_rank0_equals_zero_B_bit_identical():
+    rng = np.random.default_rng(14)
+    p = S.gen_proj(rng, 48, 256, 8)
+    x = rng.normal(size=(3, 256)).astype(np.float16)
+    p0 = S.ProjWeights(p.rows, p.cols, p.bits, p.alpha, None, None, None, None)
+    pz = S.ProjWeights(p.rows, p.cols, p.bits, p.alpha, p.A, p.sA, np.zeros_like(p.B), p.sB)
+    assert np.array_equal(O.project(x, p0).y, O.project(x, pz).y)
+    assert not np.array_equal(O.project(x, p0).y, O.project(x, p).y)
+
+
+def test_lora_bruteforce_integer_and_fp():
+    rng = np.random.default_rng(15)
+    rows, cols, rank, batch = 9, 64, 4, 2
+    p = S.gen_proj(rng, rows, cols, rank)
+    p.sA = rng.uniform(5e-4, 2e-3, size=rank).astype(np.float16)
+    p.sB = rng.uniform(5e-4, 2e-3, size=rows).astype(np.float16)
+    x = rng.normal(size=(batch, cols)).astype(np.float16)
+    tr = O.project(x, p)
+    S0 = O.unpack_signs(p.bits, cols)
+    for b in range(batch):
+        q = [int(v) for v in tr.xq[b]]
+        for j in range(rank):
+            acc = 0
+            for k in range(cols):
+                acc += int(p.A[j, k]) * q[k]
+            assert acc == int(tr.acc[b, j])
+        u = [int(tr.acc[b, j]) * float(p.sA[j]) * float(tr.sx[b]) for j in range(rank)]
+        for o in range(rows):
+            scaf = sum(int(S0[o, k]) * float(x[b, k]) for k in range(cols)) * float(p.alpha[o])
+            lo = sum(int(p.B[o, j]) * u[j] for j in range(rank)) * float(p.sB[o])
+            assert abs(tr.y[b, o] - (scaf + lo)) <= 1e-12 * max(1.0, abs(scaf + lo))
+
+
+def test_identity_like_A_picks_codes():
+    rng = np.random.default_rng(16)
+    cols, rank = 128, 8
+    p = S.gen_proj(rng, 16, cols, rank)
+    picks = rng.choice(cols, size=rank, replace=False)
+    A = np.zeros((rank, cols), dtype=np.int8)
+    A[np.arange(rank), picks] = 1
+    A[3, picks[3]] = -1
+    x = rng.normal(size=(1, cols)).astype(np.float16)
+    xq, _ = O.quantize_act(x)
+    acc = O.lora_stage1(A, xq)
+    expect = xq[0, picks].astype(np.int64)
+    expect[3] = -expect[3]
+    assert np.array_equal(acc[0], expect)
+
+
+def test_lora_worst_case_fits_int32():
+    A = np.full((1, 4096), 127, dtype=np.int8)
+    xq = np.full((1, 4096), -127, dtype=np.int8)
+    assert int(O.lora_stage1(A, xq)[0, 0]) == -4096 * 127 * 127
+    A2 = np.full((1, 2 ** 18), 127, dtype=np.int8)
+    with pytest.raises(OverflowError):
+        O.lora_stage1(A2, np.full((1, 2 ** 18), 127, dtype=np.int8))
+
+
+# ---------------------------------------------------------------- quantiser
+
+def test_quantize_ties_half_even_and_extremes():
+    x = np.array([[127.0, 2.5, 3.5, -2.5, -127.0, 0.5, 1.5, 0.0]], dtype=np.float16)
+    q, sx = O.quantize_act(x)
+    assert sx[0] == np.float32(1.0)
+    assert q.tolist() == [[127, 2, 4, -2, -127, 0, 2, 0]]
+
+
+def test_quantize_zero_row_and_bounds():
+    rng = np.random.default_rng(17)
+    x = rng.normal(size=(4, 512)).astype(np.float16)
+    x[2] = 0
+    q, sx = O.quantize_act(x)
+    assert np.all(q[2] == 0) and sx[2] == 1.0
+    for r in (0, 1, 3):
+        i = int(np.argmax(np.abs(x[r].astype(np.float32))))
+        assert abs(int(q[r, i])) == 127 and np.sign(q[r, i]) == np.sign(x[r, i])
+        err = np.abs(x[r].astype(np.float64) - q[r].astype(np.float64) * float(sx[r]))
+        assert err.max() <= 0.5 * float(sx[r]) * (1 + 1e-6)
+        assert np.all(np.abs(q[r]) <= 127)
+
+
+# ---------------------------------------------------------------- conv step
+
+def test_conv_step_matches_np_convolve():
+    rng = np.random.default_rng(18)
+    T, Cc, W = 11, 5, 4
+    u = rng.normal(size=(T, Cc))
+    w = rng.uniform(-0.5, 0.5, size=(Cc, W)).astype(np.float16)
+    b = rng.uniform(-0.5, 0.5, size=Cc).astype(np.float16)
+    st = np.zeros((1, W - 1, Cc), dtype=np.float32)
+    outs = []
+    for t in range(T):
+        y, st = O.conv_step(st, u[t:t + 1].astype(np.float32), w, b)
+        outs.append(y[0])
+    outs = np.array(outs)
+    u32 = u.astype(np.float32).astype(np.float64)
+    for c in range(Cc):
+        pre = np.convolve(u32[:, c], w[c, ::-1].astype(np.float64))[:T] + float(b[c])
+        np.testing.assert_allclose(outs[:, c], pre / (1 + np.exp(-pre)), rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("tap", [0, 1, 2, 3])
+def test_conv_one_hot_tap_delays(tap):
+    T, W = 9, 4
+    u = np.arange(1, T + 1, dtype=np.float32)[:, None] * 0.25
+    w = np.zeros((1, W), dtype=np.float16)
+    w[0, tap] = 1
+    st = np.zeros((1, W - 1, 1), dtype=np.float32)
+    for t in range(T):
+        y, st = O.conv_step(st, u[t:t + 1], w, np.zeros(1, np.float16))
+        src = t - (W - 1 - tap)
+        v = float(u[src, 0]) if src >= 0 else 0.0
+        assert y[0, 0] == pytest.approx(v / (1 + np.exp(-v)), rel=1e-14, abs=0)
+
+
+# ---------------------------------------------------------------- SSM step
+
+def _ssm_args(rng, Bb=2, H=3, P=4, N=5):
+    h = rng.normal(size=(Bb, H, P, N)).astype(np.float32)
+    x = rng.normal(size=(Bb, H, P))
+    Bv = rng.normal(size=(Bb, N))
+    Cv = rng.normal(size=(Bb, N))
+    dt_raw = rng.normal(size=(Bb, H))
+    dt_bias = rng.normal(0, 0.1, size=H).astype(np.float32)
+    A_log = rng.uniform(0, np.log(16), size=H).astype(np.float32)
+    D = rng.normal(1, 0.1, size=H).astype(np.float32)
+    return h, x, Bv, Cv, dt_raw, dt_bias, A_log, D
+
+
+def test_softplus_library():
+    v = np.linspace(-30, 20, 1001)
+    np.testing.assert_allclose(O.softplus(v), np.logaddexp(0.0, v), rtol=1e-15, atol=1e-300)
+    big = np.linspace(20.001, 60, 101)       # above the threshold: identity, off by < e^-20
+    assert np.array_equal(O.softplus(big), big)
+    assert np.max(np.abs(np.logaddexp(0.0, big) - big)) < np.exp(-20.0)
+    assert O.softplus(np.array([-1e4]))[0] == 0.0
+
+
+def test_ssm_bruteforce_scalar_loops():
+    rng = np.random.default_rng(19)
+    h, x, Bv, Cv, dt_raw, dt_bias, A_log, D = _ssm_args(rng)
+    y, hn = O.ssm_step(h, x, Bv, Cv, dt_raw, dt_bias, A_log, D)
+    import math
+    Bb, H, P, N = h.shape
+    for b in range(Bb):
+        for hh in range(H):
+            v = float(dt_raw[b, hh]) + float(dt_bias[hh])
+            dt = math.log1p(math.exp(v))
+            dA = math.exp(-dt * math.exp(float(A_log[hh])))
+            for p in range(P):
+                yy = 0.0
+                for n in range(N):
+                    hv = dA * float(h[b, hh, p, n]) + dt * float(x[b, hh, p]) * float(Bv[b, n])
+                    assert hn[b, hh, p, n] == np.float32(hv)
+                    yy += float(Cv[b, n]) * hv
+                yy += float(D[hh]) * float(x[b, hh, p])
+                assert y[b, hh, p] == pytest.approx(yy, rel=1e-12, abs=1e-12)
+
+
+def test_ssm_dt_zero_leaves_state():
+    rng = np.random.default_rng(20)
+    h, x, Bv, Cv, dt_raw, dt_bias, A_log, D = _ssm_args(rng)
+    dt_bias[:] = -1e4
+    y, hn = O.ssm_step(h, x, Bv, Cv, dt_raw, dt_bias, A_log, D)
+    assert np.array_equal(hn, h)
+    np.testing.assert_allclose(y, np.einsum("bhpn,bn->bhp", h.astype(np.float64), Cv) + D[None, :, None] * x,
+                               rtol=1e-13)
+
+
+def test_ssm_recurrence_equals_unrolled_closed_form():
+    rng = np.random.default_rng(21)
+    T = 7
+    h0, _, _, _, _, dt_bias, A_log, D = _ssm_args(rng, Bb=1)
+    h0 = h0.astype(np.float64)
+    xs = rng.normal(size=(T, 1, 3, 4))
+    Bs = rng.normal(size=(T, 1, 5))
+    Cs = rng.normal(size=(T, 1, 5))
+    dts = rng.normal(size=(T, 1, 3))
+    # fp64 recurrence (state kept in fp64 by re-deriving from the oracle's formula pieces)
+    h = h0.copy()
+    dAs, dtv = [], []
+    for t in range(T):
+        dt = O.softplus(dts[t] + dt_bias)
+        dA = np.exp(dt * -np.exp(A_log.astype(np.float64)))
+        dAs.append(dA)
+        dtv.append(dt)
+        y, hn = O.ssm_step(h.astype(np.float32), xs[t], Bs[t], Cs[t], dts[t], dt_bias, A_log, D)
+        # oracle's own step (fp32 storage) must track the fp64 recurrence closely
+        h = dA[:, :, None, None] * h + (xs[t] * dt[:, :, None])[..., None] * Bs[t][:, None, None, :]
+        np.testing.assert_allclose(hn, h, rtol=1e-5, atol=1e-6)
+    closed = np.prod(dAs, axis=0)[:, :, None, None] * h0
+    for t in range(T):
+        decay = np.ones_like(dAs[0])
+        for s in range(t + 1, T):
+            decay = decay * dAs[s]
+        closed = closed + decay[:, :, None, None] * (xs[t] * dtv[t][:, :, None])[..., None] * Bs[t][:, None, None, :]
+    np.testing.assert_allclose(h, closed, rtol=1e-12, atol=1e-12)
+
+
+def test_ssm_no_decay_is_running_sum():
+    rng = np.random.default_rng(22)
+    h, x, Bv, Cv, dt_raw, dt_bias, A_log, D = _ssm_args(rng)
+    A_log[:] = -80.0   # A = -exp(-80): dt*A rounds exp() to exactly 1
+    h[:] = 0
+    acc = np.zeros(h.shape)
+    for t in range(3):
+        _, h = O.ssm_step(h, x, Bv, Cv, dt_raw, dt_bias, A_log, D)
+        dt = np.logaddexp(0.0, dt_raw + dt_bias)
+        acc = acc + (x * dt[:, :, None])[..., None] * Bv[:, None, None, :]
+        np.testing.assert_allclose(h, acc, rtol=1e-5, atol=1e-6)
+
+
+def test_appendixB_dt_scaling_matters():
+    fix = json.load(open(os.path.join(GOLDEN, "appendixB_block_fixes.json")))
+    assert "dt" in fix["fixes"][0]["correct"]
+    rng = np.random.default_rng(23)
+    h, x, Bv, Cv, dt_raw, dt_bias, A_log, D = _ssm_args(rng)
+    _, hn = O.ssm_step(h, x, Bv, Cv, dt_raw, dt_bias, A_log, D)
+    dt = np.logaddexp(0.0, dt_raw + dt_bias)
+    dA = np.exp(-dt * np.exp(A_log))
+    buggy = dA[:, :, None, None] * h + x[..., None] * Bv[:, None, None, :]
+    assert np.max(np.abs(hn - buggy)) > 1e-2
+
+
+# ---------------------------------------------------------------- gated norm
+
+def test_gate_then_norm_order_and_unit_rms():
+    fix = json.load(open(os.path.join(GOLDEN, "appendixB_block_fixes.json")))
+    assert fix["fixes"][2]["correct"] == "norm(y * silu(z))"
+    rng = np.random.default_rng(24)
+    y = rng.normal(size=(2, 64))
+    z = rng.normal(size=(2, 64))
+    w = np.ones(64, dtype=np.float16)
+    got = O.gated_rmsnorm(y, z, w)
+    np.testing.assert_allclose(np.mean(got ** 2, axis=-1), 1.0, rtol=1e-4)
+    g = y * (z / (1 + np.exp(-z)))
+    np.testing.assert_allclose(got, g / np.sqrt(np.mean(g ** 2, axis=-1, keepdims=True) + O.EPS), rtol=1e-13)
+    wrong = O.rmsnorm(y, w) * (z / (1 + np.exp(-z)))
+    assert np.max(np.abs(got - wrong)) > 0.1
+
+
+# ---------------------------------------------------------------- layer / model
+
+def _small_layer(seed=25, batch=2):
+    d = S.LAYER_SMALL.with_batch(batch)
+    rng = np.random.default_rng(seed)
+    lw = S.gen_layer(rng, d)
+    st = S.zero_state(d)
+    st.conv[:] = rng.normal(size=st.conv.shape)
+    st.ssm[:] = rng.normal(size=st.ssm.shape)
+    res = rng.normal(size=(batch, d.d_model)).astype(np.float32)
+    return d, lw, st, res
+
+
+def test_appendixB_d_state_mismatch_rejected():
+    d, lw, st, res = _small_layer()
+    bad = S.Dims(batch=d.batch, d_model=d.d_model, d_inner=d.d_inner, nheads=d.nheads,
+                 headdim=d.headdim, d_state=d.d_state // 2, rank=d.rank)
+    with pytest.raises(ValueError):
+        O.layer_step(res, lw, st, bad)
+
+
+def test_layer_identity_when_out_proj_is_zero():
+    d, lw, st, res = _small_layer()
+    lw.out.alpha[:] = 0
+    lw.out.A = lw.out.B = lw.out.sA = lw.out.sB = None
+    t = O.layer_step(res, lw, st, d)
+    assert np.array_equal(t.res, res)
+
+
+def test_layer_conv_state_shift_and_dt_zero():
+    d, lw, st, res = _small_layer()
+    lw.dt_bias[:] = -1e4
+    t = O.layer_step(res, lw, st, d)
+    assert np.array_equal(t.conv[:, :2], st.conv[:, 1:])
+    E, C = d.d_inner, d.conv_dim
+    assert np.array_equal(t.conv[:, 2], t.zxbcdt[:, E:E + C].astype(np.float32))
+    assert np.array_equal(t.ssm, st.ssm)
+
+
+def test_layer_pieces_compose():
+    """The layer's intermediates agree with the pinned pieces applied one at a time."""
+    d, lw, st, res = _small_layer()
+    t = O.layer_step(res, lw, st, d)
+    E, C, N = d.d_inner, d.conv_dim, d.d_state
+    x_in = O.rmsnorm(res, lw.prenorm_w).astype(np.float16)
+    assert np.array_equal(x_in, t.x_in)
+    assert np.array_equal(O.project(x_in, lw.inp).y, t.zxbcdt)
+    xc, _ = O.conv_step(st.conv, t.zxbcdt[:, E:E + C], lw.conv_w, lw.conv_b)
+    y, _ = O.ssm_step(st.ssm, xc[:, :E].reshape(d.batch, d.nheads, d.headdim), xc[:, E:E + N],
+                      xc[:, E + N:], t.zxbcdt[:, E + C:], lw.dt_bias, lw.A_log, lw.D)
+    np.testing.assert_array_equal(y.reshape(d.batch, E), t.y)
+    xo = O.gated_rmsnorm(t.y, t.zxbcdt[:, :E], lw.gnorm_w).astype(np.float16)
+    assert np.array_equal(xo, t.x_out)
+
+
+def test_model_argmax_lowest_id_on_ties_and_embedding():
+    d = S.LAYER_SMALL.with_batch(2)
+    rng = np.random.default_rng(26)
+    m = S.gen_model(rng, d, 0, 40)
+    m.embed[7] = m.embed[3]
+    m.embed[3] *= 8
+    m.embed[7] = m.embed[3]
+    tr = O.model_step(np.array([3, 7], dtype=np.int32), m, [])
+    assert np.array_equal(tr.res, m.embed[[3, 7]].astype(np.float32))
+    assert tr.tokens.tolist() == [3, 3]
+
+
+# ---------------------------------------------------------------- byte model vs Table 1
+
+def test_table1_sizes_from_shapes():
+    t1 = json.load(open(os.path.join(GOLDEN, "table1_model_size.json")))
+    d = S.LAYER_1P3B
+    n = t1["n_layer"]
+    scaffold = n * (d.in_rows * d.d_model + d.d_model * d.d_inner) // 8
+    assert abs(scaffold / 1e6 - t1["scaffold_1bit_MB"]) < 0.5
+    emb = S.VOCAB_1P3B * d.d_model
+    assert abs(emb / 1e6 - t1["embedding_lm_head_int8_MB"]) < 0.5
+    r = t1["lora_rank"]
+    lora = n * r * (d.d_model + d.in_rows + d.d_inner + d.d_model)
+    assert abs(lora / 1e6 - t1["lora_int8_r16_MB"]) < 1.0
+    # the byte model counts the same scaffold and LoRA bytes
+    d16 = S.Dims(1, 2048, 4096, 64, 64, 128, rank=r)
+    bits_only = R.proj_weight_bytes(d16.in_rows, 2048, 0) - 2 * d16.in_rows \
+        + R.proj_weight_bytes(2048, 4096, 0) - 2 * 2048
+    assert n * bits_only == scaffold
+
+
+def test_decode_token_bytes_1p3b():
+    d = S.LAYER_1P3B
+    assert R.layer_weight_bytes(d) == 3_861_120
+    assert R.layer_state_bytes(d) == 4_298_752
+    tok = R.model_token_bytes(d, 48, S.VOCAB_1P3B)
+    assert abs(tok / 1e6 - 597.6) < 0.1
