@@ -1,0 +1,139 @@
+// Shared device helpers for the DF-SSM decode kernels (sm_100a).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define DFSSM_DEV __device__ __forceinline__
+
+namespace dfssm {
+
+constexpr int kTileRows = 16;    // rows per tiled sign tile (m16n8k16 M)
+constexpr int kTileCols = 256;   // columns per tiled sign tile
+constexpr int kTileWords = 128;  // 32 lanes x 4 words
+constexpr int kConvW = 4;        // supported conv width
+constexpr float kEps = 1e-5f;    // RMSNorm epsilon
+constexpr double kEpsD = 1e-5;   // RMSNorm epsilon, fp64 paths
+
+DFSSM_DEV float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+DFSSM_DEV int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+DFSSM_DEV double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+DFSSM_DEV float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum with a fixed reduction tree (deterministic).  `red` holds >= 32 floats.
+DFSSM_DEV float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = (lane < nw) ? red[lane] : 0.f;
+  t = warp_sum(t);
+  return t;  // every thread holds the total
+}
+
+DFSSM_DEV double block_sum_d(double v, double* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum_d(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double t = (lane < nw) ? red[lane] : 0.0;
+  t = warp_sum_d(t);
+  return t;
+}
+
+DFSSM_DEV int block_sum_i(int v, int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum_i(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int t = (lane < nw) ? red[lane] : 0;
+  t = warp_sum_i(t);
+  return t;
+}
+
+DFSSM_DEV float block_max(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = (lane < nw) ? red[lane] : 0.f;
+  t = warp_max(t);
+  return t;
+}
+
+DFSSM_DEV float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+DFSSM_DEV uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+
+DFSSM_DEV double h2d(uint16_t h) { return double(__half2float(__ushort_as_half(h))); }
+
+// Round-to-nearest-even fp64 -> fp16 in one step (no double rounding through fp32).
+DFSSM_DEV uint16_t d2h(double v) {
+  uint16_t r;
+  asm("cvt.rn.f16.f64 %0, %1;" : "=h"(r) : "d"(v));
+  return r;
+}
+
+DFSSM_DEV double silu_d(double v) { return v / (1.0 + exp(-v)); }
+
+DFSSM_DEV double softplus_d(double v) { return v > 20.0 ? v : log1p(exp(v)); }
+
+// Scaffold signs as 0/1 bytes: register q of 32-column chunk ch of a tiled word.
+DFSSM_DEV uint32_t sign_bytes(uint32_t word, int s) { return (word >> s) & 0x01010101u; }
+
+// D += A(16x32, s8, row) * B(32x8, s8, col), exact s32 accumulators.
+DFSSM_DEV void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Exact activation digits: an fp16 value times 2^24 is an integer X with
+// |X| < 2^40; it is written as kDigits balanced base-256 digits in [-128, 127],
+// X = sum_d D_d 256^d.  The scaffold sum over 0/1 sign bytes of each digit
+// plane is then exact in int32, and recombining the planes in int64 gives the
+// exact dot product of the +/-1 row with the fp16 activations.
+constexpr int kDigits = 6;
+
+DFSSM_DEV void fp16_digits(uint16_t h, int8_t (&dg)[kDigits]) {
+  long long X = (long long)(h2d(h) * 16777216.0);
+#pragma unroll
+  for (int d = 0; d < kDigits; ++d) {
+    const int D = int((X + 128) & 255) - 128;
+    dg[d] = int8_t(D);
+    X = (X - D) >> 8;
+  }
+}
+
+// int8 activation code, decided in fp32: clamp(rint(x / sx), -127, 127).
+DFSSM_DEV int quant_code(float x, float sx) {
+  int q = __float2int_rn(__fdiv_rn(x, sx));
+  return max(-127, min(127, q));
+}
+
+}  // namespace dfssm

@@ -1,0 +1,446 @@
+// C ABI of libdfssm.so: host-side argument validation, workspace layout and the
+// launch sequences of the DF-SSM decode step.  Declarations and semantics: dfssm.h.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "dfssm.h"
+#include "kernels.cuh"
+#include "persistent.cuh"
+
+using namespace dfssm;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return DFSSM_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, code, ...) \
+  do {                           \
+    if (!(cond)) return fail(code, __VA_ARGS__); \
+  } while (0)
+
+#define REQUIRE_PTR(p) \
+  do { \
+    REQUIRE((p) != nullptr, DFSSM_ERR_INVALID_ARG, "%s is NULL", #p); \
+    REQUIRE(aligned16(p), DFSSM_ERR_MISALIGNED, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+#define CHECK_LAUNCH(what) \
+  do { \
+    cudaError_t e_ = cudaGetLastError(); \
+    if (e_ != cudaSuccess) return fail(DFSSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+
+constexpr size_t kNone = ~size_t(0);
+constexpr int kHeadBlocks = 592;  // 4 per SM on a 148-SM B200
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Bump {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    off = align256(off);
+    size_t at = off;
+    off += bytes;
+    return at;
+  }
+};
+
+size_t tiled_words(int rows, int cols) {
+  return size_t((rows + kTileRows - 1) / kTileRows) * kTileRows * (cols / 32);
+}
+
+int check_proj(const dfssm_proj* p, int rank, const char* name) {
+  REQUIRE(p != nullptr, DFSSM_ERR_INVALID_ARG, "%s: projection is NULL", name);
+  REQUIRE(p->rows > 0 && p->cols > 0, DFSSM_ERR_INVALID_ARG, "%s: rows/cols must be positive", name);
+  REQUIRE(p->cols % kTileCols == 0, DFSSM_ERR_UNSUPPORTED_SHAPE, "%s: cols (%d) must be a multiple of 256", name, p->cols);
+  REQUIRE(p->cols <= 8192, DFSSM_ERR_UNSUPPORTED_SHAPE, "%s: cols (%d) > 8192", name, p->cols);
+  REQUIRE(rank >= 0 && rank <= 128 && rank % 4 == 0, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "%s: rank (%d) must be in [0, 128] and a multiple of 4", name, rank);
+  REQUIRE(p->bits && aligned16(p->bits), p->bits ? DFSSM_ERR_MISALIGNED : DFSSM_ERR_INVALID_ARG,
+          "%s: bits NULL or misaligned", name);
+  REQUIRE(p->alpha && aligned16(p->alpha), p->alpha ? DFSSM_ERR_MISALIGNED : DFSSM_ERR_INVALID_ARG,
+          "%s: alpha NULL or misaligned", name);
+  if (rank > 0) {
+    REQUIRE(p->A && p->sA && p->B && p->sB, DFSSM_ERR_INVALID_ARG, "%s: LoRA pointers NULL with rank %d", name, rank);
+    REQUIRE(aligned16(p->A) && aligned16(p->sA) && aligned16(p->B) && aligned16(p->sB),
+            DFSSM_ERR_MISALIGNED, "%s: LoRA pointer not 16-byte aligned", name);
+  }
+  return DFSSM_OK;
+}
+
+int check_dims(const dfssm_dims* d) {
+  REQUIRE(d != nullptr, DFSSM_ERR_INVALID_ARG, "dims is NULL");
+  REQUIRE(d->batch > 0 && d->d_model > 0 && d->d_inner > 0 && d->nheads > 0 && d->headdim > 0 &&
+              d->d_state > 0, DFSSM_ERR_INVALID_ARG, "dims must be positive");
+  REQUIRE(d->ngroups == 1, DFSSM_ERR_UNSUPPORTED_SHAPE, "ngroups (%d) must be 1", d->ngroups);
+  REQUIRE(d->d_conv == kConvW, DFSSM_ERR_UNSUPPORTED_SHAPE, "d_conv (%d) must be 4", d->d_conv);
+  REQUIRE(d->nheads * d->headdim == d->d_inner, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "d_inner (%d) != nheads*headdim (%d)", d->d_inner, d->nheads * d->headdim);
+  REQUIRE(d->d_model % kTileCols == 0 && d->d_inner % kTileCols == 0, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "d_model and d_inner must be multiples of 256");
+  REQUIRE(d->d_model <= 8192 && d->d_inner <= 8192, DFSSM_ERR_UNSUPPORTED_SHAPE, "d_model/d_inner > 8192");
+  REQUIRE(d->headdim % 16 == 0 && d->headdim <= 128, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "headdim (%d) must be a multiple of 16 and <= 128", d->headdim);
+  REQUIRE(d->d_state % 4 == 0 && d->d_state <= 256, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "d_state (%d) must be a multiple of 4 and <= 256", d->d_state);
+  REQUIRE(d->rank >= 0 && d->rank <= 128 && d->rank % 4 == 0, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "rank (%d) must be in [0,128], multiple of 4", d->rank);
+  return DFSSM_OK;
+}
+
+int in_rows(const dfssm_dims* d) { return 2 * d->d_inner + 2 * d->ngroups * d->d_state + d->nheads; }
+int conv_dim(const dfssm_dims* d) { return d->d_inner + 2 * d->ngroups * d->d_state; }
+
+int check_layer(const dfssm_dims* d, const dfssm_layer_weights* w, const dfssm_layer_state* s, int li) {
+  REQUIRE(w != nullptr && s != nullptr, DFSSM_ERR_INVALID_ARG, "layer %d: weights/state NULL", li);
+  int rc;
+  if ((rc = check_proj(&w->in, d->rank, "in_proj")) != 0) return rc;
+  if ((rc = check_proj(&w->out, d->rank, "out_proj")) != 0) return rc;
+  REQUIRE(w->in.rows == in_rows(d) && w->in.cols == d->d_model, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "layer %d: in_proj is %dx%d, dims need %dx%d (check d_state/nheads)", li, w->in.rows,
+          w->in.cols, in_rows(d), d->d_model);
+  REQUIRE(w->out.rows == d->d_model && w->out.cols == d->d_inner, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "layer %d: out_proj is %dx%d, dims need %dx%d", li, w->out.rows, w->out.cols, d->d_model,
+          d->d_inner);
+  const void* ptrs[] = {w->prenorm_w, w->conv_w, w->conv_b, w->dt_bias, w->A_log, w->D, w->gnorm_w,
+                        s->conv_state, s->ssm_state};
+  const char* names[] = {"prenorm_w", "conv_w", "conv_b", "dt_bias", "A_log", "D", "gnorm_w",
+                         "conv_state", "ssm_state"};
+  for (int i = 0; i < 9; ++i) {
+    REQUIRE(ptrs[i] != nullptr, DFSSM_ERR_INVALID_ARG, "layer %d: %s is NULL", li, names[i]);
+    REQUIRE(aligned16(ptrs[i]), DFSSM_ERR_MISALIGNED, "layer %d: %s not 16-byte aligned", li, names[i]);
+  }
+  return DFSSM_OK;
+}
+
+void layer_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* L) {
+  const size_t B = d->batch, D = d->d_model, E = d->d_inner, r = d->rank ? d->rank : 1;
+  Bump bp;
+  L->status = bp.take(256);
+  L->x_in = bp.take(2 * B * D);
+  L->xq_in = bp.take(B * D);
+  L->sx_in = bp.take(4 * B);
+  L->acc_in = bp.take(4 * B * r);
+  L->u_in = bp.take(8 * B * r);
+  L->xd_in = bp.take(B * kDigits * D);
+  L->xdsum_in = bp.take(4 * B * kDigits);
+  L->zxbcdt = bp.take(8 * B * in_rows(d));
+  L->xc = bp.take(8 * B * conv_dim(d));
+  L->g = bp.take(8 * B * E);
+  L->x_out = bp.take(2 * B * E);
+  L->xq_out = bp.take(B * E);
+  L->sx_out = bp.take(4 * B);
+  L->acc_out = bp.take(4 * B * r);
+  L->u_out = bp.take(8 * B * r);
+  L->xd_out = bp.take(B * kDigits * E);
+  L->xdsum_out = bp.take(4 * B * kDigits);
+  if (n_layer > 0) {
+    L->res = bp.take(4 * B * D);
+    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), kHeadBlocks));
+  } else {
+    L->res = kNone;
+    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), 0));
+  }
+  L->total_bytes = align256(bp.off);
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<unsigned char*>(ws) + off); }
+
+struct Act {       // one activation's preprocessing outputs
+  uint16_t* x; int8_t* xq; float* sx; int* acc; double* u; int8_t* xd; int* xdsum;
+};
+
+struct Bufs {
+  unsigned* status;
+  Act in, out;
+  double* zxbcdt; double* xc; double* g;
+  float* res; unsigned char* scratch;
+};
+
+Bufs bind(void* ws, const dfssm_ws_layout& L) {
+  Bufs b;
+  b.status = at<unsigned>(ws, L.status);
+  b.in = Act{at<uint16_t>(ws, L.x_in), at<int8_t>(ws, L.xq_in), at<float>(ws, L.sx_in), at<int>(ws, L.acc_in),
+             at<double>(ws, L.u_in), at<int8_t>(ws, L.xd_in), at<int>(ws, L.xdsum_in)};
+  b.out = Act{at<uint16_t>(ws, L.x_out), at<int8_t>(ws, L.xq_out), at<float>(ws, L.sx_out),
+              at<int>(ws, L.acc_out), at<double>(ws, L.u_out), at<int8_t>(ws, L.xd_out),
+              at<int>(ws, L.xdsum_out)};
+  b.zxbcdt = at<double>(ws, L.zxbcdt);
+  b.xc = at<double>(ws, L.xc);
+  b.g = at<double>(ws, L.g);
+  b.res = L.res == kNone ? nullptr : at<float>(ws, L.res);
+  b.scratch = at<unsigned char>(ws, L.scratch);
+  return b;
+}
+
+// ---- launch helpers ---------------------------------------------------------
+
+template <typename SrcT, int MODE>
+int launch_prologue(int K, int rank, int batch, const void* src, const uint16_t* src16, const uint16_t* w,
+                    const Act& o, const dfssm_proj* p, cudaStream_t st) {
+  PrologueArgs a{};
+  a.K = K; a.rank = rank; a.src = src; a.src16 = src16; a.w = w;
+  a.x = o.x; a.xq = o.xq; a.sx = o.sx; a.xd = o.xd; a.xdsum = o.xdsum;
+  a.A = p->A; a.sA = p->sA; a.acc = o.acc; a.u = o.u;
+  dim3 grid(rank > 0 ? (rank + kPrologueRowsPerBlock - 1) / kPrologueRowsPerBlock : 1, batch);
+  k_prologue<SrcT, MODE><<<grid, kPrologueThreads, size_t(3) * K, st>>>(a);
+  CHECK_LAUNCH("k_prologue");
+  return DFSSM_OK;
+}
+
+constexpr size_t kProjSmemCap = 200 * 1024;
+
+int pick_bt(int batch, int K, int rank) {
+  int bt = batch <= 1 ? 1 : batch <= 2 ? 2 : batch <= 4 ? 4 : 8;
+  while (bt > 1 && proj_smem_bytes(K, rank, bt) > kProjSmemCap) bt >>= 1;
+  return bt;
+}
+
+template <int EPI, int BT>
+int launch_proj_bt(const ProjArgs& a, cudaStream_t st) {
+  const size_t smem = proj_smem_bytes(a.K, a.rank, BT);
+  cudaFuncSetAttribute(k_proj<EPI, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  dim3 grid((a.rows + kTileRows - 1) / kTileRows, (a.batch + BT - 1) / BT);
+  k_proj<EPI, BT><<<grid, kProjThreads, smem, st>>>(a);
+  CHECK_LAUNCH("k_proj");
+  return DFSSM_OK;
+}
+
+template <int EPI>
+int launch_proj(const ProjArgs& a, cudaStream_t st) {
+  switch (pick_bt(a.batch, a.K, a.rank)) {
+    case 1: return launch_proj_bt<EPI, 1>(a, st);
+    case 2: return launch_proj_bt<EPI, 2>(a, st);
+    case 4: return launch_proj_bt<EPI, 4>(a, st);
+    default: return launch_proj_bt<EPI, 8>(a, st);
+  }
+}
+
+ProjArgs proj_args(const dfssm_proj* p, int rank, int batch, const Act& act) {
+  ProjArgs a{};
+  a.rows = p->rows; a.K = p->cols; a.rank = rank; a.batch = batch;
+  a.bits = p->bits; a.alpha = p->alpha; a.B = p->B; a.sB = p->sB;
+  a.xd = act.xd; a.xdsum = act.xdsum; a.u = act.u;
+  return a;
+}
+
+// The layer as five dependent launches on one stream.
+int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const dfssm_layer_state* s,
+                      float* res, const Bufs& b, cudaStream_t st) {
+  const int B = d->batch, D = d->d_model, E = d->d_inner, r = d->rank, C = conv_dim(d);
+  int rc = launch_prologue<float, 0>(D, r, B, res, nullptr, w->prenorm_w, b.in, &w->in, st);
+  if (rc) return rc;
+  ProjArgs pa = proj_args(&w->in, r, B, b.in);
+  pa.zx = b.zxbcdt;
+  pa.conv_lo = E; pa.conv_dim = C; pa.conv_w = w->conv_w; pa.conv_b = w->conv_b;
+  pa.conv_state = s->conv_state; pa.xc = b.xc;
+  if ((rc = launch_proj<EPI_INPROJ>(pa, st))) return rc;
+  SsmArgs sa{};
+  sa.H = d->nheads; sa.P = d->headdim; sa.N = d->d_state; sa.E = E; sa.conv_dim = C; sa.in_rows = in_rows(d);
+  sa.zx = b.zxbcdt; sa.xc = b.xc; sa.dt_bias = w->dt_bias; sa.A_log = w->A_log; sa.D = w->D;
+  sa.state = s->ssm_state; sa.g = b.g;
+  k_ssm<<<dim3(d->nheads * (d->headdim / kSsmRows), B), kSsmThreads, size_t(16) * d->d_state, st>>>(sa);
+  CHECK_LAUNCH("k_ssm");
+  if ((rc = launch_prologue<double, 0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
+  ProjArgs po = proj_args(&w->out, r, B, b.out);
+  po.out = res;
+  return launch_proj<EPI_RESID>(po, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dfssm_version(void) { return 100; }
+
+int dfssm_model_decode_launches(const dfssm_dims* d, int n_layer, int vocab) {
+  if (check_dims(d) || n_layer < 1 || n_layer > kMaxLayers || vocab < 1) return 0;
+  return 1 + 5 * n_layer + 2;
+}
+
+const char* dfssm_last_error(void) { return g_last_error.c_str(); }
+
+size_t dfssm_packed_words(int rows, int cols, int layout) {
+  if (rows <= 0 || cols <= 0) return 0;
+  if (layout == DFSSM_LAYOUT_ROWMAJOR) return cols % 32 ? 0 : size_t(rows) * (cols / 32);
+  if (layout == DFSSM_LAYOUT_TILED) return cols % kTileCols ? 0 : tiled_words(rows, cols);
+  return 0;
+}
+
+int dfssm_pack_weights(const void* w, int dtype, int rows, int cols, int layout, uint32_t* bits,
+                       void* stream) {
+  REQUIRE(rows > 0 && cols > 0, DFSSM_ERR_INVALID_ARG, "rows/cols must be positive");
+  REQUIRE(dtype == DFSSM_DTYPE_F16 || dtype == DFSSM_DTYPE_F32, DFSSM_ERR_INVALID_ARG, "bad dtype %d", dtype);
+  REQUIRE(layout == DFSSM_LAYOUT_ROWMAJOR || layout == DFSSM_LAYOUT_TILED, DFSSM_ERR_INVALID_ARG,
+          "bad layout %d", layout);
+  REQUIRE(cols % (layout == DFSSM_LAYOUT_TILED ? kTileCols : 32) == 0, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "cols (%d) must be a multiple of %d", cols, layout == DFSSM_LAYOUT_TILED ? kTileCols : 32);
+  REQUIRE_PTR(w);
+  REQUIRE_PTR(bits);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = dfssm_packed_words(rows, cols, layout);
+  const int blocks = int(std::min<size_t>((n + 255) / 256, 148 * 16));
+  if (layout == DFSSM_LAYOUT_ROWMAJOR)
+    k_pack_rowmajor<<<blocks, 256, 0, st>>>(w, dtype, rows, cols, bits);
+  else
+    k_pack_tiled<<<blocks, 256, 0, st>>>(w, dtype, rows, cols, bits, n);
+  CHECK_LAUNCH("pack");
+  return ok();
+}
+
+int dfssm_repack_bits(const uint32_t* rowmajor, int rows, int cols, uint32_t* tiled, void* stream) {
+  REQUIRE(rows > 0 && cols > 0, DFSSM_ERR_INVALID_ARG, "rows/cols must be positive");
+  REQUIRE(cols % kTileCols == 0, DFSSM_ERR_UNSUPPORTED_SHAPE, "cols (%d) must be a multiple of 256", cols);
+  REQUIRE_PTR(rowmajor);
+  REQUIRE_PTR(tiled);
+  const size_t n = tiled_words(rows, cols);
+  const int blocks = int(std::min<size_t>((n + 255) / 256, 148 * 16));
+  k_repack_tiled<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(rowmajor, rows, cols, tiled, n);
+  CHECK_LAUNCH("repack");
+  return ok();
+}
+
+int dfssm_proj_workspace_layout(int rows, int cols, int rank, int batch, dfssm_ws_layout* L) {
+  REQUIRE(L != nullptr, DFSSM_ERR_INVALID_ARG, "layout is NULL");
+  REQUIRE(rows > 0 && cols > 0 && batch > 0 && rank >= 0, DFSSM_ERR_INVALID_ARG, "bad sizes");
+  std::memset(L, 0xff, sizeof *L);
+  const size_t B = batch, r = rank ? rank : 1;
+  Bump bp;
+  L->status = bp.take(256);
+  L->xq_in = bp.take(B * cols);
+  L->sx_in = bp.take(4 * B);
+  L->acc_in = bp.take(4 * B * r);
+  L->u_in = bp.take(8 * B * r);
+  L->xd_in = bp.take(B * kDigits * cols);
+  L->xdsum_in = bp.take(4 * B * kDigits);
+  L->total_bytes = align256(bp.off);
+  return ok();
+}
+
+size_t dfssm_proj_workspace_bytes(int rows, int cols, int rank, int batch) {
+  dfssm_ws_layout L;
+  if (dfssm_proj_workspace_layout(rows, cols, rank, batch, &L)) return 0;
+  return L.total_bytes;
+}
+
+int dfssm_proj_forward(const dfssm_proj* p, int rank, int batch, const uint16_t* x, float* y, void* ws,
+                       size_t ws_bytes, void* stream) {
+  int rc = check_proj(p, rank, "proj");
+  if (rc) return rc;
+  REQUIRE(batch > 0, DFSSM_ERR_INVALID_ARG, "batch must be positive");
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(y);
+  REQUIRE_PTR(ws);
+  dfssm_ws_layout L;
+  dfssm_proj_workspace_layout(p->rows, p->cols, rank, batch, &L);
+  REQUIRE(ws_bytes >= L.total_bytes, DFSSM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes,
+          L.total_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Act act{nullptr, at<int8_t>(ws, L.xq_in), at<float>(ws, L.sx_in), at<int>(ws, L.acc_in),
+          at<double>(ws, L.u_in), at<int8_t>(ws, L.xd_in), at<int>(ws, L.xdsum_in)};
+  if ((rc = launch_prologue<float, 1>(p->cols, rank, batch, nullptr, x, nullptr, act, p, st))) return rc;
+  ProjArgs a = proj_args(p, rank, batch, act);
+  a.out = y;
+  if ((rc = launch_proj<EPI_STORE>(a, st))) return rc;
+  return ok();
+}
+
+int dfssm_workspace_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* L) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  REQUIRE(L != nullptr, DFSSM_ERR_INVALID_ARG, "layout is NULL");
+  REQUIRE(n_layer >= 0 && vocab >= 0 && (n_layer == 0) == (vocab == 0), DFSSM_ERR_INVALID_ARG,
+          "n_layer and vocab must both be 0 (layer step) or both positive (model decode)");
+  layer_layout(d, n_layer, vocab, L);
+  return ok();
+}
+
+size_t dfssm_workspace_bytes(const dfssm_dims* d, int n_layer, int vocab) {
+  dfssm_ws_layout L;
+  if (dfssm_workspace_layout(d, n_layer, vocab, &L)) return 0;
+  return L.total_bytes;
+}
+
+int dfssm_layer_step(const dfssm_dims* d, const dfssm_layer_weights* w, const dfssm_layer_state* s,
+                     float* residual, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if ((rc = check_layer(d, w, s, 0))) return rc;
+  REQUIRE_PTR(residual);
+  REQUIRE_PTR(ws);
+  dfssm_ws_layout L;
+  layer_layout(d, 0, 0, &L);
+  REQUIRE(ws_bytes >= L.total_bytes, DFSSM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes,
+          L.total_bytes);
+  Bufs b = bind(ws, L);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = layer_multikernel(d, w, s, residual, b, st))) return rc;
+  return ok();
+}
+
+int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16_t* embed,
+                       const dfssm_layer_weights* layers, const dfssm_layer_state* states,
+                       const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out, float* logits,
+                       void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  REQUIRE(n_layer >= 1 && n_layer <= kMaxLayers, DFSSM_ERR_INVALID_ARG, "n_layer (%d) must be in [1, %d]",
+          n_layer, kMaxLayers);
+  REQUIRE(vocab >= 1, DFSSM_ERR_INVALID_ARG, "vocab must be positive");
+  REQUIRE(layers != nullptr && states != nullptr, DFSSM_ERR_INVALID_ARG, "layers/states NULL");
+  for (int l = 0; l < n_layer; ++l)
+    if ((rc = check_layer(d, &layers[l], &states[l], l))) return rc;
+  REQUIRE_PTR(embed);
+  REQUIRE_PTR(normf_w);
+  REQUIRE_PTR(tok_in);
+  REQUIRE_PTR(tok_out);
+  REQUIRE(logits == nullptr || aligned16(logits), DFSSM_ERR_MISALIGNED, "logits not 16-byte aligned");
+  REQUIRE_PTR(ws);
+  dfssm_ws_layout L;
+  layer_layout(d, n_layer, vocab, &L);
+  REQUIRE(ws_bytes >= L.total_bytes, DFSSM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes,
+          L.total_bytes);
+  Bufs b = bind(ws, L);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int B = d->batch, D = d->d_model;
+  k_embed<<<B, 256, 0, st>>>(embed, tok_in, vocab, D, b.res, b.status);
+  CHECK_LAUNCH("k_embed");
+  for (int l = 0; l < n_layer; ++l)
+    if ((rc = layer_multikernel(d, &layers[l], &states[l], b.res, b, st))) return rc;
+  float* part_val = reinterpret_cast<float*>(b.scratch);
+  int* part_idx = reinterpret_cast<int*>(b.scratch + size_t(4) * B * kHeadBlocks);
+  HeadArgs h{};
+  h.D = D; h.vocab = vocab; h.batch = B; h.res = b.res; h.normf_w = normf_w; h.embed = embed;
+  h.logits = logits; h.part_val = part_val; h.part_idx = part_idx;
+  const size_t smem = size_t(4) * kHeadBatch * D;
+  cudaFuncSetAttribute(k_lmhead, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  k_lmhead<<<dim3(kHeadBlocks, (B + kHeadBatch - 1) / kHeadBatch), kHeadWarps * 32, smem, st>>>(h);
+  CHECK_LAUNCH("k_lmhead");
+  k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, kHeadBlocks, tok_out);
+  CHECK_LAUNCH("k_argmax");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,219 @@
+/*
+ * dfssm.h -- C ABI of libdfssm.so, the B200 (sm_100a) DF-SSM decode step.
+ *
+ * Method: "Density Field State Space Models" (C. Shinde).  Every projection of a
+ * Mamba-2 layer is a frozen 1-bit sign scaffold plus an int8 low-rank correction
+ * (Section 3.2, Eq. 3; int8 per-channel scales, Section 3.3; 1-bit packed
+ * storage, Table 1).  The scaffold feeds the causal depthwise conv1d step (a
+ * stateful shift register) and the selective-SSM recurrence over preallocated
+ * persistent state (Section 4.1), with the corrected Mamba-2 forms of Appendix B
+ * (Table 12): h = A h + (x * dt) (outer) B, and gate before norm,
+ * norm(y * silu(z)).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller (the library
+ *     never allocates, frees, creates streams or synchronises).  `stream` is a
+ *     cudaStream_t passed as void*; all work is enqueued on it, so every call
+ *     may be captured into a CUDA graph.
+ *   - fp16 values travel as uint16_t bit patterns (IEEE binary16).
+ *   - Return value: 0 on success, a negative DFSSM_ERR_* code otherwise; argument
+ *     errors are detected on the host before anything is enqueued.  The message
+ *     of the calling thread's last failure is available from dfssm_last_error().
+ *   - Alignment: every pointer must be 16-byte aligned (DFSSM_ERR_MISALIGNED).
+ */
+#ifndef DFSSM_H
+#define DFSSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DFSSM_API __attribute__((visibility("default")))
+#else
+#define DFSSM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  DFSSM_OK = 0,
+  DFSSM_ERR_INVALID_ARG = -1,        /* null pointer, non-positive size, bad enum */
+  DFSSM_ERR_UNSUPPORTED_SHAPE = -2,  /* e.g. cols % 256 != 0, d_inner != nheads*headdim, ngroups != 1 */
+  DFSSM_ERR_MISALIGNED = -3,         /* a pointer is not 16-byte aligned */
+  DFSSM_ERR_WORKSPACE_TOO_SMALL = -4,
+  DFSSM_ERR_CUDA = -5,               /* a CUDA runtime call or launch failed */
+  DFSSM_ERR_DEVICE = -6              /* no usable sm_100 device */
+};
+
+enum { DFSSM_DTYPE_F16 = 0, DFSSM_DTYPE_F32 = 1 };
+
+/* Sign-word layouts.  ROWMAJOR: uint32 [rows][cols/32], bit j of word k holds
+ * column 32k+j, bit = 1 encodes +1 and bit = 0 encodes -1.  TILED: the same bits
+ * permuted into 16-row x 256-column tiles of 128 words (rows padded up to a
+ * multiple of 16 with clear bits).  For weight (row, col) with r16 = row % 16,
+ * c = col % 256, kt = c / 64, ch = (c % 64) / 16, c16 = c % 16:
+ *   lane = (r16 % 8) * 4 + (c16 % 8) / 2,  q = r16 / 8 + 2 * (c16 / 8),  s = 4*ch + q,
+ *   bit  = 15 - s for even c16, 31 - s for odd c16,
+ *   word = ((row / 16) * (cols / 256) + col / 256) * 128 + lane * 4 + kt.
+ * Each warp lane then reads one 16-byte vector per tile and forms its m16n8k16
+ * tensor-core A fragment with one shift and one mask per fp16 pair.  The
+ * projection kernels consume TILED words only. */
+enum { DFSSM_LAYOUT_ROWMAJOR = 0, DFSSM_LAYOUT_TILED = 1 };
+
+/* Shape of one layer.  in_proj: d_model -> 2*d_inner + 2*ngroups*d_state + nheads
+ * ([z | x | B | C | dt]); conv over the conv_dim = d_inner + 2*ngroups*d_state
+ * channels [x | B | C]; out_proj: d_inner -> d_model.  Supported: ngroups == 1,
+ * d_conv == 4, d_inner == nheads*headdim, d_model and d_inner multiples of 256,
+ * headdim a multiple of 16 (<= 128), d_state a multiple of 4 (<= 256),
+ * 0 <= rank <= 128 and a multiple of 4. */
+typedef struct dfssm_dims {
+  int32_t batch, d_model, d_inner, nheads, headdim, d_state, ngroups, d_conv, rank;
+} dfssm_dims;
+
+/* One DF-SSM projection (Eq. 3 with a per-row scaffold scale):
+ *   y[o] = alpha[o] * sum_k s[o,k] x[k] + sB[o] * sum_j B[o,j] u[j],
+ *   u[j] = acc[j] * sA[j] * sx,  acc[j] = sum_k A[j,k] xq[k]  (int8 x int8 -> int32),
+ *   xq = clamp(rint(x / sx), -127, 127), sx = max|x| / 127 (fp32; sx = 1, xq = 0 for x == 0).
+ * bits : TILED sign words, dfssm_packed_words(rows, cols, DFSSM_LAYOUT_TILED) words
+ * alpha: fp16 [rows]            A : int8 [rank][cols]      sA: fp16 [rank]
+ * B    : int8 [rows][rank]      sB: fp16 [rows]
+ * A, sA, B, sB may be NULL only when the rank in use is 0. */
+typedef struct dfssm_proj {
+  int32_t rows, cols;
+  const uint32_t* bits;
+  const uint16_t* alpha;
+  const int8_t* A;
+  const uint16_t* sA;
+  const int8_t* B;
+  const uint16_t* sB;
+} dfssm_proj;
+
+/* Weights of one layer.  prenorm_w fp16 [d_model]; conv_w fp16 [conv_dim][d_conv]
+ * (tap d_conv-1 multiplies the newest input); conv_b fp16 [conv_dim]; dt_bias,
+ * A_log, D fp32 [nheads]; gnorm_w fp16 [d_inner]. */
+typedef struct dfssm_layer_weights {
+  const uint16_t* prenorm_w;
+  dfssm_proj in;
+  const uint16_t* conv_w;
+  const uint16_t* conv_b;
+  const float* dt_bias;
+  const float* A_log;
+  const float* D;
+  const uint16_t* gnorm_w;
+  dfssm_proj out;
+} dfssm_layer_weights;
+
+/* Persistent per-layer state, updated in place each step (caller-owned).
+ * conv_state fp32 [batch][d_conv-1][conv_dim], index 0 the oldest input;
+ * ssm_state fp32 [batch][nheads][headdim][d_state]. */
+typedef struct dfssm_layer_state {
+  float* conv_state;
+  float* ssm_state;
+} dfssm_layer_state;
+
+/* Byte offsets of the intermediates a step leaves in its workspace (valid after
+ * the stream has reached the end of the call).  For dfssm_model_decode they hold
+ * the LAST layer's values.  ~0 marks a region the call does not have.
+ * Digit planes: an fp16 activation x is the integer X = x * 2^24 (|X| < 2^40),
+ * written as 6 balanced base-256 digits D_d in [-128, 127] with X = sum D_d 256^d;
+ * the scaffold product is computed exactly from these planes. */
+typedef struct dfssm_ws_layout {
+  size_t total_bytes;
+  size_t status;     /* uint32 status word: 0 ok; bit 1 = a token id was out of range (clamped) */
+  size_t x_in;       /* fp16  [batch][d_model]    pre-norm output (in_proj activation) */
+  size_t xq_in;      /* int8  [batch][d_model]    its int8 LoRA codes */
+  size_t sx_in;      /* fp32  [batch]             their scales */
+  size_t acc_in;     /* int32 [batch][rank]       in_proj A.xq partials */
+  size_t u_in;       /* fp64  [batch][rank]       acc * sA * sx */
+  size_t xd_in;      /* int8  [batch][6][d_model] digit planes of x_in */
+  size_t xdsum_in;   /* int32 [batch][6]          digit-plane sums */
+  size_t zxbcdt;     /* fp64  [batch][in_rows]    in_proj output [z|x|B|C|dt] */
+  size_t xc;         /* fp64  [batch][conv_dim]   conv output after SiLU */
+  size_t g;          /* fp64  [batch][d_inner]    y * silu(z) */
+  size_t x_out;      /* fp16  [batch][d_inner]    gated-norm output (out_proj activation) */
+  size_t xq_out;     /* int8  [batch][d_inner] */
+  size_t sx_out;     /* fp32  [batch] */
+  size_t acc_out;    /* int32 [batch][rank] */
+  size_t u_out;      /* fp64  [batch][rank] */
+  size_t xd_out;     /* int8  [batch][6][d_inner] */
+  size_t xdsum_out;  /* int32 [batch][6] */
+  size_t res;        /* fp32  [batch][d_model]    residual stream (model decode only) */
+  size_t scratch;    /* internal */
+} dfssm_ws_layout;
+
+/* ---- weight packing (not on the timed path) ------------------------------ */
+
+/* Number of uint32 words of a packed [rows x cols] sign matrix in `layout`. */
+DFSSM_API size_t dfssm_packed_words(int rows, int cols, int layout);
+
+/* Pack a dense row-major matrix w ([rows][cols], fp16 or fp32 per `dtype`) into
+ * sign words: bit = 1 where w >= 0 (so -0.0 packs to +1), 0 otherwise (NaN too).
+ * cols % 32 == 0 (ROWMAJOR) or cols % 256 == 0 (TILED).  `bits` receives
+ * dfssm_packed_words(rows, cols, layout) words.  Table 1 ("1-bit packed"). */
+DFSSM_API int dfssm_pack_weights(const void* w, int dtype, int rows, int cols, int layout,
+                       uint32_t* bits, void* stream);
+
+/* Permute ROWMAJOR sign words into the TILED layout (exact bit permutation). */
+DFSSM_API int dfssm_repack_bits(const uint32_t* rowmajor, int rows, int cols, uint32_t* tiled,
+                      void* stream);
+
+/* ---- one projection (Eq. 3) --------------------------------------------- */
+
+DFSSM_API size_t dfssm_proj_workspace_bytes(int rows, int cols, int rank, int batch);
+
+/* y [batch][rows] fp32 = projection of x [batch][cols] fp16 (finite values).  The
+ * scaffold sum is exact (integer arithmetic on the activation's digit planes), the
+ * LoRA stage 2 and scaling are fp64, y is rounded once to fp32.  The workspace
+ * receives xq_in, sx_in, acc_in, u_in, xd_in and xdsum_in (see dfssm_ws_layout)
+ * at the offsets dfssm_proj_workspace_layout reports. */
+DFSSM_API int dfssm_proj_forward(const dfssm_proj* p, int rank, int batch, const uint16_t* x, float* y,
+                       void* ws, size_t ws_bytes, void* stream);
+DFSSM_API int dfssm_proj_workspace_layout(int rows, int cols, int rank, int batch, dfssm_ws_layout* out);
+
+/* ---- decode step -------------------------------------------------------- */
+
+/* Workspace for dfssm_layer_step (n_layer == 0, vocab == 0) or for
+ * dfssm_model_decode (n_layer >= 1, vocab >= 1).  The workspace must be
+ * zero-filled once before its first use; the library leaves its control words
+ * consistent after every successful call. */
+DFSSM_API size_t dfssm_workspace_bytes(const dfssm_dims* d, int n_layer, int vocab);
+DFSSM_API int dfssm_workspace_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* out);
+
+/* One decode token through one layer, residual add included:
+ *   x = fp16(rmsnorm(residual) * prenorm_w); [z|xBC|dt] = in_proj(x);
+ *   xc = silu(conv1d_step(xBC)); SSM update of ssm_state; g = y * silu(z);
+ *   xo = fp16(rmsnorm(g) * gnorm_w); residual += out_proj(xo).
+ * residual fp32 [batch][d_model] in/out; state updated in place.  RMSNorm eps 1e-5. */
+DFSSM_API int dfssm_layer_step(const dfssm_dims* d, const dfssm_layer_weights* w, const dfssm_layer_state* s,
+                     float* residual, void* ws, size_t ws_bytes, void* stream);
+
+/* One greedy decode token for all batch rows through the whole model:
+ *   residual = embed[tok_in]; n_layer layer steps; xf = rmsnorm(residual) * normf_w;
+ *   logits = embed . xf (tied LM head, fp32 accumulation); tok_out = argmax
+ *   (lowest token id wins ties).
+ * embed fp16 [vocab][d_model]; layers/states HOST arrays of n_layer entries, read at
+ * call time (under stream capture their pointers are baked into the graph);
+ * tok_in/tok_out int32 [batch] device (may alias); logits fp32 [batch][vocab] or NULL.
+ * n_layer <= 64. */
+DFSSM_API int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16_t* embed,
+                       const dfssm_layer_weights* layers, const dfssm_layer_state* states,
+                       const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out,
+                       float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* Number of kernel launches one dfssm_model_decode call enqueues for these
+ * arguments (0 if they are invalid). */
+DFSSM_API int dfssm_model_decode_launches(const dfssm_dims* d, int n_layer, int vocab);
+
+/* Message describing the calling thread's last nonzero return ("" if none). */
+DFSSM_API const char* dfssm_last_error(void);
+
+/* ABI version (major * 100 + minor). */
+DFSSM_API int dfssm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFSSM_H */

@@ -73,15 +73,15 @@ def tiled_bit_position(row, col, cols: int):
     """(word index, bit index) of weight (row, col) in the tiled sign-word layout.
 
     Works elementwise on integers or integer arrays.  The tiled layout is a
-    bijective permutation of the row-major bits, chosen so that each of the 32
-    lanes of a warp reads one 16-byte vector per 16x256 tile and obtains its
-    tensor-core A-fragment signs for an m16n8k16 product with one shift and one
-    mask per fp16 pair.  Within a tile:
-      row r16 = row % 16, column c = col % 256, k-subtile kt = c // 64,
-      16-column chunk ch = (c % 64) // 16, column in chunk c16 = c % 16,
-      lane = (r16 % 8) * 4 + (c16 % 8) // 2,
-      q = (r16 // 8) + 2 * (c16 // 8),  s = 4 * ch + q,
-      bit = 15 - s for even c16, 31 - s for odd c16,
+    bijective permutation of the row-major bits into 16-row x 256-column tiles of
+    128 words, chosen so that each of the 32 lanes of a warp reads one 16-byte
+    vector per tile and forms each int8 A-fragment register of an m16n8k32
+    tensor-core product with one shift and one mask (byte = sign bit, 0 or 1).
+    Within a tile:
+      r16 = row % 16, c = col % 256, kt = c // 64, ch = (c % 64) // 32,
+      c32 = c % 32, colhalf = c32 // 16, t = (c32 % 16) // 4, i = c32 % 4,
+      lane = (r16 % 8) * 4 + t,  q = r16 // 8 + 2 * colhalf,  s = 4 * ch + q,
+      bit = s + 8 * i,
       word = ((row // 16) * (cols // 256) + col // 256) * 128 + lane * 4 + kt.
     """
     row = np.asarray(row, dtype=np.int64)
@@ -89,12 +89,15 @@ def tiled_bit_position(row, col, cols: int):
     r16 = row % TILE_ROWS
     c = col % TILE_COLS
     kt = c // 64
-    ch = (c % 64) // 16
-    c16 = c % 16
-    lane = (r16 % 8) * 4 + (c16 % 8) // 2
-    q = (r16 // 8) + 2 * (c16 // 8)
+    ch = (c % 64) // 32
+    c32 = c % 32
+    colhalf = c32 // 16
+    t = (c32 % 16) // 4
+    i = c32 % 4
+    lane = (r16 % 8) * 4 + t
+    q = r16 // 8 + 2 * colhalf
     s = 4 * ch + q
-    bit = np.where(c16 % 2 == 0, 15 - s, 31 - s)
+    bit = s + 8 * i
     word = ((row // TILE_ROWS) * (cols // TILE_COLS) + col // TILE_COLS) * 128 + lane * 4 + kt
     return word, bit
 

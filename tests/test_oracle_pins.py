@@ -66,28 +66,29 @@ def test_tiled_layout_is_bijection():
 
 
 def test_tiled_layout_matches_mma_fragment_table():
-    """Independent check against the m16n8k16 fp16 A-fragment table of the PTX ISA:
-    lane = 4*groupID + threadID_in_group; a0,a1 -> (g, 2t..2t+1); a2,a3 -> (g+8, 2t..);
-    a4,a5 -> (g, 2t+8..); a6,a7 -> (g+8, 2t+8..).  Register q of chunk ch comes from
-    the lane's word with shift s = 4ch+q: its low half sign is bit 15-s, high half 31-s."""
+    """Independent check against the m16n8k32 .s8 A-fragment table of the PTX ISA:
+    lane = 4*groupID + threadID_in_group; register 0 holds (g, 4t..4t+3), register 1
+    (g+8, 4t..4t+3), register 2 (g, 16+4t..), register 3 (g+8, 16+4t..).  Register q
+    of 32-column chunk ch is (word >> s) & 0x01010101 with s = 4ch+q: byte i of it
+    is the sign bit of column 4t+i (+16 for q >= 2)."""
     rng = np.random.default_rng(11)
     rows, cols = 16, 256
     dense = rng.choice([-1.0, 1.0], size=(rows, cols)).astype(np.float32)
     tiled = O.tile_signs(O.pack_signs(dense), rows, cols)
-    frag_pos = {0: (0, 0), 1: (8, 0), 2: (0, 8), 3: (8, 8)}   # reg q -> (row offset, col offset)
+    frag_pos = {0: (0, 0), 1: (8, 0), 2: (0, 16), 3: (8, 16)}   # reg q -> (row offset, col offset)
     for lane in range(32):
         g, t = lane // 4, lane % 4
         for kt in range(4):
             word = int(tiled[lane * 4 + kt])
-            for ch in range(4):
+            for ch in range(2):
                 for q in range(4):
-                    s = 4 * ch + q
+                    reg = (word >> (4 * ch + q)) & 0x01010101
                     ro, co = frag_pos[q]
-                    row = g + ro
-                    col = kt * 64 + ch * 16 + 2 * t + co
-                    lo = 1.0 if (word >> (15 - s)) & 1 else -1.0
-                    hi = 1.0 if (word >> (31 - s)) & 1 else -1.0
-                    assert lo == dense[row, col] and hi == dense[row, col + 1]
+                    for i in range(4):
+                        bit = (reg >> (8 * i)) & 0xFF
+                        assert bit in (0, 1)
+                        col = kt * 64 + ch * 32 + co + 4 * t + i
+                        assert (1.0 if bit else -1.0) == dense[g + ro, col]
 
 
 def test_tiled_rows_padded():

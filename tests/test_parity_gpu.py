@@ -1,0 +1,300 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same
+seeded inputs.  Bit-exact for packing and for the int8 x int8 -> int32 low-rank
+partials; max relative error <= 2e-3 for fp outputs and states."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import dfssm_oracle as O
+from bit_scaffold_quantized_b200 import synth as S
+from bit_scaffold_quantized_b200 import dfssm as F
+from tests._util import TOL, rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+FAITHFUL = 1e-6   # observed-agreement bound for fp32 outputs of an exact/fp64 pipeline
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    F.lib()
+
+
+def _sync():
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- packing
+
+@pytest.mark.parametrize("rows,cols", [(64, 512), (1064, 256), (8512, 2048)])
+@pytest.mark.parametrize("dtype", [np.float16, np.float32])
+def test_pack_bit_exact(rows, cols, dtype):
+    rng = np.random.default_rng(rows * 7 + cols)
+    w = rng.normal(size=(rows, cols)).astype(dtype)
+    w.flat[rng.choice(w.size, 64, replace=False)] = 0.0
+    w.flat[rng.choice(w.size, 64, replace=False)] = -0.0
+    wt = torch.from_numpy(w).to(DEV)
+    for layout in (F.LAYOUT_ROWMAJOR, F.LAYOUT_TILED):
+        out = torch.full((F.packed_words(rows, cols, layout),), -1, dtype=torch.int32, device=DEV)
+        F.pack_weights(wt, rows, cols, layout, out)
+        _sync()
+        got = to_np(out).view(np.uint32)
+        ref = O.pack_signs(w)
+        if layout == F.LAYOUT_TILED:
+            ref = O.tile_signs(ref, rows, cols)
+        assert np.array_equal(got, ref.ravel())
+
+
+@pytest.mark.parametrize("rows,cols", [(16, 256), (40, 512), (1064, 256), (2048, 4096)])
+def test_repack_bit_exact(rows, cols):
+    rng = np.random.default_rng(rows + cols)
+    bits = rng.integers(0, 2 ** 32, size=(rows, cols // 32), dtype=np.uint64).astype(np.uint32)
+    src = torch.from_numpy(bits.view(np.int32)).to(DEV)
+    out = torch.full((F.packed_words(rows, cols, F.LAYOUT_TILED),), -1, dtype=torch.int32, device=DEV)
+    F.repack_bits(src, rows, cols, out)
+    _sync()
+    assert np.array_equal(to_np(out).view(np.uint32), O.tile_signs(bits, rows, cols))
+
+
+# ---------------------------------------------------------------- projection (Eq. 3)
+
+def _proj_case(p, x, rank):
+    dp = F.DeviceProj.from_host(p)
+    xt = torch.from_numpy(x).to(DEV)
+    y = torch.full((x.shape[0], p.rows), np.nan, dtype=torch.float32, device=DEV)
+    ws = F.proj_workspace(p.rows, p.cols, rank, x.shape[0])
+    F.proj_forward(dp, rank, xt, y, ws)
+    _sync()
+    L = F.proj_workspace_layout(p.rows, p.cols, rank, x.shape[0])
+    ref = O.project(x, p)
+    e = rel_err(to_np(y), ref.y)
+    assert e <= TOL, e
+    assert e <= FAITHFUL, e      # exact scaffold + fp64 epilogue: only the final fp32 rounding differs
+    B = x.shape[0]
+    _check_digits(to_np(F.ws_view(ws, L.xd_in, torch.int8, (B, 6, p.cols))),
+                  to_np(F.ws_view(ws, L.xdsum_in, torch.int32, (B, 6))), x)
+    if rank:
+        xq = to_np(F.ws_view(ws, L.xq_in, torch.int8, (B, p.cols)))
+        sx = to_np(F.ws_view(ws, L.sx_in, torch.float32, (B,)))
+        acc = to_np(F.ws_view(ws, L.acc_in, torch.int32, (B, rank)))
+        assert np.array_equal(xq, ref.xq)
+        assert np.array_equal(sx, ref.sx)
+        assert np.array_equal(acc.astype(np.int64), ref.acc)
+    return to_np(y), ref
+
+
+def _check_digits(xd, xdsum, x16):
+    """Digit planes are an exact balanced base-256 representation of x * 2^24."""
+    X = (x16.astype(np.float64) * 2.0 ** 24).astype(np.int64)
+    rec = np.zeros_like(X)
+    for dd in range(5, -1, -1):
+        rec = rec * 256 + xd[:, dd, :].astype(np.int64)
+    assert np.array_equal(rec, X)
+    assert np.array_equal(xdsum.astype(np.int64), xd.astype(np.int64).sum(axis=2))
+
+
+@pytest.mark.parametrize("d_in,d_out", S.PROJ_SWEEP_SHAPES)
+@pytest.mark.parametrize("rank", S.PROJ_SWEEP_RANKS)
+@pytest.mark.parametrize("batch", S.PROJ_SWEEP_BATCHES)
+def test_proj_sweep_parity(d_in, d_out, rank, batch):
+    p, x = S.proj_workload(d_in, d_out, rank, batch)
+    _proj_case(p, x, rank)
+
+
+@pytest.mark.parametrize("rows,cols,rank,batch", [(1064, 256, 8, 3), (40, 512, 0, 9), (17, 256, 4, 1),
+                                                   (8512, 2048, 32, 13)])
+def test_proj_ragged_and_rank0(rows, cols, rank, batch):
+    rng = np.random.default_rng(rows + cols + rank + batch)
+    p = S.gen_proj(rng, rows, cols, rank)
+    x = rng.normal(size=(batch, cols)).astype(np.float16)
+    if batch > 1:
+        x[1] = 0          # all-zero activation row: codes 0, scale 1
+    _proj_case(p, x, rank)
+
+
+def test_proj_all_plus_one_gives_alpha_sum():
+    rng = np.random.default_rng(5)
+    p = S.gen_proj(rng, 48, 512, 0)
+    p.bits[:] = 0xFFFFFFFF
+    x = rng.normal(size=(2, 512)).astype(np.float16)
+    y, _ = _proj_case(p, x, 0)
+    closed = p.alpha.astype(np.float64)[None] * x.astype(np.float64).sum(1, keepdims=True)
+    assert rel_err(y, closed) <= 1e-5
+
+
+def test_proj_rank0_bit_identical_to_zero_B():
+    rng = np.random.default_rng(6)
+    p = S.gen_proj(rng, 256, 1024, 16)
+    x = rng.normal(size=(1, 1024)).astype(np.float16)
+    p0 = S.ProjWeights(p.rows, p.cols, p.bits, p.alpha, None, None, None, None)
+    pz = S.ProjWeights(p.rows, p.cols, p.bits, p.alpha, p.A, p.sA, np.zeros_like(p.B), p.sB)
+    y0, _ = _proj_case(p0, x, 0)
+    yz, _ = _proj_case(pz, x, 16)
+    assert np.array_equal(y0, yz)
+
+
+# ---------------------------------------------------------------- layer step
+
+class LayerRun:
+    def __init__(self, d, lw, st):
+        self.d = d
+        self.dw = F.DeviceLayer.from_host(lw)
+        self.ds = F.DeviceState.from_host(st)
+        self.ws = F.workspace(d)
+        self.L = F.workspace_layout(d)
+
+    def step(self, res_np):
+        res = torch.from_numpy(np.ascontiguousarray(res_np)).to(DEV)
+        F.layer_step(self.d, self.dw, self.ds, res, self.ws)
+        _sync()
+        return to_np(res)
+
+    def view(self, name, dtype, shape):
+        return to_np(F.ws_view(self.ws, getattr(self.L, name), dtype, shape))
+
+
+def _check_layer_step(run, lw, d, ost, res_in):
+    got = run.step(res_in)
+    t = O.layer_step(res_in, lw, ost, d)
+    B, D, E = d.batch, d.d_model, d.d_inner
+    errs = {
+        "res": rel_err(got, t.res),
+        "conv": rel_err(to_np(run.ds.conv), t.conv),
+        "ssm": rel_err(to_np(run.ds.ssm), t.ssm),
+        "zxbcdt": rel_err(run.view("zxbcdt", torch.float64, (B, d.in_rows)), t.zxbcdt),
+        "xc": rel_err(run.view("xc", torch.float64, (B, d.conv_dim)), t.xc),
+        "g": rel_err(run.view("g", torch.float64, (B, E)), t.g),
+    }
+    bad = {k: v for k, v in errs.items() if v > TOL}
+    assert not bad, bad
+    loose = {k: v for k, v in errs.items() if v > FAITHFUL}
+    assert not loose, loose
+    # fp16 activations entering the projections: identical to the oracle's
+    assert np.array_equal(run.view("x_in", torch.float16, (B, D)), t.x_in)
+    assert np.array_equal(run.view("x_out", torch.float16, (B, E)), t.x_out)
+    if d.rank:
+        # int8 codes, scales and int8 x int8 -> int32 partials: bit-exact
+        for pre, tr in (("in", t.proj_in), ("out", t.proj_out)):
+            K = D if pre == "in" else E
+            assert np.array_equal(run.view(f"xq_{pre}", torch.int8, (B, K)), tr.xq)
+            assert np.array_equal(run.view(f"sx_{pre}", torch.float32, (B,)), tr.sx)
+            assert np.array_equal(run.view(f"acc_{pre}", torch.int32, (B, d.rank)).astype(np.int64), tr.acc)
+    _check_digits(run.view("xd_in", torch.int8, (B, 6, D)), run.view("xdsum_in", torch.int32, (B, 6)), t.x_in)
+    return t
+
+
+@pytest.mark.parametrize("name,steps", [("layer_d256_b1_16steps", 16), ("layer_d2048_b1_256steps", 48)])
+def test_layer_step_parity(name, steps):
+    d, lw, st, xs = S.layer_workload(name, steps=steps)
+    run = LayerRun(d, lw, st)
+    ost = st
+    for t in range(steps):
+        tr = _check_layer_step(run, lw, d, ost, xs[t])
+        ost = O.State(tr.conv, tr.ssm)
+
+
+@pytest.mark.parametrize("batch", [9, 16])
+def test_layer_step_batched_parity(batch):
+    d, lw, st, xs = S.layer_workload("layer_d256_b1_16steps", steps=4, batch=batch)
+    run = LayerRun(d, lw, st)
+    ost = st
+    for t in range(4):
+        tr = _check_layer_step(run, lw, d, ost, xs[t])
+        ost = O.State(tr.conv, tr.ssm)
+
+
+def test_layer_dt_zero_leaves_ssm_state():
+    d, lw, st, xs = S.layer_workload("layer_d256_b1_16steps", steps=2)
+    lw.dt_bias[:] = -1e4
+    rng = np.random.default_rng(3)
+    st.ssm[:] = rng.normal(size=st.ssm.shape)
+    run = LayerRun(d, lw, st)
+    run.step(xs[0])
+    assert np.array_equal(to_np(run.ds.ssm), st.ssm)
+
+
+def test_layer_graph_replay_matches_eager():
+    d, lw, st, xs = S.layer_workload("layer_d2048_b1_256steps", steps=6)
+    eager = LayerRun(d, lw, st)
+    outs = [eager.step(xs[t]) for t in range(6)]
+    g_run = LayerRun(d, lw, st)
+    res = torch.zeros((d.batch, d.d_model), dtype=torch.float32, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        res.copy_(torch.from_numpy(xs[0]).to(DEV))
+        F.layer_step(d, g_run.dw, g_run.ds, res, g_run.ws)    # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    _sync()
+    # restore state, then capture one step and replay it
+    g_run.ds.conv.zero_(); g_run.ds.ssm.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        F.layer_step(d, g_run.dw, g_run.ds, res, g_run.ws)
+    for t in range(6):
+        res.copy_(torch.from_numpy(xs[t]).to(DEV))
+        graph.replay()
+        _sync()
+        assert np.array_equal(to_np(res), outs[t])
+    assert np.array_equal(to_np(g_run.ds.ssm), to_np(eager.ds.ssm))
+
+
+def test_state_checkpoint_resume_bit_identical():
+    d, lw, st, xs = S.layer_workload("layer_d256_b1_16steps", steps=8)
+    run = LayerRun(d, lw, st)
+    for t in range(4):
+        run.step(xs[t])
+    saved = (run.ds.conv.clone(), run.ds.ssm.clone())
+    first = [run.step(xs[t]) for t in range(4, 8)]
+    run.ds.conv.copy_(saved[0]); run.ds.ssm.copy_(saved[1])
+    again = [run.step(xs[t]) for t in range(4, 8)]
+    for a, b in zip(first, again):
+        assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------------------- model decode
+
+def _teacher_forced(m, tok0, steps, n_check_tokens=True):
+    d = m.dims
+    dm = F.DeviceModel.from_host(m)
+    states = [F.DeviceState.zeros(d) for _ in m.layers]
+    call = F.ModelCall(dm, states)
+    ws = F.workspace(d, len(m.layers), m.vocab)
+    tok_in = torch.from_numpy(tok0.astype(np.int32)).to(DEV)
+    tok_out = torch.zeros(d.batch, dtype=torch.int32, device=DEV)
+    logits = torch.zeros((d.batch, m.vocab), dtype=torch.float32, device=DEV)
+    ost = [S.zero_state(d) for _ in m.layers]
+    ost = [O.State(s.conv, s.ssm) for s in ost]
+    tok = tok0.astype(np.int32)
+    for t in range(steps):
+        tok_in.copy_(torch.from_numpy(tok).to(DEV))
+        call(tok_in, tok_out, ws, logits)
+        _sync()
+        tr = O.model_step(tok, m, ost)
+        e = rel_err(to_np(logits), tr.logits)
+        assert e <= TOL, (t, e)
+        for l in (0, len(m.layers) - 1):
+            assert rel_err(to_np(states[l].ssm), tr.states[l].ssm) <= TOL
+            assert rel_err(to_np(states[l].conv), tr.states[l].conv) <= TOL
+        got = to_np(tok_out)
+        gl = to_np(logits)
+        assert np.array_equal(got, np.argmax(gl, axis=-1))          # argmax of its own logits
+        for b in range(d.batch):
+            if got[b] != tr.tokens[b]:
+                top = np.sort(tr.logits[b])[-2:]
+                assert top[1] - top[0] <= 4 * TOL * np.sqrt(np.mean(tr.logits[b] ** 2))
+        ost = tr.states
+        tok = tr.tokens
+
+
+def test_model_decode_small_parity():
+    d = S.LAYER_SMALL.with_batch(2)
+    rng = np.random.default_rng(30)
+    m = S.gen_model(rng, d, 3, 1000)
+    _teacher_forced(m, S.gen_tokens(rng, 2, 1000), 6)
+
+
+def test_model_decode_1p3b_parity():
+    m, tok = S.model_workload("model_48x2048_v50280_b1_greedy512")
+    _teacher_forced(m, tok, 2)
