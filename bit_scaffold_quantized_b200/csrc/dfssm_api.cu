@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "dfssm.h"
@@ -444,3 +445,62 @@ int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16
 }
 
 }  // extern "C"
+
+// ---- projection with library-owned scratch ----------------------------------
+//
+// For callers that cannot call cudaMalloc: dfssm_proj_forward needs a workspace,
+// and some callers have no way to obtain one (a plugin whose host framework hands
+// it no allocator, or a latency-critical thread that must not risk the device-wide
+// synchronisation cudaMalloc/cudaFree can cause).  This variant runs the same
+// kernels with its scratch in a fixed file-scope device array instead.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB per device, held until exit
+constexpr int kNoAllocMaxDevices = 64;
+
+// The name below is only a host-side handle; its device address is looked up once
+// per device with cudaGetSymbolAddress and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  REQUIRE(dev >= 0 && dev < kNoAllocMaxDevices, DFSSM_ERR_DEVICE, "device %d beyond the %d supported", dev,
+          kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(DFSSM_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return DFSSM_OK;
+}
+
+}  // namespace
+
+extern "C" int dfssm_proj_forward_noalloc(const dfssm_proj* p, int rank, int batch, const uint16_t* x,
+                                          float* y, void* stream) {
+  int rc = check_proj(p, rank, "proj");
+  if (rc) return rc;
+  REQUIRE(batch > 0, DFSSM_ERR_INVALID_ARG, "batch must be positive");
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(y);
+  dfssm_ws_layout L;
+  if ((rc = dfssm_proj_workspace_layout(p->rows, p->cols, rank, batch, &L))) return rc;
+  REQUIRE(L.total_bytes <= kNoAllocScratchBytes, DFSSM_ERR_WORKSPACE_TOO_SMALL,
+          "this projection needs %zu bytes of scratch but the built-in scratch holds %zu bytes; "
+          "use dfssm_proj_forward with a caller workspace", L.total_bytes, kNoAllocScratchBytes);
+  void* ws = nullptr;
+  if ((rc = noalloc_scratch(&ws))) return rc;
+  // Every region of the projection's scratch is written before it is read, so
+  // nothing left by an earlier call needs clearing.
+  return dfssm_proj_forward(p, rank, batch, x, y, ws, kNoAllocScratchBytes, stream);
+}

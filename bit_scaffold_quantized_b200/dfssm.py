@@ -28,7 +28,8 @@ LAYOUT_ROWMAJOR, LAYOUT_TILED = 0, 1
 
 EXPORTS = [
     "dfssm_packed_words", "dfssm_pack_weights", "dfssm_repack_bits",
-    "dfssm_proj_workspace_bytes", "dfssm_proj_forward", "dfssm_proj_workspace_layout",
+    "dfssm_proj_workspace_bytes", "dfssm_proj_forward", "dfssm_proj_forward_noalloc",
+    "dfssm_proj_workspace_layout",
     "dfssm_workspace_bytes", "dfssm_workspace_layout", "dfssm_layer_step",
     "dfssm_model_decode", "dfssm_model_decode_launches", "dfssm_last_error", "dfssm_version",
 ]
@@ -88,6 +89,7 @@ def lib() -> C.CDLL:
     L.dfssm_proj_workspace_bytes.restype = sz
     L.dfssm_proj_workspace_layout.argtypes = [i, i, i, i, C.POINTER(CWsLayout)]
     L.dfssm_proj_forward.argtypes = [C.POINTER(CProj), i, i, vp, vp, vp, sz, vp]
+    L.dfssm_proj_forward_noalloc.argtypes = [C.POINTER(CProj), i, i, vp, vp, vp]
     L.dfssm_workspace_bytes.argtypes = [C.POINTER(CDims), i, i]
     L.dfssm_workspace_bytes.restype = sz
     L.dfssm_workspace_layout.argtypes = [C.POINTER(CDims), i, i, C.POINTER(CWsLayout)]
@@ -251,6 +253,12 @@ def proj_forward(p: DeviceProj, rank: int, x, y, ws, stream=None) -> None:
     cp = p.c()
     _check(lib().dfssm_proj_forward(C.byref(cp), rank, x.shape[0], _ptr(x), _ptr(y), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def proj_forward_noalloc(p: DeviceProj, rank: int, x, y, stream=None) -> None:
+    """dfssm_proj_forward without a caller workspace (library-owned 4 MiB scratch)."""
+    cp = p.c()
+    _check(lib().dfssm_proj_forward_noalloc(C.byref(cp), rank, x.shape[0], _ptr(x), _ptr(y), _stream(stream)))
 
 
 def workspace_layout(d, n_layer: int = 0, vocab: int = 0) -> CWsLayout:

@@ -170,6 +170,20 @@ DFSSM_API size_t dfssm_proj_workspace_bytes(int rows, int cols, int rank, int ba
  * at the offsets dfssm_proj_workspace_layout reports. */
 DFSSM_API int dfssm_proj_forward(const dfssm_proj* p, int rank, int batch, const uint16_t* x, float* y,
                        void* ws, size_t ws_bytes, void* stream);
+/* Same projection as dfssm_proj_forward, for callers that cannot call cudaMalloc
+ * (no allocator is available to them, or they must not risk the device-wide
+ * synchronisation an allocation can cause).  The paper has no counterpart; this
+ * is a convenience of this library.  The scratch is a fixed 4 MiB array inside
+ * the library that every GPU which loads the library holds until exit; a call
+ * whose dfssm_proj_workspace_bytes exceeds 4 MiB returns
+ * DFSSM_ERR_WORKSPACE_TOO_SMALL without enqueueing anything.  The first call on
+ * a device looks up that device's address of the array, so make it before any
+ * stream capture.  All calls on a device share the one array, which keeps the
+ * last call's contents: calls whose kernels may overlap on the GPU (different
+ * streams without ordering) race on it.  Nothing in it needs to start at zero. */
+DFSSM_API int dfssm_proj_forward_noalloc(const dfssm_proj* p, int rank, int batch, const uint16_t* x,
+                                         float* y, void* stream);
+
 DFSSM_API int dfssm_proj_workspace_layout(int rows, int cols, int rank, int batch, dfssm_ws_layout* out);
 
 /* ---- decode step -------------------------------------------------------- */
