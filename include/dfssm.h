@@ -53,13 +53,14 @@ enum { DFSSM_DTYPE_F16 = 0, DFSSM_DTYPE_F32 = 1 };
  * column 32k+j, bit = 1 encodes +1 and bit = 0 encodes -1.  TILED: the same bits
  * permuted into 16-row x 256-column tiles of 128 words (rows padded up to a
  * multiple of 16 with clear bits).  For weight (row, col) with r16 = row % 16,
- * c = col % 256, kt = c / 64, ch = (c % 64) / 16, c16 = c % 16:
- *   lane = (r16 % 8) * 4 + (c16 % 8) / 2,  q = r16 / 8 + 2 * (c16 / 8),  s = 4*ch + q,
- *   bit  = 15 - s for even c16, 31 - s for odd c16,
+ * c = col % 256, kt = c / 64, ch = (c % 64) / 32, c32 = c % 32:
+ *   lane = (r16 % 8) * 4 + (c32 % 16) / 4,  q = r16 / 8 + 2 * (c32 / 16),
+ *   s = 4 * ch + q,  bit = s + 8 * (c32 % 4),
  *   word = ((row / 16) * (cols / 256) + col / 256) * 128 + lane * 4 + kt.
- * Each warp lane then reads one 16-byte vector per tile and forms its m16n8k16
- * tensor-core A fragment with one shift and one mask per fp16 pair.  The
- * projection kernels consume TILED words only. */
+ * Each warp lane reads one 16-byte vector per tile; (word >> s) & 0x01010101 is
+ * then its int8 A-fragment register q of 32-column chunk ch of an m16n8k32
+ * tensor-core product, with bytes 0/1 for -1/+1.  The projection kernels consume
+ * TILED words only. */
 enum { DFSSM_LAYOUT_ROWMAJOR = 0, DFSSM_LAYOUT_TILED = 1 };
 
 /* Shape of one layer.  in_proj: d_model -> 2*d_inner + 2*ngroups*d_state + nheads
