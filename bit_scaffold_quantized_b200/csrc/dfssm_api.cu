@@ -148,7 +148,7 @@ void layer_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* 
   L->xdsum_in = bp.take(4 * B * kDigits);
   L->zxbcdt = bp.take(8 * B * in_rows(d));
   L->xc = bp.take(8 * B * conv_dim(d));
-  L->g = bp.take(8 * B * E);
+  L->g = bp.take(4 * B * E);
   L->x_out = bp.take(2 * B * E);
   L->xq_out = bp.take(B * E);
   L->sx_out = bp.take(4 * B);
@@ -176,7 +176,7 @@ struct Act {       // one activation's preprocessing outputs
 struct Bufs {
   unsigned* status;
   Act in, out;
-  double* zxbcdt; double* xc; double* g;
+  double* zxbcdt; double* xc; float* g;
   float* res; unsigned char* scratch;
 };
 
@@ -190,7 +190,7 @@ Bufs bind(void* ws, const dfssm_ws_layout& L) {
               at<int>(ws, L.xdsum_out)};
   b.zxbcdt = at<double>(ws, L.zxbcdt);
   b.xc = at<double>(ws, L.xc);
-  b.g = at<double>(ws, L.g);
+  b.g = at<float>(ws, L.g);
   b.res = L.res == kNone ? nullptr : at<float>(ws, L.res);
   b.scratch = at<unsigned char>(ws, L.scratch);
   return b;
@@ -264,7 +264,7 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   sa.state = s->ssm_state; sa.g = b.g;
   k_ssm<<<dim3(d->nheads * (d->headdim / kSsmRows), B), kSsmThreads, size_t(16) * d->d_state, st>>>(sa);
   CHECK_LAUNCH("k_ssm");
-  if ((rc = launch_prologue<double, 0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
+  if ((rc = launch_prologue<float, 0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, B, b.out);
   po.out = res;
   return launch_proj<EPI_RESID>(po, st);

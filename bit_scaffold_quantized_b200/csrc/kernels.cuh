@@ -355,7 +355,7 @@ struct SsmArgs {
   const float* A_log;
   const float* D;
   float* state;          // fp32 [B][H][P][N]
-  double* g;             // fp64 [B][E]
+  float* g;              // fp32 [B][E]
 };
 
 constexpr int kSsmRows = 16;     // head rows per block
@@ -364,7 +364,7 @@ constexpr int kSsmThreads = 256;
 // grid (H * P/16, B).  One warp per state row of N fp32 values (float4 per lane),
 // arithmetic in fp64, state stored back in fp32:
 //   dt = softplus(dt_raw + dt_bias), dA = exp(-dt * exp(A_log)),
-//   h' = dA h + (x dt) B,  y = C . h' + D x,  g = y * silu(z).
+//   h' = dA h + (x dt) B,  y = C . h' + D x,  g = y * silu(z) (stored fp32).
 __global__ void __launch_bounds__(kSsmThreads) k_ssm(SsmArgs a) {
   extern __shared__ __align__(16) double sbc[];   // [2N]: B then C
   const int tiles_per_head = a.P / kSsmRows;
@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kSsmThreads) k_ssm(SsmArgs a) {
     y = warp_sum_d(y);
     if (lane == 0) {
       y = fma(Dh, x, y);
-      a.g[size_t(b) * a.E + e] = y * silu_d(zr[e]);
+      a.g[size_t(b) * a.E + e] = float(y * silu_d(zr[e]));
     }
   }
 }

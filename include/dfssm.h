@@ -132,7 +132,7 @@ typedef struct dfssm_ws_layout {
   size_t xdsum_in;   /* int32 [batch][6]          digit-plane sums */
   size_t zxbcdt;     /* fp64  [batch][in_rows]    in_proj output [z|x|B|C|dt] */
   size_t xc;         /* fp64  [batch][conv_dim]   conv output after SiLU */
-  size_t g;          /* fp64  [batch][d_inner]    y * silu(z) */
+  size_t g;          /* fp32  [batch][d_inner]    y * silu(z) */
   size_t x_out;      /* fp16  [batch][d_inner]    gated-norm output (out_proj activation) */
   size_t xq_out;     /* int8  [batch][d_inner] */
   size_t sx_out;     /* fp32  [batch] */

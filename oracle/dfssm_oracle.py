@@ -8,7 +8,8 @@ does.  It shares no code with the CUDA library and imports nothing from it.
 Arithmetic is fp64 except where the method fixes a storage format or where a
 floating-point value decides an integer:
   * activations entering a projection are stored as fp16;
-  * SSM state, conv state and the residual stream are stored as fp32;
+  * SSM state, conv state, the residual stream and the gated value y*silu(z)
+    are stored as fp32;
   * the int8 activation quantiser takes its decision in fp32 (scale = amax/127
     as an IEEE fp32 divide, code = round-half-even of x/scale in fp32), the
     precision the kernel uses, so both sides take the same integer decision;
@@ -252,7 +253,7 @@ class LayerTrace:
     zxbcdt: np.ndarray       # fp64 [B, in_rows]
     xc: np.ndarray           # fp64 [B, conv_dim] conv output
     y: np.ndarray            # fp64 [B, d_inner] SSM output (before gate)
-    g: np.ndarray            # fp64 [B, d_inner] gated value y * silu(z)
+    g: np.ndarray            # [B, d_inner] gated value y * silu(z), stored as fp32 (held in fp64)
     x_out: np.ndarray        # fp16 [B, d_inner] gated-norm output (out_proj activation)
     proj_out: ProjTrace
 
@@ -299,7 +300,9 @@ def layer_step(res: np.ndarray, lw, st, d) -> LayerTrace:
         y[:, hs], ssm_new[:, hs] = ssm_step(st.ssm[:, hs], xs[:, hs], Bg[:, gi], Cg[:, gi],
                                             dt_raw[:, hs], lw.dt_bias[hs], lw.A_log[hs], lw.D[hs])
     y = y.reshape(d.batch, E)
-    g = y * silu(z)
+    # the gated value is an activation between two kernels and is stored as fp32,
+    # like the residual stream; the gated RMSNorm reads the stored values
+    g = (y * silu(z)).astype(np.float32).astype(np.float64)
     gw = g.reshape(d.batch, G, E // G)
     xo = rmsnorm(gw, lw.gnorm_w.reshape(G, E // G)).reshape(d.batch, E)
     x_out = xo.astype(np.float16)

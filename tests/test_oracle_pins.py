@@ -429,7 +429,9 @@ def test_layer_pieces_compose():
     y, _ = O.ssm_step(st.ssm, xc[:, :E].reshape(d.batch, d.nheads, d.headdim), xc[:, E:E + N],
                       xc[:, E + N:], t.zxbcdt[:, E + C:], lw.dt_bias, lw.A_log, lw.D)
     np.testing.assert_array_equal(y.reshape(d.batch, E), t.y)
-    xo = O.gated_rmsnorm(t.y, t.zxbcdt[:, :E], lw.gnorm_w).astype(np.float16)
+    g32 = (t.y * O.silu(t.zxbcdt[:, :E])).astype(np.float32)
+    assert np.array_equal(t.g, g32.astype(np.float64))
+    xo = O.rmsnorm(g32, lw.gnorm_w).astype(np.float16)
     assert np.array_equal(xo, t.x_out)
 
 

@@ -164,7 +164,7 @@ def _check_layer_step(run, lw, d, ost, res_in):
         "ssm": rel_err(to_np(run.ds.ssm), t.ssm),
         "zxbcdt": rel_err(run.view("zxbcdt", torch.float64, (B, d.in_rows)), t.zxbcdt),
         "xc": rel_err(run.view("xc", torch.float64, (B, d.conv_dim)), t.xc),
-        "g": rel_err(run.view("g", torch.float64, (B, E)), t.g),
+        "g": rel_err(run.view("g", torch.float32, (B, E)), t.g),
     }
     bad = {k: v for k, v in errs.items() if v > TOL}
     assert not bad, bad
