@@ -130,6 +130,19 @@ DFSSM_DEV void fp16_digits(uint16_t h, int8_t (&dg)[kDigits]) {
   }
 }
 
+// Same decision as quant_code with a multiply by rcp = 1/sx (fp32, rounded) in
+// place of the divide: x * rcp is within 3 * 2^-24 |x/sx| of the correctly rounded
+// quotient, so rint agrees unless the product lies within that distance of a
+// half-integer, where the IEEE divide decides.
+DFSSM_DEV int quant_code_fast(float x, float sx, float rcp) {
+  const float t = x * rcp;
+  const float r = rintf(t);
+  const float off = fabsf(fabsf(t - r) - 0.5f);
+  int q = int(r);
+  if (off <= 4.0e-5f) q = __float2int_rn(__fdiv_rn(x, sx));
+  return max(-127, min(127, q));
+}
+
 // int8 activation code, decided in fp32: clamp(rint(x / sx), -127, 127).
 DFSSM_DEV int quant_code(float x, float sx) {
   int q = __float2int_rn(__fdiv_rn(x, sx));

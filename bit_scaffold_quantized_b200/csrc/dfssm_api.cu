@@ -270,6 +270,154 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   return launch_proj<EPI_RESID>(po, st);
 }
 
+// ---- persistent whole-token kernel (batch 1) ------------------------------------
+
+int align16i(int v) { return (v + 15) & ~15; }
+
+struct PPlan {
+  bool ok = false;
+  int grid = 0;
+  PSmem sm{};
+  char why[160] = {0};
+};
+
+int device_sm_count(int* nsm, int* smem_optin) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  return e == cudaSuccess ? 0 : -1;
+}
+
+// Whether (and how) one token of these dims runs as the persistent kernel.
+PPlan plan_persistent(const dfssm_dims* d) {
+  PPlan p;
+  auto no = [&](const char* why) {
+    snprintf(p.why, sizeof p.why, "%s", why);
+    return p;
+  };
+  int nsm = 0, optin = 0;
+  if (device_sm_count(&nsm, &optin)) return no("device query failed");
+  const int D = d->d_model, E = d->d_inner, H = d->nheads, N = d->d_state, R = d->rank;
+  if (d->batch != 1) return no("batch != 1");
+  if (N % 16 || H % 16) return no("d_state and nheads must be multiples of 16");
+  if (R % 8) return no("rank must be a multiple of 8");
+  const int units = E / 16;
+  const int grid = std::min(nsm, units);
+  if ((units + grid - 1) / grid > kPMaxUnits) return no("more than 2 SSM row units per block");
+  if (D / 16 > grid) return no("more out_proj tiles than blocks");
+  if (2 * N / 16 > grid || R > grid) return no("more B/C tiles or LoRA rows than blocks");
+  const int kg_in = D / kTileCols, kg_out = E / kTileCols, Kmax = std::max(D, E);
+  PSmem& m = p.sm;
+  int off = 0;
+  auto take = [&](int bytes) { int at = off; off = align16i(off + std::max(bytes, 16)); return at; };
+  m.in_tiles = take(kPMaxInTiles * kg_in * 512);
+  m.in_bq = take(kPMaxInTiles * 16 * R);
+  m.in_alpha = take(kPMaxInTiles * 32);
+  m.in_sb = take(kPMaxInTiles * 32);
+  m.convw_x = take(kPMaxUnits * 128);
+  m.convb_x = take(kPMaxUnits * 32);
+  m.cst_x = take(3 * kPMaxUnits * 64);
+  m.bc_bq = take(2 * N * R);
+  m.bc_sb = take(4 * N);
+  m.bc_convw = take(16 * N);
+  m.bc_convb = take(4 * N);
+  m.bc_cst = take(24 * N);
+  m.a_in = take(D);
+  m.prenorm = take(2 * D);
+  m.sa_in = take(2 * R);
+  m.hd_dtb = take(4 * H);
+  m.hd_alog = take(4 * H);
+  m.hd_d = take(4 * H);
+  m.state = take(kPMaxUnits * 16 * N * 4);
+  off = std::max(off, 2 * kHeadChunkRows * 2 * D);     // the LM-head ring reuses this group
+  m.ab_end = off;
+  m.out_tile = take(kg_out * 512);
+  m.out_bq = take(16 * R);
+  m.out_alpha = take(32);
+  m.out_sb = take(32);
+  m.a_out = take(E);
+  m.gnorm = take(2 * E);
+  m.sa_out = take(2 * R);
+  m.cd_end = off;
+  m.res = take(4 * D);
+  m.gbuf = take(4 * Kmax);
+  m.x16 = take(2 * Kmax);
+  m.digits = take(kDigits * (Kmax + 16));
+  m.xq = take(Kmax);
+  m.part = take(16 * 16 * kDigits * 4);
+  m.yin = take(kPMaxInTiles * 16 * 8);
+  m.bcx = take(2 * N * 8);
+  m.bcst_new = take(3 * 2 * N * 4);
+  m.u_in = take(8 * std::max(R, 1));
+  m.u_out = take(8 * std::max(R, 1));
+  m.misc = take(4 * std::max({D + grid, 4 * N, 2 * R, 2 * grid, kHeadChunkRows}));
+  m.total = off;
+  if (m.total > optin) return no("shared memory plan exceeds the per-block limit");
+  p.grid = grid;
+  p.ok = true;
+  return p;
+}
+
+PLayer player(const dfssm_layer_weights& w, const dfssm_layer_state& s) {
+  PLayer L;
+  L.prenorm_w = w.prenorm_w;
+  L.in_bits = w.in.bits; L.in_alpha = w.in.alpha; L.in_A = w.in.A; L.in_sA = w.in.sA; L.in_B = w.in.B;
+  L.in_sB = w.in.sB;
+  L.conv_w = w.conv_w; L.conv_b = w.conv_b; L.dt_bias = w.dt_bias; L.A_log = w.A_log; L.D = w.D;
+  L.gnorm_w = w.gnorm_w;
+  L.out_bits = w.out.bits; L.out_alpha = w.out.alpha; L.out_A = w.out.A; L.out_sA = w.out.sA;
+  L.out_B = w.out.B; L.out_sB = w.out.sB;
+  L.conv_state = s.conv_state; L.ssm_state = s.ssm_state;
+  return L;
+}
+
+// Launch one token (model mode) or one layer step (layer mode) as the persistent kernel.
+int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int vocab,
+                      const dfssm_layer_weights* layers, const dfssm_layer_state* states, const uint16_t* embed,
+                      const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out, float* logits,
+                      float* residual, void* ws, const dfssm_ws_layout& WL, int head_blocks, cudaStream_t st) {
+  static_assert(sizeof(PParams) < 32000, "kernel parameter block too large");
+  PParams a;
+  std::memset(&a, 0, sizeof a);
+  const int D = d->d_model, E = d->d_inner, N = d->d_state, R = d->rank;
+  a.n_layer = n_layer; a.D = D; a.E = E; a.H = d->nheads; a.P = d->headdim; a.N = N; a.R = R;
+  a.in_rows = in_rows(d); a.C = conv_dim(d); a.vocab = vocab;
+  a.kg_in = D / kTileCols; a.kg_out = E / kTileCols;
+  a.units = E / 16; a.grid = plan.grid;
+  a.n_bc_tiles = 2 * N / 16; a.dt_tile0 = (2 * E + 2 * N) / 16; a.out_tiles = D / 16;
+  a.layer_mode = residual != nullptr;
+  a.sm = plan.sm;
+  a.embed = embed; a.normf_w = normf_w; a.tok_in = tok_in; a.tok_out = tok_out; a.logits = logits;
+  a.residual = residual;
+  unsigned char* scratch = at<unsigned char>(ws, WL.scratch);
+  unsigned char* pbase = scratch + align256(size_t(8) * d->batch * std::max(head_blocks, 1));
+  a.status = at<unsigned>(ws, WL.status);
+  a.ctl = reinterpret_cast<unsigned*>(pbase);
+  unsigned long long* wd = reinterpret_cast<unsigned long long*>(pbase + 256);
+  a.x_r = wd;      wd += D + plan.grid;
+  a.x_g = wd;      wd += E;
+  a.x_bc = wd;     wd += 4 * N;
+  a.x_uin = wd;    wd += 2 * R;
+  a.x_uout = wd;   wd += 2 * R;
+  a.x_head = wd;   wd += 2 * plan.grid;
+  Bufs b = bind(ws, WL);
+  a.d_x_in = b.in.x; a.d_xq_in = b.in.xq; a.d_sx_in = b.in.sx; a.d_acc_in = b.in.acc; a.d_u_in = b.in.u;
+  a.d_xd_in = b.in.xd; a.d_xdsum_in = b.in.xdsum; a.d_zx = b.zxbcdt; a.d_xc = b.xc; a.d_g = b.g;
+  a.d_x_out = b.out.x; a.d_xq_out = b.out.xq; a.d_sx_out = b.out.sx; a.d_acc_out = b.out.acc;
+  a.d_u_out = b.out.u; a.d_xd_out = b.out.xd; a.d_xdsum_out = b.out.xdsum; a.d_res = b.res;
+  for (int l = 0; l < n_layer; ++l) a.L[l] = player(layers[l], states[l]);
+  cudaError_t e = cudaFuncSetAttribute(k_decode_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       plan.sm.total);
+  if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "persistent smem attribute: %s", cudaGetErrorString(e));
+  void* args[] = {&a};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_decode_persistent), dim3(plan.grid), dim3(kPBlock),
+                                  args, size_t(plan.sm.total), st);
+  if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "persistent launch: %s", cudaGetErrorString(e));
+  CHECK_LAUNCH("k_decode_persistent");
+  return DFSSM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -278,6 +426,7 @@ int dfssm_version(void) { return 100; }
 
 int dfssm_model_decode_launches(const dfssm_dims* d, int n_layer, int vocab) {
   if (check_dims(d) || n_layer < 1 || n_layer > kMaxLayers || vocab < 1) return 0;
+  if (plan_persistent(d).ok) return 1;
   return 1 + 5 * n_layer + 2;
 }
 
@@ -397,7 +546,14 @@ int dfssm_layer_step(const dfssm_dims* d, const dfssm_layer_weights* w, const df
           L.total_bytes);
   Bufs b = bind(ws, L);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((rc = layer_multikernel(d, w, s, residual, b, st))) return rc;
+  const PPlan plan = plan_persistent(d);
+  if (plan.ok) {
+    if ((rc = launch_persistent(plan, d, 1, 0, w, s, nullptr, nullptr, nullptr, nullptr, nullptr, residual, ws, L,
+                                0, st)))
+      return rc;
+  } else if ((rc = layer_multikernel(d, w, s, residual, b, st))) {
+    return rc;
+  }
   return ok();
 }
 
@@ -426,6 +582,13 @@ int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16
   Bufs b = bind(ws, L);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int B = d->batch, D = d->d_model;
+  const PPlan plan = plan_persistent(d);
+  if (plan.ok) {
+    if ((rc = launch_persistent(plan, d, n_layer, vocab, layers, states, embed, normf_w, tok_in, tok_out, logits,
+                                nullptr, ws, L, kHeadBlocks, st)))
+      return rc;
+    return ok();
+  }
   k_embed<<<B, 256, 0, st>>>(embed, tok_in, vocab, D, b.res, b.status);
   CHECK_LAUNCH("k_embed");
   for (int l = 0; l < n_layer; ++l)

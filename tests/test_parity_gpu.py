@@ -136,6 +136,10 @@ def test_proj_rank0_bit_identical_to_zero_B():
 
 # ---------------------------------------------------------------- layer step
 
+# small shape the batch-1 persistent kernel accepts (nheads and d_state multiples of 16)
+LAYER_SMALL_P = S.Dims(batch=1, d_model=256, d_inner=512, nheads=16, headdim=32, d_state=16, rank=8)
+
+
 class LayerRun:
     def __init__(self, d, lw, st):
         self.d = d
@@ -148,6 +152,7 @@ class LayerRun:
         res = torch.from_numpy(np.ascontiguousarray(res_np)).to(DEV)
         F.layer_step(self.d, self.dw, self.ds, res, self.ws)
         _sync()
+        assert int(self.view("status", torch.int32, (1,))[0]) == 0
         return to_np(res)
 
     def view(self, name, dtype, shape):
@@ -190,6 +195,20 @@ def test_layer_step_parity(name, steps):
     run = LayerRun(d, lw, st)
     ost = st
     for t in range(steps):
+        tr = _check_layer_step(run, lw, d, ost, xs[t])
+        ost = O.State(tr.conv, tr.ssm)
+
+
+def test_layer_step_persistent_small_parity():
+    rng = np.random.default_rng(40)
+    d = LAYER_SMALL_P
+    lw = S.gen_layer(rng, d)
+    st = S.zero_state(d)
+    xs = S.gen_layer_inputs(rng, d, 12)
+    assert F.launches_per_decode_step(d, 1, 1000) == 1      # takes the persistent kernel
+    run = LayerRun(d, lw, st)
+    ost = st
+    for t in range(12):
         tr = _check_layer_step(run, lw, d, ost, xs[t])
         ost = O.State(tr.conv, tr.ssm)
 
@@ -261,6 +280,7 @@ def _teacher_forced(m, tok0, steps, n_check_tokens=True):
     states = [F.DeviceState.zeros(d) for _ in m.layers]
     call = F.ModelCall(dm, states)
     ws = F.workspace(d, len(m.layers), m.vocab)
+    L = F.workspace_layout(d, len(m.layers), m.vocab)
     tok_in = torch.from_numpy(tok0.astype(np.int32)).to(DEV)
     tok_out = torch.zeros(d.batch, dtype=torch.int32, device=DEV)
     logits = torch.zeros((d.batch, m.vocab), dtype=torch.float32, device=DEV)
@@ -271,6 +291,7 @@ def _teacher_forced(m, tok0, steps, n_check_tokens=True):
         tok_in.copy_(torch.from_numpy(tok).to(DEV))
         call(tok_in, tok_out, ws, logits)
         _sync()
+        assert int(to_np(F.ws_view(ws, L.status, torch.int32, (1,)))[0]) == 0
         tr = O.model_step(tok, m, ost)
         e = rel_err(to_np(logits), tr.logits)
         assert e <= TOL, (t, e)
@@ -286,6 +307,13 @@ def _teacher_forced(m, tok0, steps, n_check_tokens=True):
                 assert top[1] - top[0] <= 4 * TOL * np.sqrt(np.mean(tr.logits[b] ** 2))
         ost = tr.states
         tok = tr.tokens
+
+
+def test_model_decode_small_persistent_parity():
+    rng = np.random.default_rng(31)
+    m = S.gen_model(rng, LAYER_SMALL_P, 3, 1000)
+    assert F.launches_per_decode_step(LAYER_SMALL_P, 3, 1000) == 1
+    _teacher_forced(m, S.gen_tokens(rng, 1, 1000), 6)
 
 
 def test_model_decode_small_parity():
