@@ -340,7 +340,7 @@ PPlan plan_persistent(const dfssm_dims* d) {
   m.gnorm = take(2 * E);
   m.sa_out = take(2 * R);
   m.cd_end = off;
-  m.res = take(4 * D);
+  m.res = take(4 * (D + grid));      // residual words + the exchange's token words
   m.gbuf = take(4 * Kmax);
   m.x16 = take(2 * Kmax);
   m.digits = take(kDigits * (Kmax + 16));

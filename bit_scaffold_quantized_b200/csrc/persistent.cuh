@@ -393,35 +393,82 @@ DFSSM_DEV void produce_cd(const PParams& a, const PWork& w, const PLayer& L, uns
 
 // ------------------------------------------------------------------ activation prep
 
-// fp16 of z = (v * rs) * w, correctly rounded from the fp64 product.  The fp32
-// product is within 4 * 2^-24 |z| of it; when that window holds no fp16 rounding
-// midpoint the fp32 result is already the answer, otherwise fp64 decides.
-DFSSM_DEV uint16_t norm_fp16(float v, double rs, float rs32, uint16_t wbits) {
-  const float wf = h2f(wbits);
+// Exact fp16 -> fp32 by bit construction for normal values (no convert
+// instruction); zero, subnormal and non-finite values take the hardware path.
+DFSSM_DEV float half_to_float_bits(uint32_t h) {
+  const uint32_t e = (h >> 10) & 0x1fu;
+  if (e == 0u || e == 31u) return h2f(uint16_t(h));
+  return __uint_as_float(((h & 0x8000u) << 16) | ((e + 112u) << 23) | ((h & 0x3ffu) << 13));
+}
+
+// x * 2^24 as an integer, exact for every finite fp16 (|result| < 2^40 fits int64;
+// the packed-digit path only calls it when |x| <= 127, where it fits int32).
+DFSSM_DEV int half_times_2p24(uint32_t h) {
+  const uint32_t e = (h >> 10) & 0x1fu, m = h & 0x3ffu;
+  const int X = e == 0u ? int(m) : int((m | 0x400u) << (e - 1u));
+  return (h & 0x8000u) ? -X : X;
+}
+
+// fp16 bits of z = (v * rs) * w, correctly rounded from the fp64 product.  The
+// fp32 product lies within 4 fp32 ulps of it; if its low 13 mantissa bits are more
+// than 4 away from the fp16 rounding midpoint (0x1000) and z is in the fp16 normal
+// range, rounding the fp32 value is already the answer (done here with integer
+// ops); otherwise fp64 decides.
+DFSSM_DEV uint16_t norm_fp16(float v, double rs, float rs32, float wf) {
   const float z = (v * rs32) * wf;
-  const uint16_t h = f2h(z);
-  const float az = fabsf(z);
-  const uint16_t hm = h & 0x7fffu;
-  const float ah = h2f(hm);
-  const float r = az - ah;
-  bool safe = (r == 0.f);
-  if (!safe && hm < 0x7bffu && hm > 0x0400u) {               // finite normal neighbours on both sides
-    const uint16_t nb = r > 0.f ? uint16_t(hm + 1) : uint16_t(hm - 1);
-    const float mid = 0.5f * (ah + h2f(nb));
-    safe = fabsf(az - mid) > 4.0f * 5.9604645e-8f * az;
+  const uint32_t bits = __float_as_uint(z);
+  const uint32_t ez = (bits >> 23) & 0xffu;
+  const int low13 = int(bits & 0x1fffu);
+  if (ez >= 113u && ez <= 141u && abs(low13 - 0x1000) > 4) {
+    uint32_t hm = ((ez - 112u) << 10) | ((bits >> 13) & 0x3ffu);
+    hm += low13 > 0x1000 ? 1u : 0u;
+    return uint16_t(hm | ((bits >> 16) & 0x8000u));
   }
-  if (safe) return h;
   return d2h((double(v) * rs) * double(wf));
 }
 
+// Round-to-nearest-even of |t| < 2^22 via the 1.5 * 2^23 add (no convert instruction).
+DFSSM_DEV int rint_small(float t, float* r) {
+  const float m = t + 12582912.0f;
+  *r = m - 12582912.0f;
+  return __float_as_int(m) - 0x4B400000;
+}
+
+// Same decision as quant_code: clamp(rint(x / sx), -127, 127) with the fp32 IEEE
+// divide; the product x * rcp is within 3 * 2^-24 |x/sx| of the correctly rounded
+// quotient, so the divide is only needed near a half-integer.
+DFSSM_DEV int quant_code_bits(float x, float sx, float rcp) {
+  const float t = x * rcp;
+  float r;
+  int q = rint_small(t, &r);
+  if (fabsf(fabsf(t - r) - 0.5f) <= 4.0e-5f) q = __float2int_rn(__fdiv_rn(x, sx));
+  return max(-127, min(127, q));
+}
+
+// Four consecutive fp16 values -> their packed balanced base-256 digit bytes, one
+// 32-bit word per digit plane (byte e = element e); |x| <= 127 (4 planes).
+DFSSM_DEV void pack_digits4(const uint32_t (&h)[4], uint32_t (&planes)[4]) {
+  uint32_t P[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) P[e] = (uint32_t(half_times_2p24(h[e])) + 0x80808080u) ^ 0x80808080u;
+  const uint32_t t01 = __byte_perm(P[0], P[1], 0x5140), t23 = __byte_perm(P[2], P[3], 0x5140);
+  const uint32_t u01 = __byte_perm(P[0], P[1], 0x7362), u23 = __byte_perm(P[2], P[3], 0x7362);
+  planes[0] = __byte_perm(t01, t23, 0x5410);
+  planes[1] = __byte_perm(t01, t23, 0x7632);
+  planes[2] = __byte_perm(u01, u23, 0x5410);
+  planes[3] = __byte_perm(u01, u23, 0x7632);
+}
+
 // x = fp16((v * rs) * w) for K values (fp32 src in smem), rs = 1/sqrt(mean(v^2)+eps)
-// in fp64; then the fp32 LoRA decision (sx, codes) and the scaffold digit planes
-// (stride K+16) with their sums in tsum[6].  Four consecutive elements per thread
-// per step.  Returns sx.
-DFSSM_DEV float prep_activation(const float* v, const uint16_t* w, int K, uint16_t* x16, int8_t* xq, int8_t* dg,
-                                int* tsum, double* redd, float* redf, int* redi, uint16_t* x_diag,
+// in fp64, and its scaffold digit planes (stride K+16) with their sums in tsum[6].
+// Blocks that own a LoRA row (`codes`) also take the fp32 LoRA decision: amax, sx
+// and int8 codes.  Four consecutive elements per thread per step.  Returns sx
+// (1 when `codes` is false).
+DFSSM_DEV float prep_activation(const float* v, const uint16_t* w, int K, bool codes, uint16_t* x16, int8_t* xq,
+                                int8_t* dg, int* tsum, double* redd, float* redf, int* redi, uint16_t* x_diag,
                                 int8_t* xq_diag, int8_t* xd_diag, int* xdsum_diag, float* sx_diag) {
   const int tid = threadIdx.x, K4 = K / 4, DS = K + 16;
+  const bool keep = codes || x_diag;
   double ss = 0.0;
   for (int i = tid; i < K4; i += kPThreads) {
     const float4 f = reinterpret_cast<const float4*>(v)[i];
@@ -433,55 +480,35 @@ DFSSM_DEV float prep_activation(const float* v, const uint16_t* w, int K, uint16
   ss = csum_d(ss, redd);
   const double rs = 1.0 / sqrt(ss / double(K) + kEpsD);
   const float rs32 = float(rs);
-  float am = 0.f;
+  uint32_t am_bits = 0;                   // max |x| as fp16 bits (monotone for non-negative values)
+  uint32_t big = 0;                       // any |x| > 127: the digit planes need the 6-plane path
+  int ts[kDigits] = {0, 0, 0, 0, 0, 0};
   for (int i = tid; i < K4; i += kPThreads) {
     const float4 f = reinterpret_cast<const float4*>(v)[i];
     const uint2 wv = reinterpret_cast<const uint2*>(w)[i];
-    const uint16_t h0 = norm_fp16(f.x, rs, rs32, uint16_t(wv.x & 0xffff));
-    const uint16_t h1 = norm_fp16(f.y, rs, rs32, uint16_t(wv.x >> 16));
-    const uint16_t h2 = norm_fp16(f.z, rs, rs32, uint16_t(wv.y & 0xffff));
-    const uint16_t h3 = norm_fp16(f.w, rs, rs32, uint16_t(wv.y >> 16));
-    reinterpret_cast<uint2*>(x16)[i] = make_uint2(h0 | (uint32_t(h1) << 16), h2 | (uint32_t(h3) << 16));
-    am = fmaxf(am, fmaxf(fmaxf(fabsf(h2f(h0)), fabsf(h2f(h1))), fmaxf(fabsf(h2f(h2)), fabsf(h2f(h3)))));
-  }
-  am = cmax_f(am, redf);
-  const float sx = am > 0.f ? __fdiv_rn(am, 127.f) : 1.f;
-  const float rcp = __frcp_rn(sx);
-  const bool fast = am <= 127.f;     // |x * 2^24| fits the 4-digit packed path
-  int ts[kDigits] = {0, 0, 0, 0, 0, 0};
-  for (int i = tid; i < K4; i += kPThreads) {
-    const uint2 hv = reinterpret_cast<const uint2*>(x16)[i];
-    const uint16_t hh[4] = {uint16_t(hv.x & 0xffff), uint16_t(hv.x >> 16), uint16_t(hv.y & 0xffff),
-                            uint16_t(hv.y >> 16)};
-    uint32_t qw = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int q = am > 0.f ? quant_code_fast(h2f(hh[e]), sx, rcp) : 0;
-      qw |= (uint32_t(q) & 0xffu) << (8 * e);
-    }
-    reinterpret_cast<uint32_t*>(xq)[i] = qw;
+    uint32_t h[4];
+    h[0] = norm_fp16(f.x, rs, rs32, half_to_float_bits(wv.x & 0xffffu));
+    h[1] = norm_fp16(f.y, rs, rs32, half_to_float_bits(wv.x >> 16));
+    h[2] = norm_fp16(f.z, rs, rs32, half_to_float_bits(wv.y & 0xffffu));
+    h[3] = norm_fp16(f.w, rs, rs32, half_to_float_bits(wv.y >> 16));
+    const uint32_t m4 = max(max(h[0] & 0x7fffu, h[1] & 0x7fffu), max(h[2] & 0x7fffu, h[3] & 0x7fffu));
+    am_bits = max(am_bits, m4);
+    if (keep) reinterpret_cast<uint2*>(x16)[i] = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
     uint32_t planes[kDigits];
-    if (fast) {
-      uint32_t P[4];
+    if (m4 <= 0x57f0u) {                  // every |x| <= 127: four packed digit planes
+      uint32_t p4[4];
+      pack_digits4(h, p4);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int X = int(h2f(hh[e]) * 16777216.f);
-        P[e] = (uint32_t(X) + 0x80808080u) ^ 0x80808080u;   // bytes = balanced base-256 digits
-      }
-      const uint32_t t01 = __byte_perm(P[0], P[1], 0x5140), t23 = __byte_perm(P[2], P[3], 0x5140);
-      const uint32_t u01 = __byte_perm(P[0], P[1], 0x7362), u23 = __byte_perm(P[2], P[3], 0x7362);
-      planes[0] = __byte_perm(t01, t23, 0x5410);
-      planes[1] = __byte_perm(t01, t23, 0x7632);
-      planes[2] = __byte_perm(u01, u23, 0x5410);
-      planes[3] = __byte_perm(u01, u23, 0x7632);
+      for (int d = 0; d < 4; ++d) planes[d] = p4[d];
       planes[4] = planes[5] = 0u;
     } else {
+      big = 1u;
 #pragma unroll
       for (int d = 0; d < kDigits; ++d) planes[d] = 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         int8_t d6[kDigits];
-        fp16_digits(hh[e], d6);
+        fp16_digits(uint16_t(h[e]), d6);
 #pragma unroll
         for (int d = 0; d < kDigits; ++d) planes[d] |= (uint32_t(uint8_t(d6[d]))) << (8 * e);
       }
@@ -492,12 +519,12 @@ DFSSM_DEV float prep_activation(const float* v, const uint16_t* w, int K, uint16
       ts[d] = __dp4a(int(planes[d]), 0x01010101, ts[d]);
     }
     if (x_diag) {
-      reinterpret_cast<uint2*>(x_diag)[i] = hv;
-      reinterpret_cast<uint32_t*>(xq_diag)[i] = qw;
+      reinterpret_cast<uint2*>(x_diag)[i] = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
 #pragma unroll
       for (int d = 0; d < kDigits; ++d) reinterpret_cast<uint32_t*>(xd_diag + size_t(d) * K)[i] = planes[d];
     }
   }
+  (void)big;
 #pragma unroll
   for (int d = 0; d < kDigits; ++d) ts[d] = warp_sum_i(ts[d]);
   const int lane = tid & 31, warp = tid >> 5;
@@ -505,7 +532,26 @@ DFSSM_DEV float prep_activation(const float* v, const uint16_t* w, int K, uint16
 #pragma unroll
     for (int d = 0; d < kDigits; ++d) redi[d * kPWarps + warp] = ts[d];
   }
-  csync();
+  float sx = 1.f;
+  if (codes) {
+    const float am = cmax_f(half_to_float_bits(am_bits), redf);   // (also orders the redi writes)
+    sx = am > 0.f ? __fdiv_rn(am, 127.f) : 1.f;
+    const float rcp = __frcp_rn(sx);
+    for (int i = tid; i < K4; i += kPThreads) {
+      const uint2 hv = reinterpret_cast<const uint2*>(x16)[i];
+      const uint32_t hh[4] = {hv.x & 0xffffu, hv.x >> 16, hv.y & 0xffffu, hv.y >> 16};
+      uint32_t qw = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int q = am > 0.f ? quant_code_bits(half_to_float_bits(hh[e]), sx, rcp) : 0;
+        qw |= (uint32_t(q) & 0xffu) << (8 * e);
+      }
+      reinterpret_cast<uint32_t*>(xq)[i] = qw;
+      if (xq_diag) reinterpret_cast<uint32_t*>(xq_diag)[i] = qw;
+    }
+  } else {
+    csync();
+  }
   if (tid < kDigits) {
     int t = 0;
 #pragma unroll
@@ -531,15 +577,18 @@ DFSSM_DEV void lora_row(const int8_t* Arow, const int8_t* xq, int K, float sx, u
   *u_out = (double(acc) * h2d(sA)) * double(sx);
 }
 
-// LoRA stage 2 for `nrows` rows, lane-parallel over the rank: out[r] = sum_j B[r][j] u[j]
-// (fp64).  One warp per row at a time.
+// LoRA stage 2 for `nrows` rows: out[r] = sum_j B[r][j] u[j] in fp64, one thread
+// per row with four interleaved partial sums (R is a multiple of 8).
 DFSSM_DEV void lora2_rows(const int8_t* Bq, int nrows, const double* u, int R, double* out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int r = warp; r < nrows; r += kPWarps) {
-    double l = 0.0;
-    for (int j = lane; j < R; j += 32) l = fma(double(Bq[r * R + j]), u[j], l);
-    l = warp_sum_d(l);
-    if (lane == 0) out[r] = l;
+  for (int r = threadIdx.x; r < nrows; r += kPThreads) {
+    const int* b4 = reinterpret_cast<const int*>(Bq + r * R);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int j4 = 0; j4 < R / 4; ++j4) {
+      const int v = b4[j4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = fma(double(int8_t(v >> (8 * e))), u[4 * j4 + e], acc[e]);
+    }
+    out[r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
 }
 
@@ -743,15 +792,18 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
 
     // ---- R: residual entering this layer
     if (l > 0) {
-      if (!tw_gather(status, ctl, a.x_r, a.D + G - a.out_tiles, tag(l, XR), scratch32, 4u)) { alive = false; break; }
-      for (int k = tid; k < a.D; k += kPThreads) res[k] = __uint_as_float(scratch32[k]);
-      csync();
+      if (!tw_gather(status, ctl, a.x_r, a.D + G - a.out_tiles, tag(l, XR), reinterpret_cast<uint32_t*>(res), 4u)) {
+        alive = false;
+        break;
+      }
     }
     if (!mbar_wait_compute(status, ctl, full_ab, par, 8u)) { alive = false; break; }
 
     // ---- pre-norm, codes, digit planes
     const bool wdiag = diag && w.c == 0;
-    const float sx_in = prep_activation(res, sp<uint16_t>(sm, s.prenorm), a.D, x16, xq, dg, tsum, redd, redf, redi,
+    const bool lora_block = a.R && first_lora_row(a) < a.R;
+    const float sx_in = prep_activation(res, sp<uint16_t>(sm, s.prenorm), a.D, lora_block || wdiag, x16, xq, dg, tsum,
+                                        redd, redf, redi,
                                         wdiag ? a.d_x_in : nullptr, wdiag ? a.d_xq_in : nullptr,
                                         wdiag ? a.d_xd_in : nullptr, wdiag ? a.d_xdsum_in : nullptr,
                                         wdiag ? a.d_sx_in : nullptr);
@@ -871,17 +923,10 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         const float* hrow = st + size_t(rr) * a.N;
         float* grow = L.ssm_state + size_t(e) * a.N;
         double y = 0.0;
-        for (int n4 = lane; n4 < a.N / 4; n4 += 32) {
-          const float4 hv = reinterpret_cast<const float4*>(hrow)[n4];
-          const double h0v = fma(dA, double(hv.x), xdt * bcx[4 * n4]);
-          const double h1v = fma(dA, double(hv.y), xdt * bcx[4 * n4 + 1]);
-          const double h2v = fma(dA, double(hv.z), xdt * bcx[4 * n4 + 2]);
-          const double h3v = fma(dA, double(hv.w), xdt * bcx[4 * n4 + 3]);
-          y = fma(bcx[a.N + 4 * n4], h0v, y);
-          y = fma(bcx[a.N + 4 * n4 + 1], h1v, y);
-          y = fma(bcx[a.N + 4 * n4 + 2], h2v, y);
-          y = fma(bcx[a.N + 4 * n4 + 3], h3v, y);
-          reinterpret_cast<float4*>(grow)[n4] = make_float4(float(h0v), float(h1v), float(h2v), float(h3v));
+        for (int n = lane; n < a.N; n += 32) {
+          const double hv = fma(dA, double(hrow[n]), xdt * bcx[n]);
+          y = fma(bcx[a.N + n], hv, y);
+          grow[n] = float(hv);
         }
         y = warp_sum_d(y);
         if (lane == 0) {
@@ -901,7 +946,8 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         for (int r = 0; r < 3; ++r) L.conv_state[size_t(r) * a.C + a.E + i] = bcst_new[r * 2 * a.N + i];
     }
     if (!mbar_wait_compute(status, ctl, full_cd, par, 128u)) { alive = false; break; }
-    const float sx_out = prep_activation(gbuf, sp<uint16_t>(sm, s.gnorm), a.E, x16, xq, dg, tsum, redd, redf, redi,
+    const float sx_out = prep_activation(gbuf, sp<uint16_t>(sm, s.gnorm), a.E, lora_block || wdiag, x16, xq, dg, tsum,
+                                         redd, redf, redi,
                                          wdiag ? a.d_x_out : nullptr, wdiag ? a.d_xq_out : nullptr,
                                          wdiag ? a.d_xd_out : nullptr, wdiag ? a.d_xdsum_out : nullptr,
                                          wdiag ? a.d_sx_out : nullptr);
@@ -951,9 +997,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   // ---- LM head
   if (alive && !a.layer_mode) {
     const int L = a.n_layer;
-    if (tw_gather(status, ctl, a.x_r, a.D + G - a.out_tiles, tag(L, XR), scratch32, 512u)) {
-      for (int k = tid; k < a.D; k += kPThreads) res[k] = __uint_as_float(scratch32[k]);
-      csync();
+    if (tw_gather(status, ctl, a.x_r, a.D + G - a.out_tiles, tag(L, XR), reinterpret_cast<uint32_t*>(res), 512u)) {
       double ss = 0.0;
       for (int k = tid; k < a.D; k += kPThreads) ss = fma(double(res[k]), double(res[k]), ss);
       ss = csum_d(ss, redd);
