@@ -15,7 +15,9 @@ replica on its own GPU (replicas only: no collective on the data path).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -42,6 +44,27 @@ THROTTLE_BITS = {
 }
 
 
+def profiled_traffic():
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary.
+
+    Returns None when the kernel source has changed since those counters were taken.
+    """
+    path = os.path.join(ROOT, "profiles", "k_decode_persistent_model_48x2048_v50280_b1_launches.md")
+    src = os.path.join(ROOT, "bit_scaffold_quantized_b200", "csrc", "persistent.cuh")
+    try:
+        with open(path) as f:
+            text = f.read()
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    t = re.search(r"^traffic_bytes_per_launch: (\d+)$", text, re.M)
+    h = re.search(r"^kernel_source_sha256: ([0-9a-f]{64})$", text, re.M)
+    if not t or not h or h.group(1) != sha:
+        return None
+    return int(t.group(1))
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -59,6 +82,17 @@ class ClockSampler:
         self.rows = []
         self.proc = None
         self.thread = None
+        self.window = None
+
+    def wait_first(self, limit_s: float):
+        """Let nvidia-smi start up before the region it has to cover (bounded)."""
+        t_end = time.monotonic() + limit_s
+        while self.proc is not None and not self.rows and time.monotonic() < t_end:
+            time.sleep(0.02)
+
+    def mark(self, t0: float, t1: float):
+        """Restrict the summary to samples taken between two monotonic times."""
+        self.window = (t0, t1)
 
     def __enter__(self):
         cmd = ["nvidia-smi", "-i", str(self.gpu),
@@ -72,7 +106,7 @@ class ClockSampler:
 
         def reader():
             for line in self.proc.stdout:
-                self.rows.append(line.strip())
+                self.rows.append((time.monotonic(), line.strip()))
         self.thread = threading.Thread(target=reader, daemon=True)
         self.thread.start()
         return self
@@ -88,7 +122,11 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], [], set()
-        for r in self.rows:
+        rows = self.rows
+        if self.window is not None:
+            inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
+            rows = inside or rows[-1:]
+        for _, r in rows:
             parts = [p.strip() for p in r.split(",")]
             if len(parts) < 3:
                 continue
@@ -177,23 +215,26 @@ def run_ours(args, rank, world, local_rank):
         call(tok, tok, ws, None, stream)
     launches_per_step = F.launches_per_decode_step(d, len(m.layers), m.vocab)
 
-    for _ in range(args.warmup):
-        with torch.cuda.stream(stream):
-            graph.replay()
-    stream.synchronize()
-
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
+        clk.wait_first(3.0)
+        for _ in range(args.warmup):
+            with torch.cuda.stream(stream):
+                graph.replay()
+        stream.synchronize()
+
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        t_begin = time.monotonic()
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(args.steps):
                 graph.replay()
             e1.record(stream)
         stream.synchronize()
+        clk.mark(t_begin, time.monotonic())
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -251,7 +292,7 @@ def run_ours(args, rank, world, local_rank):
                    "cuda_graph": True,
                    "l2": f"no flush: each step streams {bytes_tok / 1e6:.1f} MB > 126 MB L2"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
                      "kernel": "whole decode step (graph replay)",
                      "algorithmic_bytes_per_step": bytes_tok, "peak_source": peak_kind},
         "roofline_tokens_per_s": round(peak * 1e9 / bytes_tok, 1),
@@ -304,8 +345,8 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64)
-    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
