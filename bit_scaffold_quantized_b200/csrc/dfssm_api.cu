@@ -1,11 +1,13 @@
 // C ABI of libdfssm.so: host-side argument validation, workspace layout and the
 // launch sequences of the DF-SSM decode step.  Declarations and semantics: dfssm.h.
 #include <algorithm>
+#include <array>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "dfssm.h"
 #include "kernels.cuh"
@@ -272,22 +274,58 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
 
 // ---- persistent whole-token kernel (batch 1) ------------------------------------
 
-int align16i(int v) { return (v + 15) & ~15; }
 
 struct PPlan {
   bool ok = false;
-  int grid = 0;
+  bool spec = false;   // the compile-time shape instantiation applies
+  int grid = 0, Q = 0;
   PSmem sm{};
   char why[160] = {0};
 };
 
-int device_sm_count(int* nsm, int* smem_optin) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(nsm, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+int device_sm_count(int* dev, int* nsm, int* smem_optin) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(nsm, cudaDevAttrMultiProcessorCount, *dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, *dev);
   return e == cudaSuccess ? 0 : -1;
 }
+
+// Clusters of Q persistent CTAs that can be resident at once (cached per device,
+// cluster size and shared-memory size; the query is not a stream operation).
+using PKernel = void (*)(PParams);
+PKernel persistent_kernel(bool spec) {
+  return spec ? k_decode_persistent<Shape2048> : k_decode_persistent<ShapeAny>;
+}
+
+int max_active_clusters(int dev, int Q, int smem, bool spec) {
+  static std::mutex mu;
+  static std::vector<std::array<int, 5>> cache;   // dev, Q, smem, spec, result
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& c : cache)
+    if (c[0] == dev && c[1] == Q && c[2] == smem && c[3] == int(spec)) return c[4];
+  int n = 0;
+  const PKernel kfn = persistent_kernel(spec);
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = unsigned(Q);
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(unsigned(Q));
+    cfg.blockDim = dim3(kPBlock);
+    cfg.dynamicSmemBytes = size_t(smem);
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kfn), &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cache.push_back({dev, Q, smem, int(spec), n});
+  return n;
+}
+
+bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+int ilog2(int v) { int l = 0; while ((1 << l) < v) ++l; return l; }
 
 // Whether (and how) one token of these dims runs as the persistent kernel.
 PPlan plan_persistent(const dfssm_dims* d) {
@@ -296,65 +334,36 @@ PPlan plan_persistent(const dfssm_dims* d) {
     snprintf(p.why, sizeof p.why, "%s", why);
     return p;
   };
-  int nsm = 0, optin = 0;
-  if (device_sm_count(&nsm, &optin)) return no("device query failed");
-  const int D = d->d_model, E = d->d_inner, H = d->nheads, N = d->d_state, R = d->rank;
+  int dev = 0, nsm = 0, optin = 0;
+  if (device_sm_count(&dev, &nsm, &optin)) return no("device query failed");
+  const int D = d->d_model, E = d->d_inner, H = d->nheads, N = d->d_state, R = d->rank, P = d->headdim;
   if (d->batch != 1) return no("batch != 1");
   if (N % 16 || H % 16) return no("d_state and nheads must be multiples of 16");
-  if (R % 8) return no("rank must be a multiple of 8");
-  const int units = E / 16;
-  const int grid = std::min(nsm, units);
-  if ((units + grid - 1) / grid > kPMaxUnits) return no("more than 2 SSM row units per block");
-  if (D / 16 > grid) return no("more out_proj tiles than blocks");
-  if (2 * N / 16 > grid || R > grid) return no("more B/C tiles or LoRA rows than blocks");
-  const int kg_in = D / kTileCols, kg_out = E / kTileCols, Kmax = std::max(D, E);
-  PSmem& m = p.sm;
-  int off = 0;
-  auto take = [&](int bytes) { int at = off; off = align16i(off + std::max(bytes, 16)); return at; };
-  m.in_tiles = take(kPMaxInTiles * kg_in * 512);
-  m.in_bq = take(kPMaxInTiles * 16 * R);
-  m.in_alpha = take(kPMaxInTiles * 32);
-  m.in_sb = take(kPMaxInTiles * 32);
-  m.convw_x = take(kPMaxUnits * 128);
-  m.convb_x = take(kPMaxUnits * 32);
-  m.cst_x = take(3 * kPMaxUnits * 64);
-  m.bc_bq = take(2 * N * R);
-  m.bc_sb = take(4 * N);
-  m.bc_convw = take(16 * N);
-  m.bc_convb = take(4 * N);
-  m.bc_cst = take(24 * N);
-  m.a_in = take(D);
-  m.prenorm = take(2 * D);
-  m.sa_in = take(2 * R);
-  m.hd_dtb = take(4 * H);
-  m.hd_alog = take(4 * H);
-  m.hd_d = take(4 * H);
-  m.state = take(kPMaxUnits * 16 * N * 4);
-  off = std::max(off, 2 * kHeadChunkRows * 2 * D);     // the LM-head ring reuses this group
-  m.ab_end = off;
-  m.out_tile = take(kg_out * 512);
-  m.out_bq = take(16 * R);
-  m.out_alpha = take(32);
-  m.out_sb = take(32);
-  m.a_out = take(E);
-  m.gnorm = take(2 * E);
-  m.sa_out = take(2 * R);
-  m.cd_end = off;
-  m.res = take(4 * (D + grid));      // residual words + the exchange's token words
-  m.gbuf = take(4 * Kmax);
-  m.x16 = take(2 * Kmax);
-  m.digits = take(kDigits * (Kmax + 16));
-  m.xq = take(Kmax);
-  m.part = take(16 * 16 * kDigits * 4);
-  m.yin = take(kPMaxInTiles * 16 * 8);
-  m.bcx = take(2 * N * 8);
-  m.bcst_new = take(3 * 2 * N * 4);
-  m.u_in = take(8 * std::max(R, 1));
-  m.u_out = take(8 * std::max(R, 1));
-  m.misc = take(4 * std::max({D + grid, 4 * N, 2 * R, 2 * grid, kHeadChunkRows}));
-  m.total = off;
-  if (m.total > optin) return no("shared memory plan exceeds the per-block limit");
+  if (R != 0 && (!pow2(R) || R < 8 || R > kPThreads)) return no("rank must be 0 or a power of two in [8, 512]");
+  const int Q = kPMaxCluster;
+  const int SD = D / Q, SE = E / Q;
+  if (D % Q || E % Q || !pow2(SD) || !pow2(SE) || SD < 32 || SE < 32 || SD > 2 * kPThreads || SE > 2 * kPThreads)
+    return no("d_model / 8 and d_inner / 8 must be powers of two in [32, 512]");
+  const int units = E / 16, out_tiles = D / 16, nbc = 2 * N / 16;
+  p.sm = plan_smem(D, E, H, N, R, Q);
+  const PSmem& m = p.sm;
+  p.spec = D == Shape2048::D && E == Shape2048::E && H == Shape2048::H && P == Shape2048::P && N == Shape2048::N &&
+           R == Shape2048::R && Q == Shape2048::Q;
+  if (p.spec && std::memcmp(&p.sm, &Shape2048::kPlan, sizeof(PSmem)) != 0) return no("compile-time plan mismatch");
+  if (m.total + int(sizeof(PParams)) + 1024 > optin) return no("shared memory plan exceeds the per-block limit");
+  if (m.head_slots < 2) return no("fewer than two LM-head chunk slots fit in shared memory");
+  const int maxc = max_active_clusters(dev, Q, m.total, p.spec);
+  const int grid = std::min(std::min(maxc, kPlanSMs / Q), std::min(units, out_tiles) / Q) * Q;
+  if (grid < Q) return no("no co-resident cluster of persistent CTAs");
+  for (int c = 0; c < grid; ++c) {
+    const PWork w = assign_cta(c, grid, Q, units, P, nbc, out_tiles);
+    if (w.nu < 1 || w.nu > kPMaxUnits) return no("SSM row units per CTA out of range");
+    if (w.no < 1 || w.no > kPMaxOutTiles) return no("out_proj tiles per CTA out of range");
+    if (w.NS > kPMaxSharedTiles || w.ns > kPMaxShared || w.ntile > kPMaxInTiles) return no("too many in_proj tiles");
+    if (w.h1 - w.h0 + 1 > kPMaxHeads) return no("too many heads per CTA");
+  }
   p.grid = grid;
+  p.Q = Q;
   p.ok = true;
   return p;
 }
@@ -384,8 +393,10 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.n_layer = n_layer; a.D = D; a.E = E; a.H = d->nheads; a.P = d->headdim; a.N = N; a.R = R;
   a.in_rows = in_rows(d); a.C = conv_dim(d); a.vocab = vocab;
   a.kg_in = D / kTileCols; a.kg_out = E / kTileCols;
-  a.units = E / 16; a.grid = plan.grid;
+  a.units = E / 16; a.grid = plan.grid; a.Q = plan.Q;
   a.n_bc_tiles = 2 * N / 16; a.dt_tile0 = (2 * E + 2 * N) / 16; a.out_tiles = D / 16;
+  a.SD = D / plan.Q; a.SE = E / plan.Q; a.lgSD = ilog2(a.SD); a.lgSE = ilog2(a.SE);
+  a.BSD = kDigits * (a.SD + 16) + 16; a.BSE = kDigits * (a.SE + 16) + 16;
   a.layer_mode = residual != nullptr;
   a.sm = plan.sm;
   a.embed = embed; a.normf_w = normf_w; a.tok_in = tok_in; a.tok_out = tok_out; a.logits = logits;
@@ -395,11 +406,10 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.status = at<unsigned>(ws, WL.status);
   a.ctl = reinterpret_cast<unsigned*>(pbase);
   unsigned long long* wd = reinterpret_cast<unsigned long long*>(pbase + 256);
-  a.x_r = wd;      wd += D + plan.grid;
+  a.x_r = wd;      wd += D;
+  a.x_rs = wd;     wd += 2 * plan.grid;
   a.x_g = wd;      wd += E;
-  a.x_bc = wd;     wd += 4 * N;
-  a.x_uin = wd;    wd += 2 * R;
-  a.x_uout = wd;   wd += 2 * R;
+  a.x_gs = wd;     wd += 2 * plan.grid;
   a.x_head = wd;   wd += 2 * plan.grid;
   Bufs b = bind(ws, WL);
   a.d_x_in = b.in.x; a.d_xq_in = b.in.xq; a.d_sx_in = b.in.sx; a.d_acc_in = b.in.acc; a.d_u_in = b.in.u;
@@ -407,12 +417,25 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.d_x_out = b.out.x; a.d_xq_out = b.out.xq; a.d_sx_out = b.out.sx; a.d_acc_out = b.out.acc;
   a.d_u_out = b.out.u; a.d_xd_out = b.out.xd; a.d_xdsum_out = b.out.xdsum; a.d_res = b.res;
   for (int l = 0; l < n_layer; ++l) a.L[l] = player(layers[l], states[l]);
-  cudaError_t e = cudaFuncSetAttribute(k_decode_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       plan.sm.total);
+  const PKernel kfn = persistent_kernel(plan.spec);
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.sm.total);
   if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "persistent smem attribute: %s", cudaGetErrorString(e));
-  void* args[] = {&a};
-  e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_decode_persistent), dim3(plan.grid), dim3(kPBlock),
-                                  args, size_t(plan.sm.total), st);
+  // clusters of Q CTAs, all co-resident (cooperative): the CTAs wait on one another
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = unsigned(plan.Q);
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeCooperative;
+  at[1].val.cooperative = 1;
+  cfg.gridDim = dim3(unsigned(plan.grid));
+  cfg.blockDim = dim3(kPBlock);
+  cfg.dynamicSmemBytes = size_t(plan.sm.total);
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, kfn, a);
   if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "persistent launch: %s", cudaGetErrorString(e));
   CHECK_LAUNCH("k_decode_persistent");
   return DFSSM_OK;

@@ -325,4 +325,6 @@ def test_model_decode_small_parity():
 
 def test_model_decode_1p3b_parity():
     m, tok = S.model_workload("model_48x2048_v50280_b1_greedy512")
+    # the benchmark shape must take the single-launch persistent kernel
+    assert F.launches_per_decode_step(m.dims, len(m.layers), m.vocab) == 1
     _teacher_forced(m, tok, 2)
