@@ -782,9 +782,8 @@ DFSSM_DEV void plane_sums(const unsigned char* asmb, int Q, int S, int BS, int* 
 }
 
 // int8 codes of the slice (from its fp16 bits), then LoRA stage-1 partials of the
-// slice for all R rows: stage[j] = sum_k A[j][k] q[k] over the slice, with
-// kPThreads / R threads per row (their sums through `scratch`, in a fixed order),
-// fenced for the async proxy.
+// slice for all R rows: stage[j] = sum_k A[j][k] q[k] over the slice, fenced for the
+// async proxy.
 DFSSM_DEV void codes_and_lora_partials(const uint16_t* xs, int S, float sx, float rcp, bool nonzero, int8_t* xqs,
                                        const int8_t* Aslice, int R, int* scratch, int* stage, int8_t* xq_diag) {
   const int tid = threadIdx.x;
@@ -795,21 +794,20 @@ DFSSM_DEV void codes_and_lora_partials(const uint16_t* xs, int S, float sx, floa
   }
   csync();
   if (R > 0) {
-    const int tpr = kPThreads / R;                 // threads per row
-    const int j = tid / tpr, g = tid % tpr;
-    int acc = 0;
-    if (j < R) {
+    // 16 lanes per row, two rows per warp; rows beyond the first pass of the warps
+    // come round again
+    const int half = (tid & 31) >> 4, sub = tid & 15;
+    for (int j = 2 * (tid >> 5) + half; j < R; j += 2 * kPWarps) {
       const int* A4 = reinterpret_cast<const int*>(Aslice + j * S);
       const int* q4 = reinterpret_cast<const int*>(xqs);
-      for (int i = g; i < S / 4; i += tpr) acc = __dp4a(A4[i], q4[i], acc);
-    }
-    scratch[tid] = acc;
-    csync();
-    if (tid < R) {
-      int t = 0;
-      for (int i = 0; i < tpr; ++i) t += scratch[tid * tpr + i];
-      stage[tid] = t;
-      fence_async_smem();
+      int acc = 0;
+      for (int i = sub; i < S / 4; i += 16) acc = __dp4a(A4[i], q4[i], acc);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (sub == 0) {
+        stage[j] = acc;
+        fence_async_smem();
+      }
     }
   }
 }
@@ -1222,30 +1220,30 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
           for (int i = 0; i < kPSsmRows; ++i) yv[i] += __shfl_xor_sync(0xffffffffu, yv[i], o);
-        if (lane == 0) {
+        // lane i finishes row warp + kPWarps i: D skip, gate, publish g
+        double g2 = 0.0;
 #pragma unroll
-          for (int i = 0; i < kPSsmRows; ++i) {
-            const int rr = warp + kPWarps * i;
-            double g2 = 0.0;
-            if (rr < nrow) {
-              const int e = 16 * w.u0 + rr;
-              const double x = yin[(xslot + rr / 16) * 16 + rr % 16];
-              const double gate = yin[(zslot + rr / 16) * 16 + rr % 16];
-              const double y = fma(double(sp<float>(sm, PSM(hd_d))[e / P]), x, yv[i]);
-              const float gv = float(y * gate);
-              tw_put(a.x_g + e, __float_as_uint(gv), tag(l, XG));
-              if (diag) a.d_g[e] = gv;
-              g2 = double(gv) * double(gv);
-            }
-            ssw[warp * kPSsmRows + i] = g2;
+        for (int i = 0; i < kPSsmRows; ++i) {
+          const int rr = warp + kPWarps * i;
+          if (lane == i && rr < nrow) {
+            const int e = 16 * w.u0 + rr;
+            const double x = yin[(xslot + rr / 16) * 16 + rr % 16];
+            const double gate = yin[(zslot + rr / 16) * 16 + rr % 16];
+            const double y = fma(double(sp<float>(sm, PSM(hd_d))[e / P]), x, yv[i]);
+            const float gv = float(y * gate);
+            tw_put(a.x_g + e, __float_as_uint(gv), tag(l, XG));
+            if (diag) a.d_g[e] = gv;
+            g2 = double(gv) * double(gv);
           }
         }
+        if (lane < kPSsmRows) ssw[warp * kPSsmRows + lane] = g2;
       }
       csync();
-      if (tid == 0) {
+      if (warp == 0) {          // sum of squares of the CTA's gated values (fixed order)
         double t = 0.0;
-        for (int rr = 0; rr < w.nu * 16; ++rr) t += ssw[(rr % kPWarps) * kPSsmRows + rr / kPWarps];   // row order
-        tw_put_f64(a.x_gs + 2 * w.c, t, tag(l, XG));
+        for (int i = lane; i < kPWarps * kPSsmRows; i += 32) t += ssw[i];
+        t = warp_sum_d(t);
+        if (lane == 0) tw_put_f64(a.x_gs + 2 * w.c, t, tag(l, XG));
       }
       if (tid == 0) mbar_arrive(empty_ab);      // AB group consumed: the copy warp may refill it
       // ---- G: own slice of the gated value and the sums of squares
@@ -1305,10 +1303,11 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         }
       }
       csync();
-      if (tid == 0) {
+      if (warp == 0) {          // sum of squares of the CTA's residual rows (fixed order)
         double t = 0.0;
-        for (int i = 0; i < w.no * 16; ++i) t = fma(double(resown[i]), double(resown[i]), t);
-        if (!(last && a.layer_mode)) tw_put_f64(a.x_rs + 2 * w.c, t, tag(l + 1, XR));
+        for (int i = lane; i < w.no * 16; i += 32) t = fma(double(resown[i]), double(resown[i]), t);
+        t = warp_sum_d(t);
+        if (lane == 0 && !(last && a.layer_mode)) tw_put_f64(a.x_rs + 2 * w.c, t, tag(l + 1, XR));
       }
       if (tid == 0) mbar_arrive(empty_cd);      // CD group consumed
     }
