@@ -31,6 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from bit_scaffold_quantized_b200 import synth as S  # noqa: E402
+from bit_scaffold_quantized_b200 import replicas as RP  # noqa: E402
 from bit_scaffold_quantized_b200 import roofline as R  # noqa: E402
 
 WORKLOAD = "model_48x2048_v50280_b1_greedy512"
@@ -222,8 +223,7 @@ def run_ours(args, rank, world, local_rank):
                 graph.replay()
         stream.synchronize()
 
-        if world > 1:
-            torch.distributed.barrier()
+        RP.barrier(world)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -236,8 +236,7 @@ def run_ours(args, rank, world, local_rank):
         stream.synchronize()
         clk.mark(t_begin, time.monotonic())
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    RP.barrier(world)
     ms = e0.elapsed_time(e1)
 
     # end-to-end: host token in (pinned) -> decode step -> host token out, every step
@@ -258,17 +257,14 @@ def run_ours(args, rank, world, local_rank):
     stream.synchronize()
     ms_e2e = f0.elapsed_time(f1)
 
-    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = RP.max_over_ranks([ms, ms_e2e], world, device=dev)
     del graph
 
     if rank != 0:
         return None
     peaks, peak_kind = load_peaks()
     tokens = args.steps * d.batch * world
-    tok_s = tokens / (ms / 1e3)
+    tok_s = RP.job_tokens_per_s(args.steps, d.batch, world, ms)
     bytes_tok = R.model_token_bytes(d, len(m.layers), m.vocab)
     step_s = ms / 1e3 / args.steps
     achieved = bytes_tok / step_s / 1e9        # GB/s; one step = one token for every batch row
@@ -296,7 +292,7 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": "whole decode step (graph replay)",
                      "algorithmic_bytes_per_step": bytes_tok, "peak_source": peak_kind},
         "roofline_tokens_per_s": round(peak * 1e9 / bytes_tok, 1),
-        "e2e": {"value": round(tokens / (ms_e2e / 1e3), 2), "unit": "tokens/s",
+        "e2e": {"value": round(RP.job_tokens_per_s(args.steps, d.batch, world, ms_e2e), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * d.batch, "d2h_bytes_per_step": 4 * d.batch},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
