@@ -197,7 +197,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     F.lib()
-    m, tok0 = S.model_workload(WORKLOAD)
+    m, tok0 = S.model_workload(args.workload)
     d = m.dims
     dm = F.DeviceModel.from_host(m, device=dev)
     states = [F.DeviceState.zeros(d, device=dev) for _ in m.layers]
@@ -282,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "1-bit scaffold x fp16 act (fp32 acc), int8 LoRA (int32 acc), fp32 SSM state",
         "data": "synthetic (seeded random-init weights, random 1-token prompt)",
-        "config": {"workload": WORKLOAD, "n_layer": len(m.layers), "d_model": d.d_model,
+        "config": {"workload": args.workload, "n_layer": len(m.layers), "d_model": d.d_model,
                    "d_inner": d.d_inner, "nheads": d.nheads, "headdim": d.headdim, "d_state": d.d_state,
                    "rank": d.rank, "vocab": m.vocab, "batch": d.batch, "parallelism": f"replicas x{world}",
                    "cuda_graph": True,
@@ -309,11 +309,67 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def run_sweep(args):
+    """The isolated scaffold + int8-LoRA projection sweep: one JSON line per point.
+
+    Each point cycles through enough copies of the packed sign words to exceed 4x L2,
+    as a CUDA graph of one call per copy, and times 1000+ calls with CUDA events."""
+    import torch
+    from bit_scaffold_quantized_b200 import dfssm as F
+    dev = torch.device("cuda", 0)
+    F.lib()
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    int8_tops = 2.0 * float(peaks["bf16_tflops"])      # int8 dense = 2x the measured bf16 rate (nominal ratio)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    for d_in, d_out in S.PROJ_SWEEP_SHAPES:
+        for r in S.PROJ_SWEEP_RANKS:
+            for b in S.PROJ_SWEEP_BATCHES:
+                pw, x_h = S.proj_workload(d_in, d_out, r, b)
+                p = F.DeviceProj.from_host(pw, device=dev)
+                wbytes = R.proj_weight_bytes(d_out, d_in, r)
+                ncopy = max(1, min(128, -(-4 * l2 // wbytes)))
+                copies = [p.bits.clone() for _ in range(ncopy)]
+                x = torch.from_numpy(x_h).to(dev)
+                y = torch.empty((b, d_out), dtype=torch.float32, device=dev)
+                ws = F.proj_workspace(d_out, d_in, r, b, device=dev)
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=stream):
+                    for c in copies:
+                        p.bits = c
+                        F.proj_forward(p, r, x, y, ws, stream)
+                reps = max(1, -(-1000 // ncopy))
+                for _ in range(2):
+                    graph.replay()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(reps):
+                        graph.replay()
+                    e1.record(stream)
+                stream.synchronize()
+                us = e0.elapsed_time(e1) * 1e3 / (reps * ncopy)
+                gbs = R.proj_bytes(d_out, d_in, r, b) / (us * 1e-6) / 1e9
+                tops = R.proj_flops(d_out, d_in, r, b) / (us * 1e-6) / 1e12
+                print(json.dumps({
+                    "metric": "fused scaffold + int8-LoRA projection", "value": round(us, 3), "unit": "us/call",
+                    "higher_is_better": False, "config": {"d_in": d_in, "d_out": d_out, "rank": r, "batch": b,
+                                                          "weight_copies": ncopy, "calls": reps * ncopy},
+                    "hbm": {"achieved_gbs": round(gbs, 1), "peak": hbm, "frac": round(gbs / hbm, 4)},
+                    "tensor": {"achieved_tops": round(tops, 2), "peak_int8_tops": int8_tops,
+                               "frac": round(tops / int8_tops, 5)},
+                    "peak_source": peak_kind}), flush=True)
+                del graph, copies
+
+
 def run_reference(args, rank, world):
     """Reference arm: the CPU oracle as it stands, on this machine's host cores."""
     if rank != 0:
         return None
-    m, tok0 = S.model_workload(WORKLOAD)
+    m, tok0 = S.model_workload(args.workload)
     nl, vr = 1, m.vocab // 48
     frac = slice_fraction(m, nl, vr)
     for _ in range(args.warmup):
@@ -330,7 +386,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded random-init weights, random 1-token prompt)",
-        "config": {"workload": WORKLOAD, "batch": d.batch, "n_layer": len(m.layers), "vocab": m.vocab},
+        "config": {"workload": args.workload, "batch": d.batch, "n_layer": len(m.layers), "vocab": m.vocab},
         "cpu_baseline": {"value": round(value, 5), "unit": "tokens/s", "cores": _blas_threads(),
                          "kind": "oracle",
                          "sample": f"each step = 1 of 48 layers + {vr} LM-head rows = {frac:.4f} token"},
@@ -345,10 +401,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[k for k in S.WORKLOADS if k.startswith("model_")],
+                    help="model decode workload (default: the batch-1 greedy decode)")
+    ap.add_argument("--sweep", action="store_true", help="time the isolated projection sweep instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.sweep:
+        run_sweep(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

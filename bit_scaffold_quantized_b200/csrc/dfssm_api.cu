@@ -221,11 +221,27 @@ int pick_bt(int batch, int K, int rank) {
   return bt;
 }
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
+        cudaSuccess && v > 0)
+      n = v;
+    else
+      n = 148;
+  }
+  return n;
+}
+
 template <int EPI, int BT>
 int launch_proj_bt(const ProjArgs& a, cudaStream_t st) {
   const size_t smem = proj_smem_bytes(a.K, a.rank, BT);
   cudaFuncSetAttribute(k_proj<EPI, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  dim3 grid((a.rows + kTileRows - 1) / kTileRows, (a.batch + BT - 1) / BT);
+  // about two blocks per SM; each block reuses its staged digit planes over several tiles
+  const int ntiles = (a.rows + kTileRows - 1) / kTileRows, gy = (a.batch + BT - 1) / BT;
+  const int gx = std::max(1, std::min(ntiles, (2 * sm_count() + gy - 1) / gy));
+  dim3 grid(gx, gy);
   k_proj<EPI, BT><<<grid, kProjThreads, smem, st>>>(a);
   CHECK_LAUNCH("k_proj");
   return DFSSM_OK;
@@ -264,7 +280,7 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   sa.H = d->nheads; sa.P = d->headdim; sa.N = d->d_state; sa.E = E; sa.conv_dim = C; sa.in_rows = in_rows(d);
   sa.zx = b.zxbcdt; sa.xc = b.xc; sa.dt_bias = w->dt_bias; sa.A_log = w->A_log; sa.D = w->D;
   sa.state = s->ssm_state; sa.g = b.g;
-  k_ssm<<<dim3(d->nheads * (d->headdim / kSsmRows), B), kSsmThreads, size_t(16) * d->d_state, st>>>(sa);
+  k_ssm<<<dim3(d->nheads, B), kSsmThreads, size_t(16) * d->d_state, st>>>(sa);
   CHECK_LAUNCH("k_ssm");
   if ((rc = launch_prologue<float, 0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, B, b.out);

@@ -128,8 +128,11 @@ __global__ void __launch_bounds__(kPrologueThreads) k_prologue(PrologueArgs a) {
     }
     ss = block_sum_d(ss, redd);
     const double rs = 1.0 / sqrt(ss / double(K) + kEpsD);
+    const float rs32 = float(rs);
     for (int k = tid; k < K; k += blockDim.x) {
-      const uint16_t h = d2h((double(v[k]) * rs) * h2d(a.w[k]));
+      uint16_t h;
+      if constexpr (sizeof(SrcT) == 4) h = norm_fp16(float(v[k]), rs, rs32, half_to_float_bits(a.w[k]));
+      else h = d2h((double(v[k]) * rs) * h2d(a.w[k]));
       xs[k] = h;
       if (writer && a.x) a.x[size_t(b) * K + k] = h;
     }
@@ -144,17 +147,20 @@ __global__ void __launch_bounds__(kPrologueThreads) k_prologue(PrologueArgs a) {
   int dsum[kDigits];
 #pragma unroll
   for (int d = 0; d < kDigits; ++d) dsum[d] = 0;
+  const float rcp = __frcp_rn(sx);
   for (int k = tid; k < K; k += blockDim.x) {
-    const int8_t q = am > 0.f ? int8_t(quant_code(h2f(xs[k]), sx)) : int8_t(0);
+    const int8_t q = am > 0.f ? int8_t(quant_code_bits(half_to_float_bits(xs[k]), sx, rcp)) : int8_t(0);
     qs[k] = q;
     if (writer) {
       a.xq[size_t(b) * K + k] = q;
-      int8_t dg[kDigits];
-      fp16_digits(xs[k], dg);
+      uint32_t lo, hi;
+      digits_of(xs[k], &lo, &hi);
+      const uint32_t w6[kDigits] = {lo, lo >> 8, lo >> 16, lo >> 24, hi, hi >> 8};
 #pragma unroll
       for (int d = 0; d < kDigits; ++d) {
-        a.xd[(size_t(b) * kDigits + d) * K + k] = dg[d];
-        dsum[d] += dg[d];
+        const int8_t dg = int8_t(w6[d] & 0xffu);
+        a.xd[(size_t(b) * kDigits + d) * K + k] = dg;
+        dsum[d] += dg;
       }
     }
   }
@@ -227,8 +233,9 @@ DFSSM_DEV double scaffold_value(const int (&q)[kDigits], const int* T) {
   return double(S) * (1.0 / 16777216.0);
 }
 
-// grid (ceil(rows/16), ceil(batch/BT)).  One 16-row tile per block; the 8 warps
-// split K in 256-column groups.  Each warp expands its lane's 16-byte vector of
+// grid (row-tile blocks, ceil(batch/BT)).  A block stages the digit planes of its
+// BT batch rows once and then loops over 16-row tiles rt = blockIdx.x, +gridDim.x,
+// ...; per tile the 8 warps split K in 256-column groups.  Each warp expands its lane's 16-byte vector of
 // sign words into 0/1 int8 A fragments (one shift + one mask per register) and
 // runs m16n8k32 int8 MMAs against the activation digit planes; int32 partials are
 // summed in a fixed order in shared memory, recombined exactly, and the epilogue
@@ -243,8 +250,9 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
   int* part = reinterpret_cast<int*>(us + BT * rk);                               // [warps][16][NC]
   int* T = part + kProjWarps * 16 * NC;                                           // [BT][kDigits]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rt = blockIdx.x, b0 = blockIdx.y * BT;
+  const int b0 = blockIdx.y * BT;
   const int kgroups = K / kTileCols;
+  const int ntiles = (a.rows + kTileRows - 1) / kTileRows;
 
   // stage digit planes: column c = bb * kDigits + d (zero past the batch and past 6*BT)
   for (int i = tid; i < NC * (K / 16); i += blockDim.x) {
@@ -263,10 +271,11 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
     T[i] = (b0 + i / kDigits < a.batch) ? a.xdsum[size_t(b0) * kDigits + i] : 0;
   __syncthreads();
 
+  const int g = lane >> 2, t = lane & 3;
+  for (int rt = blockIdx.x; rt < ntiles; rt += gridDim.x) {
   int acc[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
-  const int g = lane >> 2, t = lane & 3;
   const uint4* tiles = reinterpret_cast<const uint4*>(a.bits) + size_t(rt) * kgroups * 32;
   for (int kg = warp; kg < kgroups; kg += kProjWarps) {
     const uint4 wv = __ldg(tiles + kg * 32 + lane);
@@ -343,6 +352,8 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
       }
     }
   }
+  __syncthreads();   // the partials of this tile are consumed before the next tile's
+  }
 }
 
 // ------------------------------------------------------------------ SSM step
@@ -358,50 +369,65 @@ struct SsmArgs {
   float* g;              // fp32 [B][E]
 };
 
-constexpr int kSsmRows = 16;     // head rows per block
 constexpr int kSsmThreads = 256;
 
-// grid (H * P/16, B).  One warp per state row of N fp32 values (float4 per lane),
-// arithmetic in fp64, state stored back in fp32:
+// grid (H, B): one block per head and batch row.  One warp per state row of N fp32
+// values (float4 per lane, four rows of a warp in flight together), arithmetic in
+// fp64, state stored back in fp32:
 //   dt = softplus(dt_raw + dt_bias), dA = exp(-dt * exp(A_log)),
 //   h' = dA h + (x dt) B,  y = C . h' + D x,  g = y * silu(z) (stored fp32).
 __global__ void __launch_bounds__(kSsmThreads) k_ssm(SsmArgs a) {
   extern __shared__ __align__(16) double sbc[];   // [2N]: B then C
-  const int tiles_per_head = a.P / kSsmRows;
-  const int h = blockIdx.x / tiles_per_head, p0 = (blockIdx.x % tiles_per_head) * kSsmRows;
-  const int b = blockIdx.y;
+  const int h = blockIdx.x, b = blockIdx.y;
   const double* xcb = a.xc + size_t(b) * a.conv_dim;
   for (int i = threadIdx.x; i < 2 * a.N; i += blockDim.x) sbc[i] = xcb[a.E + i];
-  __syncthreads();
   const double* zr = a.zx + size_t(b) * a.in_rows;
   const double dt = softplus_d(zr[a.E + a.conv_dim + h] + double(a.dt_bias[h]));
   const double dA = exp(dt * -exp(double(a.A_log[h])));
   const double Dh = a.D[h];
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < kSsmRows; r += kSsmThreads / 32) {
-    const int p = p0 + r, e = h * a.P + p;
-    const double x = xcb[e];
-    const double xdt = x * dt;
-    float4* st = reinterpret_cast<float4*>(a.state + ((size_t(b) * a.H + h) * a.P + p) * a.N);
-    double y = 0.0;
+  constexpr int kW = kSsmThreads / 32;
+  // warp w takes rows w, w + kW, ...; four rows at a time so that their state loads
+  // are in flight together
+  for (int r0 = warp; r0 < a.P; r0 += 4 * kW) {
+    double xdt[4], y[4] = {0.0, 0.0, 0.0, 0.0};
+    float4* st[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int p = min(r0 + i * kW, a.P - 1), e = h * a.P + p;
+      xdt[i] = xcb[e] * dt;
+      st[i] = reinterpret_cast<float4*>(a.state + ((size_t(b) * a.H + h) * a.P + p) * a.N);
+    }
     for (int n4 = lane; n4 < a.N / 4; n4 += 32) {
-      float4 hv = st[n4];
+      float4 hv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) hv[i] = st[i][n4];
       const double* Bv = sbc + 4 * n4;
       const double* Cv = sbc + a.N + 4 * n4;
-      const double h0 = fma(dA, double(hv.x), xdt * Bv[0]);
-      const double h1 = fma(dA, double(hv.y), xdt * Bv[1]);
-      const double h2 = fma(dA, double(hv.z), xdt * Bv[2]);
-      const double h3 = fma(dA, double(hv.w), xdt * Bv[3]);
-      y = fma(Cv[0], h0, y);
-      y = fma(Cv[1], h1, y);
-      y = fma(Cv[2], h2, y);
-      y = fma(Cv[3], h3, y);
-      st[n4] = make_float4(float(h0), float(h1), float(h2), float(h3));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (r0 + i * kW >= a.P) continue;
+        const double h0 = fma(dA, double(hv[i].x), xdt[i] * Bv[0]);
+        const double h1 = fma(dA, double(hv[i].y), xdt[i] * Bv[1]);
+        const double h2 = fma(dA, double(hv[i].z), xdt[i] * Bv[2]);
+        const double h3 = fma(dA, double(hv[i].w), xdt[i] * Bv[3]);
+        y[i] = fma(Cv[0], h0, y[i]);
+        y[i] = fma(Cv[1], h1, y[i]);
+        y[i] = fma(Cv[2], h2, y[i]);
+        y[i] = fma(Cv[3], h3, y[i]);
+        st[i][n4] = make_float4(float(h0), float(h1), float(h2), float(h3));
+      }
     }
-    y = warp_sum_d(y);
-    if (lane == 0) {
-      y = fma(Dh, x, y);
-      a.g[size_t(b) * a.E + e] = float(y * silu_d(zr[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) y[i] += __shfl_xor_sync(0xffffffffu, y[i], o);
+    if (lane < 4 && r0 + lane * kW < a.P) {
+      const int e = h * a.P + r0 + lane * kW;
+      double yy = lane == 0 ? y[0] : lane == 1 ? y[1] : lane == 2 ? y[2] : y[3];
+      yy = fma(Dh, xcb[e], yy);
+      a.g[size_t(b) * a.E + e] = float(yy * silu_d(zr[e]));
     }
   }
 }

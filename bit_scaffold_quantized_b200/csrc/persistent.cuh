@@ -616,80 +616,6 @@ DFSSM_DEV void produce_cd(const PParams& a, const PWork& w, const PLayer& L, uns
 
 // ------------------------------------------------------------------ activation prep
 
-// Exact fp16 -> fp32 by bit construction for normal values (no convert
-// instruction); zero, subnormal and non-finite values take the hardware path.
-DFSSM_DEV float half_to_float_bits(uint32_t h) {
-  const uint32_t e = (h >> 10) & 0x1fu;
-  if (e == 0u || e == 31u) return h2f(uint16_t(h));
-  return __uint_as_float(((h & 0x8000u) << 16) | ((e + 112u) << 23) | ((h & 0x3ffu) << 13));
-}
-
-// x * 2^24 as an integer, exact for every finite fp16 (|X| < 2^40).
-DFSSM_DEV long long half_times_2p24_64(uint32_t h) {
-  const uint32_t e = (h >> 10) & 0x1fu, m = h & 0x3ffu;
-  const long long X = e == 0u ? (long long)m : ((long long)(m | 0x400u) << (e - 1u));
-  return (h & 0x8000u) ? -X : X;
-}
-
-// fp16 bits of z = (v * rs) * w, correctly rounded from the fp64 product.  The
-// fp32 product lies within 4 fp32 ulps of it; if its low 13 mantissa bits are more
-// than 4 away from the fp16 rounding midpoint (0x1000) and z is in the fp16 normal
-// range, rounding the fp32 value is already the answer (done here with integer
-// ops); otherwise fp64 decides.
-DFSSM_DEV uint16_t norm_fp16(float v, double rs, float rs32, float wf) {
-  const float z = (v * rs32) * wf;
-  const uint32_t bits = __float_as_uint(z);
-  const uint32_t ez = (bits >> 23) & 0xffu;
-  const int low13 = int(bits & 0x1fffu);
-  if (ez >= 113u && ez <= 141u && abs(low13 - 0x1000) > 4) {
-    uint32_t hm = ((ez - 112u) << 10) | ((bits >> 13) & 0x3ffu);
-    hm += low13 > 0x1000 ? 1u : 0u;
-    return uint16_t(hm | ((bits >> 16) & 0x8000u));
-  }
-  return d2h((double(v) * rs) * double(wf));
-}
-
-// Round-to-nearest-even of |t| < 2^22 via the 1.5 * 2^23 add (no convert instruction).
-DFSSM_DEV int rint_small(float t, float* r) {
-  const float m = t + 12582912.0f;
-  *r = m - 12582912.0f;
-  return __float_as_int(m) - 0x4B400000;
-}
-
-// Same decision as quant_code: clamp(rint(x / sx), -127, 127) with the fp32 IEEE
-// divide; the product x * rcp is within 3 * 2^-24 |x/sx| of the correctly rounded
-// quotient, so the divide is only needed near a half-integer.
-DFSSM_DEV int quant_code_bits(float x, float sx, float rcp) {
-  const float t = x * rcp;
-  float r;
-  int q = rint_small(t, &r);
-  if (fabsf(fabsf(t - r) - 0.5f) <= 4.0e-5f) q = __float2int_rn(__fdiv_rn(x, sx));
-  return max(-127, min(127, q));
-}
-
-// Balanced base-256 digits of X = x * 2^24 for one fp16 value, packed: planes 0-3
-// in `lo` (byte d = digit d), planes 4-5 in the low two bytes of `hi`.
-DFSSM_DEV void digits_of(uint32_t h, uint32_t* lo, uint32_t* hi) {
-  if ((h & 0x7fffu) <= 0x57f0u) {          // |x| <= 127: |X| < 2^31, four digits
-    const uint32_t e = (h >> 10) & 0x1fu, m = h & 0x3ffu;
-    int X = e == 0u ? int(m) : int((m | 0x400u) << (e - 1u));
-    X = (h & 0x8000u) ? -X : X;
-    *lo = (uint32_t(X) + 0x80808080u) ^ 0x80808080u;
-    *hi = 0u;
-    return;
-  }
-  long long X = half_times_2p24_64(h);
-  uint32_t b[kDigits];
-#pragma unroll
-  for (int d = 0; d < kDigits; ++d) {
-    const long long Dd = ((X + 128) & 255) - 128;
-    b[d] = uint32_t(Dd) & 0xffu;
-    X = (X - Dd) >> 8;
-  }
-  *lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-  *hi = b[4] | (b[5] << 8);
-}
-
 // Slice preparation (elements tid, tid + kPThreads, ...): x = fp16((v rs) w) into
 // xs, its six digit planes into the staging block (plane stride S + 16), and the
 // block tail: the exact sum of the slice's X = x 2^24 (int64) and max |x| (fp16 bits).
