@@ -365,6 +365,23 @@ def run_sweep(args):
                 del graph, copies
 
 
+def run_proj_point(args):
+    """One projection sweep point, called a few times (a short target for profilers)."""
+    import torch
+    from bit_scaffold_quantized_b200 import dfssm as F
+    d_in, d_out, r, b = args.proj
+    F.lib()
+    pw, x_h = S.proj_workload(d_in, d_out, r, b)
+    p = F.DeviceProj.from_host(pw)
+    x = torch.from_numpy(x_h).cuda()
+    y = torch.empty((b, d_out), dtype=torch.float32, device="cuda")
+    ws = F.proj_workspace(d_out, d_in, r, b)
+    for _ in range(3):
+        F.proj_forward(p, r, x, y, ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"proj": [d_in, d_out, r, b], "calls": 3, "ok": True}))
+
+
 def run_reference(args, rank, world):
     """Reference arm: the CPU oracle as it stands, on this machine's host cores."""
     if rank != 0:
@@ -405,12 +422,17 @@ def main():
                     choices=[k for k in S.WORKLOADS if k.startswith("model_")],
                     help="model decode workload (default: the batch-1 greedy decode)")
     ap.add_argument("--sweep", action="store_true", help="time the isolated projection sweep instead")
+    ap.add_argument("--proj", type=int, nargs=4, metavar=("D_IN", "D_OUT", "RANK", "BATCH"),
+                    help="call one projection sweep point three times (a target for profilers)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.proj:
+        run_proj_point(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
