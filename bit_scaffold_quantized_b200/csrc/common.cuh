@@ -113,6 +113,15 @@ DFSSM_DEV void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D (fp32 16x8) += A (fp16 16x16, row) * B (fp16 16x8, col).
+DFSSM_DEV void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Exact activation digits: an fp16 value times 2^24 is an integer X with
 // |X| < 2^40; it is written as kDigits balanced base-256 digits in [-128, 127],
 // X = sum_d D_d 256^d.  The scaffold sum over 0/1 sign bytes of each digit

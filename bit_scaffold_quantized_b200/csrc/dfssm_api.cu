@@ -158,12 +158,15 @@ void layer_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* 
   L->u_out = bp.take(8 * B * r);
   L->xd_out = bp.take(B * kDigits * E);
   L->xdsum_out = bp.take(4 * B * kDigits);
+  // internal scratch: persistent-kernel / LM-head words, then the multi-launch
+  // path's per-(batch, head) step size and decay (fp64 pairs)
+  const size_t dta = 16 * B * size_t(d->nheads);
   if (n_layer > 0) {
     L->res = bp.take(4 * B * D);
-    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), kHeadBlocks));
+    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), kHeadBlocks) + dta);
   } else {
     L->res = kNone;
-    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), 0));
+    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), 0) + dta);
   }
   L->total_bytes = align256(bp.off);
 }
@@ -180,9 +183,10 @@ struct Bufs {
   Act in, out;
   double* zxbcdt; double* xc; float* g;
   float* res; unsigned char* scratch;
+  double* dta;     // [batch][nheads][2] step size and decay (multi-launch path)
 };
 
-Bufs bind(void* ws, const dfssm_ws_layout& L) {
+Bufs bind(void* ws, const dfssm_ws_layout& L, const dfssm_dims* d) {
   Bufs b;
   b.status = at<unsigned>(ws, L.status);
   b.in = Act{at<uint16_t>(ws, L.x_in), at<int8_t>(ws, L.xq_in), at<float>(ws, L.sx_in), at<int>(ws, L.acc_in),
@@ -195,20 +199,23 @@ Bufs bind(void* ws, const dfssm_ws_layout& L) {
   b.g = at<float>(ws, L.g);
   b.res = L.res == kNone ? nullptr : at<float>(ws, L.res);
   b.scratch = at<unsigned char>(ws, L.scratch);
+  b.dta = at<double>(ws, L.total_bytes) - 2 * size_t(d->batch) * d->nheads;
   return b;
 }
 
 // ---- launch helpers ---------------------------------------------------------
 
-template <typename SrcT, int MODE>
-int launch_prologue(int K, int rank, int batch, const void* src, const uint16_t* src16, const uint16_t* w,
+static_assert(kPrologueThreads * kPrologueVals >= 8192, "the prologue holds K <= 8192 elements in registers");
+
+template <int MODE>
+int launch_prologue(int K, int rank, int batch, const float* src, const uint16_t* src16, const uint16_t* w,
                     const Act& o, const dfssm_proj* p, cudaStream_t st) {
   PrologueArgs a{};
   a.K = K; a.rank = rank; a.src = src; a.src16 = src16; a.w = w;
   a.x = o.x; a.xq = o.xq; a.sx = o.sx; a.xd = o.xd; a.xdsum = o.xdsum;
   a.A = p->A; a.sA = p->sA; a.acc = o.acc; a.u = o.u;
   dim3 grid(rank > 0 ? (rank + kPrologueRowsPerBlock - 1) / kPrologueRowsPerBlock : 1, batch);
-  k_prologue<SrcT, MODE><<<grid, kPrologueThreads, size_t(3) * K, st>>>(a);
+  k_prologue<MODE><<<grid, kPrologueThreads, size_t(K), st>>>(a);
   CHECK_LAUNCH("k_prologue");
   return DFSSM_OK;
 }
@@ -238,9 +245,19 @@ template <int EPI, int BT>
 int launch_proj_bt(const ProjArgs& a, cudaStream_t st) {
   const size_t smem = proj_smem_bytes(a.K, a.rank, BT);
   cudaFuncSetAttribute(k_proj<EPI, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  // about two blocks per SM; each block reuses its staged digit planes over several tiles
+  // one wave of resident blocks; each reuses its staged digit planes over several tiles
+  static int occ_smem = -1, occ_blocks = 1;
+  if (occ_smem != int(smem)) {
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_proj<EPI, BT>, kProjThreads, smem) != cudaSuccess ||
+        nb < 1)
+      nb = 1;
+    occ_smem = int(smem);
+    occ_blocks = nb;
+  }
   const int ntiles = (a.rows + kTileRows - 1) / kTileRows, gy = (a.batch + BT - 1) / BT;
-  const int gx = std::max(1, std::min(ntiles, (2 * sm_count() + gy - 1) / gy));
+  const int wave = std::max(1, occ_blocks * sm_count() / gy);
+  const int gx = std::max(1, std::min((ntiles + kProjWarps - 1) / kProjWarps, wave));
   dim3 grid(gx, gy);
   k_proj<EPI, BT><<<grid, kProjThreads, smem, st>>>(a);
   CHECK_LAUNCH("k_proj");
@@ -265,24 +282,68 @@ ProjArgs proj_args(const dfssm_proj* p, int rank, int batch, const Act& act) {
   return a;
 }
 
+// LM head of the multi-launch path: the tensor-core kernel (16 or 8 batch rows per
+// block) when its normalised rows fit in shared memory, else the fp32 kernel.
+// `*nparts` receives the partials per batch row that k_argmax reduces.
+constexpr size_t kHeadTcSmemCap = 200 * 1024;
+size_t head_tc_smem(int D, int nb) { return size_t(2) * 8 * nb * (D + 4) * 2; }
+
+template <int NB>
+int launch_head_tc(const HeadArgs& h, cudaStream_t st, int* nparts) {
+  const size_t smem = head_tc_smem(h.D, NB);
+  static int occ_smem = -1, occ_blocks = 1;
+  if (occ_smem != int(smem)) {
+    cudaFuncSetAttribute(k_lmhead_tc<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_lmhead_tc<NB>, kHeadWarps * 32, smem) != cudaSuccess ||
+        nb < 1)
+      nb = 1;
+    occ_smem = int(smem);
+    occ_blocks = nb;
+  }
+  const int gx = (h.batch + 8 * NB - 1) / (8 * NB);
+  const int tiles = (h.vocab + 15) / 16;
+  int gy = std::max(1, occ_blocks * sm_count() / gx);
+  gy = std::min(gy, std::min(kHeadBlocks, (tiles + kHeadWarps - 1) / kHeadWarps));
+  k_lmhead_tc<NB><<<dim3(gx, gy), kHeadWarps * 32, smem, st>>>(h);
+  CHECK_LAUNCH("k_lmhead_tc");
+  *nparts = gy;
+  return DFSSM_OK;
+}
+
+int launch_head(const HeadArgs& h, cudaStream_t st, int* nparts) {
+  if (h.D % 64 == 0) {
+    if (h.batch > 8 && head_tc_smem(h.D, 2) <= kHeadTcSmemCap) return launch_head_tc<2>(h, st, nparts);
+    if (head_tc_smem(h.D, 1) <= kHeadTcSmemCap) return launch_head_tc<1>(h, st, nparts);
+  }
+  const size_t smem = size_t(4) * kHeadBatch * h.D;
+  cudaFuncSetAttribute(k_lmhead, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  k_lmhead<<<dim3(kHeadBlocks, (h.batch + kHeadBatch - 1) / kHeadBatch), kHeadWarps * 32, smem, st>>>(h);
+  CHECK_LAUNCH("k_lmhead");
+  *nparts = kHeadBlocks;
+  return DFSSM_OK;
+}
+
 // The layer as five dependent launches on one stream.
 int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const dfssm_layer_state* s,
                       float* res, const Bufs& b, cudaStream_t st) {
   const int B = d->batch, D = d->d_model, E = d->d_inner, r = d->rank, C = conv_dim(d);
-  int rc = launch_prologue<float, 0>(D, r, B, res, nullptr, w->prenorm_w, b.in, &w->in, st);
+  int rc = launch_prologue<0>(D, r, B, res, nullptr, w->prenorm_w, b.in, &w->in, st);
   if (rc) return rc;
   ProjArgs pa = proj_args(&w->in, r, B, b.in);
   pa.zx = b.zxbcdt;
   pa.conv_lo = E; pa.conv_dim = C; pa.conv_w = w->conv_w; pa.conv_b = w->conv_b;
   pa.conv_state = s->conv_state; pa.xc = b.xc;
+  pa.dt_lo = E + C; pa.nheads = d->nheads; pa.dt_bias = w->dt_bias; pa.A_log = w->A_log; pa.dta = b.dta;
   if ((rc = launch_proj<EPI_INPROJ>(pa, st))) return rc;
   SsmArgs sa{};
   sa.H = d->nheads; sa.P = d->headdim; sa.N = d->d_state; sa.E = E; sa.conv_dim = C; sa.in_rows = in_rows(d);
   sa.zx = b.zxbcdt; sa.xc = b.xc; sa.dt_bias = w->dt_bias; sa.A_log = w->A_log; sa.D = w->D;
-  sa.state = s->ssm_state; sa.g = b.g;
-  k_ssm<<<dim3(d->nheads, B), kSsmThreads, size_t(16) * d->d_state, st>>>(sa);
+  sa.state = s->ssm_state; sa.g = b.g; sa.dta = b.dta;
+  if (d->d_state <= 128) k_ssm<1><<<dim3(d->nheads, B), kSsmThreads, 0, st>>>(sa);
+  else k_ssm<2><<<dim3(d->nheads, B), kSsmThreads, 0, st>>>(sa);
   CHECK_LAUNCH("k_ssm");
-  if ((rc = launch_prologue<float, 0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
+  if ((rc = launch_prologue<0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, B, b.out);
   po.out = res;
   return launch_proj<EPI_RESID>(po, st);
@@ -427,7 +488,7 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.x_g = wd;      wd += E;
   a.x_gs = wd;     wd += 2 * plan.grid;
   a.x_head = wd;   wd += 2 * plan.grid;
-  Bufs b = bind(ws, WL);
+  Bufs b = bind(ws, WL, d);
   a.d_x_in = b.in.x; a.d_xq_in = b.in.xq; a.d_sx_in = b.in.sx; a.d_acc_in = b.in.acc; a.d_u_in = b.in.u;
   a.d_xd_in = b.in.xd; a.d_xdsum_in = b.in.xdsum; a.d_zx = b.zxbcdt; a.d_xc = b.xc; a.d_g = b.g;
   a.d_x_out = b.out.x; a.d_xq_out = b.out.xq; a.d_sx_out = b.out.sx; a.d_acc_out = b.out.acc;
@@ -549,7 +610,7 @@ int dfssm_proj_forward(const dfssm_proj* p, int rank, int batch, const uint16_t*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Act act{nullptr, at<int8_t>(ws, L.xq_in), at<float>(ws, L.sx_in), at<int>(ws, L.acc_in),
           at<double>(ws, L.u_in), at<int8_t>(ws, L.xd_in), at<int>(ws, L.xdsum_in)};
-  if ((rc = launch_prologue<float, 1>(p->cols, rank, batch, nullptr, x, nullptr, act, p, st))) return rc;
+  if ((rc = launch_prologue<1>(p->cols, rank, batch, nullptr, x, nullptr, act, p, st))) return rc;
   ProjArgs a = proj_args(p, rank, batch, act);
   a.out = y;
   if ((rc = launch_proj<EPI_STORE>(a, st))) return rc;
@@ -583,7 +644,7 @@ int dfssm_layer_step(const dfssm_dims* d, const dfssm_layer_weights* w, const df
   layer_layout(d, 0, 0, &L);
   REQUIRE(ws_bytes >= L.total_bytes, DFSSM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes,
           L.total_bytes);
-  Bufs b = bind(ws, L);
+  Bufs b = bind(ws, L, d);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const PPlan plan = plan_persistent(d);
   if (plan.ok) {
@@ -618,7 +679,7 @@ int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16
   layer_layout(d, n_layer, vocab, &L);
   REQUIRE(ws_bytes >= L.total_bytes, DFSSM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes,
           L.total_bytes);
-  Bufs b = bind(ws, L);
+  Bufs b = bind(ws, L, d);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int B = d->batch, D = d->d_model;
   const PPlan plan = plan_persistent(d);
@@ -637,11 +698,9 @@ int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16
   HeadArgs h{};
   h.D = D; h.vocab = vocab; h.batch = B; h.res = b.res; h.normf_w = normf_w; h.embed = embed;
   h.logits = logits; h.part_val = part_val; h.part_idx = part_idx;
-  const size_t smem = size_t(4) * kHeadBatch * D;
-  cudaFuncSetAttribute(k_lmhead, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  k_lmhead<<<dim3(kHeadBlocks, (B + kHeadBatch - 1) / kHeadBatch), kHeadWarps * 32, smem, st>>>(h);
-  CHECK_LAUNCH("k_lmhead");
-  k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, kHeadBlocks, tok_out);
+  int nparts = kHeadBlocks;
+  if ((rc = launch_head(h, st, &nparts))) return rc;
+  k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, nparts, tok_out);
   CHECK_LAUNCH("k_argmax");
   return ok();
 }

@@ -83,7 +83,7 @@ __global__ void k_repack_tiled(const uint32_t* __restrict__ src, int rows, int c
 
 struct PrologueArgs {
   int K, rank;
-  const void* src;        // mode 0: [B][K] fp32 (residual) or fp64 (gated value) to normalise
+  const float* src;       // mode 0: [B][K] fp32 value to normalise (residual or gated value)
   const uint16_t* src16;  // mode 1: fp16 [B][K] activation as given
   const uint16_t* w;      // fp16 [K] norm weight (mode 0)
   uint16_t* x;            // fp16 [B][K] out (mode 0; may be null)
@@ -97,90 +97,135 @@ struct PrologueArgs {
   double* u;              // fp64 [B][rank] out
 };
 
-constexpr int kPrologueThreads = 256;
+constexpr int kPrologueThreads = 512;
 constexpr int kPrologueRowsPerBlock = kPrologueThreads / 32;  // one LoRA row per warp
+constexpr int kPrologueVals = 16;                             // elements per thread: K <= 8192
 
-// grid (max(1, ceil(rank/8)), B).  Every block recomputes the activation of its
+// grid (max(1, ceil(rank/16)), B).  Every block recomputes the activation of its
 // batch row (same arithmetic, same result); block 0 also writes the activation,
-// its int8 codes and its digit planes, and each warp computes one LoRA row.
+// its int8 codes and its digit planes, and each warp computes one LoRA row.  A
+// thread holds its elements k = tid + 512 i in registers, so the block waits for
+// global memory once: the LoRA row's A bytes, the source and the norm weight are
+// all requested before any arithmetic.
 //   mode 0: x = fp16(src * (1/sqrt(mean(src^2) + eps)) * w), all in fp64
 //   mode 1: x = src16
 //   sx = max|x| / 127, xq = clamp(rint(x / sx), -127, 127) (fp32 decision)
 //   acc[j] = sum_k A[j,k] xq[k] (exact), u[j] = acc[j] * sA[j] * sx (fp64)
-template <typename SrcT, int MODE>
+template <int MODE>
 __global__ void __launch_bounds__(kPrologueThreads) k_prologue(PrologueArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int K = a.K;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);            // [K]
-  int8_t* qs = reinterpret_cast<int8_t*>(smem + 2 * K);        // [K]
+  int8_t* qs = reinterpret_cast<int8_t*>(smem);                // [K] codes
   __shared__ double redd[32];
   __shared__ float red[32];
-  __shared__ int redi[32];
-  const int b = blockIdx.y, tid = threadIdx.x;
+  __shared__ int red6[kPrologueRowsPerBlock][kDigits];
+  const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool writer = blockIdx.x == 0;
 
+  // this warp's LoRA row, 16 bytes per lane and step (K <= 32 * 16 * kAV in registers)
+  constexpr int kAV = 8;
+  const int j = blockIdx.x * kPrologueRowsPerBlock + warp;
+  const int nv = K / 16;
+  const uint4* Arow = reinterpret_cast<const uint4*>(a.A + size_t(j < a.rank ? j : 0) * K);
+  uint4 av[kAV];
+#pragma unroll
+  for (int m = 0; m < kAV; ++m)
+    av[m] = (j < a.rank && lane + 32 * m < nv) ? __ldg(Arow + lane + 32 * m) : make_uint4(0, 0, 0, 0);
+
+  uint32_t h[kPrologueVals];     // fp16 bits of x
+  float am = 0.f;
   if (MODE == 0) {
-    const SrcT* v = reinterpret_cast<const SrcT*>(a.src) + size_t(b) * K;
-    double ss = 0.0;
-    for (int k = tid; k < K; k += blockDim.x) {
-      const double t = double(v[k]);
-      ss = fma(t, t, ss);
+    const float* v = a.src + size_t(b) * K;
+    float vf[kPrologueVals];
+    uint16_t wh[kPrologueVals];
+#pragma unroll
+    for (int i = 0; i < kPrologueVals; ++i) {
+      const int k = tid + i * kPrologueThreads;
+      vf[i] = k < K ? v[k] : 0.f;
+      wh[i] = k < K ? a.w[k] : uint16_t(0);
     }
+    double ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < kPrologueVals; ++i) ss = fma(double(vf[i]), double(vf[i]), ss);
     ss = block_sum_d(ss, redd);
     const double rs = 1.0 / sqrt(ss / double(K) + kEpsD);
     const float rs32 = float(rs);
-    for (int k = tid; k < K; k += blockDim.x) {
-      uint16_t h;
-      if constexpr (sizeof(SrcT) == 4) h = norm_fp16(float(v[k]), rs, rs32, half_to_float_bits(a.w[k]));
-      else h = d2h((double(v[k]) * rs) * h2d(a.w[k]));
-      xs[k] = h;
-      if (writer && a.x) a.x[size_t(b) * K + k] = h;
+#pragma unroll
+    for (int i = 0; i < kPrologueVals; ++i) {
+      const int k = tid + i * kPrologueThreads;
+      h[i] = k < K ? norm_fp16(vf[i], rs, rs32, half_to_float_bits(wh[i])) : 0u;
+      am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
+      if (k < K && writer && a.x) a.x[size_t(b) * K + k] = uint16_t(h[i]);
     }
   } else {
-    for (int k = tid; k < K; k += blockDim.x) xs[k] = a.src16[size_t(b) * K + k];
+#pragma unroll
+    for (int i = 0; i < kPrologueVals; ++i) {
+      const int k = tid + i * kPrologueThreads;
+      h[i] = k < K ? a.src16[size_t(b) * K + k] : 0u;
+      am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
+    }
   }
-  __syncthreads();
-  float am = 0.f;
-  for (int k = tid; k < K; k += blockDim.x) am = fmaxf(am, fabsf(h2f(xs[k])));
   am = block_max(am, red);
   const float sx = am > 0.f ? __fdiv_rn(am, 127.f) : 1.f;
+  const float rcp = __frcp_rn(sx);
   int dsum[kDigits];
 #pragma unroll
   for (int d = 0; d < kDigits; ++d) dsum[d] = 0;
-  const float rcp = __frcp_rn(sx);
-  for (int k = tid; k < K; k += blockDim.x) {
-    const int8_t q = am > 0.f ? int8_t(quant_code_bits(half_to_float_bits(xs[k]), sx, rcp)) : int8_t(0);
-    qs[k] = q;
-    if (writer) {
-      a.xq[size_t(b) * K + k] = q;
-      uint32_t lo, hi;
-      digits_of(xs[k], &lo, &hi);
-      const uint32_t w6[kDigits] = {lo, lo >> 8, lo >> 16, lo >> 24, hi, hi >> 8};
 #pragma unroll
-      for (int d = 0; d < kDigits; ++d) {
-        const int8_t dg = int8_t(w6[d] & 0xffu);
-        a.xd[(size_t(b) * kDigits + d) * K + k] = dg;
-        dsum[d] += dg;
+  for (int i = 0; i < kPrologueVals; ++i) {
+    const int k = tid + i * kPrologueThreads;
+    if (k < K) {
+      const int8_t q = am > 0.f ? int8_t(quant_code_bits(half_to_float_bits(h[i]), sx, rcp)) : int8_t(0);
+      qs[k] = q;
+      if (writer) {
+        a.xq[size_t(b) * K + k] = q;
+        uint32_t lo, hi;
+        digits_of(h[i], &lo, &hi);
+        const uint32_t w6[kDigits] = {lo, lo >> 8, lo >> 16, lo >> 24, hi, hi >> 8};
+#pragma unroll
+        for (int d = 0; d < kDigits; ++d) {
+          const int8_t dg = int8_t(w6[d] & 0xffu);
+          a.xd[(size_t(b) * kDigits + d) * K + k] = dg;
+          dsum[d] += dg;
+        }
       }
     }
   }
   if (writer) {
 #pragma unroll
     for (int d = 0; d < kDigits; ++d) {
-      const int t = block_sum_i(dsum[d], redi);
-      if (tid == 0) a.xdsum[b * kDigits + d] = t;
+      const int t = __reduce_add_sync(0xffffffffu, dsum[d]);
+      if (lane == 0) red6[warp][d] = t;
     }
+  }
+  __syncthreads();             // codes (and the warps' plane sums) complete
+  if (writer && tid < kDigits) {
+    int t = 0;
+    for (int w = 0; w < kPrologueRowsPerBlock; ++w) t += red6[w][tid];
+    a.xdsum[b * kDigits + tid] = t;
     if (tid == 0) a.sx[b] = sx;
   }
-  __syncthreads();
 
-  const int warp = tid >> 5, lane = tid & 31;
-  const int j = blockIdx.x * kPrologueRowsPerBlock + warp;
   if (j < a.rank) {
-    const int* Arow = reinterpret_cast<const int*>(a.A + size_t(j) * K);
-    const int* q4 = reinterpret_cast<const int*>(qs);
+    const uint4* q16 = reinterpret_cast<const uint4*>(qs);
     int acc = 0;
-    for (int i = lane; i < K / 4; i += 32) acc = __dp4a(Arow[i], q4[i], acc);
+#pragma unroll
+    for (int m = 0; m < kAV; ++m) {
+      if (lane + 32 * m < nv) {
+        const uint4 q = q16[lane + 32 * m];
+        acc = __dp4a(int(av[m].x), int(q.x), acc);
+        acc = __dp4a(int(av[m].y), int(q.y), acc);
+        acc = __dp4a(int(av[m].z), int(q.z), acc);
+        acc = __dp4a(int(av[m].w), int(q.w), acc);
+      }
+    }
+    for (int i = lane + 32 * kAV; i < nv; i += 32) {   // rows longer than the register window
+      const uint4 av2 = __ldg(Arow + i), q = q16[i];
+      acc = __dp4a(int(av2.x), int(q.x), acc);
+      acc = __dp4a(int(av2.y), int(q.y), acc);
+      acc = __dp4a(int(av2.z), int(q.z), acc);
+      acc = __dp4a(int(av2.w), int(q.w), acc);
+    }
     acc = warp_sum_i(acc);
     if (lane == 0) {
       a.acc[size_t(b) * a.rank + j] = acc;
@@ -210,6 +255,11 @@ struct ProjArgs {
   const uint16_t* conv_b;  // [conv_dim]
   float* conv_state;       // fp32 [batch][3][conv_dim]
   double* xc;              // fp64 [batch][conv_dim]
+  // EPI_INPROJ step sizes: rows [dt_lo, dt_lo + nheads) are dt_raw of each head
+  int dt_lo, nheads;
+  const float* dt_bias;    // [nheads]
+  const float* A_log;      // [nheads]
+  double* dta;             // fp64 [batch][nheads][2]: dt = softplus(dt_raw + dt_bias), dA = exp(-dt exp(A_log))
 };
 
 constexpr int kProjWarps = 8;
@@ -217,10 +267,11 @@ constexpr int kProjThreads = kProjWarps * 32;
 
 __host__ __device__ constexpr int proj_cols(int bt) { return ((kDigits * bt + 7) / 8) * 8; }
 __host__ __device__ __forceinline__ int proj_dstride(int K) { return K + 16; }  // bytes; spreads banks
+__host__ __device__ constexpr int proj_pstride(int bt) { return proj_cols(bt) + 1; }  // odd: spreads banks
 __host__ __device__ __forceinline__ size_t proj_smem_bytes(int K, int rank, int bt) {
   return size_t(proj_cols(bt)) * proj_dstride(K)                 // digit planes
          + size_t(8) * bt * (rank > 0 ? rank : 1)                 // u (fp64)
-         + size_t(4) * kProjWarps * 16 * proj_cols(bt)            // int32 partials
+         + size_t(4) * kProjWarps * 16 * proj_pstride(bt)         // per-warp int32 tile sums
          + size_t(4) * bt * kDigits;                              // digit sums
 }
 
@@ -233,22 +284,24 @@ DFSSM_DEV double scaffold_value(const int (&q)[kDigits], const int* T) {
   return double(S) * (1.0 / 16777216.0);
 }
 
-// grid (row-tile blocks, ceil(batch/BT)).  A block stages the digit planes of its
-// BT batch rows once and then loops over 16-row tiles rt = blockIdx.x, +gridDim.x,
-// ...; per tile the 8 warps split K in 256-column groups.  Each warp expands its lane's 16-byte vector of
-// sign words into 0/1 int8 A fragments (one shift + one mask per register) and
-// runs m16n8k32 int8 MMAs against the activation digit planes; int32 partials are
-// summed in a fixed order in shared memory, recombined exactly, and the epilogue
-// adds the LoRA stage 2 in fp64.
+// grid (gx, ceil(batch/BT)), gx sized to the resident blocks.  A block stages the
+// digit planes of its BT batch rows once; each warp then owns whole 16-row tiles
+// (rt = 8 blockIdx.x + warp, then + 8 gridDim.x, ...) over the full K, so the
+// integer sums never leave the warp and no block barrier follows the staging.  Per
+// 256-column group the warp expands its lane's 16-byte vector of sign words (loaded
+// two groups ahead) into 0/1 int8 A fragments (one shift + one mask per register)
+// and runs m16n8k32 int8 MMAs against the planes; the epilogue recombines the
+// planes exactly (lane = row, batch rows split over the two half-warps) and adds
+// the LoRA stage 2 in fp64.
 template <int EPI, int BT>
 __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  constexpr int NC = proj_cols(BT), NT = NC / 8;
+  constexpr int NC = proj_cols(BT), NT = NC / 8, PS = proj_pstride(BT);
   const int K = a.K, DS = proj_dstride(K), rk = a.rank > 0 ? a.rank : 1;
   int8_t* dg = reinterpret_cast<int8_t*>(smem);                                   // [NC][DS]
   double* us = reinterpret_cast<double*>(smem + size_t(NC) * DS);                 // [BT][rank]
-  int* part = reinterpret_cast<int*>(us + BT * rk);                               // [warps][16][NC]
-  int* T = part + kProjWarps * 16 * NC;                                           // [BT][kDigits]
+  int* part = reinterpret_cast<int*>(us + BT * rk);                               // [warps][16][PS]
+  int* T = part + kProjWarps * 16 * PS;                                           // [BT][kDigits]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b0 = blockIdx.y * BT;
   const int kgroups = K / kTileCols;
@@ -272,87 +325,99 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
   __syncthreads();
 
   const int g = lane >> 2, t = lane & 3;
-  for (int rt = blockIdx.x; rt < ntiles; rt += gridDim.x) {
-  int acc[NT][4];
+  int* wp = part + warp * 16 * PS;
+  const uint4 zero4 = make_uint4(0, 0, 0, 0);
+  for (int rt = blockIdx.x * kProjWarps + warp; rt < ntiles; rt += gridDim.x * kProjWarps) {
+    int acc[NT][4];
 #pragma unroll
-  for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
-  const uint4* tiles = reinterpret_cast<const uint4*>(a.bits) + size_t(rt) * kgroups * 32;
-  for (int kg = warp; kg < kgroups; kg += kProjWarps) {
-    const uint4 wv = __ldg(tiles + kg * 32 + lane);
-    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
+    const uint4* tiles = reinterpret_cast<const uint4*>(a.bits) + size_t(rt) * kgroups * 32 + lane;
+    uint4 w0 = __ldg(tiles), w1 = kgroups > 1 ? __ldg(tiles + 32) : zero4;
+    for (int kg = 0; kg < kgroups; ++kg) {
+      const uint4 wv = w0;
+      w0 = w1;
+      w1 = kg + 2 < kgroups ? __ldg(tiles + (kg + 2) * 32) : zero4;
+      const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-    for (int kt = 0; kt < 4; ++kt) {
+      for (int kt = 0; kt < 4; ++kt) {
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t af[4];
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t af[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) af[q] = sign_bytes(words[kt], 4 * ch + q);
-        const int k0 = kg * kTileCols + kt * 64 + ch * 32 + 4 * t;
+          for (int q = 0; q < 4; ++q) af[q] = sign_bytes(words[kt], 4 * ch + q);
+          const int k0 = kg * kTileCols + kt * 64 + ch * 32 + 4 * t;
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          const int8_t* dr = dg + size_t(n * 8 + g) * DS + k0;
-          const uint32_t bf0 = *reinterpret_cast<const uint32_t*>(dr);
-          const uint32_t bf1 = *reinterpret_cast<const uint32_t*>(dr + 16);
-          mma_s8_16832(acc[n], af, bf0, bf1);
+          for (int n = 0; n < NT; ++n) {
+            const int8_t* dr = dg + size_t(n * 8 + g) * DS + k0;
+            const uint32_t bf0 = *reinterpret_cast<const uint32_t*>(dr);
+            const uint32_t bf1 = *reinterpret_cast<const uint32_t*>(dr + 16);
+            mma_s8_16832(acc[n], af, bf0, bf1);
+          }
         }
       }
     }
-  }
 #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    int* p = part + size_t(warp) * 16 * NC;
-    p[g * NC + n * 8 + 2 * t] = acc[n][0];
-    p[g * NC + n * 8 + 2 * t + 1] = acc[n][1];
-    p[(g + 8) * NC + n * 8 + 2 * t] = acc[n][2];
-    p[(g + 8) * NC + n * 8 + 2 * t + 1] = acc[n][3];
-  }
-  __syncthreads();
+    for (int n = 0; n < NT; ++n) {
+      wp[g * PS + n * 8 + 2 * t] = acc[n][0];
+      wp[g * PS + n * 8 + 2 * t + 1] = acc[n][1];
+      wp[(g + 8) * PS + n * 8 + 2 * t] = acc[n][2];
+      wp[(g + 8) * PS + n * 8 + 2 * t + 1] = acc[n][3];
+    }
+    __syncwarp();
 
-  for (int i = tid; i < 16 * BT; i += blockDim.x) {
-    const int r = i / BT, bb = i % BT;
-    const int o = rt * kTileRows + r, b = b0 + bb;
-    if (o >= a.rows || b >= a.batch) continue;
-    int q[kDigits];
+    const int r = lane & 15, o = rt * kTileRows + r;
+    if (o < a.rows) {
+      const int* Br4 = reinterpret_cast<const int*>(a.B + size_t(o) * a.rank);
+      const double al = h2d(a.alpha[o]);
+      const double sb = a.rank > 0 ? h2d(a.sB[o]) : 0.0;
+      for (int bb = lane >> 4; bb < BT; bb += 2) {
+        const int b = b0 + bb;
+        if (b >= a.batch) break;
+        int q[kDigits];
 #pragma unroll
-    for (int d = 0; d < kDigits; ++d) {
-      int s = 0;
+        for (int d = 0; d < kDigits; ++d) q[d] = wp[r * PS + bb * kDigits + d];
+        double y = al * scaffold_value(q, T + bb * kDigits);
+        if (a.rank > 0) {
+          const double* ur = us + bb * a.rank;
+          double l = 0.0;
+          for (int j4 = 0; j4 < a.rank / 4; ++j4) {
+            const int v = __ldg(Br4 + j4);
 #pragma unroll
-      for (int w = 0; w < kProjWarps; ++w) s += part[(w * 16 + r) * NC + bb * kDigits + d];
-      q[d] = s;
-    }
-    double y = h2d(a.alpha[o]) * scaffold_value(q, T + bb * kDigits);
-    if (a.rank > 0) {
-      const int8_t* Br = a.B + size_t(o) * a.rank;
-      const double* ur = us + bb * a.rank;
-      double l = 0.0;
-      for (int j = 0; j < a.rank; ++j) l = fma(double(Br[j]), ur[j], l);
-      y = fma(h2d(a.sB[o]), l, y);
-    }
-    const size_t oi = size_t(b) * a.rows + o;
-    if (EPI == EPI_RESID) {
-      a.out[oi] = float(double(a.out[oi]) + y);
-    } else if (EPI == EPI_STORE) {
-      a.out[oi] = float(y);
-    } else {
-      a.zx[oi] = y;
-      const int c = o - a.conv_lo;
-      if (c >= 0 && c < a.conv_dim) {
-        float* cs = a.conv_state + size_t(b) * 3 * a.conv_dim;
-        const uint2 wv = *reinterpret_cast<const uint2*>(a.conv_w + size_t(c) * 4);
-        const double s0 = cs[c], s1 = cs[a.conv_dim + c], s2 = cs[2 * a.conv_dim + c];
-        double pre = h2d(a.conv_b[c]);
-        pre = fma(h2d(uint16_t(wv.x & 0xffff)), s0, pre);
-        pre = fma(h2d(uint16_t(wv.x >> 16)), s1, pre);
-        pre = fma(h2d(uint16_t(wv.y & 0xffff)), s2, pre);
-        pre = fma(h2d(uint16_t(wv.y >> 16)), y, pre);
-        a.xc[size_t(b) * a.conv_dim + c] = silu_d(pre);
-        cs[c] = float(s1);
-        cs[a.conv_dim + c] = float(s2);
-        cs[2 * a.conv_dim + c] = float(y);
+            for (int e = 0; e < 4; ++e) l = fma(double(int8_t(v >> (8 * e))), ur[4 * j4 + e], l);
+          }
+          y = fma(sb, l, y);
+        }
+        const size_t oi = size_t(b) * a.rows + o;
+        if (EPI == EPI_RESID) {
+          a.out[oi] = float(double(a.out[oi]) + y);
+        } else if (EPI == EPI_STORE) {
+          a.out[oi] = float(y);
+        } else {
+          a.zx[oi] = y;
+          const int c = o - a.conv_lo;
+          if (c >= 0 && c < a.conv_dim) {
+            float* cs = a.conv_state + size_t(b) * 3 * a.conv_dim;
+            const uint2 wv = *reinterpret_cast<const uint2*>(a.conv_w + size_t(c) * 4);
+            const double s0 = cs[c], s1 = cs[a.conv_dim + c], s2 = cs[2 * a.conv_dim + c];
+            double pre = h2d(a.conv_b[c]);
+            pre = fma(h2d(uint16_t(wv.x & 0xffff)), s0, pre);
+            pre = fma(h2d(uint16_t(wv.x >> 16)), s1, pre);
+            pre = fma(h2d(uint16_t(wv.y & 0xffff)), s2, pre);
+            pre = fma(h2d(uint16_t(wv.y >> 16)), y, pre);
+            a.xc[size_t(b) * a.conv_dim + c] = silu_d(pre);
+            cs[c] = float(s1);
+            cs[a.conv_dim + c] = float(s2);
+            cs[2 * a.conv_dim + c] = float(y);
+          } else if (o >= a.dt_lo && o < a.dt_lo + a.nheads) {
+            const int hh = o - a.dt_lo;
+            const double dt = softplus_d(y + double(a.dt_bias[hh]));
+            a.dta[(size_t(b) * a.nheads + hh) * 2] = dt;
+            a.dta[(size_t(b) * a.nheads + hh) * 2 + 1] = exp(dt * -exp(double(a.A_log[hh])));
+          }
+        }
       }
     }
-  }
-  __syncthreads();   // the partials of this tile are consumed before the next tile's
+    __syncwarp();   // the warp's tile sums are consumed before its next tile's
   }
 }
 
@@ -367,66 +432,106 @@ struct SsmArgs {
   const float* D;
   float* state;          // fp32 [B][H][P][N]
   float* g;              // fp32 [B][E]
+  const double* dta;     // fp64 [B][H][2]: step size and decay (from the in_proj epilogue)
 };
 
 constexpr int kSsmThreads = 256;
 
-// grid (H, B): one block per head and batch row.  One warp per state row of N fp32
-// values (float4 per lane, four rows of a warp in flight together), arithmetic in
-// fp64, state stored back in fp32:
-//   dt = softplus(dt_raw + dt_bias), dA = exp(-dt * exp(A_log)),
-//   h' = dA h + (x dt) B,  y = C . h' + D x,  g = y * silu(z) (stored fp32).
-__global__ void __launch_bounds__(kSsmThreads) k_ssm(SsmArgs a) {
-  extern __shared__ __align__(16) double sbc[];   // [2N]: B then C
-  const int h = blockIdx.x, b = blockIdx.y;
-  const double* xcb = a.xc + size_t(b) * a.conv_dim;
-  for (int i = threadIdx.x; i < 2 * a.N; i += blockDim.x) sbc[i] = xcb[a.E + i];
-  const double* zr = a.zx + size_t(b) * a.in_rows;
-  const double dt = softplus_d(zr[a.E + a.conv_dim + h] + double(a.dt_bias[h]));
-  const double dA = exp(dt * -exp(double(a.A_log[h])));
-  const double Dh = a.D[h];
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kW = kSsmThreads / 32;
-  // warp w takes rows w, w + kW, ...; four rows at a time so that their state loads
-  // are in flight together
-  for (int r0 = warp; r0 < a.P; r0 += 4 * kW) {
-    double xdt[4], y[4] = {0.0, 0.0, 0.0, 0.0};
-    float4* st[4];
+// Sum over the warp of R per-lane values, folded so that each shuffle level halves
+// the values a lane carries: afterwards every lane holds the full sum of value
+// `*sel` (lanes that differ only in their low bits hold the same one).
+template <int R>
+DFSSM_DEV double fold_rows(double (&y)[R], int lane, int* sel) {
+  int s = 0, off = 16;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int p = min(r0 + i * kW, a.P - 1), e = h * a.P + p;
-      xdt[i] = xcb[e] * dt;
-      st[i] = reinterpret_cast<float4*>(a.state + ((size_t(b) * a.H + h) * a.P + p) * a.N);
+  for (int n = R; n > 1; n >>= 1, off >>= 1) {
+    const bool hi = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const double keep = hi ? y[j + n / 2] : y[j];
+      const double send = hi ? y[j] : y[j + n / 2];
+      y[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
     }
-    for (int n4 = lane; n4 < a.N / 4; n4 += 32) {
-      float4 hv[4];
+    s = 2 * s + (hi ? 1 : 0);
+  }
+  double v = y[0];
+  for (; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  *sel = s;
+  return v;
+}
+
+// grid (H, B): one block per head and batch row; warp w owns state rows w, w + 8, ...
+// A lane holds NCH float4 of a row (columns 4 (lane + 32 c)), and a warp keeps
+// 8 / NCH rows in flight: their state loads are issued before anything else (they
+// depend on nothing), then B, C, x and the step size and decay arrive (computed once
+// per head by the in_proj epilogue: dt = softplus(dt_raw + dt_bias),
+// dA = exp(-dt * exp(A_log))).  Arithmetic in fp64, state stored back in fp32 with
+// streaming hints (read and written once per step):
+//   h' = dA h + (x dt) B,  y = C . h' + D x,  g = y * silu(z) (stored fp32).
+template <int NCH>
+__global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
+  constexpr int RW = 8 / NCH;                  // rows of a warp in flight
+  constexpr int kW = kSsmThreads / 32;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N4 = a.N / 4, P = a.P;
+  float* sbase = a.state + (size_t(b) * a.H + h) * size_t(P) * a.N;
+  const double* xcb = a.xc + size_t(b) * a.conv_dim;
+  const double* zr = a.zx + size_t(b) * a.in_rows;
+  for (int r0 = warp; r0 < P; r0 += RW * kW) {
+    float4 hv[RW][NCH];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) hv[i] = st[i][n4];
-      const double* Bv = sbc + 4 * n4;
-      const double* Cv = sbc + a.N + 4 * n4;
+    for (int i = 0; i < RW; ++i)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (r0 + i * kW >= a.P) continue;
-        const double h0 = fma(dA, double(hv[i].x), xdt[i] * Bv[0]);
-        const double h1 = fma(dA, double(hv[i].y), xdt[i] * Bv[1]);
-        const double h2 = fma(dA, double(hv[i].z), xdt[i] * Bv[2]);
-        const double h3 = fma(dA, double(hv[i].w), xdt[i] * Bv[3]);
-        y[i] = fma(Cv[0], h0, y[i]);
-        y[i] = fma(Cv[1], h1, y[i]);
-        y[i] = fma(Cv[2], h2, y[i]);
-        y[i] = fma(Cv[3], h3, y[i]);
-        st[i][n4] = make_float4(float(h0), float(h1), float(h2), float(h3));
+      for (int c = 0; c < NCH; ++c) {
+        const int p = r0 + i * kW, n4 = lane + 32 * c;
+        hv[i][c] = (p < P && n4 < N4) ? __ldcs(reinterpret_cast<const float4*>(sbase + size_t(p) * a.N) + n4)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    double Bv[NCH][4], Cv[NCH][4];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int n4 = lane + 32 * c;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        Bv[c][e] = n4 < N4 ? xcb[a.E + 4 * n4 + e] : 0.0;
+        Cv[c][e] = n4 < N4 ? xcb[a.E + a.N + 4 * n4 + e] : 0.0;
       }
     }
+    double xv[RW];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
+    for (int i = 0; i < RW; ++i) xv[i] = r0 + i * kW < P ? xcb[h * P + r0 + i * kW] : 0.0;
+    const double dt = a.dta[(size_t(b) * a.H + h) * 2], dA = a.dta[(size_t(b) * a.H + h) * 2 + 1];
+    double y[RW];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) y[i] += __shfl_xor_sync(0xffffffffu, y[i], o);
-    if (lane < 4 && r0 + lane * kW < a.P) {
-      const int e = h * a.P + r0 + lane * kW;
-      double yy = lane == 0 ? y[0] : lane == 1 ? y[1] : lane == 2 ? y[2] : y[3];
-      yy = fma(Dh, xcb[e], yy);
+    for (int i = 0; i < RW; ++i) {
+      const double xdt = xv[i] * dt;
+      const int p = r0 + i * kW;
+      double acc = 0.0;
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        const int n4 = lane + 32 * c;
+        const double h0 = fma(dA, double(hv[i][c].x), xdt * Bv[c][0]);
+        const double h1 = fma(dA, double(hv[i][c].y), xdt * Bv[c][1]);
+        const double h2 = fma(dA, double(hv[i][c].z), xdt * Bv[c][2]);
+        const double h3 = fma(dA, double(hv[i][c].w), xdt * Bv[c][3]);
+        acc = fma(Cv[c][0], h0, acc);
+        acc = fma(Cv[c][1], h1, acc);
+        acc = fma(Cv[c][2], h2, acc);
+        acc = fma(Cv[c][3], h3, acc);
+        if (p < P && n4 < N4)
+          __stcs(reinterpret_cast<float4*>(sbase + size_t(p) * a.N) + n4,
+                 make_float4(float(h0), float(h1), float(h2), float(h3)));
+      }
+      y[i] = acc;
+    }
+    int sel;
+    const double ys = fold_rows<RW>(y, lane, &sel);
+    // lanes 0, 32/RW, ... hold distinct rows
+    const int p = r0 + sel * kW;
+    if ((lane & (32 / RW - 1)) == 0 && p < P) {
+      const int e = h * P + p;
+      const double yy = fma(double(a.D[h]), xcb[e], ys);
       a.g[size_t(b) * a.E + e] = float(yy * silu_d(zr[e]));
     }
   }
@@ -543,6 +648,136 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead(HeadArgs a) {
     a.part_idx[size_t(b0 + bb) * gridDim.x + blockIdx.x] = bi;
   }
 }
+// Tensor-core LM head for batches: grid (ceil(B / (8 NB)), gy).  Blocks with the same
+// blockIdx.y read the same vocabulary rows and are launched next to each other, so
+// the rows come from HBM about once.  A block normalises its 8 NB batch rows (fp64,
+// kept as fp32, as k_lmhead) and splits each value into fp16 hi + lo parts
+// (x = hi + lo to 2^-22 relative), so that the fp16 tensor-core products of the fp16
+// head rows with both parts are exact and only the fp32 accumulation rounds.  Each
+// warp owns 16-row vocabulary tiles (tile = 8 blockIdx.y + warp, + 8 gy, ...); per
+// 64-column chunk, lane (g, t) loads 16 bytes x 2 of rows g and g + 8 at columns
+// 16 t.. (coalesced, one chunk ahead) and runs four m16n8k16 MMAs per batch n-tile
+// and part.  The MMA's k index i maps to column 64 c + 16 t + 4 s + (i & 1) + 2 (i >> 3)
+// for A and B alike, so the chunk's 64 columns are each summed once.  Per batch row
+// the block keeps the best (logit, id), lowest id on ties.
+template <int NB>
+__global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
+  extern __shared__ __align__(16) uint32_t xsw[];         // [2][8 NB][XS] words: hi rows, then lo rows
+  __shared__ float wbest[kHeadWarps][8 * NB];
+  __shared__ int wbesti[kHeadWarps][8 * NB];
+  const int D = a.D, XS = D / 2 + 2;                       // row stride in words (== 2 mod 32)
+  const int b0 = blockIdx.x * 8 * NB;
+  const int nb = min(8 * NB, a.batch - b0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  uint16_t* xh = reinterpret_cast<uint16_t*>(xsw);
+  uint16_t* xl = reinterpret_cast<uint16_t*>(xsw + 8 * NB * XS);
+  for (int rr = warp; rr < 8 * NB; rr += kHeadWarps) {
+    if (rr < nb) {
+      const float* v = a.res + size_t(b0 + rr) * D;
+      double ss = 0.0;
+      for (int k = lane; k < D; k += 32) ss = fma(double(v[k]), double(v[k]), ss);
+      ss = warp_sum_d(ss);
+      const double rs = 1.0 / sqrt(ss / double(D) + kEpsD);
+      for (int k = lane; k < D; k += 32) {
+        const float xv = float((double(v[k]) * rs) * h2d(a.normf_w[k]));
+        const __half hi = __float2half_rn(xv);
+        xh[rr * 2 * XS + k] = __half_as_ushort(hi);
+        xl[rr * 2 * XS + k] = f2h(xv - __half2float(hi));
+      }
+    } else {
+      for (int k = lane; k < D; k += 32) xh[rr * 2 * XS + k] = xl[rr * 2 * XS + k] = 0;
+    }
+  }
+  __syncthreads();
+
+  float best[NB][2];
+  int besti[NB][2];
+#pragma unroll
+  for (int n = 0; n < NB; ++n) best[n][0] = best[n][1] = -INFINITY, besti[n][0] = besti[n][1] = 0x7fffffff;
+  const int ntiles = (a.vocab + 15) / 16, nch = D / 64;
+  const uint2* xh2 = reinterpret_cast<const uint2*>(xsw) + g * (XS / 2) + 4 * t;
+  const uint2* xl2 = reinterpret_cast<const uint2*>(xsw + 8 * NB * XS) + g * (XS / 2) + 4 * t;
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  for (int tile = blockIdx.y * kHeadWarps + warp; tile < ntiles; tile += gridDim.y * kHeadWarps) {
+    const int v0 = tile * 16 + g, v1 = v0 + 8;
+    const uint4* r0 = reinterpret_cast<const uint4*>(a.embed + size_t(min(v0, a.vocab - 1)) * D) + 2 * t;
+    const uint4* r1 = reinterpret_cast<const uint4*>(a.embed + size_t(min(v1, a.vocab - 1)) * D) + 2 * t;
+    const bool ok0 = v0 < a.vocab, ok1 = v1 < a.vocab;
+    float acc[NB][4];
+#pragma unroll
+    for (int n = 0; n < NB; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    uint4 c00 = ok0 ? __ldg(r0) : z4, c01 = ok0 ? __ldg(r0 + 1) : z4;
+    uint4 c10 = ok1 ? __ldg(r1) : z4, c11 = ok1 ? __ldg(r1 + 1) : z4;
+    for (int c = 0; c < nch; ++c) {
+      const uint32_t p0[8] = {c00.x, c00.y, c00.z, c00.w, c01.x, c01.y, c01.z, c01.w};
+      const uint32_t p1[8] = {c10.x, c10.y, c10.z, c10.w, c11.x, c11.y, c11.z, c11.w};
+      if (c + 1 < nch) {
+        c00 = ok0 ? __ldg(r0 + 8 * (c + 1)) : z4;
+        c01 = ok0 ? __ldg(r0 + 8 * (c + 1) + 1) : z4;
+        c10 = ok1 ? __ldg(r1 + 8 * (c + 1)) : z4;
+        c11 = ok1 ? __ldg(r1 + 8 * (c + 1) + 1) : z4;
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint32_t af[4] = {p0[2 * s], p1[2 * s], p0[2 * s + 1], p1[2 * s + 1]};
+#pragma unroll
+        for (int n = 0; n < NB; ++n) {
+          const uint2 bh = xh2[n * 8 * (XS / 2) + 16 * c + s];
+          const uint2 bl = xl2[n * 8 * (XS / 2) + 16 * c + s];
+          mma_f16_16816(acc[n], af, bh.x, bh.y);
+          mma_f16_16816(acc[n], af, bl.x, bl.y);
+        }
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < NB; ++n)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int bc = n * 8 + 2 * t + e;
+        if (bc < nb) {
+          if (ok0) {
+            if (a.logits) a.logits[size_t(b0 + bc) * a.vocab + v0] = acc[n][e];
+            if (better(acc[n][e], v0, best[n][e], besti[n][e])) { best[n][e] = acc[n][e]; besti[n][e] = v0; }
+          }
+          if (ok1) {
+            if (a.logits) a.logits[size_t(b0 + bc) * a.vocab + v1] = acc[n][2 + e];
+            if (better(acc[n][2 + e], v1, best[n][e], besti[n][e])) { best[n][e] = acc[n][2 + e]; besti[n][e] = v1; }
+          }
+        }
+      }
+  }
+  // best over the lanes of equal t (they hold the same batch columns), then over warps
+#pragma unroll
+  for (int n = 0; n < NB; ++n)
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best[n][e], o);
+        const int oi = __shfl_xor_sync(0xffffffffu, besti[n][e], o);
+        if (better(ov, oi, best[n][e], besti[n][e])) { best[n][e] = ov; besti[n][e] = oi; }
+      }
+  if (g == 0) {
+#pragma unroll
+    for (int n = 0; n < NB; ++n)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        wbest[warp][n * 8 + 2 * t + e] = best[n][e];
+        wbesti[warp][n * 8 + 2 * t + e] = besti[n][e];
+      }
+  }
+  __syncthreads();
+  if (threadIdx.x < nb) {
+    const int bc = threadIdx.x;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int w = 0; w < kHeadWarps; ++w)
+      if (better(wbest[w][bc], wbesti[w][bc], bv, bi)) { bv = wbest[w][bc]; bi = wbesti[w][bc]; }
+    a.part_val[size_t(b0 + bc) * gridDim.y + blockIdx.y] = bv;
+    a.part_idx[size_t(b0 + bc) * gridDim.y + blockIdx.y] = bi;
+  }
+}
+
 // grid (B).  Reduces the per-block (logit, id) pairs of one batch row.
 __global__ void k_argmax(const float* __restrict__ part_val, const int* __restrict__ part_idx,
                          int nparts, int32_t* __restrict__ tok_out) {
