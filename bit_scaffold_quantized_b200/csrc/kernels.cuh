@@ -20,19 +20,20 @@ DFSSM_DEV float load_dense(const void* w, int dtype, size_t i) {
 }
 
 // Inverse of the tiled layout: (tile word, bit) -> (row, col) inside the matrix.
-// Bit s + 8i of a lane's word kt is byte i of A-fragment register q = s & 3 of
-// 32-column chunk ch = s >> 2 (m16n8k32 .s8 fragment: rows g / g+8, columns
-// 4t + i / 16 + 4t + i).
+// Word q of a lane holds register q of the A fragments of the tile's eight
+// 32-column m16n8k32 .s8 products s = 0..7: bit s + 8 i is byte i of that register
+// (m16n8k32 .s8 fragment: rows g / g+8, columns 4t + i / 16 + 4t + i of the
+// product).  Product s = 2 m + e covers tile columns 64 m + 16 t + 8 e + [0, 8) of
+// lane t, so the B bytes of products 2m and 2m + 1 are 16 consecutive columns.
 DFSSM_DEV void tiled_coord(size_t word, int bit, int kgroups, int* row, int* col) {
   const size_t tile = word / kTileWords;
   const int within = int(word % kTileWords);
-  const int lane = within >> 2, kt = within & 3;
+  const int lane = within >> 2, q = within & 3;
   const int rt = int(tile / kgroups), kg = int(tile % kgroups);
-  const int i = bit >> 3, s = bit & 7;
-  const int ch = s >> 2, q = s & 3;
+  const int s = bit & 7, i = bit >> 3;
   const int g = lane >> 2, t = lane & 3;
   *row = rt * kTileRows + g + 8 * (q & 1);
-  *col = kg * kTileCols + kt * 64 + ch * 32 + 16 * (q >> 1) + 4 * t + i;
+  *col = kg * kTileCols + 64 * (s >> 1) + 16 * t + 8 * (s & 1) + 4 * (q >> 1) + i;
 }
 
 __global__ void k_pack_rowmajor(const void* __restrict__ w, int dtype, int rows, int cols,
@@ -262,11 +263,11 @@ struct ProjArgs {
   double* dta;             // fp64 [batch][nheads][2]: dt = softplus(dt_raw + dt_bias), dA = exp(-dt exp(A_log))
 };
 
-constexpr int kProjWarps = 8;
+constexpr int kProjWarps = 16;
 constexpr int kProjThreads = kProjWarps * 32;
 
 __host__ __device__ constexpr int proj_cols(int bt) { return ((kDigits * bt + 7) / 8) * 8; }
-__host__ __device__ __forceinline__ int proj_dstride(int K) { return K + 16; }  // bytes; spreads banks
+__host__ __device__ __forceinline__ int proj_dstride(int K) { return K + 64; }  // bytes; == 64 mod 128: conflict-free 16-byte B loads
 __host__ __device__ constexpr int proj_pstride(int bt) { return proj_cols(bt) + 1; }  // odd: spreads banks
 __host__ __device__ __forceinline__ size_t proj_smem_bytes(int K, int rank, int bt) {
   return size_t(proj_cols(bt)) * proj_dstride(K)                 // digit planes
@@ -286,13 +287,13 @@ DFSSM_DEV double scaffold_value(const int (&q)[kDigits], const int* T) {
 
 // grid (gx, ceil(batch/BT)), gx sized to the resident blocks.  A block stages the
 // digit planes of its BT batch rows once; each warp then owns whole 16-row tiles
-// (rt = 8 blockIdx.x + warp, then + 8 gridDim.x, ...) over the full K, so the
+// (rt = 16 blockIdx.x + warp, then + 16 gridDim.x, ...) over the full K, so the
 // integer sums never leave the warp and no block barrier follows the staging.  Per
 // 256-column group the warp expands its lane's 16-byte vector of sign words (loaded
 // two groups ahead) into 0/1 int8 A fragments (one shift + one mask per register)
-// and runs m16n8k32 int8 MMAs against the planes; the epilogue recombines the
-// planes exactly (lane = row, batch rows split over the two half-warps) and adds
-// the LoRA stage 2 in fp64.
+// and runs m16n8k32 int8 MMAs against the planes, one 16-byte B load per plane row
+// serving two products; the epilogue recombines the planes exactly (lane = row,
+// batch rows split over the two half-warps) and adds the LoRA stage 2 in fp64.
 template <int EPI, int BT>
 __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -339,20 +340,18 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
       w1 = kg + 2 < kgroups ? __ldg(tiles + (kg + 2) * 32) : zero4;
       const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-      for (int kt = 0; kt < 4; ++kt) {
+      for (int m = 0; m < 4; ++m) {
+        uint32_t a0[4], a1[4];
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t af[4];
+        for (int q = 0; q < 4; ++q) {
+          a0[q] = sign_bytes(words[q], 2 * m);
+          a1[q] = sign_bytes(words[q], 2 * m + 1);
+        }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) af[q] = sign_bytes(words[kt], 4 * ch + q);
-          const int k0 = kg * kTileCols + kt * 64 + ch * 32 + 4 * t;
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const int8_t* dr = dg + size_t(n * 8 + g) * DS + k0;
-            const uint32_t bf0 = *reinterpret_cast<const uint32_t*>(dr);
-            const uint32_t bf1 = *reinterpret_cast<const uint32_t*>(dr + 16);
-            mma_s8_16832(acc[n], af, bf0, bf1);
-          }
+        for (int n = 0; n < NT; ++n) {
+          const uint4 bq = *reinterpret_cast<const uint4*>(dg + size_t(n * 8 + g) * DS + kg * kTileCols + 64 * m + 16 * t);
+          mma_s8_16832(acc[n], a0, bq.x, bq.y);
+          mma_s8_16832(acc[n], a1, bq.z, bq.w);
         }
       }
     }

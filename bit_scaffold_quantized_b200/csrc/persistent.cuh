@@ -711,7 +711,7 @@ DFSSM_DEV void plane_sums(const unsigned char* asmb, int Q, int S, int BS, int* 
 // slice for all R rows: stage[j] = sum_k A[j][k] q[k] over the slice, fenced for the
 // async proxy.
 DFSSM_DEV void codes_and_lora_partials(const uint16_t* xs, int S, float sx, float rcp, bool nonzero, int8_t* xqs,
-                                       const int8_t* Aslice, int R, int* scratch, int* stage, int8_t* xq_diag) {
+                                       const int8_t* Aslice, int R, int* stage, int8_t* xq_diag) {
   const int tid = threadIdx.x;
   for (int i = tid; i < S; i += kPThreads) {
     const int q = nonzero ? quant_code_bits(half_to_float_bits(xs[i]), sx, rcp) : 0;
@@ -773,55 +773,63 @@ DFSSM_DEV void lora2_rows(const int8_t* Bq, int nrows, const double* u, int R, d
 // Exact scaffold MMA over `ntile` tiles (smem, kg groups each), split into units
 // (tile, kgroup chunk); int32 partials to part[unit][16][kDigits].  The activation
 // digit planes come from the cluster's slice blocks: column k lies in block
-// k >> lgS at offset k & (S - 1) of each plane (stride S + 16).  Four independent
-// accumulator sets (one per 64-column subtile) keep the tensor pipe busy instead
-// of one serial MMA chain.  Returns the chunks per tile.
+// k >> lgS at offset k & (S - 1) of each plane (stride S + 16).  Register q of the
+// A fragment of product s is word q of the lane's sign vector masked to bits
+// s, s + 8, s + 16, s + 24: unsigned bytes 0 or 2^s, one instruction per register.
+// Product s accumulates into its own set, 2^s times its 0/1 sums (|sum| < 2^27),
+// and the sets are recombined exactly with right shifts.  One 16-byte load per
+// plane row gives the B fragments of products 2m and 2m + 1.  Returns the chunks
+// per tile.
 DFSSM_DEV int scaffold_mma(const unsigned char* tiles, int ntile, int kg, const unsigned char* asmb, int lgS, int BS,
                            int* part) {
+  constexpr int nw = kPWarps;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  int nchunk = kPWarps / ntile;
+  int nchunk = nw / ntile;
   if (nchunk < 1) nchunk = 1;
   if (nchunk > kg) nchunk = kg;
   const int S = 1 << lgS;
   const int nunits = ntile * nchunk;
-  const unsigned char* dbase = asmb + (g < kDigits ? g : 0) * (S + 16) + 4 * t;
-  for (int unit = warp; unit < nunits; unit += kPWarps) {
+  const unsigned char* dbase = asmb + (g < kDigits ? g : 0) * (S + 16);
+  for (int unit = warp; unit < nunits; unit += nw) {
     const int ti = unit / nchunk, ci = unit % nchunk;
     const int kg_lo = ci * kg / nchunk, kg_hi = (ci + 1) * kg / nchunk;
-    int acc[4][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
+    int acc[8][4];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) acc[s][0] = acc[s][1] = acc[s][2] = acc[s][3] = 0;
     const uint4* tw = reinterpret_cast<const uint4*>(tiles + size_t(ti) * kg * 512);
     for (int kgi = kg_lo; kgi < kg_hi; ++kgi) {
       const uint4 wv = tw[kgi * 32 + lane];
       const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
+      for (int m = 0; m < 4; ++m) {
+        // 16 aligned columns never straddle a slice block (S >= 16)
+        const int k0 = kgi * kTileCols + 64 * m + 16 * t;
+        uint4 bq = make_uint4(0, 0, 0, 0);
+        if (g < kDigits) bq = *reinterpret_cast<const uint4*>(dbase + (k0 >> lgS) * BS + (k0 & (S - 1)));
 #pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-          uint32_t af[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) af[q] = sign_bytes(words[kt], 4 * ch + q);
-          const int k0 = kgi * kTileCols + kt * 64 + ch * 32;
-          const unsigned char* p = dbase + (k0 >> lgS) * BS + (k0 & (S - 1));
-          uint32_t b0 = 0, b1 = 0;
-          if (g < kDigits) {
-            b0 = *reinterpret_cast<const uint32_t*>(p);
-            b1 = *reinterpret_cast<const uint32_t*>(p + 16);
-          }
-          mma_s8_16832(acc[kt], af, b0, b1);
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t mask = 0x01010101u << (2 * m + e);
+          const uint32_t af[4] = {words[0] & mask, words[1] & mask, words[2] & mask, words[3] & mask};
+          mma_u8s8_16832(acc[2 * m + e], af, e ? bq.z : bq.x, e ? bq.w : bq.y);
         }
       }
     }
+    int tot[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[0][i] += acc[1][i] + acc[2][i] + acc[3][i];
+    for (int i = 0; i < 4; ++i) {
+      tot[i] = acc[0][i];
+#pragma unroll
+      for (int s = 1; s < 8; ++s) tot[i] += acc[s][i] >> s;   // exact: acc[s] is a multiple of 2^s
+    }
     int* pp = part + unit * 16 * kDigits;
     if (2 * t < kDigits) {
-      pp[g * kDigits + 2 * t] = acc[0][0];
-      pp[(g + 8) * kDigits + 2 * t] = acc[0][2];
+      pp[g * kDigits + 2 * t] = tot[0];
+      pp[(g + 8) * kDigits + 2 * t] = tot[2];
     }
     if (2 * t + 1 < kDigits) {
-      pp[g * kDigits + 2 * t + 1] = acc[0][1];
-      pp[(g + 8) * kDigits + 2 * t + 1] = acc[0][3];
+      pp[g * kDigits + 2 * t + 1] = tot[1];
+      pp[(g + 8) * kDigits + 2 * t + 1] = tot[3];
     }
   }
   csync();
@@ -1026,7 +1034,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         plane_sums(asm_a, Q, SD, BSD, redi, a.d_xdsum_in);
       }
       // ---- B: codes and LoRA partials of the slice -> the cluster
-      codes_and_lora_partials(xs, SD, sx_in, __frcp_rn(sx_in), am_in > 0.f, xqs, sp<int8_t>(sm, PSM(a_in)), R, part,
+      codes_and_lora_partials(xs, SD, sx_in, __frcp_rn(sx_in), am_in > 0.f, xqs, sp<int8_t>(sm, PSM(a_in)), R,
                               stg_b, cdiag ? a.d_xq_in + r0D : nullptr);
       if (R) xsend(stg_b, rcv_b + w.r * R, unsigned(4 * R), &xbars[EX_B_IN], Q);
       // ---- in_proj scaffold on own tiles
@@ -1203,7 +1211,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       }
       // ---- B': codes and LoRA partials of the slice -> the cluster
       codes_and_lora_partials(xs, SE, sx_out, __frcp_rn(sx_out), am_out > 0.f, xqs, sp<int8_t>(sm, PSM(a_out)), R,
-                              part, stg_b, cdiag ? a.d_xq_out + r0E : nullptr);
+                              stg_b, cdiag ? a.d_xq_out + r0E : nullptr);
       if (R) xsend(stg_b, rcv_b + w.r * R, unsigned(4 * R), &xbars[EX_B_OUT], Q);
       // ---- out_proj scaffold on own tiles
       int nch_out = 1;

@@ -75,31 +75,37 @@ def tiled_bit_position(row, col, cols: int):
 
     Works elementwise on integers or integer arrays.  The tiled layout is a
     bijective permutation of the row-major bits into 16-row x 256-column tiles of
-    128 words, chosen so that each of the 32 lanes of a warp reads one 16-byte
-    vector per tile and forms each int8 A-fragment register of an m16n8k32
-    tensor-core product with one shift and one mask (byte = sign bit, 0 or 1).
+    128 words (32 lanes x 4 words), built for m16n8k32 int8 tensor-core products.
+    A tile's 256 columns are 8 products of 32 columns, s = 0..7.  Register q of the
+    A fragment of product s, for every lane, is bits s, s + 8, s + 16, s + 24 of the
+    lane's word q (byte i = bit s + 8 i).  A register is therefore one mask of word
+    q, or a shift and a mask.  The columns of products 2m and 2m + 1 are interleaved
+    so that lane t finds its B-fragment bytes for both at 16 consecutive columns,
+    64 m + 16 t .. 64 m + 16 t + 15.
     Within a tile:
-      r16 = row % 16, c = col % 256, kt = c // 64, ch = (c % 64) // 32,
-      c32 = c % 32, colhalf = c32 // 16, t = (c32 % 16) // 4, i = c32 % 4,
-      lane = (r16 % 8) * 4 + t,  q = r16 // 8 + 2 * colhalf,  s = 4 * ch + q,
+      r16 = row % 16, c = col % 256, m = c // 64, p = c % 64,
+      t = p // 16, e = (p % 16) // 8, h = (p % 8) // 4, i = p % 4,
+      lane = (r16 % 8) * 4 + t,  q = r16 // 8 + 2 * h,  s = 2 * m + e,
       bit = s + 8 * i,
-      word = ((row // 16) * (cols // 256) + col // 256) * 128 + lane * 4 + kt.
+      word = ((row // 16) * (cols // 256) + col // 256) * 128 + lane * 4 + q.
+    For product s the fragment's column 4t + i (+16 when q >= 2) is therefore
+    column 64 m + 16 t + 8 e + i (+4) of the tile.
     """
     row = np.asarray(row, dtype=np.int64)
     col = np.asarray(col, dtype=np.int64)
     r16 = row % TILE_ROWS
     c = col % TILE_COLS
-    kt = c // 64
-    ch = (c % 64) // 32
-    c32 = c % 32
-    colhalf = c32 // 16
-    t = (c32 % 16) // 4
-    i = c32 % 4
+    m = c // 64
+    p = c % 64
+    t = p // 16
+    e = (p % 16) // 8
+    h = (p % 8) // 4
+    i = p % 4
     lane = (r16 % 8) * 4 + t
-    q = r16 // 8 + 2 * colhalf
-    s = 4 * ch + q
+    q = r16 // 8 + 2 * h
+    s = 2 * m + e
     bit = s + 8 * i
-    word = ((row // TILE_ROWS) * (cols // TILE_COLS) + col // TILE_COLS) * 128 + lane * 4 + kt
+    word = ((row // TILE_ROWS) * (cols // TILE_COLS) + col // TILE_COLS) * 128 + lane * 4 + q
     return word, bit
 
 

@@ -69,26 +69,35 @@ def test_tiled_layout_matches_mma_fragment_table():
     """Independent check against the m16n8k32 .s8 A-fragment table of the PTX ISA:
     lane = 4*groupID + threadID_in_group; register 0 holds (g, 4t..4t+3), register 1
     (g+8, 4t..4t+3), register 2 (g, 16+4t..), register 3 (g+8, 16+4t..).  Register q
-    of 32-column chunk ch is (word >> s) & 0x01010101 with s = 4ch+q: byte i of it
-    is the sign bit of column 4t+i (+16 for q >= 2)."""
+    of product s is (word_q >> s) & 0x01010101; byte i of it is the sign bit of the
+    fragment's column 4t+i (+16 for q >= 2), which the layout places at tile column
+    64 (s // 2) + 16 t + 8 (s % 2) + i (+4 for q >= 2).  The B fragment of lane t
+    (columns 4t..4t+3 and 16+4t..16+4t+3 of the product) is then the 8 bytes at
+    64 (s // 2) + 16 t + 8 (s % 2): products 2m and 2m+1 read 16 consecutive bytes."""
     rng = np.random.default_rng(11)
     rows, cols = 16, 256
     dense = rng.choice([-1.0, 1.0], size=(rows, cols)).astype(np.float32)
     tiled = O.tile_signs(O.pack_signs(dense), rows, cols)
     frag_pos = {0: (0, 0), 1: (8, 0), 2: (0, 16), 3: (8, 16)}   # reg q -> (row offset, col offset)
+    seen = np.zeros((rows, cols), dtype=int)
     for lane in range(32):
         g, t = lane // 4, lane % 4
-        for kt in range(4):
-            word = int(tiled[lane * 4 + kt])
-            for ch in range(2):
-                for q in range(4):
-                    reg = (word >> (4 * ch + q)) & 0x01010101
-                    ro, co = frag_pos[q]
-                    for i in range(4):
-                        bit = (reg >> (8 * i)) & 0xFF
-                        assert bit in (0, 1)
-                        col = kt * 64 + ch * 32 + co + 4 * t + i
-                        assert (1.0 if bit else -1.0) == dense[g + ro, col]
+        for s in range(8):
+            for q in range(4):
+                reg = (int(tiled[lane * 4 + q]) >> s) & 0x01010101
+                ro, co = frag_pos[q]
+                for i in range(4):
+                    bit = (reg >> (8 * i)) & 0xFF
+                    assert bit in (0, 1)
+                    kcol = co + 4 * t + i                            # fragment column 0..31
+                    col = 64 * (s // 2) + 16 * t + 8 * (s % 2) + 4 * (co // 16) + i
+                    # the same fragment column of the B operand (lane t: b0 = 4t..4t+3,
+                    # b1 = 16+4t..) sits at byte 8 * (s % 2) + 4 * (co // 16) + i of the
+                    # lane's 16 bytes from 64 (s // 2) + 16 t
+                    assert col == 64 * (s // 2) + 16 * t + (8 * (s % 2) + 4 * (kcol // 16) + kcol % 4)
+                    assert (1.0 if bit else -1.0) == dense[g + ro, col]
+                    seen[g + ro, col] += 1
+    assert np.all(seen == 1)
 
 
 def test_tiled_rows_padded():
