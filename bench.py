@@ -291,7 +291,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
                      "kernel": "whole decode step (graph replay)",
                      "algorithmic_bytes_per_step": bytes_tok, "peak_source": peak_kind},
-        "roofline_tokens_per_s": round(peak * 1e9 / bytes_tok, 1),
+        "roofline_tokens_per_s": round(peak * 1e9 / bytes_tok * d.batch, 1),   # one step = batch tokens
         "e2e": {"value": round(RP.job_tokens_per_s(args.steps, d.batch, world, ms_e2e), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * d.batch, "d2h_bytes_per_step": 4 * d.batch},
         "gpu_launches": launches_per_step * args.steps,
