@@ -324,6 +324,45 @@ int launch_head(const HeadArgs& h, cudaStream_t st, int* nparts) {
   return DFSSM_OK;
 }
 
+// SSM update of the multi-launch path: the streaming kernel when an item's inputs
+// fit two shared-memory buffers and every bulk copy is 16-byte aligned, else k_ssm.
+constexpr int kSsmStreamSmemCap = 96 * 1024;
+
+template <int NCH>
+int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
+  static int occ_smem = -1, occ_blocks = 1;
+  if (occ_smem != smem) {
+    cudaFuncSetAttribute(k_ssm_stream<NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_ssm_stream<NCH>, kSsmStreamThreads, smem) !=
+            cudaSuccess || nb < 1)
+      nb = 1;
+    occ_smem = smem;
+    occ_blocks = nb;
+  }
+  const int items = sa.batch * sa.H;
+  const int grid = std::max(1, std::min(items, occ_blocks * sm_count()));
+  k_ssm_stream<NCH><<<grid, kSsmStreamThreads, smem, st>>>(sa);
+  CHECK_LAUNCH("k_ssm_stream");
+  return DFSSM_OK;
+}
+
+int launch_ssm(const SsmArgs& sa, cudaStream_t st) {
+  const SsmItem it = ssm_item(sa.P, sa.N);
+  const int smem = 2 * ((it.bytes + 127) & ~127);
+  const bool aligned = (size_t(sa.conv_dim) * 8) % 16 == 0 && (size_t(sa.in_rows) * 8) % 16 == 0 &&
+                       (size_t(sa.E) * 8) % 16 == 0 && (size_t(sa.P) * 8) % 16 == 0 &&
+                       aligned16(sa.state) && aligned16(sa.xc) && aligned16(sa.zx) && aligned16(sa.dta);
+  if (aligned && smem <= kSsmStreamSmemCap) {
+    if (sa.N <= 128) return launch_ssm_stream<1>(sa, smem, st);
+    return launch_ssm_stream<2>(sa, smem, st);
+  }
+  if (sa.N <= 128) k_ssm<1><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
+  else k_ssm<2><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
+  CHECK_LAUNCH("k_ssm");
+  return DFSSM_OK;
+}
+
 // The layer as five dependent launches on one stream.
 int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const dfssm_layer_state* s,
                       float* res, const Bufs& b, cudaStream_t st) {
@@ -339,10 +378,8 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   SsmArgs sa{};
   sa.H = d->nheads; sa.P = d->headdim; sa.N = d->d_state; sa.E = E; sa.conv_dim = C; sa.in_rows = in_rows(d);
   sa.zx = b.zxbcdt; sa.xc = b.xc; sa.dt_bias = w->dt_bias; sa.A_log = w->A_log; sa.D = w->D;
-  sa.state = s->ssm_state; sa.g = b.g; sa.dta = b.dta;
-  if (d->d_state <= 128) k_ssm<1><<<dim3(d->nheads, B), kSsmThreads, 0, st>>>(sa);
-  else k_ssm<2><<<dim3(d->nheads, B), kSsmThreads, 0, st>>>(sa);
-  CHECK_LAUNCH("k_ssm");
+  sa.state = s->ssm_state; sa.g = b.g; sa.dta = b.dta; sa.batch = B; sa.status = b.status;
+  if ((rc = launch_ssm(sa, st))) return rc;
   if ((rc = launch_prologue<0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, B, b.out);
   po.out = res;

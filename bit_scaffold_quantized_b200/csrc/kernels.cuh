@@ -432,6 +432,8 @@ struct SsmArgs {
   float* state;          // fp32 [B][H][P][N]
   float* g;              // fp32 [B][E]
   const double* dta;     // fp64 [B][H][2]: step size and decay (from the in_proj epilogue)
+  int batch;
+  unsigned* status;      // bit 4096 set if a streamed copy did not land (k_ssm_stream)
 };
 
 constexpr int kSsmThreads = 256;
@@ -533,6 +535,142 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
       const double yy = fma(double(a.D[h]), xcb[e], ys);
       a.g[size_t(b) * a.E + e] = float(yy * silu_d(zr[e]));
     }
+  }
+}
+
+// Bytes of one (batch, head) item of k_ssm_stream and their offsets in a buffer:
+// state [P][N] fp32, then B and C [2N] fp64, x [P] fp64, z [P] fp64, (dt, dA) fp64.
+struct SsmItem {
+  int st, bc, x, z, dta, bytes;
+};
+__host__ __device__ inline SsmItem ssm_item(int P, int N) {
+  SsmItem it;
+  it.st = 0;
+  it.bc = 4 * P * N;
+  it.x = it.bc + 16 * N;
+  it.z = it.x + 8 * P;
+  it.dta = it.z + 8 * P;
+  it.bytes = it.dta + 16;
+  return it;
+}
+constexpr int kSsmStreamThreads = 256;
+
+// Streaming SSM update: grid of resident blocks; block c takes the (batch, head)
+// items c, c + gridDim.x, ...  Each item's inputs (its 4 P N bytes of state, the
+// batch row's B and C, the head's x and z, its step size and decay) arrive by bulk
+// copies into one of two shared-memory buffers, the next item's while this one is
+// computed, so HBM always has a block's worth of state in flight per block.  Warp w
+// takes rows w, w + 8, ... four at a time; a lane holds NCH float4 of a row.  Same
+// arithmetic as k_ssm (fp64, state stored back in fp32 with a streaming hint).
+template <int NCH>
+__global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
+  extern __shared__ __align__(16) unsigned char sbuf[];
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int s_ok;
+  constexpr int RW = 4, kW = kSsmStreamThreads / 32;
+  const int P = a.P, N = a.N, H = a.H, N4 = N / 4;
+  const SsmItem it = ssm_item(P, N);
+  const int bufb = (it.bytes + 127) & ~127;
+  const int nitems = a.batch * H;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int item, int buf) {
+    const int b = item / H, h = item % H;
+    unsigned char* base = sbuf + buf * bufb;
+    mbar_expect_tx(&bar[buf], unsigned(it.bytes));
+    bulk_g2s(base + it.st, a.state + (size_t(b) * H + h) * P * N, unsigned(4 * P * N), &bar[buf]);
+    bulk_g2s(base + it.bc, a.xc + size_t(b) * a.conv_dim + a.E, unsigned(16 * N), &bar[buf]);
+    bulk_g2s(base + it.x, a.xc + size_t(b) * a.conv_dim + size_t(h) * P, unsigned(8 * P), &bar[buf]);
+    bulk_g2s(base + it.z, a.zx + size_t(b) * a.in_rows + size_t(h) * P, unsigned(8 * P), &bar[buf]);
+    bulk_g2s(base + it.dta, a.dta + (size_t(b) * H + h) * 2, 16u, &bar[buf]);
+  };
+  if (tid == 0) {
+    if (int(blockIdx.x) < nitems) issue(blockIdx.x, 0);
+    if (int(blockIdx.x + gridDim.x) < nitems) issue(blockIdx.x + gridDim.x, 1);
+  }
+  for (int k = 0;; ++k) {
+    const int item = int(blockIdx.x) + k * int(gridDim.x);
+    if (item >= nitems) break;
+    const int buf = k & 1;
+    const unsigned par = unsigned(k >> 1) & 1u;
+    if (tid == 0) {
+      long long spins = 0;
+      bool ok = true;
+      while (!mbar_try_wait(&bar[buf], par))
+        if (++spins > (1 << 22)) { ok = false; break; }
+      s_ok = ok ? 1 : 0;
+      if (!ok) atomicOr(a.status, 4096u);
+    }
+    __syncthreads();
+    if (!s_ok) {
+      // give copies that may still be in flight time to land, then leave
+      const long long t0 = clock64();
+      while (clock64() - t0 < 200000) __nanosleep(1000);
+      return;
+    }
+    (void)mbar_try_wait(&bar[buf], par);   // every thread acquires the copies' writes
+    const unsigned char* base = sbuf + buf * bufb;
+    const float* st = reinterpret_cast<const float*>(base + it.st);
+    const double* Bs = reinterpret_cast<const double*>(base + it.bc);
+    const double* Cs = Bs + N;
+    const double* xs = reinterpret_cast<const double*>(base + it.x);
+    const double* zs = reinterpret_cast<const double*>(base + it.z);
+    const double dt = reinterpret_cast<const double*>(base + it.dta)[0];
+    const double dA = reinterpret_cast<const double*>(base + it.dta)[1];
+    const int b = item / H, h = item % H;
+    float* gst = a.state + (size_t(b) * H + h) * P * N;
+    double Bv[NCH][4], Cv[NCH][4];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int n4 = lane + 32 * c;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        Bv[c][e] = n4 < N4 ? Bs[4 * n4 + e] : 0.0;
+        Cv[c][e] = n4 < N4 ? Cs[4 * n4 + e] : 0.0;
+      }
+    }
+    for (int r0 = warp; r0 < P; r0 += RW * kW) {
+      double y[RW];
+#pragma unroll
+      for (int i = 0; i < RW; ++i) {
+        const int p = r0 + i * kW;
+        const double xdt = p < P ? xs[p] * dt : 0.0;
+        double acc = 0.0;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          const int n4 = lane + 32 * c;
+          if (p < P && n4 < N4) {
+            const float4 hv = reinterpret_cast<const float4*>(st + size_t(p) * N)[n4];
+            const double h0 = fma(dA, double(hv.x), xdt * Bv[c][0]);
+            const double h1 = fma(dA, double(hv.y), xdt * Bv[c][1]);
+            const double h2 = fma(dA, double(hv.z), xdt * Bv[c][2]);
+            const double h3 = fma(dA, double(hv.w), xdt * Bv[c][3]);
+            acc = fma(Cv[c][0], h0, acc);
+            acc = fma(Cv[c][1], h1, acc);
+            acc = fma(Cv[c][2], h2, acc);
+            acc = fma(Cv[c][3], h3, acc);
+            __stcs(reinterpret_cast<float4*>(gst + size_t(p) * N) + n4,
+                   make_float4(float(h0), float(h1), float(h2), float(h3)));
+          }
+        }
+        y[i] = acc;
+      }
+      int sel;
+      const double ys = fold_rows<RW>(y, lane, &sel);
+      const int p = r0 + sel * kW;
+      if ((lane & (32 / RW - 1)) == 0 && p < P) {
+        const int e = h * P + p;
+        const double yy = fma(double(a.D[h]), xs[p], ys);
+        a.g[size_t(b) * a.E + e] = float(yy * silu_d(zs[p]));
+      }
+    }
+    __syncthreads();   // buffer consumed
+    if (tid == 0 && item + 2 * int(gridDim.x) < nitems) issue(item + 2 * int(gridDim.x), buf);
   }
 }
 

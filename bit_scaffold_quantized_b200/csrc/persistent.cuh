@@ -223,25 +223,6 @@ static_assert((1 << Shape2048::lgSD) == Shape2048::SD && (1 << Shape2048::lgSE) 
 
 // ------------------------------------------------------------------ primitives
 
-DFSSM_DEV uint32_t smem_u32(const void* p) { return uint32_t(__cvta_generic_to_shared(p)); }
-
-DFSSM_DEV void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
-}
-DFSSM_DEV void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-DFSSM_DEV void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
-}
-DFSSM_DEV bool mbar_try_wait(uint64_t* bar, unsigned parity) {
-  unsigned ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-  return ok != 0;
-}
 DFSSM_DEV bool mbar_try_wait_cluster(uint64_t* bar, unsigned parity) {
   unsigned ok;
   asm volatile(
@@ -250,11 +231,6 @@ DFSSM_DEV bool mbar_try_wait_cluster(uint64_t* bar, unsigned parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-DFSSM_DEV void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
 // Shared memory of this CTA -> shared memory of a CTA of the cluster (addresses
 // from cluster_map), completion counted on that CTA's mbarrier.
 DFSSM_DEV void bulk_s2c(uint32_t dst, const void* src, unsigned bytes, uint32_t bar) {
@@ -262,9 +238,6 @@ DFSSM_DEV void bulk_s2c(uint32_t dst, const void* src, unsigned bytes, uint32_t 
       "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :: "r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(bar) : "memory");
 }
-// Generic-proxy writes of this thread to shared memory become visible to later
-// bulk copies (async proxy) that read them.
-DFSSM_DEV void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 DFSSM_DEV uint32_t cluster_map(uint32_t saddr, unsigned rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
