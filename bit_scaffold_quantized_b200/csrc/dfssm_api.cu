@@ -214,6 +214,12 @@ int launch_prologue(int K, int rank, int batch, const float* src, const uint16_t
   a.K = K; a.rank = rank; a.src = src; a.src16 = src16; a.w = w;
   a.x = o.x; a.xq = o.xq; a.sx = o.sx; a.xd = o.xd; a.xdsum = o.xdsum;
   a.A = p->A; a.sA = p->sA; a.acc = o.acc; a.u = o.u;
+  if (K % (16 * kPrologueCQ) == 0 && K <= kPrologueCQ * kPrologueClThreads * kPrologueClVals &&
+      rank <= kPrologueMaxRank) {
+    k_prologue_cl<MODE><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a);
+    CHECK_LAUNCH("k_prologue_cl");
+    return DFSSM_OK;
+  }
   dim3 grid(rank > 0 ? (rank + kPrologueRowsPerBlock - 1) / kPrologueRowsPerBlock : 1, batch);
   k_prologue<MODE><<<grid, kPrologueThreads, size_t(K), st>>>(a);
   CHECK_LAUNCH("k_prologue");
@@ -312,7 +318,7 @@ int launch_head_tc(const HeadArgs& h, cudaStream_t st, int* nparts) {
 }
 
 int launch_head(const HeadArgs& h, cudaStream_t st, int* nparts) {
-  if (h.D % 64 == 0) {
+  if (h.D % 256 == 0) {
     if (h.batch > 8 && head_tc_smem(h.D, 2) <= kHeadTcSmemCap) return launch_head_tc<2>(h, st, nparts);
     if (head_tc_smem(h.D, 1) <= kHeadTcSmemCap) return launch_head_tc<1>(h, st, nparts);
   }

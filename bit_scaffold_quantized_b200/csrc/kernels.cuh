@@ -235,6 +235,170 @@ __global__ void __launch_bounds__(kPrologueThreads) k_prologue(PrologueArgs a) {
   }
 }
 
+// Cluster prologue: one cluster of kPrologueCQ CTAs per batch row (grid (CQ, B));
+// CTA rank q owns columns [q K/CQ, (q+1) K/CQ), at most 4 per thread.  The row's
+// sum of squares and max |x| are all-reduced through distributed shared memory
+// (each CTA stores its partial into every CTA; all sum in rank order, so every CTA
+// holds the same value); each CTA writes its columns' x, codes and digit planes;
+// the digit-plane sums and the LoRA stage-1 partials of its columns go to rank 0,
+// which adds them in rank order (exact) and writes xdsum, acc, u and sx.
+// Same arithmetic as k_prologue.
+constexpr int kPrologueCQ = 4;
+constexpr int kPrologueClThreads = 512;  // two CTAs per SM (64 registers): a batch of 64 rows runs in one wave
+constexpr int kPrologueClVals = 4;      // K / CQ / 512 <= 4: K <= 8192
+constexpr int kPrologueMaxRank = 128;
+
+template <int MODE>
+__global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueClThreads, 2)
+    k_prologue_cl(PrologueArgs a) {
+  constexpr int CQ = kPrologueCQ, NW = kPrologueClThreads / 32;
+  __shared__ double xss[CQ];
+  __shared__ float xam[CQ];
+  __shared__ int xpart[CQ][kDigits + kPrologueMaxRank];
+  __shared__ double redd[32];
+  __shared__ float red[32];
+  __shared__ int red6[NW][kDigits];
+  __shared__ __align__(16) int8_t qs[8192 / CQ];
+  const int K = a.K, Kq = K / CQ;
+  const int q = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k0 = q * Kq;
+
+  // this warp's first two LoRA rows over the CTA's columns (loads issued first)
+  const int nvq = Kq / 16;                                  // 16-byte chunks of a row slice (<= 128)
+  uint4 av[2][4];
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int j = warp + NW * rr, c = lane + 32 * m;
+      av[rr][m] = (j < a.rank && c < nvq) ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K + k0) + c)
+                                          : make_uint4(0, 0, 0, 0);
+    }
+  uint32_t h[kPrologueClVals];
+  float am = 0.f;
+  if (MODE == 0) {
+    const float* v = a.src + size_t(b) * K + k0;
+    float vf[kPrologueClVals];
+    uint16_t wh[kPrologueClVals];
+#pragma unroll
+    for (int i = 0; i < kPrologueClVals; ++i) {
+      const int k = tid + i * kPrologueClThreads;
+      vf[i] = k < Kq ? v[k] : 0.f;
+      wh[i] = k < Kq ? a.w[k0 + k] : uint16_t(0);
+    }
+    double ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < kPrologueClVals; ++i) ss = fma(double(vf[i]), double(vf[i]), ss);
+    ss = block_sum_d(ss, redd);
+    cluster_sync_all();                    // every CTA of the cluster runs: remote stores allowed
+    if (tid < CQ) st_cluster_f64(cluster_map(smem_u32(&xss[q]), tid), ss);
+    cluster_sync_all();
+    double sst = 0.0;
+#pragma unroll
+    for (int r = 0; r < CQ; ++r) sst += xss[r];
+    const double rs = 1.0 / sqrt(sst / double(K) + kEpsD);
+    const float rs32 = float(rs);
+#pragma unroll
+    for (int i = 0; i < kPrologueClVals; ++i) {
+      const int k = tid + i * kPrologueClThreads;
+      h[i] = k < Kq ? norm_fp16(vf[i], rs, rs32, half_to_float_bits(wh[i])) : 0u;
+      am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
+      if (k < Kq && a.x) a.x[size_t(b) * K + k0 + k] = uint16_t(h[i]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPrologueClVals; ++i) {
+      const int k = tid + i * kPrologueClThreads;
+      h[i] = k < Kq ? a.src16[size_t(b) * K + k0 + k] : 0u;
+      am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
+    }
+    cluster_sync_all();                    // every CTA of the cluster runs: remote stores allowed
+  }
+  am = block_max(am, red);
+  if (tid < CQ) st_cluster_u32(cluster_map(smem_u32(&xam[q]), tid), __float_as_uint(am));
+  cluster_sync_all();
+  float amt = 0.f;
+#pragma unroll
+  for (int r = 0; r < CQ; ++r) amt = fmaxf(amt, xam[r]);
+  const float sx = amt > 0.f ? __fdiv_rn(amt, 127.f) : 1.f;
+  const float rcp = __frcp_rn(sx);
+  int dsum[kDigits];
+#pragma unroll
+  for (int d = 0; d < kDigits; ++d) dsum[d] = 0;
+#pragma unroll
+  for (int i = 0; i < kPrologueClVals; ++i) {
+    const int k = tid + i * kPrologueClThreads;
+    if (k < Kq) {
+      const int8_t c = amt > 0.f ? int8_t(quant_code_bits(half_to_float_bits(h[i]), sx, rcp)) : int8_t(0);
+      qs[k] = c;
+      a.xq[size_t(b) * K + k0 + k] = c;
+      uint32_t lo, hi;
+      digits_of(h[i], &lo, &hi);
+      const uint32_t w6[kDigits] = {lo, lo >> 8, lo >> 16, lo >> 24, hi, hi >> 8};
+#pragma unroll
+      for (int d = 0; d < kDigits; ++d) {
+        const int8_t dg = int8_t(w6[d] & 0xffu);
+        a.xd[(size_t(b) * kDigits + d) * K + k0 + k] = dg;
+        dsum[d] += dg;
+      }
+    }
+  }
+#pragma unroll
+  for (int d = 0; d < kDigits; ++d) {
+    const int t = __reduce_add_sync(0xffffffffu, dsum[d]);
+    if (lane == 0) red6[warp][d] = t;
+  }
+  __syncthreads();                         // codes and the warps' plane sums complete
+  if (tid < kDigits) {
+    int t = 0;
+    for (int w = 0; w < NW; ++w) t += red6[w][tid];
+    st_cluster_u32(cluster_map(smem_u32(&xpart[q][tid]), 0), uint32_t(t));
+  }
+  // LoRA stage-1 partials of this CTA's columns: warp w takes rows w, w + 16, ...
+  const uint4* q16 = reinterpret_cast<const uint4*>(qs);
+  for (int j = warp, rr = 0; j < a.rank; j += NW, ++rr) {
+    int acc = 0;
+    if (rr < 2) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        if (c < nvq) {
+          const uint4 x4 = q16[c], w4 = rr == 0 ? av[0][m] : av[1][m];
+          acc = __dp4a(int(w4.x), int(x4.x), acc);
+          acc = __dp4a(int(w4.y), int(x4.y), acc);
+          acc = __dp4a(int(w4.z), int(x4.z), acc);
+          acc = __dp4a(int(w4.w), int(x4.w), acc);
+        }
+      }
+    } else {
+      for (int c = lane; c < nvq; c += 32) {
+        const uint4 x4 = q16[c], w4 = __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K + k0) + c);
+        acc = __dp4a(int(w4.x), int(x4.x), acc);
+        acc = __dp4a(int(w4.y), int(x4.y), acc);
+        acc = __dp4a(int(w4.z), int(x4.z), acc);
+        acc = __dp4a(int(w4.w), int(x4.w), acc);
+      }
+    }
+    acc = warp_sum_i(acc);
+    if (lane == 0) st_cluster_u32(cluster_map(smem_u32(&xpart[q][kDigits + j]), 0), uint32_t(acc));
+  }
+  cluster_sync_all();                      // rank 0 holds every CTA's partials
+  if (q == 0) {
+    if (tid < kDigits) {
+      int t = 0;
+      for (int r = 0; r < CQ; ++r) t += xpart[r][tid];
+      a.xdsum[b * kDigits + tid] = t;
+      if (tid == 0) a.sx[b] = sx;
+    }
+    for (int j = tid; j < a.rank; j += kPrologueClThreads) {
+      int acc = 0;
+      for (int r = 0; r < CQ; ++r) acc += xpart[r][kDigits + j];
+      a.acc[size_t(b) * a.rank + j] = acc;
+      a.u[size_t(b) * a.rank + j] = (double(acc) * h2d(a.sA[j])) * double(sx);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ projection
 
 enum { EPI_STORE = 0, EPI_RESID = 1, EPI_INPROJ = 2 };
@@ -793,7 +957,7 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead(HeadArgs a) {
 // head rows with both parts are exact and only the fp32 accumulation rounds.  Each
 // warp owns 16-row vocabulary tiles (tile = 8 blockIdx.y + warp, + 8 gy, ...); per
 // 64-column chunk, lane (g, t) loads 16 bytes x 2 of rows g and g + 8 at columns
-// 16 t.. (coalesced, one chunk ahead) and runs four m16n8k16 MMAs per batch n-tile
+// 16 t.. (coalesced, three chunks ahead) and runs four m16n8k16 MMAs per batch n-tile
 // and part.  The MMA's k index i maps to column 64 c + 16 t + 4 s + (i & 1) + 2 (i >> 3)
 // for A and B alike, so the chunk's 64 columns are each summed once.  Per batch row
 // the block keeps the best (logit, id), lowest id on ties.
@@ -843,26 +1007,35 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
     float acc[NB][4];
 #pragma unroll
     for (int n = 0; n < NB; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    uint4 c00 = ok0 ? __ldg(r0) : z4, c01 = ok0 ? __ldg(r0 + 1) : z4;
-    uint4 c10 = ok1 ? __ldg(r1) : z4, c11 = ok1 ? __ldg(r1 + 1) : z4;
-    for (int c = 0; c < nch; ++c) {
-      const uint32_t p0[8] = {c00.x, c00.y, c00.z, c00.w, c01.x, c01.y, c01.z, c01.w};
-      const uint32_t p1[8] = {c10.x, c10.y, c10.z, c10.w, c11.x, c11.y, c11.z, c11.w};
-      if (c + 1 < nch) {
-        c00 = ok0 ? __ldg(r0 + 8 * (c + 1)) : z4;
-        c01 = ok0 ? __ldg(r0 + 8 * (c + 1) + 1) : z4;
-        c10 = ok1 ? __ldg(r1 + 8 * (c + 1)) : z4;
-        c11 = ok1 ? __ldg(r1 + 8 * (c + 1) + 1) : z4;
-      }
+    // rows g and g + 8, 64-column chunks in a 4-slot register ring, three chunks ahead
+    uint4 ring[4][4];
+    auto fetch = [&](uint4 (&dst)[4], int c) {
+      dst[0] = ok0 ? __ldg(r0 + 8 * c) : z4;
+      dst[1] = ok0 ? __ldg(r0 + 8 * c + 1) : z4;
+      dst[2] = ok1 ? __ldg(r1 + 8 * c) : z4;
+      dst[3] = ok1 ? __ldg(r1 + 8 * c + 1) : z4;
+    };
 #pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const uint32_t af[4] = {p0[2 * s], p1[2 * s], p0[2 * s + 1], p1[2 * s + 1]};
+    for (int u = 0; u < 3; ++u)
+      if (u < nch) fetch(ring[u], u);
+    for (int c0 = 0; c0 < nch; c0 += 4) {      // nch is a multiple of 4 (D % 256 == 0)
 #pragma unroll
-        for (int n = 0; n < NB; ++n) {
-          const uint2 bh = xh2[n * 8 * (XS / 2) + 16 * c + s];
-          const uint2 bl = xl2[n * 8 * (XS / 2) + 16 * c + s];
-          mma_f16_16816(acc[n], af, bh.x, bh.y);
-          mma_f16_16816(acc[n], af, bl.x, bl.y);
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u;
+        if (c + 3 < nch) fetch(ring[(u + 3) & 3], c + 3);
+        const uint4* cur = ring[u];
+        const uint32_t p0[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+        const uint32_t p1[8] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t af[4] = {p0[2 * s], p1[2 * s], p0[2 * s + 1], p1[2 * s + 1]};
+#pragma unroll
+          for (int n = 0; n < NB; ++n) {
+            const uint2 bh = xh2[n * 8 * (XS / 2) + 16 * c + s];
+            const uint2 bl = xl2[n * 8 * (XS / 2) + 16 * c + s];
+            mma_f16_16816(acc[n], af, bh.x, bh.y);
+            mma_f16_16816(acc[n], af, bl.x, bl.y);
+          }
         }
       }
     }

@@ -238,16 +238,6 @@ DFSSM_DEV void bulk_s2c(uint32_t dst, const void* src, unsigned bytes, uint32_t 
       "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :: "r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(bar) : "memory");
 }
-DFSSM_DEV uint32_t cluster_map(uint32_t saddr, unsigned rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-// Every thread of every CTA of the cluster.
-DFSSM_DEV void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // Named barrier 1 over the CTA's 16 warps.
 DFSSM_DEV void csync() { asm volatile("bar.sync 1, %0;" :: "n"(kPThreads) : "memory"); }
 DFSSM_DEV bool csync_and(bool v) {
