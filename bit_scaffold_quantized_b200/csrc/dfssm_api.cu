@@ -229,7 +229,9 @@ int launch_prologue(int K, int rank, int batch, const float* src, const uint16_t
 constexpr size_t kProjSmemCap = 200 * 1024;
 
 int pick_bt(int batch, int K, int rank) {
-  int bt = batch <= 1 ? 1 : batch <= 2 ? 2 : batch <= 4 ? 4 : 8;
+  // at most 4 batch rows per block: two blocks (32 warps) fit an SM, which hides
+  // more latency than the better A-fragment reuse of 8 rows (measured)
+  int bt = batch <= 1 ? 1 : batch <= 2 ? 2 : 4;
   while (bt > 1 && proj_smem_bytes(K, rank, bt) > kProjSmemCap) bt >>= 1;
   return bt;
 }
