@@ -277,8 +277,7 @@ int launch_proj(const ProjArgs& a, cudaStream_t st) {
   switch (pick_bt(a.batch, a.K, a.rank)) {
     case 1: return launch_proj_bt<EPI, 1>(a, st);
     case 2: return launch_proj_bt<EPI, 2>(a, st);
-    case 4: return launch_proj_bt<EPI, 4>(a, st);
-    default: return launch_proj_bt<EPI, 8>(a, st);
+    default: return launch_proj_bt<EPI, 4>(a, st);
   }
 }
 
