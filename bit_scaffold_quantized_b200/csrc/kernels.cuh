@@ -597,7 +597,7 @@ struct SsmArgs {
   float* g;              // fp32 [B][E]
   const double* dta;     // fp64 [B][H][2]: step size and decay (from the in_proj epilogue)
   int batch;
-  unsigned* status;      // bit 4096 set if a streamed copy did not land (k_ssm_stream)
+  unsigned* status;      // value 32768 is or-ed in if a streamed copy did not land (k_ssm_stream)
 };
 
 constexpr int kSsmThreads = 256;
@@ -768,7 +768,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
       while (!mbar_try_wait(&bar[buf], par))
         if (++spins > (1 << 22)) { ok = false; break; }
       s_ok = ok ? 1 : 0;
-      if (!ok) atomicOr(a.status, 4096u);
+      if (!ok) atomicOr(a.status, 32768u);
     }
     __syncthreads();
     if (!s_ok) {

@@ -122,7 +122,12 @@ typedef struct dfssm_layer_state {
  * the scaffold product is computed exactly from these planes. */
 typedef struct dfssm_ws_layout {
   size_t total_bytes;
-  size_t status;     /* uint32 status word: 0 ok; bit 1 = a token id was out of range (clamped) */
+  size_t status;     /* uint32 status word, 0 = ok.  Value 2: a token id was out of range
+                        (clamped).  Values 4 .. 16384: a bounded wait of the batch-1 token
+                        kernel gave up (each wait has its own value) and the call's outputs
+                        are invalid.  Value 32768: a streamed SSM-state copy did not land
+                        in time (multi-launch path); outputs invalid.  Bits are or-ed in and
+                        never cleared by the library. */
   size_t x_in;       /* fp16  [batch][d_model]    pre-norm output (in_proj activation) */
   size_t xq_in;      /* int8  [batch][d_model]    its int8 LoRA codes */
   size_t sx_in;      /* fp32  [batch]             their scales */
