@@ -205,8 +205,6 @@ Bufs bind(void* ws, const dfssm_ws_layout& L, const dfssm_dims* d) {
 
 // ---- launch helpers ---------------------------------------------------------
 
-static_assert(kPrologueThreads * kPrologueVals >= 8192, "the prologue holds K <= 8192 elements in registers");
-
 template <int MODE>
 int launch_prologue(int K, int rank, int batch, const float* src, const uint16_t* src16, const uint16_t* w,
                     const Act& o, const dfssm_proj* p, cudaStream_t st) {
@@ -214,15 +212,12 @@ int launch_prologue(int K, int rank, int batch, const float* src, const uint16_t
   a.K = K; a.rank = rank; a.src = src; a.src16 = src16; a.w = w;
   a.x = o.x; a.xq = o.xq; a.sx = o.sx; a.xd = o.xd; a.xdsum = o.xdsum;
   a.A = p->A; a.sA = p->sA; a.acc = o.acc; a.u = o.u;
-  if (K % (16 * kPrologueCQ) == 0 && K <= kPrologueCQ * kPrologueClThreads * kPrologueClVals &&
-      rank <= kPrologueMaxRank) {
-    k_prologue_cl<MODE><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a);
-    CHECK_LAUNCH("k_prologue_cl");
-    return DFSSM_OK;
-  }
-  dim3 grid(rank > 0 ? (rank + kPrologueRowsPerBlock - 1) / kPrologueRowsPerBlock : 1, batch);
-  k_prologue<MODE><<<grid, kPrologueThreads, size_t(K), st>>>(a);
-  CHECK_LAUNCH("k_prologue");
+  // the API limits (K a multiple of 256 and <= 8192, rank <= 128) are the kernel's
+  REQUIRE(K % (16 * kPrologueCQ) == 0 && K <= kPrologueCQ * kPrologueClThreads * kPrologueClVals &&
+              rank <= kPrologueMaxRank,
+          DFSSM_ERR_UNSUPPORTED_SHAPE, "prologue: K (%d) or rank (%d) out of range", K, rank);
+  k_prologue_cl<MODE><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a);
+  CHECK_LAUNCH("k_prologue_cl");
   return DFSSM_OK;
 }
 

@@ -1,6 +1,6 @@
 // DF-SSM decode-step kernels ("Density Field State Space Models", Section 3.2 Eq. 3,
 // Section 3.3, Section 4.1, Appendix B).  Layer path, one launch per stage:
-//   k_prologue  RMSNorm -> fp16 activation -> int8 codes -> LoRA stage 1 (A_q . x_q)
+//   k_prologue_cl  RMSNorm -> fp16 activation -> int8 codes -> LoRA stage 1 (A_q . x_q)
 //   k_proj      1-bit scaffold on int8 tensor cores (0/1 sign bytes x exact activation
 //               digit planes, exact integer accumulation) + LoRA stage 2 (fp64)
 //               + epilogue (store | residual add | conv1d shift-register step)
@@ -98,143 +98,6 @@ struct PrologueArgs {
   double* u;              // fp64 [B][rank] out
 };
 
-constexpr int kPrologueThreads = 512;
-constexpr int kPrologueRowsPerBlock = kPrologueThreads / 32;  // one LoRA row per warp
-constexpr int kPrologueVals = 16;                             // elements per thread: K <= 8192
-
-// grid (max(1, ceil(rank/16)), B).  Every block recomputes the activation of its
-// batch row (same arithmetic, same result); block 0 also writes the activation,
-// its int8 codes and its digit planes, and each warp computes one LoRA row.  A
-// thread holds its elements k = tid + 512 i in registers, so the block waits for
-// global memory once: the LoRA row's A bytes, the source and the norm weight are
-// all requested before any arithmetic.
-//   mode 0: x = fp16(src * (1/sqrt(mean(src^2) + eps)) * w), all in fp64
-//   mode 1: x = src16
-//   sx = max|x| / 127, xq = clamp(rint(x / sx), -127, 127) (fp32 decision)
-//   acc[j] = sum_k A[j,k] xq[k] (exact), u[j] = acc[j] * sA[j] * sx (fp64)
-template <int MODE>
-__global__ void __launch_bounds__(kPrologueThreads) k_prologue(PrologueArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int K = a.K;
-  int8_t* qs = reinterpret_cast<int8_t*>(smem);                // [K] codes
-  __shared__ double redd[32];
-  __shared__ float red[32];
-  __shared__ int red6[kPrologueRowsPerBlock][kDigits];
-  const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool writer = blockIdx.x == 0;
-
-  // this warp's LoRA row, 16 bytes per lane and step (K <= 32 * 16 * kAV in registers)
-  constexpr int kAV = 8;
-  const int j = blockIdx.x * kPrologueRowsPerBlock + warp;
-  const int nv = K / 16;
-  const uint4* Arow = reinterpret_cast<const uint4*>(a.A + size_t(j < a.rank ? j : 0) * K);
-  uint4 av[kAV];
-#pragma unroll
-  for (int m = 0; m < kAV; ++m)
-    av[m] = (j < a.rank && lane + 32 * m < nv) ? __ldg(Arow + lane + 32 * m) : make_uint4(0, 0, 0, 0);
-
-  uint32_t h[kPrologueVals];     // fp16 bits of x
-  float am = 0.f;
-  if (MODE == 0) {
-    const float* v = a.src + size_t(b) * K;
-    float vf[kPrologueVals];
-    uint16_t wh[kPrologueVals];
-#pragma unroll
-    for (int i = 0; i < kPrologueVals; ++i) {
-      const int k = tid + i * kPrologueThreads;
-      vf[i] = k < K ? v[k] : 0.f;
-      wh[i] = k < K ? a.w[k] : uint16_t(0);
-    }
-    double ss = 0.0;
-#pragma unroll
-    for (int i = 0; i < kPrologueVals; ++i) ss = fma(double(vf[i]), double(vf[i]), ss);
-    ss = block_sum_d(ss, redd);
-    const double rs = 1.0 / sqrt(ss / double(K) + kEpsD);
-    const float rs32 = float(rs);
-#pragma unroll
-    for (int i = 0; i < kPrologueVals; ++i) {
-      const int k = tid + i * kPrologueThreads;
-      h[i] = k < K ? norm_fp16(vf[i], rs, rs32, half_to_float_bits(wh[i])) : 0u;
-      am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
-      if (k < K && writer && a.x) a.x[size_t(b) * K + k] = uint16_t(h[i]);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < kPrologueVals; ++i) {
-      const int k = tid + i * kPrologueThreads;
-      h[i] = k < K ? a.src16[size_t(b) * K + k] : 0u;
-      am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
-    }
-  }
-  am = block_max(am, red);
-  const float sx = am > 0.f ? __fdiv_rn(am, 127.f) : 1.f;
-  const float rcp = __frcp_rn(sx);
-  int dsum[kDigits];
-#pragma unroll
-  for (int d = 0; d < kDigits; ++d) dsum[d] = 0;
-#pragma unroll
-  for (int i = 0; i < kPrologueVals; ++i) {
-    const int k = tid + i * kPrologueThreads;
-    if (k < K) {
-      const int8_t q = am > 0.f ? int8_t(quant_code_bits(half_to_float_bits(h[i]), sx, rcp)) : int8_t(0);
-      qs[k] = q;
-      if (writer) {
-        a.xq[size_t(b) * K + k] = q;
-        uint32_t lo, hi;
-        digits_of(h[i], &lo, &hi);
-        const uint32_t w6[kDigits] = {lo, lo >> 8, lo >> 16, lo >> 24, hi, hi >> 8};
-#pragma unroll
-        for (int d = 0; d < kDigits; ++d) {
-          const int8_t dg = int8_t(w6[d] & 0xffu);
-          a.xd[(size_t(b) * kDigits + d) * K + k] = dg;
-          dsum[d] += dg;
-        }
-      }
-    }
-  }
-  if (writer) {
-#pragma unroll
-    for (int d = 0; d < kDigits; ++d) {
-      const int t = __reduce_add_sync(0xffffffffu, dsum[d]);
-      if (lane == 0) red6[warp][d] = t;
-    }
-  }
-  __syncthreads();             // codes (and the warps' plane sums) complete
-  if (writer && tid < kDigits) {
-    int t = 0;
-    for (int w = 0; w < kPrologueRowsPerBlock; ++w) t += red6[w][tid];
-    a.xdsum[b * kDigits + tid] = t;
-    if (tid == 0) a.sx[b] = sx;
-  }
-
-  if (j < a.rank) {
-    const uint4* q16 = reinterpret_cast<const uint4*>(qs);
-    int acc = 0;
-#pragma unroll
-    for (int m = 0; m < kAV; ++m) {
-      if (lane + 32 * m < nv) {
-        const uint4 q = q16[lane + 32 * m];
-        acc = __dp4a(int(av[m].x), int(q.x), acc);
-        acc = __dp4a(int(av[m].y), int(q.y), acc);
-        acc = __dp4a(int(av[m].z), int(q.z), acc);
-        acc = __dp4a(int(av[m].w), int(q.w), acc);
-      }
-    }
-    for (int i = lane + 32 * kAV; i < nv; i += 32) {   // rows longer than the register window
-      const uint4 av2 = __ldg(Arow + i), q = q16[i];
-      acc = __dp4a(int(av2.x), int(q.x), acc);
-      acc = __dp4a(int(av2.y), int(q.y), acc);
-      acc = __dp4a(int(av2.z), int(q.z), acc);
-      acc = __dp4a(int(av2.w), int(q.w), acc);
-    }
-    acc = warp_sum_i(acc);
-    if (lane == 0) {
-      a.acc[size_t(b) * a.rank + j] = acc;
-      a.u[size_t(b) * a.rank + j] = (double(acc) * h2d(a.sA[j])) * double(sx);
-    }
-  }
-}
-
 // Cluster prologue: one cluster of kPrologueCQ CTAs per batch row (grid (CQ, B));
 // CTA rank q owns columns [q K/CQ, (q+1) K/CQ), at most 4 per thread.  The row's
 // sum of squares and max |x| are all-reduced through distributed shared memory
@@ -242,7 +105,11 @@ __global__ void __launch_bounds__(kPrologueThreads) k_prologue(PrologueArgs a) {
 // holds the same value); each CTA writes its columns' x, codes and digit planes;
 // the digit-plane sums and the LoRA stage-1 partials of its columns go to rank 0,
 // which adds them in rank order (exact) and writes xdsum, acc, u and sx.
-// Same arithmetic as k_prologue.
+// Arithmetic:
+//   mode 0: x = fp16(src * (1/sqrt(mean(src^2) + eps)) * w), all in fp64
+//   mode 1: x = src16
+//   sx = max|x| / 127, xq = clamp(rint(x / sx), -127, 127) (fp32 decision)
+//   acc[j] = sum_k A[j,k] xq[k] (exact), u[j] = acc[j] * sA[j] * sx (fp64)
 constexpr int kPrologueCQ = 4;
 constexpr int kPrologueClThreads = 512;  // two CTAs per SM (64 registers): a batch of 64 rows runs in one wave
 constexpr int kPrologueClVals = 4;      // K / CQ / 512 <= 4: K <= 8192

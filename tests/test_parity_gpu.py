@@ -223,6 +223,35 @@ def test_layer_step_batched_parity(batch):
         ost = O.State(tr.conv, tr.ssm)
 
 
+def test_layer_step_1p3b_batched_parity():
+    """The 1.3B layer at batch 3: cluster prologue at K = 2048 and 4096 with rank 32,
+    4-row projection tiles with a ragged batch tile, streaming SSM with N = 128."""
+    d, lw, st, xs = S.layer_workload("layer_d2048_b1_256steps", steps=2, batch=3)
+    run = LayerRun(d, lw, st)
+    ost = st
+    for t in range(2):
+        tr = _check_layer_step(run, lw, d, ost, xs[t])
+        ost = O.State(tr.conv, tr.ssm)
+
+
+@pytest.mark.parametrize("headdim,d_state,rank", [(64, 256, 8), (128, 128, 0)])
+def test_layer_step_large_state_items_parity(headdim, d_state, rank):
+    """(batch, head) state items too large for two shared-memory buffers take the
+    one-block-per-item SSM kernel (d_state 256 also takes its two-chunk form);
+    rank 0 runs the prologue without LoRA rows."""
+    d = S.Dims(batch=2, d_model=256, d_inner=512, nheads=512 // headdim, headdim=headdim, d_state=d_state,
+               rank=rank)
+    rng = np.random.default_rng(41 + headdim)
+    lw = S.gen_layer(rng, d)
+    st = S.zero_state(d)
+    xs = S.gen_layer_inputs(rng, d, 3)
+    run = LayerRun(d, lw, st)
+    ost = st
+    for t in range(3):
+        tr = _check_layer_step(run, lw, d, ost, xs[t])
+        ost = O.State(tr.conv, tr.ssm)
+
+
 def test_layer_dt_zero_leaves_ssm_state():
     d, lw, st, xs = S.layer_workload("layer_d256_b1_16steps", steps=2)
     lw.dt_bias[:] = -1e4
@@ -321,6 +350,15 @@ def test_model_decode_small_parity():
     rng = np.random.default_rng(30)
     m = S.gen_model(rng, d, 3, 1000)
     _teacher_forced(m, S.gen_tokens(rng, 2, 1000), 6)
+
+
+def test_model_decode_batched_tc_head_parity():
+    """Batch 12: the tensor-core LM head with 16 batch rows per block (a ragged second
+    n-tile) and a vocabulary whose last 16-row tile is half empty."""
+    d = S.LAYER_SMALL.with_batch(12)
+    rng = np.random.default_rng(34)
+    m = S.gen_model(rng, d, 3, 1000)
+    _teacher_forced(m, S.gen_tokens(rng, 12, 1000), 4)
 
 
 def test_model_decode_1p3b_parity():
