@@ -331,18 +331,41 @@ class ModelTrace:
     states: list             # [State] per layer, fp32
 
 
-def model_step(tokens: np.ndarray, m, states) -> ModelTrace:
+def quantize_embedding(embed16: np.ndarray):
+    """Per-row int8 quantisation of the tied embedding / LM-head matrix (Section 3.3:
+    the embedding is quantised to int8 per row; Table 1: embedding + LM head int8).
+    The pages do not give the quantiser; this reading uses the activations' symmetric
+    one: scale = max|row| / 127 and code = round-half-even(e / scale) clamped to
+    [-127, 127], both decided in fp32; an all-zero row gets codes 0 and scale 1.
+    Returns (int8 codes [V, D], fp32 scales [V])."""
+    return quantize_act(embed16)
+
+
+def model_step(tokens: np.ndarray, m, states, emb_q=None) -> ModelTrace:
     """One greedy decode token for the whole model: embedding gather, all layers,
     final RMSNorm, tied LM head (logits = E . norm(res)), argmax with the lowest
-    token id winning ties."""
+    token id winning ties.
+
+    emb_q = (codes, scales) from quantize_embedding selects the int8 embedding: the
+    gathered row is scale * code (an fp32 product) and logit v is
+    scale_v * sum_k code[v, k] * norm(res)[k]."""
     d = m.dims
-    res = m.embed[np.asarray(tokens, dtype=np.int64)].astype(np.float32)
+    tok = np.asarray(tokens, dtype=np.int64)
+    if emb_q is None:
+        res = m.embed[tok].astype(np.float32)
+    else:
+        q, sc = emb_q
+        res = (sc[tok].astype(np.float32)[:, None] * q[tok].astype(np.float32)).astype(np.float32)
     new_states = []
     for lw, st in zip(m.layers, states):
         t = layer_step(res, lw, st, d)
         res = t.res
         new_states.append(State(t.conv, t.ssm))
     xf = rmsnorm(res, m.normf_w)
-    logits = xf @ m.embed.astype(np.float64).T
+    if emb_q is None:
+        logits = xf @ m.embed.astype(np.float64).T
+    else:
+        q, sc = emb_q
+        logits = (xf @ q.astype(np.float64).T) * sc.astype(np.float64)[None, :]
     toks = np.argmax(logits, axis=-1).astype(np.int32)
     return ModelTrace(logits, toks, res, new_states)

@@ -456,6 +456,35 @@ def test_model_argmax_lowest_id_on_ties_and_embedding():
     assert tr.tokens.tolist() == [3, 3]
 
 
+def test_int8_embedding_rows_and_logits_brute_force():
+    """Section 3.3 int8 per-row embedding: the gathered row is scale * code in fp32,
+    and the logits of the tied head are scale_v * (codes . norm(res)); checked
+    element by element against a plain loop, plus the quantiser's bound and the
+    zero-row case."""
+    d = S.LAYER_SMALL.with_batch(2)
+    rng = np.random.default_rng(27)
+    m = S.gen_model(rng, d, 0, 24)
+    m.embed[5] = 0
+    q, sc = O.quantize_embedding(m.embed)
+    assert q.dtype == np.int8 and sc.dtype == np.float32 and sc[5] == 1.0 and np.all(q[5] == 0)
+    for v in (0, 9, 23):
+        e = m.embed[v].astype(np.float64)
+        i = int(np.argmax(np.abs(e)))
+        assert abs(int(q[v, i])) == 127
+        assert np.max(np.abs(e - q[v].astype(np.float64) * float(sc[v]))) <= 0.5 * float(sc[v]) * (1 + 1e-6)
+    toks = np.array([9, 5], dtype=np.int32)
+    tr = O.model_step(toks, m, [], emb_q=(q, sc))
+    for b, t in enumerate(toks):
+        for k in (0, 17, 255):
+            assert tr.res[b, k] == np.float32(np.float32(sc[t]) * np.float32(q[t, k]))
+    xf = O.rmsnorm(tr.res, m.normf_w)
+    for b in range(2):
+        for v in (0, 3, 23):
+            ref = float(sc[v]) * sum(float(q[v, k]) * xf[b, k] for k in range(d.d_model))
+            assert abs(tr.logits[b, v] - ref) <= 1e-12 * max(1.0, abs(ref))
+    assert tr.tokens.tolist() == np.argmax(tr.logits, axis=-1).tolist()
+
+
 # ---------------------------------------------------------------- byte model vs Table 1
 
 def test_table1_sizes_from_shapes():
