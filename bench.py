@@ -199,7 +199,7 @@ def run_ours(args, rank, world, local_rank):
     F.lib()
     m, tok0 = S.model_workload(args.workload)
     d = m.dims
-    dm = F.DeviceModel.from_host(m, device=dev)
+    dm = F.DeviceModel.from_host(m, device=dev, head=args.head)
     states = [F.DeviceState.zeros(d, device=dev) for _ in m.layers]
     call = F.ModelCall(dm, states)
     ws = F.workspace(d, len(m.layers), m.vocab, device=dev)
@@ -265,7 +265,7 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_kind = load_peaks()
     tokens = args.steps * d.batch * world
     tok_s = RP.job_tokens_per_s(args.steps, d.batch, world, ms)
-    bytes_tok = R.model_token_bytes(d, len(m.layers), m.vocab)
+    bytes_tok = R.model_token_bytes(d, len(m.layers), m.vocab, head=args.head)
     step_s = ms / 1e3 / args.steps
     achieved = bytes_tok / step_s / 1e9        # GB/s; one step = one token for every batch row
     peak = float(peaks["hbm_gbs"])
@@ -282,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "1-bit scaffold x fp16 act (fp32 acc), int8 LoRA (int32 acc), fp32 SSM state",
         "data": "synthetic (seeded random-init weights, random 1-token prompt)",
-        "config": {"workload": args.workload, "n_layer": len(m.layers), "d_model": d.d_model,
+        "config": {"workload": args.workload, "head": args.head, "n_layer": len(m.layers), "d_model": d.d_model,
                    "d_inner": d.d_inner, "nheads": d.nheads, "headdim": d.headdim, "d_state": d.d_state,
                    "rank": d.rank, "vocab": m.vocab, "batch": d.batch, "parallelism": f"replicas x{world}",
                    "cuda_graph": True,
@@ -421,6 +421,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=[k for k in S.WORKLOADS if k.startswith("model_")],
                     help="model decode workload (default: the batch-1 greedy decode)")
+    ap.add_argument("--head", choices=["fp16", "int8"], default="fp16",
+                    help="tied embedding / LM head precision (int8: per-row codes + fp32 scales)")
     ap.add_argument("--sweep", action="store_true", help="time the isolated projection sweep instead")
     ap.add_argument("--proj", type=int, nargs=4, metavar=("D_IN", "D_OUT", "RANK", "BATCH"),
                     help="call one projection sweep point three times (a target for profilers)")

@@ -113,6 +113,29 @@ DFSSM_DEV void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Four int8 values (little-endian in a word) as two fp16 pairs, exactly: each
+// byte x + 128 goes into the low mantissa byte of 1024.0 (fp16 0x6400 | u = 1024 + u)
+// and 1152 = 1024 + 128 is subtracted.  lo = (x0, x1), hi = (x2, x3).
+DFSSM_DEV void i8x4_to_half2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const __half2 off = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+  const uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);
+  const uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);
+  const __half2 ha = __hsub2(*reinterpret_cast<const __half2*>(&a), off);
+  const __half2 hb = __hsub2(*reinterpret_cast<const __half2*>(&b), off);
+  lo = *reinterpret_cast<const uint32_t*>(&ha);
+  hi = *reinterpret_cast<const uint32_t*>(&hb);
+}
+
+// Eight int8 values (little-endian in a uint2) as floats.
+DFSSM_DEV void i8x8_to_float(uint2 v, float (&f)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[i] = float(int8_t(v.x >> (8 * i)));
+    f[4 + i] = float(int8_t(v.y >> (8 * i)));
+  }
+}
+
 // D (s32 16x8) += A (u8 16x32, row) * B (s8 32x8, col).
 DFSSM_DEV void mma_u8s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(

@@ -290,14 +290,15 @@ ProjArgs proj_args(const dfssm_proj* p, int rank, int batch, const Act& act) {
 constexpr size_t kHeadTcSmemCap = 200 * 1024;
 size_t head_tc_smem(int D, int nb) { return size_t(2) * 8 * nb * (D + 4) * 2; }
 
-template <int NB>
+template <int NB, bool Q8>
 int launch_head_tc(const HeadArgs& h, cudaStream_t st, int* nparts) {
   const size_t smem = head_tc_smem(h.D, NB);
   static int occ_smem = -1, occ_blocks = 1;
   if (occ_smem != int(smem)) {
-    cudaFuncSetAttribute(k_lmhead_tc<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    cudaFuncSetAttribute(k_lmhead_tc<NB, Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_lmhead_tc<NB>, kHeadWarps * 32, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_lmhead_tc<NB, Q8>, kHeadWarps * 32, smem) !=
+            cudaSuccess ||
         nb < 1)
       nb = 1;
     occ_smem = int(smem);
@@ -307,23 +308,28 @@ int launch_head_tc(const HeadArgs& h, cudaStream_t st, int* nparts) {
   const int tiles = (h.vocab + 15) / 16;
   int gy = std::max(1, occ_blocks * sm_count() / gx);
   gy = std::min(gy, std::min(kHeadBlocks, (tiles + kHeadWarps - 1) / kHeadWarps));
-  k_lmhead_tc<NB><<<dim3(gx, gy), kHeadWarps * 32, smem, st>>>(h);
+  k_lmhead_tc<NB, Q8><<<dim3(gx, gy), kHeadWarps * 32, smem, st>>>(h);
   CHECK_LAUNCH("k_lmhead_tc");
   *nparts = gy;
   return DFSSM_OK;
 }
 
-int launch_head(const HeadArgs& h, cudaStream_t st, int* nparts) {
+template <bool Q8>
+int launch_head_q(const HeadArgs& h, cudaStream_t st, int* nparts) {
   if (h.D % 256 == 0) {
-    if (h.batch > 8 && head_tc_smem(h.D, 2) <= kHeadTcSmemCap) return launch_head_tc<2>(h, st, nparts);
-    if (head_tc_smem(h.D, 1) <= kHeadTcSmemCap) return launch_head_tc<1>(h, st, nparts);
+    if (h.batch > 8 && head_tc_smem(h.D, 2) <= kHeadTcSmemCap) return launch_head_tc<2, Q8>(h, st, nparts);
+    if (head_tc_smem(h.D, 1) <= kHeadTcSmemCap) return launch_head_tc<1, Q8>(h, st, nparts);
   }
   const size_t smem = size_t(4) * kHeadBatch * h.D;
-  cudaFuncSetAttribute(k_lmhead, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  k_lmhead<<<dim3(kHeadBlocks, (h.batch + kHeadBatch - 1) / kHeadBatch), kHeadWarps * 32, smem, st>>>(h);
+  cudaFuncSetAttribute(k_lmhead<Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  k_lmhead<Q8><<<dim3(kHeadBlocks, (h.batch + kHeadBatch - 1) / kHeadBatch), kHeadWarps * 32, smem, st>>>(h);
   CHECK_LAUNCH("k_lmhead");
   *nparts = kHeadBlocks;
   return DFSSM_OK;
+}
+
+int launch_head(const HeadArgs& h, cudaStream_t st, int* nparts) {
+  return h.embed_q ? launch_head_q<true>(h, st, nparts) : launch_head_q<false>(h, st, nparts);
 }
 
 // SSM update of the multi-launch path: the streaming kernel when an item's inputs
@@ -409,8 +415,9 @@ int device_sm_count(int* dev, int* nsm, int* smem_optin) {
 // Clusters of Q persistent CTAs that can be resident at once (cached per device,
 // cluster size and shared-memory size; the query is not a stream operation).
 using PKernel = void (*)(PParams);
-PKernel persistent_kernel(bool spec) {
-  return spec ? k_decode_persistent<Shape2048> : k_decode_persistent<ShapeAny>;
+PKernel persistent_kernel(bool spec, bool q8 = false) {
+  if (q8) return spec ? k_decode_persistent<Shape2048, true> : k_decode_persistent<ShapeAny, true>;
+  return spec ? k_decode_persistent<Shape2048, false> : k_decode_persistent<ShapeAny, false>;
 }
 
 int max_active_clusters(int dev, int Q, int smem, bool spec) {
@@ -498,8 +505,15 @@ PLayer player(const dfssm_layer_weights& w, const dfssm_layer_state& s) {
 }
 
 // Launch one token (model mode) or one layer step (layer mode) as the persistent kernel.
+// The tied embedding / LM-head matrix: fp16 rows, or int8 codes with fp32 row scales.
+struct EmbedRef {
+  const uint16_t* f16 = nullptr;
+  const int8_t* q = nullptr;
+  const float* s = nullptr;
+};
+
 int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int vocab,
-                      const dfssm_layer_weights* layers, const dfssm_layer_state* states, const uint16_t* embed,
+                      const dfssm_layer_weights* layers, const dfssm_layer_state* states, const EmbedRef& emb,
                       const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out, float* logits,
                       float* residual, void* ws, const dfssm_ws_layout& WL, int head_blocks, cudaStream_t st) {
   static_assert(sizeof(PParams) < 32000, "kernel parameter block too large");
@@ -515,7 +529,8 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.BSD = kDigits * (a.SD + 16) + 16; a.BSE = kDigits * (a.SE + 16) + 16;
   a.layer_mode = residual != nullptr;
   a.sm = plan.sm;
-  a.embed = embed; a.normf_w = normf_w; a.tok_in = tok_in; a.tok_out = tok_out; a.logits = logits;
+  a.embed = emb.f16; a.embed_q = emb.q; a.embed_s = emb.s;
+  a.normf_w = normf_w; a.tok_in = tok_in; a.tok_out = tok_out; a.logits = logits;
   a.residual = residual;
   unsigned char* scratch = at<unsigned char>(ws, WL.scratch);
   unsigned char* pbase = scratch + align256(size_t(8) * d->batch * std::max(head_blocks, 1));
@@ -533,7 +548,7 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.d_x_out = b.out.x; a.d_xq_out = b.out.xq; a.d_sx_out = b.out.sx; a.d_acc_out = b.out.acc;
   a.d_u_out = b.out.u; a.d_xd_out = b.out.xd; a.d_xdsum_out = b.out.xdsum; a.d_res = b.res;
   for (int l = 0; l < n_layer; ++l) a.L[l] = player(layers[l], states[l]);
-  const PKernel kfn = persistent_kernel(plan.spec);
+  const PKernel kfn = persistent_kernel(plan.spec, emb.q != nullptr);
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.sm.total);
   if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "persistent smem attribute: %s", cudaGetErrorString(e));
   // clusters of Q CTAs, all co-resident (cooperative): the CTAs wait on one another
@@ -687,7 +702,7 @@ int dfssm_layer_step(const dfssm_dims* d, const dfssm_layer_weights* w, const df
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const PPlan plan = plan_persistent(d);
   if (plan.ok) {
-    if ((rc = launch_persistent(plan, d, 1, 0, w, s, nullptr, nullptr, nullptr, nullptr, nullptr, residual, ws, L,
+    if ((rc = launch_persistent(plan, d, 1, 0, w, s, EmbedRef{}, nullptr, nullptr, nullptr, nullptr, residual, ws, L,
                                 0, st)))
       return rc;
   } else if ((rc = layer_multikernel(d, w, s, residual, b, st))) {
@@ -696,10 +711,13 @@ int dfssm_layer_step(const dfssm_dims* d, const dfssm_layer_weights* w, const df
   return ok();
 }
 
-int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16_t* embed,
-                       const dfssm_layer_weights* layers, const dfssm_layer_state* states,
-                       const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out, float* logits,
-                       void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int model_decode(const dfssm_dims* d, int n_layer, int vocab, const EmbedRef& emb,
+                 const dfssm_layer_weights* layers, const dfssm_layer_state* states, const uint16_t* normf_w,
+                 const int32_t* tok_in, int32_t* tok_out, float* logits, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_dims(d);
   if (rc) return rc;
   REQUIRE(n_layer >= 1 && n_layer <= kMaxLayers, DFSSM_ERR_INVALID_ARG, "n_layer (%d) must be in [1, %d]",
@@ -708,7 +726,12 @@ int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16
   REQUIRE(layers != nullptr && states != nullptr, DFSSM_ERR_INVALID_ARG, "layers/states NULL");
   for (int l = 0; l < n_layer; ++l)
     if ((rc = check_layer(d, &layers[l], &states[l], l))) return rc;
-  REQUIRE_PTR(embed);
+  if (emb.q) {
+    REQUIRE_PTR(emb.q);
+    REQUIRE_PTR(emb.s);
+  } else {
+    REQUIRE_PTR(emb.f16);
+  }
   REQUIRE_PTR(normf_w);
   REQUIRE_PTR(tok_in);
   REQUIRE_PTR(tok_out);
@@ -723,24 +746,63 @@ int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16
   const int B = d->batch, D = d->d_model;
   const PPlan plan = plan_persistent(d);
   if (plan.ok) {
-    if ((rc = launch_persistent(plan, d, n_layer, vocab, layers, states, embed, normf_w, tok_in, tok_out, logits,
+    if ((rc = launch_persistent(plan, d, n_layer, vocab, layers, states, emb, normf_w, tok_in, tok_out, logits,
                                 nullptr, ws, L, kHeadBlocks, st)))
       return rc;
     return ok();
   }
-  k_embed<<<B, 256, 0, st>>>(embed, tok_in, vocab, D, b.res, b.status);
+  k_embed<<<B, 256, 0, st>>>(emb.f16, emb.q, emb.s, tok_in, vocab, D, b.res, b.status);
   CHECK_LAUNCH("k_embed");
   for (int l = 0; l < n_layer; ++l)
     if ((rc = layer_multikernel(d, &layers[l], &states[l], b.res, b, st))) return rc;
   float* part_val = reinterpret_cast<float*>(b.scratch);
   int* part_idx = reinterpret_cast<int*>(b.scratch + size_t(4) * B * kHeadBlocks);
   HeadArgs h{};
-  h.D = D; h.vocab = vocab; h.batch = B; h.res = b.res; h.normf_w = normf_w; h.embed = embed;
+  h.D = D; h.vocab = vocab; h.batch = B; h.res = b.res; h.normf_w = normf_w;
+  h.embed = emb.f16; h.embed_q = emb.q; h.embed_s = emb.s;
   h.logits = logits; h.part_val = part_val; h.part_idx = part_idx;
   int nparts = kHeadBlocks;
   if ((rc = launch_head(h, st, &nparts))) return rc;
   k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, nparts, tok_out);
   CHECK_LAUNCH("k_argmax");
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, const uint16_t* embed,
+                       const dfssm_layer_weights* layers, const dfssm_layer_state* states,
+                       const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out, float* logits,
+                       void* ws, size_t ws_bytes, void* stream) {
+  EmbedRef e;
+  e.f16 = embed;
+  REQUIRE_PTR(embed);
+  return model_decode(d, n_layer, vocab, e, layers, states, normf_w, tok_in, tok_out, logits, ws, ws_bytes,
+                      stream);
+}
+
+int dfssm_model_decode_q8(const dfssm_dims* d, int n_layer, int vocab, const int8_t* embed_q,
+                          const float* embed_scale, const dfssm_layer_weights* layers,
+                          const dfssm_layer_state* states, const uint16_t* normf_w, const int32_t* tok_in,
+                          int32_t* tok_out, float* logits, void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE_PTR(embed_q);
+  REQUIRE_PTR(embed_scale);
+  EmbedRef e;
+  e.q = embed_q;
+  e.s = embed_scale;
+  return model_decode(d, n_layer, vocab, e, layers, states, normf_w, tok_in, tok_out, logits, ws, ws_bytes,
+                      stream);
+}
+
+int dfssm_quantize_rows_int8(const uint16_t* w, int rows, int cols, int8_t* q, float* scale, void* stream) {
+  REQUIRE(rows > 0 && cols > 0, DFSSM_ERR_INVALID_ARG, "rows/cols must be positive");
+  REQUIRE_PTR(w);
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(scale);
+  k_quant_rows<<<rows, 256, 0, static_cast<cudaStream_t>(stream)>>>(w, cols, q, scale);
+  CHECK_LAUNCH("k_quant_rows");
   return ok();
 }
 

@@ -707,7 +707,10 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
 
 // ------------------------------------------------------------------ embedding / LM head
 
-__global__ void k_embed(const uint16_t* __restrict__ embed, const int32_t* __restrict__ tok,
+// grid (B).  residual row b = embedding row tok[b]: fp16 as given, or int8 codes times
+// the row's fp32 scale (an fp32 product) when embed_q is not null.
+__global__ void k_embed(const uint16_t* __restrict__ embed, const int8_t* __restrict__ embed_q,
+                        const float* __restrict__ embed_s, const int32_t* __restrict__ tok,
                         int vocab, int D, float* __restrict__ res, unsigned* status) {
   const int b = blockIdx.x;
   int t = tok[b];
@@ -715,15 +718,40 @@ __global__ void k_embed(const uint16_t* __restrict__ embed, const int32_t* __res
     if (threadIdx.x == 0) atomicOr(status, 2u);
     t = t < 0 ? 0 : vocab - 1;
   }
-  for (int k = threadIdx.x; k < D; k += blockDim.x)
-    res[size_t(b) * D + k] = h2f(embed[size_t(t) * D + k]);
+  if (embed_q) {
+    const float sc = embed_s[t];
+    for (int k = threadIdx.x; k < D; k += blockDim.x)
+      res[size_t(b) * D + k] = sc * float(embed_q[size_t(t) * D + k]);
+  } else {
+    for (int k = threadIdx.x; k < D; k += blockDim.x)
+      res[size_t(b) * D + k] = h2f(embed[size_t(t) * D + k]);
+  }
+}
+
+// grid (rows), 256 threads.  Per-row int8 quantisation of an fp16 matrix: scale =
+// max|row| / 127 (fp32 divide; 1 for an all-zero row), code = round-half-even(w /
+// scale) clamped to [-127, 127], decided in fp32 (the activation quantiser's rule).
+__global__ void __launch_bounds__(256) k_quant_rows(const uint16_t* __restrict__ w, int cols,
+                                                    int8_t* __restrict__ q, float* __restrict__ scale) {
+  __shared__ float red[32];
+  const size_t r = blockIdx.x;
+  float am = 0.f;
+  for (int k = threadIdx.x; k < cols; k += blockDim.x) am = fmaxf(am, fabsf(h2f(w[r * cols + k])));
+  am = block_max(am, red);
+  const float sx = am > 0.f ? __fdiv_rn(am, 127.f) : 1.f;
+  const float rcp = __frcp_rn(sx);
+  for (int k = threadIdx.x; k < cols; k += blockDim.x)
+    q[r * cols + k] = am > 0.f ? int8_t(quant_code_bits(h2f(w[r * cols + k]), sx, rcp)) : int8_t(0);
+  if (threadIdx.x == 0) scale[r] = sx;
 }
 
 struct HeadArgs {
   int D, vocab, batch;
   const float* res;        // [B][D]
   const uint16_t* normf_w; // [D]
-  const uint16_t* embed;   // [V][D]
+  const uint16_t* embed;   // [V][D] fp16, or
+  const int8_t* embed_q;   // [V][D] int8 codes (when not null) with
+  const float* embed_s;    // [V] fp32 row scales
   float* logits;           // [B][V] or null
   float* part_val;         // [B][gridDim.x]
   int* part_idx;           // [B][gridDim.x]
@@ -740,6 +768,7 @@ DFSSM_DEV bool better(float v, int i, float bv, int bi) {
 // (fp64, kept as fp32), streams its share of LM-head rows (one warp per row,
 // 16-byte loads, fp32 accumulation) and keeps the best (logit, id) per batch row;
 // the lowest id wins ties.
+template <bool Q8>
 __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead(HeadArgs a) {
   extern __shared__ __align__(16) float xf[];   // [8][D]
   __shared__ double red[32];
@@ -765,19 +794,22 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead(HeadArgs a) {
   for (int bb = 0; bb < kHeadBatch; ++bb) { best[bb] = -INFINITY; besti[bb] = 0x7fffffff; }
   const int nwarps = gridDim.x * kHeadWarps;
   for (int v = blockIdx.x * kHeadWarps + warp; v < a.vocab; v += nwarps) {
-    const uint4* row = reinterpret_cast<const uint4*>(a.embed + size_t(v) * D);
     float s[kHeadBatch];
 #pragma unroll
     for (int bb = 0; bb < kHeadBatch; ++bb) s[bb] = 0.f;
     for (int c = lane; c < D / 8; c += 32) {
-      const uint4 w = __ldg(row + c);
-      const __half2* wh = reinterpret_cast<const __half2*>(&w);
       float wf[8];
+      if constexpr (Q8) {
+        i8x8_to_float(__ldg(reinterpret_cast<const uint2*>(a.embed_q + size_t(v) * D) + c), wf);
+      } else {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(a.embed + size_t(v) * D) + c);
+        const __half2* wh = reinterpret_cast<const __half2*>(&w);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(wh[i]);
-        wf[2 * i] = f.x;
-        wf[2 * i + 1] = f.y;
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(wh[i]);
+          wf[2 * i] = f.x;
+          wf[2 * i + 1] = f.y;
+        }
       }
 #pragma unroll
       for (int bb = 0; bb < kHeadBatch; ++bb) {
@@ -796,7 +828,7 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead(HeadArgs a) {
 #pragma unroll
     for (int bb = 0; bb < kHeadBatch; ++bb) {
       if (bb < nb) {
-        const float l = warp_sum(s[bb]);
+        const float l = Q8 ? warp_sum(s[bb]) * a.embed_s[v] : warp_sum(s[bb]);
         if (a.logits && lane == 0) a.logits[size_t(b0 + bb) * a.vocab + v] = l;
         if (better(l, v, best[bb], besti[bb])) { best[bb] = l; besti[bb] = v; }
       }
@@ -828,7 +860,7 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead(HeadArgs a) {
 // and part.  The MMA's k index i maps to column 64 c + 16 t + 4 s + (i & 1) + 2 (i >> 3)
 // for A and B alike, so the chunk's 64 columns are each summed once.  Per batch row
 // the block keeps the best (logit, id), lowest id on ties.
-template <int NB>
+template <int NB, bool Q8>
 __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
   extern __shared__ __align__(16) uint32_t xsw[];         // [2][8 NB][XS] words: hi rows, then lo rows
   __shared__ float wbest[kHeadWarps][8 * NB];
@@ -868,19 +900,24 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
   const uint4 z4 = make_uint4(0, 0, 0, 0);
   for (int tile = blockIdx.y * kHeadWarps + warp; tile < ntiles; tile += gridDim.y * kHeadWarps) {
     const int v0 = tile * 16 + g, v1 = v0 + 8;
-    const uint4* r0 = reinterpret_cast<const uint4*>(a.embed + size_t(min(v0, a.vocab - 1)) * D) + 2 * t;
-    const uint4* r1 = reinterpret_cast<const uint4*>(a.embed + size_t(min(v1, a.vocab - 1)) * D) + 2 * t;
+    // fp16 rows: 2 x 16 bytes per 64-column chunk and lane; int8 rows: 16 bytes
+    constexpr int kLV = Q8 ? 1 : 2;
+    const uint4* r0 = Q8 ? reinterpret_cast<const uint4*>(a.embed_q + size_t(min(v0, a.vocab - 1)) * D) + t
+                         : reinterpret_cast<const uint4*>(a.embed + size_t(min(v0, a.vocab - 1)) * D) + 2 * t;
+    const uint4* r1 = Q8 ? reinterpret_cast<const uint4*>(a.embed_q + size_t(min(v1, a.vocab - 1)) * D) + t
+                         : reinterpret_cast<const uint4*>(a.embed + size_t(min(v1, a.vocab - 1)) * D) + 2 * t;
     const bool ok0 = v0 < a.vocab, ok1 = v1 < a.vocab;
     float acc[NB][4];
 #pragma unroll
     for (int n = 0; n < NB; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
     // rows g and g + 8, 64-column chunks in a 4-slot register ring, three chunks ahead
-    uint4 ring[4][4];
-    auto fetch = [&](uint4 (&dst)[4], int c) {
-      dst[0] = ok0 ? __ldg(r0 + 8 * c) : z4;
-      dst[1] = ok0 ? __ldg(r0 + 8 * c + 1) : z4;
-      dst[2] = ok1 ? __ldg(r1 + 8 * c) : z4;
-      dst[3] = ok1 ? __ldg(r1 + 8 * c + 1) : z4;
+    uint4 ring[4][2 * kLV];
+    auto fetch = [&](uint4 (&dst)[2 * kLV], int c) {
+#pragma unroll
+      for (int i = 0; i < kLV; ++i) {
+        dst[i] = ok0 ? __ldg(r0 + 4 * kLV * c + i) : z4;
+        dst[kLV + i] = ok1 ? __ldg(r1 + 4 * kLV * c + i) : z4;
+      }
     };
 #pragma unroll
     for (int u = 0; u < 3; ++u)
@@ -891,8 +928,24 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
         const int c = c0 + u;
         if (c + 3 < nch) fetch(ring[(u + 3) & 3], c + 3);
         const uint4* cur = ring[u];
-        const uint32_t p0[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
-        const uint32_t p1[8] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
+        uint32_t p0[8], p1[8];
+        if constexpr (Q8) {   // 16 int8 columns per row -> 8 exact fp16 pairs
+          const uint32_t w0[4] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w};
+          const uint32_t w1[4] = {cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            i8x4_to_half2x2(w0[i], p0[2 * i], p0[2 * i + 1]);
+            i8x4_to_half2x2(w1[i], p1[2 * i], p1[2 * i + 1]);
+          }
+        } else {              // rows g and g + 8: two 16-byte vectors each
+          const uint32_t q0[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+          const uint32_t q1[8] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            p0[i] = q0[i];
+            p1[i] = q1[i];
+          }
+        }
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           const uint32_t af[4] = {p0[2 * s], p1[2 * s], p0[2 * s + 1], p1[2 * s + 1]};
@@ -904,6 +957,16 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
             mma_f16_16816(acc[n], af, bl.x, bl.y);
           }
         }
+      }
+    }
+    if constexpr (Q8) {      // logit = row scale * (codes . x)
+      const float s0 = ok0 ? a.embed_s[v0] : 0.f, s1 = ok1 ? a.embed_s[v1] : 0.f;
+#pragma unroll
+      for (int n = 0; n < NB; ++n) {
+        acc[n][0] *= s0;
+        acc[n][1] *= s0;
+        acc[n][2] *= s1;
+        acc[n][3] *= s1;
       }
     }
 #pragma unroll

@@ -113,6 +113,8 @@ struct __align__(16) PParams {
   PSmem sm;
   // io
   const uint16_t* embed; const uint16_t* normf_w; const int32_t* tok_in; int32_t* tok_out; float* logits;
+  const int8_t* embed_q;         // int8 per-row embedding (replaces embed when not null)
+  const float* embed_s;          // its fp32 row scales
   float* residual;               // layer mode: [D] in/out
   // workspace
   unsigned* status;              // status word
@@ -814,7 +816,7 @@ DFSSM_DEV double tile_row_value(const int* part, int ti, int nchunk, int r, long
 
 // ------------------------------------------------------------------ the kernel
 
-template <class SH>
+template <class SH, bool Q8>
 __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_constant__ PParams pa) {
   extern __shared__ __align__(128) unsigned char sm[];
   // The parameter block (~11 KB, mostly the per-layer pointer table) is read with
@@ -855,13 +857,18 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.grid;
   const int v0 = int((long long)w.c * a.vocab / G), v1 = int((long long)(w.c + 1) * a.vocab / G);
-  const int head_chunks = (v1 - v0 + kHeadChunkRows - 1) / kHeadChunkRows;
-  const unsigned head_row_bytes = 2u * D;
+  // LM-head rows: fp16, or (Q8) int8 codes with a per-row scale.  Slots are spaced for
+  // 7 fp16 rows, which is 14 int8 rows: an int8 chunk is 14 rows (half the chunks).
+  // A compile-time choice keeps the fp16 kernel's registers as they were.
+  constexpr bool q8 = Q8;
+  constexpr int CR = Q8 ? 2 * kHeadChunkRows : kHeadChunkRows;
+  const unsigned head_row_bytes = q8 ? unsigned(D) : 2u * D;
+  const int head_chunks = (v1 - v0 + CR - 1) / CR;
 
   // LM-head chunk slots tile the shared memory below `ring_end`; the slots inside
   // the AB group are free after the last layer's SSM, the others after its out_proj
   const int NH = PSM(head_slots);
-  const int chunk_bytes = kHeadChunkRows * int(head_row_bytes);
+  const int chunk_bytes = kHeadChunkRows * 2 * D;
   auto head_slot = [&](int b) { return sm + b * chunk_bytes; };
   if (warp == kPWarps) {
     // ============================================================== copy warp
@@ -874,10 +881,12 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
     };
     auto issue_head = [&](int ci) {
       const int b = ci % NH;
-      const int r0 = v0 + ci * kHeadChunkRows, nr = min(kHeadChunkRows, v1 - r0);
+      const int r0 = v0 + ci * CR, nr = min(CR, v1 - r0);
       if (lane == 0) {
         mbar_expect_tx(full_h + b, nr * head_row_bytes);
-        bulk_g2s(head_slot(b), a.embed + size_t(r0) * D, nr * head_row_bytes, full_h + b);
+        const void* src = q8 ? static_cast<const void*>(a.embed_q + size_t(r0) * D)
+                             : static_cast<const void*>(a.embed + size_t(r0) * D);
+        bulk_g2s(head_slot(b), src, nr * head_row_bytes, full_h + b);
       }
       ++h_issued[b];
     };
@@ -951,7 +960,11 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         }
       }
       const uint16_t* erow = a.embed + size_t(t) * D;
-      auto res0 = [&](int k) { return a.layer_mode ? a.residual[k] : h2f(erow[k]); };
+      const int8_t* eqrow = q8 ? a.embed_q + size_t(t) * D : nullptr;
+      const float es = q8 ? a.embed_s[t] : 0.f;
+      auto res0 = [&](int k) {
+        return a.layer_mode ? a.residual[k] : q8 ? es * float(eqrow[k]) : h2f(erow[k]);
+      };
       double acc = 0.0;
       for (int k = tid; k < D; k += kPThreads) {
         const double v = double(res0(k));
@@ -1221,7 +1234,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         csync();
         float best = -INFINITY;
         int besti = 0x7fffffff;
-        float* hsum = sp<float>(sm, PSM(part));     // [2][kHeadChunkRows][2]
+        float* hsum = sp<float>(sm, PSM(part));     // [2][CR][2]
         // warp 2 r + h takes half h of row r of every chunk; its lanes keep their
         // columns of the normalised residual in registers (kHV 8-column groups each)
         constexpr int kHV = 4;
@@ -1235,47 +1248,60 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         for (int ci = 0; ci < head_chunks && alive; ++ci) {
           const int b = ci % NH;
           if (!mbar_wait_compute(status, ctl, full_h + b, unsigned(ci / NH) & 1u, 1024u)) { alive = false; break; }
-          const int r0 = v0 + ci * kHeadChunkRows, nr = min(kHeadChunkRows, v1 - r0);
-          float* hs = hsum + (ci & 1) * 2 * kHeadChunkRows;
-          if (hrow < nr) {
-            const uint4* wr = reinterpret_cast<const uint4*>(head_slot(b) + size_t(hrow) * head_row_bytes) + hb;
+          const int r0 = v0 + ci * CR, nr = min(CR, v1 - r0);
+          float* hs = hsum + (ci & 1) * 2 * CR;
+#pragma unroll
+          for (int rsub = 0; rsub < CR / kHeadChunkRows; ++rsub) {
+          const int row = hrow + kHeadChunkRows * rsub;
+          if (row < nr) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            auto acc8 = [&](const float (&f)[8], const float* x) {
+              acc[0] = fmaf(f[0], x[0], acc[0]); acc[1] = fmaf(f[1], x[1], acc[1]);
+              acc[2] = fmaf(f[2], x[2], acc[2]); acc[3] = fmaf(f[3], x[3], acc[3]);
+              acc[0] = fmaf(f[4], x[4], acc[0]); acc[1] = fmaf(f[5], x[5], acc[1]);
+              acc[2] = fmaf(f[6], x[6], acc[2]); acc[3] = fmaf(f[7], x[7], acc[3]);
+            };
+            auto f16x8 = [](const uint4& wv, float (&f)[8]) {
+              const __half2* wh = reinterpret_cast<const __half2*>(&wv);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 t2 = __half22float2(wh[i]);
+                f[2 * i] = t2.x;
+                f[2 * i + 1] = t2.y;
+              }
+            };
+            const unsigned char* wrow = head_slot(b) + size_t(row) * head_row_bytes;
 #pragma unroll
             for (int m = 0; m < kHV; ++m) {
               if (lane + 32 * m < hn) {
-                const uint4 wv = wr[lane + 32 * m];
-                const __half2* wh = reinterpret_cast<const __half2*>(&wv);
-                float2 f;
-                f = __half22float2(wh[0]); acc[0] = fmaf(f.x, xr[m][0], acc[0]); acc[1] = fmaf(f.y, xr[m][1], acc[1]);
-                f = __half22float2(wh[1]); acc[2] = fmaf(f.x, xr[m][2], acc[2]); acc[3] = fmaf(f.y, xr[m][3], acc[3]);
-                f = __half22float2(wh[2]); acc[0] = fmaf(f.x, xr[m][4], acc[0]); acc[1] = fmaf(f.y, xr[m][5], acc[1]);
-                f = __half22float2(wh[3]); acc[2] = fmaf(f.x, xr[m][6], acc[2]); acc[3] = fmaf(f.y, xr[m][7], acc[3]);
+                float f[8];
+                if (q8) i8x8_to_float(reinterpret_cast<const uint2*>(wrow)[hb + lane + 32 * m], f);
+                else f16x8(reinterpret_cast<const uint4*>(wrow)[hb + lane + 32 * m], f);
+                acc8(f, xr[m]);
               }
             }
             for (int c = lane + 32 * kHV; c < hn; c += 32) {   // half rows wider than kHV groups per lane
-              const uint4 wv = wr[c];
-              const __half2* wh = reinterpret_cast<const __half2*>(&wv);
-              const float* xc = xn + (hb + c) * 8;
-              float2 f;
-              f = __half22float2(wh[0]); acc[0] = fmaf(f.x, xc[0], acc[0]); acc[1] = fmaf(f.y, xc[1], acc[1]);
-              f = __half22float2(wh[1]); acc[2] = fmaf(f.x, xc[2], acc[2]); acc[3] = fmaf(f.y, xc[3], acc[3]);
-              f = __half22float2(wh[2]); acc[0] = fmaf(f.x, xc[4], acc[0]); acc[1] = fmaf(f.y, xc[5], acc[1]);
-              f = __half22float2(wh[3]); acc[2] = fmaf(f.x, xc[6], acc[2]); acc[3] = fmaf(f.y, xc[7], acc[3]);
+              float f[8];
+              if (q8) i8x8_to_float(reinterpret_cast<const uint2*>(wrow)[hb + c], f);
+              else f16x8(reinterpret_cast<const uint4*>(wrow)[hb + c], f);
+              acc8(f, xn + (hb + c) * 8);
             }
             const float v = warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
-            if (lane == 0) hs[hrow * 2 + hhalf] = v;
+            if (lane == 0) hs[row * 2 + hhalf] = v;
+          }
           }
           csync();
           if (tid == 0) mbar_arrive(empty_h + b);      // the slot may be refilled
           if (tid < nr) {
-            const float lg = hs[tid * 2] + hs[tid * 2 + 1];
+            float lg = hs[tid * 2] + hs[tid * 2 + 1];
+            if (q8) lg *= a.embed_s[r0 + tid];
             if (a.logits) a.logits[r0 + tid] = lg;
             if (lg > best || (lg == best && r0 + tid < besti)) { best = lg; besti = r0 + tid; }
           }
         }
         csync();
         // best over the threads that held rows
-        if (tid < kHeadChunkRows) {
+        if (tid < CR) {
           scratch32[2 * tid] = __float_as_uint(best);
           scratch32[2 * tid + 1] = uint32_t(besti);
         }
@@ -1283,7 +1309,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         if (tid == 0) {
           float bv = -INFINITY;
           int bi = 0x7fffffff;
-          for (int i = 0; i < kHeadChunkRows; ++i) {
+          for (int i = 0; i < CR; ++i) {
             const float v = __uint_as_float(scratch32[2 * i]);
             const int id = int(scratch32[2 * i + 1]);
             if (v > bv || (v == bv && id < bi)) { bv = v; bi = id; }

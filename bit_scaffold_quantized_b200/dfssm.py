@@ -32,6 +32,7 @@ EXPORTS = [
     "dfssm_proj_workspace_layout",
     "dfssm_workspace_bytes", "dfssm_workspace_layout", "dfssm_layer_step",
     "dfssm_model_decode", "dfssm_model_decode_launches", "dfssm_last_error", "dfssm_version",
+    "dfssm_model_decode_q8", "dfssm_quantize_rows_int8",
 ]
 
 
@@ -98,6 +99,9 @@ def lib() -> C.CDLL:
     L.dfssm_model_decode.argtypes = [C.POINTER(CDims), i, i, vp, C.POINTER(CLayerWeights),
                                      C.POINTER(CLayerState), vp, vp, vp, vp, vp, sz, vp]
     L.dfssm_model_decode_launches.argtypes = [C.POINTER(CDims), i, i]
+    L.dfssm_model_decode_q8.argtypes = [C.POINTER(CDims), i, i, vp, vp, C.POINTER(CLayerWeights),
+                                        C.POINTER(CLayerState), vp, vp, vp, vp, vp, sz, vp]
+    L.dfssm_quantize_rows_int8.argtypes = [vp, i, i, vp, vp, vp]
     L.dfssm_last_error.restype = C.c_char_p
     L.dfssm_version.restype = C.c_int
     for name in EXPORTS:
@@ -217,17 +221,36 @@ class DeviceState:
 class DeviceModel:
     dims: object
     vocab: int
-    embed: object
+    embed: object                  # fp16 [vocab][d_model]
     normf_w: object
     layers: List[DeviceLayer]
+    embed_q: object = None         # head="int8": int8 codes [vocab][d_model] ...
+    embed_scale: object = None     # ... and fp32 row scales [vocab]
 
     @classmethod
-    def from_host(cls, m, device="cuda", stream=None) -> "DeviceModel":
-        return cls(m.dims, m.vocab, _dev(m.embed, device), _dev(m.normf_w, device),
-                   [DeviceLayer.from_host(lw, device, stream) for lw in m.layers])
+    def from_host(cls, m, device="cuda", stream=None, head: str = "fp16") -> "DeviceModel":
+        """head="int8" quantises the tied embedding per row on the device
+        (dfssm_quantize_rows_int8) and decodes through dfssm_model_decode_q8."""
+        if head not in ("fp16", "int8"):
+            raise ValueError("head must be 'fp16' or 'int8'")
+        dm = cls(m.dims, m.vocab, _dev(m.embed, device), _dev(m.normf_w, device),
+                 [DeviceLayer.from_host(lw, device, stream) for lw in m.layers])
+        if head == "int8":
+            dm.embed_q, dm.embed_scale = quantize_rows_int8(dm.embed, stream)
+        return dm
 
 
 # ------------------------------------------------------------------ entry points
+
+def quantize_rows_int8(w16, stream=None):
+    """Per-row int8 codes and fp32 scales of a device fp16 matrix (dfssm_quantize_rows_int8)."""
+    import torch
+    rows, cols = w16.shape
+    q = torch.empty((rows, cols), dtype=torch.int8, device=w16.device)
+    sc = torch.empty((rows,), dtype=torch.float32, device=w16.device)
+    _check(lib().dfssm_quantize_rows_int8(_ptr(w16), rows, cols, _ptr(q), _ptr(sc), _stream(stream)))
+    return q, sc
+
 
 def packed_words(rows: int, cols: int, layout: int) -> int:
     return int(lib().dfssm_packed_words(rows, cols, layout))
@@ -299,6 +322,12 @@ class ModelCall:
 
     def __call__(self, tok_in, tok_out, ws, logits=None, stream=None) -> None:
         m = self.m
+        if m.embed_q is not None:
+            _check(lib().dfssm_model_decode_q8(C.byref(self.cd), len(m.layers), m.vocab, _ptr(m.embed_q),
+                                               _ptr(m.embed_scale), self.cw, self.cs, _ptr(m.normf_w),
+                                               _ptr(tok_in), _ptr(tok_out), _ptr(logits), _ptr(ws), ws.numel(),
+                                               _stream(stream)))
+            return
         _check(lib().dfssm_model_decode(C.byref(self.cd), len(m.layers), m.vocab, _ptr(m.embed), self.cw,
                                         self.cs, _ptr(m.normf_w), _ptr(tok_in), _ptr(tok_out), _ptr(logits),
                                         _ptr(ws), ws.numel(), _stream(stream)))

@@ -40,13 +40,17 @@ def layer_step_bytes(d: Dims) -> int:
     return layer_weight_bytes(d) + layer_state_bytes(d) + 2 * 4 * d.batch * d.d_model
 
 
-def model_token_bytes(d: Dims, n_layer: int, vocab: int) -> int:
+def model_token_bytes(d: Dims, n_layer: int, vocab: int, head: str = "fp16") -> int:
     """One greedy token for all batch rows: embedding rows, all layers, final norm,
-    fp16 tied LM head, token ids in and out."""
-    return (d.batch * 2 * d.d_model
+    tied LM head (fp16, or int8 codes + an fp32 scale per row), token ids in and out."""
+    if head == "int8":
+        emb_row, head_bytes = d.d_model + 4, vocab * (d.d_model + 4)
+    else:
+        emb_row, head_bytes = 2 * d.d_model, 2 * vocab * d.d_model
+    return (d.batch * emb_row
             + n_layer * (layer_weight_bytes(d) + layer_state_bytes(d))
             + 2 * d.d_model
-            + 2 * vocab * d.d_model
+            + head_bytes
             + 2 * 4 * d.batch)
 
 

@@ -222,6 +222,27 @@ DFSSM_API int dfssm_model_decode(const dfssm_dims* d, int n_layer, int vocab, co
                        const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out,
                        float* logits, void* ws, size_t ws_bytes, void* stream);
 
+/* dfssm_model_decode with the int8 per-row embedding / tied LM head ("Density Field
+ * State Space Models", Section 3.3: the embedding is quantised to int8 per row;
+ * Table 1: embedding + LM head int8).  embed_q int8 [vocab][d_model] and embed_scale
+ * fp32 [vocab] (device, 16-byte aligned; from dfssm_quantize_rows_int8 or any
+ * per-row quantiser).  The gathered row is embed_scale[t] * embed_q[t] (an fp32
+ * product); logit v = embed_scale[v] * (embed_q[v] . xf), fp32 accumulation.
+ * Everything else as dfssm_model_decode, same workspace. */
+DFSSM_API int dfssm_model_decode_q8(const dfssm_dims* d, int n_layer, int vocab, const int8_t* embed_q,
+                                    const float* embed_scale, const dfssm_layer_weights* layers,
+                                    const dfssm_layer_state* states, const uint16_t* normf_w,
+                                    const int32_t* tok_in, int32_t* tok_out, float* logits, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* Per-row int8 quantisation of a dense fp16 matrix w [rows][cols] (device):
+ * scale[r] = max_k |w[r][k]| / 127 (an fp32 divide; 1 for an all-zero row) and
+ * q[r][k] = round-half-even(w[r][k] / scale[r]) clamped to [-127, 127], the
+ * decision taken in fp32.  q int8 [rows][cols], scale fp32 [rows], caller-owned,
+ * 16-byte aligned.  Not on the timed path (done once when a model is loaded). */
+DFSSM_API int dfssm_quantize_rows_int8(const uint16_t* w, int rows, int cols, int8_t* q, float* scale,
+                                       void* stream);
+
 /* Number of kernel launches one dfssm_model_decode call enqueues for these
  * arguments (0 if they are invalid). */
 DFSSM_API int dfssm_model_decode_launches(const dfssm_dims* d, int n_layer, int vocab);

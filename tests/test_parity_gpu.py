@@ -303,9 +303,15 @@ def test_state_checkpoint_resume_bit_identical():
 
 # ---------------------------------------------------------------- model decode
 
-def _teacher_forced(m, tok0, steps, n_check_tokens=True):
+def _teacher_forced(m, tok0, steps, n_check_tokens=True, head="fp16"):
     d = m.dims
-    dm = F.DeviceModel.from_host(m)
+    dm = F.DeviceModel.from_host(m, head=head)
+    emb_q = None
+    if head == "int8":
+        emb_q = O.quantize_embedding(m.embed)
+        # the device quantiser takes the oracle's integer decisions
+        assert np.array_equal(to_np(dm.embed_q), emb_q[0])
+        assert np.array_equal(to_np(dm.embed_scale), emb_q[1])
     states = [F.DeviceState.zeros(d) for _ in m.layers]
     call = F.ModelCall(dm, states)
     ws = F.workspace(d, len(m.layers), m.vocab)
@@ -321,7 +327,7 @@ def _teacher_forced(m, tok0, steps, n_check_tokens=True):
         call(tok_in, tok_out, ws, logits)
         _sync()
         assert int(to_np(F.ws_view(ws, L.status, torch.int32, (1,)))[0]) == 0
-        tr = O.model_step(tok, m, ost)
+        tr = O.model_step(tok, m, ost, emb_q=emb_q)
         e = rel_err(to_np(logits), tr.logits)
         assert e <= TOL, (t, e)
         for l in (0, len(m.layers) - 1):
@@ -359,6 +365,43 @@ def test_model_decode_batched_tc_head_parity():
     rng = np.random.default_rng(34)
     m = S.gen_model(rng, d, 3, 1000)
     _teacher_forced(m, S.gen_tokens(rng, 12, 1000), 4)
+
+
+def test_quantize_rows_int8_bit_exact():
+    """Per-row int8 quantiser (Section 3.3) against the oracle: zero row, exact
+    half-way codes, the largest fp16, subnormals, and random rows."""
+    rng = np.random.default_rng(35)
+    w = rng.normal(0.0, 0.02, size=(37, 512)).astype(np.float16)
+    w[3] = 0
+    w[4, :4] = [127.0, 2.5, -3.5, 0.5]          # scale 1: codes 127, 2, -4, 0 (half-even)
+    w[4, 4:] = 0
+    w[5, 0], w[5, 1] = np.float16(65504.0), np.float16(-65504.0)
+    w[6] = np.float16(2.0 ** -24) * rng.integers(-3, 4, size=512)
+    q, sc = F.quantize_rows_int8(torch.from_numpy(w).to(DEV))
+    _sync()
+    rq, rs = O.quantize_embedding(w)
+    assert np.array_equal(to_np(q), rq)
+    assert np.array_equal(to_np(sc), rs)
+    assert to_np(q)[4, :4].tolist() == [127, 2, -4, 0]
+
+
+@pytest.mark.parametrize("case", ["persistent_b1", "multi_b2", "multi_b12"])
+def test_model_decode_int8_head_parity(case):
+    """The int8 per-row embedding / tied LM head on both paths and all head kernels."""
+    rng = np.random.default_rng(36)
+    if case == "persistent_b1":
+        d = LAYER_SMALL_P
+    else:
+        d = S.LAYER_SMALL.with_batch(2 if case == "multi_b2" else 12)
+    m = S.gen_model(rng, d, 3, 1000)
+    assert (F.launches_per_decode_step(d, 3, 1000) == 1) == (case == "persistent_b1")
+    _teacher_forced(m, S.gen_tokens(rng, d.batch, 1000), 4, head="int8")
+
+
+def test_model_decode_1p3b_int8_head_parity():
+    m, tok = S.model_workload("model_48x2048_v50280_b1_greedy512")
+    assert F.launches_per_decode_step(m.dims, len(m.layers), m.vocab) == 1
+    _teacher_forced(m, tok, 2, head="int8")
 
 
 def test_model_decode_1p3b_parity():
