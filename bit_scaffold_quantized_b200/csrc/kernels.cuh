@@ -1,11 +1,16 @@
 // DF-SSM decode-step kernels ("Density Field State Space Models", Section 3.2 Eq. 3,
-// Section 3.3, Section 4.1, Appendix B).  Layer path, one launch per stage:
-//   k_prologue_cl  RMSNorm -> fp16 activation -> int8 codes -> LoRA stage 1 (A_q . x_q)
-//   k_proj      1-bit scaffold on int8 tensor cores (0/1 sign bytes x exact activation
-//               digit planes, exact integer accumulation) + LoRA stage 2 (fp64)
-//               + epilogue (store | residual add | conv1d shift-register step)
-//   k_ssm       selective-SSM state update + D skip + gate y * silu(z)
-//   k_lmhead    final RMSNorm + tied fp16 LM head + per-block argmax; k_argmax finishes it
+// Section 3.3, Section 4.1, Appendix B), multi-launch path (any batch), one launch
+// per stage:
+//   k_prologue_cl   RMSNorm -> fp16 activation -> int8 codes, digit planes -> LoRA
+//                   stage 1 (A_q . x_q); one cluster of 4 CTAs per batch row
+//   k_proj          1-bit scaffold on int8 tensor cores (0/1 sign bytes x exact
+//                   activation digit planes, exact integer accumulation) + LoRA stage 2
+//                   (fp64) + epilogue (store | residual add | conv1d step + step sizes)
+//   k_ssm_stream    selective-SSM state update + D skip + gate y * silu(z), state items
+//                   streamed through shared memory by bulk copies (k_ssm: large items)
+//   k_lmhead_tc     final RMSNorm + tied LM head (fp16 or int8 rows) on tensor cores +
+//                   per-block argmax (k_lmhead: fp32 fallback); k_argmax finishes it
+//   k_embed, k_quant_rows, k_pack_*   embedding gather, int8 row quantiser, sign packing
 #pragma once
 
 #include "common.cuh"
