@@ -44,6 +44,7 @@ class Dims:
     ngroups: int = 1
     d_conv: int = 4
     rank: int = 0
+    ssm_state_dtype: int = 0      # SSM state storage: 0 fp32, 1 fp16
 
     @property
     def in_rows(self) -> int:
@@ -168,7 +169,8 @@ def gen_layer(rng: np.random.Generator, d: Dims) -> LayerWeights:
 def zero_state(d: Dims) -> LayerState:
     return LayerState(
         conv=np.zeros((d.batch, d.d_conv - 1, d.conv_dim), dtype=np.float32),
-        ssm=np.zeros((d.batch, d.nheads, d.headdim, d.d_state), dtype=np.float32),
+        ssm=np.zeros((d.batch, d.nheads, d.headdim, d.d_state),
+                     dtype=np.float16 if d.ssm_state_dtype == 1 else np.float32),
     )
 
 

@@ -222,14 +222,16 @@ def conv_step(conv_state: np.ndarray, xBC: np.ndarray, w: np.ndarray, b: np.ndar
 
 
 def ssm_step(h: np.ndarray, x: np.ndarray, Bv: np.ndarray, Cv: np.ndarray,
-             dt_raw: np.ndarray, dt_bias: np.ndarray, A_log: np.ndarray, D: np.ndarray):
+             dt_raw: np.ndarray, dt_bias: np.ndarray, A_log: np.ndarray, D: np.ndarray,
+             state_dtype=np.float32):
     """Selective-SSM state update for one token (Appendix B, corrected form).
 
     h [B, H, P, N], x [B, H, P], Bv/Cv [B, N] (one group), dt_raw [B, H].
       dt = softplus(dt_raw + dt_bias),  A = -exp(A_log),  dA = exp(dt * A)
       h' = dA * h + (x * dt) (outer) B
       y  = sum_n C[n] h'[.., n] + D * x
-    Returns (y fp64 [B, H, P], h' fp32).
+    Returns (y fp64 [B, H, P], h' rounded once from fp64 to the state's storage
+    type: fp32, or fp16 for the half-precision state of the survey's next items).
     """
     h = np.asarray(h, dtype=np.float64)
     x = np.asarray(x, dtype=np.float64)
@@ -240,7 +242,7 @@ def ssm_step(h: np.ndarray, x: np.ndarray, Bv: np.ndarray, Cv: np.ndarray,
     hn = dA[:, :, None, None] * h + xdt[:, :, :, None] * np.asarray(Bv, dtype=np.float64)[:, None, None, :]
     y = np.einsum("bhpn,bn->bhp", hn, np.asarray(Cv, dtype=np.float64))
     y = y + np.asarray(D, dtype=np.float64)[None, :, None] * x
-    return y, hn.astype(np.float32)
+    return y, hn.astype(state_dtype)
 
 
 def gated_rmsnorm(y: np.ndarray, z: np.ndarray, w: np.ndarray, eps: float = EPS) -> np.ndarray:
@@ -304,7 +306,8 @@ def layer_step(res: np.ndarray, lw, st, d) -> LayerTrace:
     for gi in range(G):
         hs = slice(gi * heads_per_group, (gi + 1) * heads_per_group)
         y[:, hs], ssm_new[:, hs] = ssm_step(st.ssm[:, hs], xs[:, hs], Bg[:, gi], Cg[:, gi],
-                                            dt_raw[:, hs], lw.dt_bias[hs], lw.A_log[hs], lw.D[hs])
+                                            dt_raw[:, hs], lw.dt_bias[hs], lw.A_log[hs], lw.D[hs],
+                                            state_dtype=st.ssm.dtype)
     y = y.reshape(d.batch, E)
     # the gated value is an activation between two kernels and is stored as fp32,
     # like the residual stream; the gated RMSNorm reads the stored values

@@ -456,6 +456,40 @@ def test_model_argmax_lowest_id_on_ties_and_embedding():
     assert tr.tokens.tolist() == [3, 3]
 
 
+def test_ssm_fp16_state_is_the_fp64_update_rounded_once():
+    """Half-precision state storage: the new state is the fp64 update h' rounded once
+    to fp16 (checked per element against a plain loop), y is computed from the
+    unrounded h' exactly as with fp32 storage, and a layer step whose state is fp16
+    keeps it fp16."""
+    rng = np.random.default_rng(28)
+    Bsz, H, P, N = 2, 3, 4, 8
+    h = rng.normal(size=(Bsz, H, P, N)).astype(np.float16)
+    x = rng.normal(size=(Bsz, H, P))
+    Bv, Cv = rng.normal(size=(Bsz, N)), rng.normal(size=(Bsz, N))
+    dt_raw = rng.normal(size=(Bsz, H))
+    dt_bias = rng.normal(0, 0.1, size=H).astype(np.float32)
+    A_log = rng.uniform(0, np.log(16), size=H).astype(np.float32)
+    D = rng.normal(1, 0.1, size=H).astype(np.float32)
+    y16, h16 = O.ssm_step(h, x, Bv, Cv, dt_raw, dt_bias, A_log, D, state_dtype=np.float16)
+    y32, h32 = O.ssm_step(h, x, Bv, Cv, dt_raw, dt_bias, A_log, D)
+    assert h16.dtype == np.float16 and h32.dtype == np.float32
+    assert np.array_equal(y16, y32)
+    for b in range(Bsz):
+        for hh in range(H):
+            dt = float(np.log1p(np.exp(float(dt_raw[b, hh]) + float(dt_bias[hh]))))
+            dA = np.exp(-dt * np.exp(float(A_log[hh])))
+            for p in range(P):
+                for n in range(N):
+                    v = dA * float(h[b, hh, p, n]) + (float(x[b, hh, p]) * dt) * float(Bv[b, n])
+                    assert h16[b, hh, p, n] == np.float16(v)
+    d = S.Dims(batch=2, d_model=256, d_inner=512, nheads=8, headdim=64, d_state=16, rank=8, ssm_state_dtype=1)
+    lw = S.gen_layer(rng, d)
+    st = S.zero_state(d)
+    assert st.ssm.dtype == np.float16
+    t = O.layer_step(S.gen_layer_inputs(rng, d, 1)[0], lw, st, d)
+    assert t.ssm.dtype == np.float16 and t.conv.dtype == np.float32
+
+
 def test_int8_embedding_rows_and_logits_brute_force():
     """Section 3.3 int8 per-row embedding: the gathered row is scale * code in fp32,
     and the logits of the tied head are scale_v * (codes . norm(res)); checked
