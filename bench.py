@@ -17,6 +17,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+from dataclasses import replace
 import re
 import os
 import statistics
@@ -198,6 +199,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     F.lib()
     m, tok0 = S.model_workload(args.workload)
+    if args.state == "fp16":
+        m.dims = replace(m.dims, ssm_state_dtype=1)
     d = m.dims
     dm = F.DeviceModel.from_host(m, device=dev, head=args.head)
     states = [F.DeviceState.zeros(d, device=dev) for _ in m.layers]
@@ -280,9 +283,10 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "1-bit scaffold x fp16 act (fp32 acc), int8 LoRA (int32 acc), fp32 SSM state",
+        "dtype": f"1-bit scaffold x fp16 act (fp32 acc), int8 LoRA (int32 acc), {args.state} SSM state",
         "data": "synthetic (seeded random-init weights, random 1-token prompt)",
-        "config": {"workload": args.workload, "head": args.head, "n_layer": len(m.layers), "d_model": d.d_model,
+        "config": {"workload": args.workload, "head": args.head, "ssm_state": args.state,
+                   "n_layer": len(m.layers), "d_model": d.d_model,
                    "d_inner": d.d_inner, "nheads": d.nheads, "headdim": d.headdim, "d_state": d.d_state,
                    "rank": d.rank, "vocab": m.vocab, "batch": d.batch, "parallelism": f"replicas x{world}",
                    "cuda_graph": True,
@@ -423,6 +427,8 @@ def main():
                     help="model decode workload (default: the batch-1 greedy decode)")
     ap.add_argument("--head", choices=["fp16", "int8"], default="fp16",
                     help="tied embedding / LM head precision (int8: per-row codes + fp32 scales)")
+    ap.add_argument("--state", choices=["fp32", "fp16"], default="fp32",
+                    help="SSM state storage (fp16: multi-launch path at every batch size)")
     ap.add_argument("--sweep", action="store_true", help="time the isolated projection sweep instead")
     ap.add_argument("--proj", type=int, nargs=4, metavar=("D_IN", "D_OUT", "RANK", "BATCH"),
                     help="call one projection sweep point three times (a target for profilers)")

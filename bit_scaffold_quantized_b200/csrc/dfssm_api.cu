@@ -105,6 +105,8 @@ int check_dims(const dfssm_dims* d) {
   REQUIRE(d->d_model <= 8192 && d->d_inner <= 8192, DFSSM_ERR_UNSUPPORTED_SHAPE, "d_model/d_inner > 8192");
   REQUIRE(d->headdim % 16 == 0 && d->headdim <= 128, DFSSM_ERR_UNSUPPORTED_SHAPE,
           "headdim (%d) must be a multiple of 16 and <= 128", d->headdim);
+  REQUIRE(d->ssm_state_dtype == 0 || d->ssm_state_dtype == 1, DFSSM_ERR_INVALID_ARG,
+          "ssm_state_dtype (%d) must be 0 (fp32) or 1 (fp16)", d->ssm_state_dtype);
   REQUIRE(d->d_state % 4 == 0 && d->d_state <= 256, DFSSM_ERR_UNSUPPORTED_SHAPE,
           "d_state (%d) must be a multiple of 4 and <= 256", d->d_state);
   REQUIRE(d->rank >= 0 && d->rank <= 128 && d->rank % 4 == 0, DFSSM_ERR_UNSUPPORTED_SHAPE,
@@ -336,13 +338,13 @@ int launch_head(const HeadArgs& h, cudaStream_t st, int* nparts) {
 // fit two shared-memory buffers and every bulk copy is 16-byte aligned, else k_ssm.
 constexpr int kSsmStreamSmemCap = 96 * 1024;
 
-template <int NCH>
+template <int NCH, typename ST>
 int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
   static int occ_smem = -1, occ_blocks = 1;
   if (occ_smem != smem) {
-    cudaFuncSetAttribute(k_ssm_stream<NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaFuncSetAttribute(k_ssm_stream<NCH, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_ssm_stream<NCH>, kSsmStreamThreads, smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_ssm_stream<NCH, ST>, kSsmStreamThreads, smem) !=
             cudaSuccess || nb < 1)
       nb = 1;
     occ_smem = smem;
@@ -350,25 +352,31 @@ int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
   }
   const int items = sa.batch * sa.H;
   const int grid = std::max(1, std::min(items, occ_blocks * sm_count()));
-  k_ssm_stream<NCH><<<grid, kSsmStreamThreads, smem, st>>>(sa);
+  k_ssm_stream<NCH, ST><<<grid, kSsmStreamThreads, smem, st>>>(sa);
   CHECK_LAUNCH("k_ssm_stream");
   return DFSSM_OK;
 }
 
-int launch_ssm(const SsmArgs& sa, cudaStream_t st) {
-  const SsmItem it = ssm_item(sa.P, sa.N);
+template <typename ST>
+int launch_ssm_t(const SsmArgs& sa, cudaStream_t st) {
+  const SsmItem it = ssm_item(sa.P, sa.N, int(sizeof(ST)));
   const int smem = 2 * ((it.bytes + 127) & ~127);
   const bool aligned = (size_t(sa.conv_dim) * 8) % 16 == 0 && (size_t(sa.in_rows) * 8) % 16 == 0 &&
                        (size_t(sa.E) * 8) % 16 == 0 && (size_t(sa.P) * 8) % 16 == 0 &&
+                       (size_t(sa.P) * sa.N * sizeof(ST)) % 16 == 0 &&
                        aligned16(sa.state) && aligned16(sa.xc) && aligned16(sa.zx) && aligned16(sa.dta);
   if (aligned && smem <= kSsmStreamSmemCap) {
-    if (sa.N <= 128) return launch_ssm_stream<1>(sa, smem, st);
-    return launch_ssm_stream<2>(sa, smem, st);
+    if (sa.N <= 128) return launch_ssm_stream<1, ST>(sa, smem, st);
+    return launch_ssm_stream<2, ST>(sa, smem, st);
   }
-  if (sa.N <= 128) k_ssm<1><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
-  else k_ssm<2><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
+  if (sa.N <= 128) k_ssm<1, ST><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
+  else k_ssm<2, ST><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
   CHECK_LAUNCH("k_ssm");
   return DFSSM_OK;
+}
+
+int launch_ssm(const SsmArgs& sa, cudaStream_t st) {
+  return sa.state16 ? launch_ssm_t<__half>(sa, st) : launch_ssm_t<float>(sa, st);
 }
 
 // The layer as five dependent launches on one stream.
@@ -386,7 +394,8 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   SsmArgs sa{};
   sa.H = d->nheads; sa.P = d->headdim; sa.N = d->d_state; sa.E = E; sa.conv_dim = C; sa.in_rows = in_rows(d);
   sa.zx = b.zxbcdt; sa.xc = b.xc; sa.dt_bias = w->dt_bias; sa.A_log = w->A_log; sa.D = w->D;
-  sa.state = s->ssm_state; sa.g = b.g; sa.dta = b.dta; sa.batch = B; sa.status = b.status;
+  sa.state = s->ssm_state; sa.state16 = d->ssm_state_dtype == 1;
+  sa.g = b.g; sa.dta = b.dta; sa.batch = B; sa.status = b.status;
   if ((rc = launch_ssm(sa, st))) return rc;
   if ((rc = launch_prologue<0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, B, b.out);
@@ -461,6 +470,7 @@ PPlan plan_persistent(const dfssm_dims* d) {
   if (device_sm_count(&dev, &nsm, &optin)) return no("device query failed");
   const int D = d->d_model, E = d->d_inner, H = d->nheads, N = d->d_state, R = d->rank, P = d->headdim;
   if (d->batch != 1) return no("batch != 1");
+  if (d->ssm_state_dtype != 0) return no("the token kernel holds fp32 SSM state");
   if (N % 16 || H % 16) return no("d_state and nheads must be multiples of 16");
   if (R != 0 && (!pow2(R) || R < 8 || R > kPThreads)) return no("rank must be 0 or a power of two in [8, 512]");
   const int Q = kPMaxCluster;
@@ -500,7 +510,7 @@ PLayer player(const dfssm_layer_weights& w, const dfssm_layer_state& s) {
   L.gnorm_w = w.gnorm_w;
   L.out_bits = w.out.bits; L.out_alpha = w.out.alpha; L.out_A = w.out.A; L.out_sA = w.out.sA;
   L.out_B = w.out.B; L.out_sB = w.out.sB;
-  L.conv_state = s.conv_state; L.ssm_state = s.ssm_state;
+  L.conv_state = s.conv_state; L.ssm_state = static_cast<float*>(s.ssm_state);   // fp32 (planner)
   return L;
 }
 

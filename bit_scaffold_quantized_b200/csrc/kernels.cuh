@@ -465,7 +465,8 @@ struct SsmArgs {
   const float* dt_bias;
   const float* A_log;
   const float* D;
-  float* state;          // fp32 [B][H][P][N]
+  void* state;           // [B][H][P][N], fp32 or (state16) fp16
+  bool state16;
   float* g;              // fp32 [B][E]
   const double* dta;     // fp64 [B][H][2]: step size and decay (from the in_proj epilogue)
   int batch;
@@ -505,14 +506,32 @@ DFSSM_DEV double fold_rows(double (&y)[R], int lane, int* sel) {
 // dA = exp(-dt * exp(A_log))).  Arithmetic in fp64, state stored back in fp32 with
 // streaming hints (read and written once per step):
 //   h' = dA h + (x dt) B,  y = C . h' + D x,  g = y * silu(z) (stored fp32).
-template <int NCH>
+// Four consecutive state values (16-byte aligned for fp32, 8-byte for fp16) as
+// floats, with a streaming hint; and four fp64 updates stored back, rounded once to
+// the state's type.
+DFSSM_DEV float4 ld_state4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+DFSSM_DEV float4 ld_state4(const __half* p) {
+  const uint2 v = __ldcs(reinterpret_cast<const uint2*>(p));
+  return make_float4(h2f(uint16_t(v.x & 0xffffu)), h2f(uint16_t(v.x >> 16)), h2f(uint16_t(v.y & 0xffffu)),
+                     h2f(uint16_t(v.y >> 16)));
+}
+DFSSM_DEV void st_state4(float* p, double h0, double h1, double h2, double h3) {
+  __stcs(reinterpret_cast<float4*>(p), make_float4(float(h0), float(h1), float(h2), float(h3)));
+}
+DFSSM_DEV void st_state4(__half* p, double h0, double h1, double h2, double h3) {
+  const uint2 v = make_uint2(uint32_t(d2h(h0)) | (uint32_t(d2h(h1)) << 16),
+                             uint32_t(d2h(h2)) | (uint32_t(d2h(h3)) << 16));
+  __stcs(reinterpret_cast<uint2*>(p), v);
+}
+
+template <int NCH, typename ST>
 __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
   constexpr int RW = 8 / NCH;                  // rows of a warp in flight
   constexpr int kW = kSsmThreads / 32;
   const int h = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N4 = a.N / 4, P = a.P;
-  float* sbase = a.state + (size_t(b) * a.H + h) * size_t(P) * a.N;
+  ST* sbase = static_cast<ST*>(a.state) + (size_t(b) * a.H + h) * size_t(P) * a.N;
   const double* xcb = a.xc + size_t(b) * a.conv_dim;
   const double* zr = a.zx + size_t(b) * a.in_rows;
   for (int r0 = warp; r0 < P; r0 += RW * kW) {
@@ -522,7 +541,7 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
         const int p = r0 + i * kW, n4 = lane + 32 * c;
-        hv[i][c] = (p < P && n4 < N4) ? __ldcs(reinterpret_cast<const float4*>(sbase + size_t(p) * a.N) + n4)
+        hv[i][c] = (p < P && n4 < N4) ? ld_state4(sbase + size_t(p) * a.N + 4 * n4)
                                       : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     double Bv[NCH][4], Cv[NCH][4];
@@ -556,9 +575,7 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
         acc = fma(Cv[c][1], h1, acc);
         acc = fma(Cv[c][2], h2, acc);
         acc = fma(Cv[c][3], h3, acc);
-        if (p < P && n4 < N4)
-          __stcs(reinterpret_cast<float4*>(sbase + size_t(p) * a.N) + n4,
-                 make_float4(float(h0), float(h1), float(h2), float(h3)));
+        if (p < P && n4 < N4) st_state4(sbase + size_t(p) * a.N + 4 * n4, h0, h1, h2, h3);
       }
       y[i] = acc;
     }
@@ -575,14 +592,15 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
 }
 
 // Bytes of one (batch, head) item of k_ssm_stream and their offsets in a buffer:
-// state [P][N] fp32, then B and C [2N] fp64, x [P] fp64, z [P] fp64, (dt, dA) fp64.
+// state [P][N] (es bytes per value), then B and C [2N] fp64, x [P] fp64, z [P] fp64,
+// (dt, dA) fp64.
 struct SsmItem {
   int st, bc, x, z, dta, bytes;
 };
-__host__ __device__ inline SsmItem ssm_item(int P, int N) {
+__host__ __device__ inline SsmItem ssm_item(int P, int N, int es) {
   SsmItem it;
   it.st = 0;
-  it.bc = 4 * P * N;
+  it.bc = ((es * P * N + 15) / 16) * 16;
   it.x = it.bc + 16 * N;
   it.z = it.x + 8 * P;
   it.dta = it.z + 8 * P;
@@ -592,20 +610,27 @@ __host__ __device__ inline SsmItem ssm_item(int P, int N) {
 constexpr int kSsmStreamThreads = 256;
 
 // Streaming SSM update: grid of resident blocks; block c takes the (batch, head)
-// items c, c + gridDim.x, ...  Each item's inputs (its 4 P N bytes of state, the
+// items c, c + gridDim.x, ...  Each item's inputs (its P N values of state, the
 // batch row's B and C, the head's x and z, its step size and decay) arrive by bulk
 // copies into one of two shared-memory buffers, the next item's while this one is
 // computed, so HBM always has a block's worth of state in flight per block.  Warp w
 // takes rows w, w + 8, ... four at a time; a lane holds NCH float4 of a row.  Same
-// arithmetic as k_ssm (fp64, state stored back in fp32 with a streaming hint).
-template <int NCH>
+// arithmetic as k_ssm (fp64, state stored back in its own type with a streaming hint).
+DFSSM_DEV float4 ld_smem_state4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+DFSSM_DEV float4 ld_smem_state4(const __half* p) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  return make_float4(h2f(uint16_t(v.x & 0xffffu)), h2f(uint16_t(v.x >> 16)), h2f(uint16_t(v.y & 0xffffu)),
+                     h2f(uint16_t(v.y >> 16)));
+}
+
+template <int NCH, typename ST>
 __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
   extern __shared__ __align__(16) unsigned char sbuf[];
   __shared__ __align__(8) uint64_t bar[2];
   __shared__ int s_ok;
   constexpr int RW = 4, kW = kSsmStreamThreads / 32;
   const int P = a.P, N = a.N, H = a.H, N4 = N / 4;
-  const SsmItem it = ssm_item(P, N);
+  const SsmItem it = ssm_item(P, N, int(sizeof(ST)));
   const int bufb = (it.bytes + 127) & ~127;
   const int nitems = a.batch * H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -619,7 +644,8 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     const int b = item / H, h = item % H;
     unsigned char* base = sbuf + buf * bufb;
     mbar_expect_tx(&bar[buf], unsigned(it.bytes));
-    bulk_g2s(base + it.st, a.state + (size_t(b) * H + h) * P * N, unsigned(4 * P * N), &bar[buf]);
+    bulk_g2s(base + it.st, static_cast<const ST*>(a.state) + (size_t(b) * H + h) * P * N,
+             unsigned(sizeof(ST) * P * N), &bar[buf]);
     bulk_g2s(base + it.bc, a.xc + size_t(b) * a.conv_dim + a.E, unsigned(16 * N), &bar[buf]);
     bulk_g2s(base + it.x, a.xc + size_t(b) * a.conv_dim + size_t(h) * P, unsigned(8 * P), &bar[buf]);
     bulk_g2s(base + it.z, a.zx + size_t(b) * a.in_rows + size_t(h) * P, unsigned(8 * P), &bar[buf]);
@@ -651,7 +677,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     }
     (void)mbar_try_wait(&bar[buf], par);   // every thread acquires the copies' writes
     const unsigned char* base = sbuf + buf * bufb;
-    const float* st = reinterpret_cast<const float*>(base + it.st);
+    const ST* st = reinterpret_cast<const ST*>(base + it.st);
     const double* Bs = reinterpret_cast<const double*>(base + it.bc);
     const double* Cs = Bs + N;
     const double* xs = reinterpret_cast<const double*>(base + it.x);
@@ -659,7 +685,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     const double dt = reinterpret_cast<const double*>(base + it.dta)[0];
     const double dA = reinterpret_cast<const double*>(base + it.dta)[1];
     const int b = item / H, h = item % H;
-    float* gst = a.state + (size_t(b) * H + h) * P * N;
+    ST* gst = static_cast<ST*>(a.state) + (size_t(b) * H + h) * P * N;
     double Bv[NCH][4], Cv[NCH][4];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
@@ -681,7 +707,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
         for (int c = 0; c < NCH; ++c) {
           const int n4 = lane + 32 * c;
           if (p < P && n4 < N4) {
-            const float4 hv = reinterpret_cast<const float4*>(st + size_t(p) * N)[n4];
+            const float4 hv = ld_smem_state4(st + size_t(p) * N + 4 * n4);
             const double h0 = fma(dA, double(hv.x), xdt * Bv[c][0]);
             const double h1 = fma(dA, double(hv.y), xdt * Bv[c][1]);
             const double h2 = fma(dA, double(hv.z), xdt * Bv[c][2]);
@@ -690,8 +716,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
             acc = fma(Cv[c][1], h1, acc);
             acc = fma(Cv[c][2], h2, acc);
             acc = fma(Cv[c][3], h3, acc);
-            __stcs(reinterpret_cast<float4*>(gst + size_t(p) * N) + n4,
-                   make_float4(float(h0), float(h1), float(h2), float(h3)));
+            st_state4(gst + size_t(p) * N + 4 * n4, h0, h1, h2, h3);
           }
         }
         y[i] = acc;

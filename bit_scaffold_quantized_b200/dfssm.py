@@ -44,7 +44,8 @@ class DfssmError(RuntimeError):
 
 class CDims(C.Structure):
     _fields_ = [(n, C.c_int32) for n in
-                ("batch", "d_model", "d_inner", "nheads", "headdim", "d_state", "ngroups", "d_conv", "rank")]
+                ("batch", "d_model", "d_inner", "nheads", "headdim", "d_state", "ngroups", "d_conv", "rank",
+                 "ssm_state_dtype")]
 
 
 class CProj(C.Structure):
@@ -130,7 +131,8 @@ def _stream(stream) -> Optional[int]:
 
 
 def cdims(d) -> CDims:
-    return CDims(d.batch, d.d_model, d.d_inner, d.nheads, d.headdim, d.d_state, d.ngroups, d.d_conv, d.rank)
+    return CDims(d.batch, d.d_model, d.d_inner, d.nheads, d.headdim, d.d_state, d.ngroups, d.d_conv, d.rank,
+                 getattr(d, "ssm_state_dtype", 0))
 
 
 # ------------------------------------------------------------------ host -> device
@@ -201,13 +203,14 @@ class DeviceLayer:
 @dataclass
 class DeviceState:
     conv: object   # fp32 [B, W-1, conv_dim]
-    ssm: object    # fp32 [B, H, P, N]
+    ssm: object    # [B, H, P, N], fp32 or fp16 (d.ssm_state_dtype == 1)
 
     @classmethod
     def zeros(cls, d, device="cuda") -> "DeviceState":
         import torch
+        sdt = torch.float16 if getattr(d, "ssm_state_dtype", 0) == 1 else torch.float32
         return cls(torch.zeros((d.batch, d.d_conv - 1, d.conv_dim), dtype=torch.float32, device=device),
-                   torch.zeros((d.batch, d.nheads, d.headdim, d.d_state), dtype=torch.float32, device=device))
+                   torch.zeros((d.batch, d.nheads, d.headdim, d.d_state), dtype=sdt, device=device))
 
     @classmethod
     def from_host(cls, st, device="cuda") -> "DeviceState":

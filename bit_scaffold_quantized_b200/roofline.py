@@ -30,8 +30,10 @@ def layer_weight_bytes(d: Dims) -> int:
 
 
 def layer_state_bytes(d: Dims) -> int:
-    """fp32 conv + SSM state of all batch rows, read once and written once."""
-    per_row = 4 * ((d.d_conv - 1) * d.conv_dim + d.nheads * d.headdim * d.d_state)
+    """fp32 conv state + SSM state (fp32, or fp16 when d.ssm_state_dtype == 1) of all
+    batch rows, read once and written once."""
+    ssm_es = 2 if getattr(d, "ssm_state_dtype", 0) == 1 else 4
+    per_row = 4 * (d.d_conv - 1) * d.conv_dim + ssm_es * d.nheads * d.headdim * d.d_state
     return 2 * d.batch * per_row
 
 

@@ -71,6 +71,10 @@ enum { DFSSM_LAYOUT_ROWMAJOR = 0, DFSSM_LAYOUT_TILED = 1 };
  * 0 <= rank <= 128 and a multiple of 4. */
 typedef struct dfssm_dims {
   int32_t batch, d_model, d_inner, nheads, headdim, d_state, ngroups, d_conv, rank;
+  /* SSM state storage: 0 fp32; 1 fp16 (each step's fp64 update rounded once to
+   * fp16; halves the state stream).  fp16 state runs the multi-launch path at
+   * every batch size: the batch-1 token kernel holds fp32 state. */
+  int32_t ssm_state_dtype;
 } dfssm_dims;
 
 /* One DF-SSM projection (Eq. 3 with a per-row scaffold scale):
@@ -108,10 +112,10 @@ typedef struct dfssm_layer_weights {
 
 /* Persistent per-layer state, updated in place each step (caller-owned).
  * conv_state fp32 [batch][d_conv-1][conv_dim], index 0 the oldest input;
- * ssm_state fp32 [batch][nheads][headdim][d_state]. */
+ * ssm_state [batch][nheads][headdim][d_state], fp32 or fp16 per dims->ssm_state_dtype. */
 typedef struct dfssm_layer_state {
   float* conv_state;
-  float* ssm_state;
+  void* ssm_state;
 } dfssm_layer_state;
 
 /* Byte offsets of the intermediates a step leaves in its workspace (valid after

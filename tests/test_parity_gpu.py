@@ -4,6 +4,7 @@ partials; max relative error <= 2e-3 for fp outputs and states."""
 import numpy as np
 import pytest
 import torch
+from dataclasses import replace
 
 from oracle import dfssm_oracle as O
 from bit_scaffold_quantized_b200 import synth as S
@@ -250,6 +251,33 @@ def test_layer_step_large_state_items_parity(headdim, d_state, rank):
     for t in range(3):
         tr = _check_layer_step(run, lw, d, ost, xs[t])
         ost = O.State(tr.conv, tr.ssm)
+
+
+@pytest.mark.parametrize("name,batch", [("layer_d256_b1_16steps", 3), ("layer_d2048_b1_256steps", 2)])
+def test_layer_step_fp16_state_parity(name, batch):
+    """Half-precision SSM state (streaming kernel, fp64 update rounded once to fp16);
+    the oracle stores the same rounding, so states compare exactly up to rounding-order
+    differences far below an fp16 ulp."""
+    d, lw, st, xs = S.layer_workload(name, steps=3, batch=batch)
+    d = replace(d, ssm_state_dtype=1)
+    st = S.zero_state(d)
+    assert st.ssm.dtype == np.float16
+    run = LayerRun(d, lw, st)
+    ost = st
+    for t in range(3):
+        tr = _check_layer_step(run, lw, d, ost, xs[t])
+        assert tr.ssm.dtype == np.float16 and run.ds.ssm.dtype == torch.float16
+        assert np.array_equal(to_np(run.ds.ssm), tr.ssm)
+        ost = O.State(tr.conv, tr.ssm)
+
+
+def test_model_decode_fp16_state_parity():
+    """Batch-1 model with fp16 state takes the multi-launch path and matches the oracle."""
+    d = replace(LAYER_SMALL_P, ssm_state_dtype=1)
+    rng = np.random.default_rng(37)
+    m = S.gen_model(rng, d, 3, 1000)
+    assert F.launches_per_decode_step(d, 3, 1000) > 1
+    _teacher_forced(m, S.gen_tokens(rng, 1, 1000), 4)
 
 
 def test_layer_dt_zero_leaves_ssm_state():
