@@ -9,7 +9,8 @@ Arithmetic is fp64 except where the method fixes a storage format or where a
 floating-point value decides an integer:
   * activations entering a projection are stored as fp16;
   * SSM state, conv state, the residual stream and the gated value y*silu(z)
-    are stored as fp32;
+    are stored as fp32 (the SSM state in fp16 when the given state array is fp16:
+    the fp64 update rounded once);
   * the int8 activation quantiser takes its decision in fp32 (scale = amax/127
     as an IEEE fp32 divide, code = round-half-even of x/scale in fp32), the
     precision the kernel uses, so both sides take the same integer decision;
