@@ -5,6 +5,7 @@ Space Models" (Table 1, Appendix B).  A plausible slip anywhere in the oracle
 (a dropped term, a wrong sign or index, a transposed operand) fails one of these.
 """
 import json
+from dataclasses import replace
 import os
 
 import numpy as np
@@ -520,6 +521,20 @@ def test_int8_embedding_rows_and_logits_brute_force():
 
 
 # ---------------------------------------------------------------- byte model vs Table 1
+
+def test_byte_model_head_and_state_variants():
+    """int8 head: 1 byte per element plus a 4-byte scale per row (embedding row and
+    head); fp16 SSM state: 2 bytes per state element, conv state unchanged."""
+    d = S.LAYER_1P3B
+    V, L = S.VOCAB_1P3B, 48
+    f16 = R.model_token_bytes(d, L, V)
+    i8 = R.model_token_bytes(d, L, V, head="int8")
+    assert f16 - i8 == (2 * d.d_model - (d.d_model + 4)) + V * (2 * d.d_model - (d.d_model + 4))
+    d16 = replace(d, ssm_state_dtype=1)
+    ssm = d.nheads * d.headdim * d.d_state
+    assert R.layer_state_bytes(d) - R.layer_state_bytes(d16) == 2 * d.batch * 2 * ssm
+    assert f16 == 597_628_936
+
 
 def test_table1_sizes_from_shapes():
     t1 = json.load(open(os.path.join(GOLDEN, "table1_model_size.json")))
