@@ -616,11 +616,24 @@ constexpr int kSsmStreamThreads = 256;
 // computed, so HBM always has a block's worth of state in flight per block.  Warp w
 // takes rows w, w + 8, ... four at a time; a lane holds NCH float4 of a row.  Same
 // arithmetic as k_ssm (fp64, state stored back in its own type with a streaming hint).
-DFSSM_DEV float4 ld_smem_state4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-DFSSM_DEV float4 ld_smem_state4(const __half* p) {
+// Four consecutive state values from shared memory, converted once to fp64 (fp16
+// goes straight to fp64: one exact conversion per value).
+struct D4 {
+  double x, y, z, w;
+};
+DFSSM_DEV double h2d_direct(uint16_t h) {
+  double r;
+  asm("cvt.f64.f16 %0, %1;" : "=d"(r) : "h"(h));
+  return r;
+}
+DFSSM_DEV D4 ld_smem_state4(const float* p) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  return D4{double(v.x), double(v.y), double(v.z), double(v.w)};
+}
+DFSSM_DEV D4 ld_smem_state4(const __half* p) {
   const uint2 v = *reinterpret_cast<const uint2*>(p);
-  return make_float4(h2f(uint16_t(v.x & 0xffffu)), h2f(uint16_t(v.x >> 16)), h2f(uint16_t(v.y & 0xffffu)),
-                     h2f(uint16_t(v.y >> 16)));
+  return D4{h2d_direct(uint16_t(v.x & 0xffffu)), h2d_direct(uint16_t(v.x >> 16)),
+            h2d_direct(uint16_t(v.y & 0xffffu)), h2d_direct(uint16_t(v.y >> 16))};
 }
 
 template <int NCH, typename ST>
@@ -707,11 +720,11 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
         for (int c = 0; c < NCH; ++c) {
           const int n4 = lane + 32 * c;
           if (p < P && n4 < N4) {
-            const float4 hv = ld_smem_state4(st + size_t(p) * N + 4 * n4);
-            const double h0 = fma(dA, double(hv.x), xdt * Bv[c][0]);
-            const double h1 = fma(dA, double(hv.y), xdt * Bv[c][1]);
-            const double h2 = fma(dA, double(hv.z), xdt * Bv[c][2]);
-            const double h3 = fma(dA, double(hv.w), xdt * Bv[c][3]);
+            const D4 hv = ld_smem_state4(st + size_t(p) * N + 4 * n4);
+            const double h0 = fma(dA, hv.x, xdt * Bv[c][0]);
+            const double h1 = fma(dA, hv.y, xdt * Bv[c][1]);
+            const double h2 = fma(dA, hv.z, xdt * Bv[c][2]);
+            const double h3 = fma(dA, hv.w, xdt * Bv[c][3]);
             acc = fma(Cv[c][0], h0, acc);
             acc = fma(Cv[c][1], h1, acc);
             acc = fma(Cv[c][2], h2, acc);
