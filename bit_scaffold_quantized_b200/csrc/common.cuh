@@ -101,7 +101,7 @@ DFSSM_DEV double silu_d(double v) { return v / (1.0 + exp(-v)); }
 
 DFSSM_DEV double softplus_d(double v) { return v > 20.0 ? v : log1p(exp(v)); }
 
-// Scaffold signs as 0/1 bytes: register q of 32-column chunk ch of a tiled word.
+// Scaffold signs as 0/1 bytes: A-fragment register of product s from tiled word q.
 DFSSM_DEV uint32_t sign_bytes(uint32_t word, int s) { return (word >> s) & 0x01010101u; }
 
 // D += A(16x32, s8, row) * B(32x8, s8, col), exact s32 accumulators.

@@ -53,14 +53,18 @@ enum { DFSSM_DTYPE_F16 = 0, DFSSM_DTYPE_F32 = 1 };
  * column 32k+j, bit = 1 encodes +1 and bit = 0 encodes -1.  TILED: the same bits
  * permuted into 16-row x 256-column tiles of 128 words (rows padded up to a
  * multiple of 16 with clear bits).  For weight (row, col) with r16 = row % 16,
- * c = col % 256, kt = c / 64, ch = (c % 64) / 32, c32 = c % 32:
- *   lane = (r16 % 8) * 4 + (c32 % 16) / 4,  q = r16 / 8 + 2 * (c32 / 16),
- *   s = 4 * ch + q,  bit = s + 8 * (c32 % 4),
- *   word = ((row / 16) * (cols / 256) + col / 256) * 128 + lane * 4 + kt.
- * Each warp lane reads one 16-byte vector per tile; (word >> s) & 0x01010101 is
- * then its int8 A-fragment register q of 32-column chunk ch of an m16n8k32
- * tensor-core product, with bytes 0/1 for -1/+1.  The projection kernels consume
- * TILED words only. */
+ * c = col % 256, m = c / 64, p = c % 64, t = p / 16, e = (p % 16) / 8,
+ * h = (p % 8) / 4, i = p % 4:
+ *   lane = (r16 % 8) * 4 + t,  q = r16 / 8 + 2 * h,  s = 2 * m + e,
+ *   bit = s + 8 * i,
+ *   word = ((row / 16) * (cols / 256) + col / 256) * 128 + lane * 4 + q.
+ * Each warp lane reads one 16-byte vector (words q = 0..3) per tile; for each of
+ * the tile's eight 32-column m16n8k32 tensor-core products s, (word_q >> s) &
+ * 0x01010101 is the lane's int8 A-fragment register q with bytes 0/1 for -1/+1
+ * (fragment column 4t+i, +16 for q >= 2, is tile column 64m + 16t + 8e + i, +4).
+ * Products 2m and 2m+1 together cover tile columns 64m .. 64m+63, lane t's
+ * B-fragment bytes of both being the 16 consecutive columns 64m + 16t ...  The
+ * projection kernels consume TILED words only. */
 enum { DFSSM_LAYOUT_ROWMAJOR = 0, DFSSM_LAYOUT_TILED = 1 };
 
 /* Shape of one layer.  in_proj: d_model -> 2*d_inner + 2*ngroups*d_state + nheads
