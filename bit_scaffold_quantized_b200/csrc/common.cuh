@@ -40,18 +40,7 @@ DFSSM_DEV float warp_max(float v) {
   return v;
 }
 
-// Block-wide sum with a fixed reduction tree (deterministic).  `red` holds >= 32 floats.
-DFSSM_DEV float block_sum(float v, float* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  v = warp_sum(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float t = (lane < nw) ? red[lane] : 0.f;
-  t = warp_sum(t);
-  return t;  // every thread holds the total
-}
-
+// Block-wide reductions with a fixed tree (deterministic); `red` holds >= 32 entries.
 DFSSM_DEV double block_sum_d(double v, double* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   v = warp_sum_d(v);
@@ -60,17 +49,6 @@ DFSSM_DEV double block_sum_d(double v, double* red) {
   __syncthreads();
   double t = (lane < nw) ? red[lane] : 0.0;
   t = warp_sum_d(t);
-  return t;
-}
-
-DFSSM_DEV int block_sum_i(int v, int* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  v = warp_sum_i(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  int t = (lane < nw) ? red[lane] : 0;
-  t = warp_sum_i(t);
   return t;
 }
 
@@ -161,29 +139,6 @@ DFSSM_DEV void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
 // exact dot product of the +/-1 row with the fp16 activations.
 constexpr int kDigits = 6;
 
-DFSSM_DEV void fp16_digits(uint16_t h, int8_t (&dg)[kDigits]) {
-  long long X = (long long)(h2d(h) * 16777216.0);
-#pragma unroll
-  for (int d = 0; d < kDigits; ++d) {
-    const int D = int((X + 128) & 255) - 128;
-    dg[d] = int8_t(D);
-    X = (X - D) >> 8;
-  }
-}
-
-// Same decision as quant_code with a multiply by rcp = 1/sx (fp32, rounded) in
-// place of the divide: x * rcp is within 3 * 2^-24 |x/sx| of the correctly rounded
-// quotient, so rint agrees unless the product lies within that distance of a
-// half-integer, where the IEEE divide decides.
-DFSSM_DEV int quant_code_fast(float x, float sx, float rcp) {
-  const float t = x * rcp;
-  const float r = rintf(t);
-  const float off = fabsf(fabsf(t - r) - 0.5f);
-  int q = int(r);
-  if (off <= 4.0e-5f) q = __float2int_rn(__fdiv_rn(x, sx));
-  return max(-127, min(127, q));
-}
-
 // Exact fp16 -> fp32 by bit construction for normal values (no convert
 // instruction); zero, subnormal and non-finite values take the hardware path.
 DFSSM_DEV float half_to_float_bits(uint32_t h) {
@@ -224,9 +179,10 @@ DFSSM_DEV int rint_small(float t, float* r) {
   return __float_as_int(m) - 0x4B400000;
 }
 
-// Same decision as quant_code: clamp(rint(x / sx), -127, 127) with the fp32 IEEE
-// divide; the product x * rcp is within 3 * 2^-24 |x/sx| of the correctly rounded
-// quotient, so the divide is only needed near a half-integer.
+// int8 activation code, decided in fp32: clamp(rint(x / sx), -127, 127) with the
+// IEEE fp32 divide.  The product x * rcp (rcp = 1/sx rounded) is within
+// 3 * 2^-24 |x/sx| of the correctly rounded quotient, so the divide is only needed
+// near a half-integer.
 DFSSM_DEV int quant_code_bits(float x, float sx, float rcp) {
   const float t = x * rcp;
   float r;
@@ -256,12 +212,6 @@ DFSSM_DEV void digits_of(uint32_t h, uint32_t* lo, uint32_t* hi) {
   }
   *lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
   *hi = b[4] | (b[5] << 8);
-}
-
-// int8 activation code, decided in fp32: clamp(rint(x / sx), -127, 127).
-DFSSM_DEV int quant_code(float x, float sx) {
-  int q = __float2int_rn(__fdiv_rn(x, sx));
-  return max(-127, min(127, q));
 }
 
 // ---- mbarriers and bulk copies (global -> this CTA's shared memory)
