@@ -252,6 +252,48 @@ def gated_rmsnorm(y: np.ndarray, z: np.ndarray, w: np.ndarray, eps: float = EPS)
     return rmsnorm(g, w, eps)
 
 
+def ssd_scan(h0: np.ndarray, x: np.ndarray, Bm: np.ndarray, Cm: np.ndarray, dt_raw: np.ndarray,
+             dt_bias: np.ndarray, A_log: np.ndarray, D: np.ndarray, chunk: int = 64):
+    """Selective-SSM over a whole prompt of T tokens in the chunked (state space
+    duality, "SSD") form of Mamba-2, which the pages name (Section 2) and use with
+    block_len = 64 (Appendix B, DF-SSD).  One group.
+
+    h0 [B, H, P, N] state before the prompt, x [B, T, H, P], Bm/Cm [B, T, N],
+    dt_raw [B, T, H].  Per token dt = softplus(dt_raw + dt_bias), a = dt * A with
+    A = -exp(A_log).  Within a chunk starting at c0, cs[t] = sum_{r=c0..t} a_r, so
+    prod_{r=s+1..t} dA_r = exp(cs[t] - cs[s]):
+      y_t = sum_{s=c0..t} (C_t . B_s) exp(cs[t] - cs[s]) dt_s x_s       (within the chunk)
+          + exp(cs[t]) C_t . h_prev                                      (from the carried state)
+          + D x_t,
+      h_next = exp(cs[end]) h_prev + sum_s exp(cs[end] - cs[s]) dt_s x_s (outer) B_s.
+    This is the recurrence h_t = dA_t h_{t-1} + (x_t dt_t) (outer) B_t, y_t = C_t . h_t
+    + D x_t unrolled over a chunk, in fp64 throughout (no rounding of the state
+    between tokens).  Returns (y fp64 [B, T, H, P], final state fp64 [B, H, P, N])."""
+    x = np.asarray(x, dtype=np.float64)
+    Bm = np.asarray(Bm, dtype=np.float64)
+    Cm = np.asarray(Cm, dtype=np.float64)
+    dt = softplus(np.asarray(dt_raw, dtype=np.float64) + np.asarray(dt_bias, dtype=np.float64))
+    A = -np.exp(np.asarray(A_log, dtype=np.float64))
+    a = dt * A                                                      # [B, T, H]
+    T = x.shape[1]
+    h = np.asarray(h0, dtype=np.float64).copy()
+    y = np.zeros(x.shape)
+    for c0 in range(0, T, chunk):
+        c1 = min(c0 + chunk, T)
+        cs = np.cumsum(a[:, c0:c1], axis=1)                         # [B, L, H]
+        L = c1 - c0
+        seg = np.exp(cs[:, :, None, :] - cs[:, None, :, :])         # [B, t, s, H]
+        seg = seg * np.tril(np.ones((L, L)))[None, :, :, None]
+        CB = np.einsum("btn,bsn->bts", Cm[:, c0:c1], Bm[:, c0:c1])   # [B, t, s]
+        xdt = x[:, c0:c1] * dt[:, c0:c1, :, None]                   # [B, L, H, P]
+        y[:, c0:c1] = np.einsum("bts,btsh,bshp->bthp", CB, seg, xdt)
+        y[:, c0:c1] += np.exp(cs)[..., None] * np.einsum("btn,bhpn->bthp", Cm[:, c0:c1], h)
+        tail = np.exp(cs[:, -1:, :] - cs)                           # [B, L, H]: decay from s+1 to the end
+        h = np.exp(cs[:, -1, :])[:, :, None, None] * h + np.einsum("bsh,bshp,bsn->bhpn", tail, xdt, Bm[:, c0:c1])
+    y += np.asarray(D, dtype=np.float64)[None, None, :, None] * x
+    return y, h
+
+
 @dataclass
 class LayerTrace:
     res: np.ndarray          # fp32 [B, D] residual after the layer
