@@ -124,3 +124,29 @@ def test_model_decode_rejects_bad_arguments():
     assert L.dfssm_model_decode(*bad) == F.ERR_MISALIGNED
     bad = list(args); bad[11] = 64
     assert L.dfssm_model_decode(*bad) == F.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_int8_head_and_state_dtype_reject_bad_arguments():
+    from dataclasses import replace
+    d = S.LAYER_SMALL
+    w, s = _layer_structs(d)
+    cd = F.cdims(d)
+    L = F.lib()
+    ws_ = (F.CLayerWeights * 1)(w)
+    ss_ = (F.CLayerState * 1)(s)
+    args = [C.byref(cd), 1, 100, FAKE, FAKE, ws_, ss_, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None]
+    bad = list(args); bad[3] = None                 # int8 codes NULL
+    assert L.dfssm_model_decode_q8(*bad) == F.ERR_INVALID_ARG
+    bad = list(args); bad[4] = FAKE + 4             # scales misaligned
+    assert L.dfssm_model_decode_q8(*bad) == F.ERR_MISALIGNED
+    bad = list(args); bad[12] = 64
+    assert L.dfssm_model_decode_q8(*bad) == F.ERR_WORKSPACE_TOO_SMALL
+    # SSM state storage type must be 0 (fp32) or 1 (fp16)
+    cd_bad = F.cdims(replace(d, ssm_state_dtype=2))
+    assert L.dfssm_layer_step(C.byref(cd_bad), C.byref(w), C.byref(s), FAKE, FAKE, 1 << 30, None) == \
+        F.ERR_INVALID_ARG
+    assert "ssm_state_dtype" in F.last_error()
+    # the row quantiser
+    assert L.dfssm_quantize_rows_int8(FAKE, 0, 16, FAKE, FAKE, None) == F.ERR_INVALID_ARG
+    assert L.dfssm_quantize_rows_int8(FAKE, 4, 16, FAKE + 1, FAKE, None) == F.ERR_MISALIGNED
+    assert L.dfssm_quantize_rows_int8(None, 4, 16, FAKE, FAKE, None) == F.ERR_INVALID_ARG
