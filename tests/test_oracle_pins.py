@@ -5,6 +5,7 @@ Space Models" (Table 1, Appendix B).  A plausible slip anywhere in the oracle
 (a dropped term, a wrong sign or index, a transposed operand) fails one of these.
 """
 import json
+import math
 from dataclasses import replace
 import os
 
@@ -583,3 +584,138 @@ def test_decode_token_bytes_1p3b():
     assert R.layer_state_bytes(d) == 4_298_752
     tok = R.model_token_bytes(d, 48, S.VOCAB_1P3B)
     assert abs(tok / 1e6 - 597.6) < 0.1
+
+
+# ---------------------------------------------------------------- layer wiring, by hand
+
+def _scalar_rmsnorm(v, w, eps=1e-5):
+    ms = sum(float(a) * float(a) for a in v) / len(v)
+    r = 1.0 / math.sqrt(ms + eps)
+    return [float(a) * r * float(b) for a, b in zip(v, w)]
+
+
+def _scalar_silu(v):
+    return v / (1.0 + math.exp(-v))
+
+
+def test_rmsnorm_weight_is_applied_per_element():
+    """RMSNorm with a non-unit, non-uniform weight against a scalar loop: a dropped,
+    inverted or reversed weight fails."""
+    rng = np.random.default_rng(30)
+    v = rng.normal(size=(3, 40))
+    w = rng.uniform(0.25, 3.0, size=40).astype(np.float16)
+    got = O.rmsnorm(v, w)
+    for b in range(3):
+        ref = _scalar_rmsnorm(v[b], w)
+        for k in range(40):
+            assert got[b, k] == pytest.approx(ref[k], rel=1e-13, abs=0)
+    assert np.max(np.abs(got - O.rmsnorm(v, np.ones(40)))) > 0.1
+    assert np.max(np.abs(got - O.rmsnorm(v, 1.0 / w.astype(np.float64)))) > 0.1
+
+
+def test_final_norm_weight_and_tied_head_by_hand():
+    """Model with no layers: logits[b, v] = sum_k E[v, k] * rmsnorm(E[tok_b])[k] * wf[k],
+    written out as scalar loops with a non-uniform final norm weight."""
+    d = S.LAYER_SMALL.with_batch(2)
+    rng = np.random.default_rng(31)
+    m = S.gen_model(rng, d, 0, 12)
+    m.normf_w = rng.uniform(0.2, 2.5, size=d.d_model).astype(np.float16)
+    toks = np.array([4, 9], dtype=np.int32)
+    tr = O.model_step(toks, m, [])
+    for b, t in enumerate(toks):
+        xn = _scalar_rmsnorm(m.embed[t].astype(np.float32), m.normf_w)
+        for v in range(12):
+            ref = sum(float(m.embed[v, k]) * xn[k] for k in range(d.d_model))
+            assert tr.logits[b, v] == pytest.approx(ref, rel=1e-12, abs=1e-15)
+    m.normf_w = np.ones(d.d_model, dtype=np.float16)
+    assert np.max(np.abs(O.model_step(toks, m, []).logits - tr.logits)) > 1e-3
+
+
+def _hand_layer(seed):
+    """A hand-sized layer: d_model 32, two heads of headdim 16 (d_inner 32), d_state 2,
+    rank 0, random signs and non-uniform weights, nonzero conv and SSM state."""
+    d = S.Dims(batch=1, d_model=32, d_inner=32, nheads=2, headdim=16, d_state=2, rank=0)
+    rng = np.random.default_rng(seed)
+    lw = S.gen_layer(rng, d)
+    lw.prenorm_w = rng.uniform(0.3, 2.0, size=32).astype(np.float16)
+    lw.gnorm_w = rng.uniform(0.3, 2.0, size=32).astype(np.float16)
+    lw.inp.alpha = rng.uniform(0.05, 0.6, size=d.in_rows).astype(np.float16)
+    lw.out.alpha = rng.uniform(0.05, 0.6, size=32).astype(np.float16)
+    lw.dt_bias = np.array([0.3, -0.4], dtype=np.float32)
+    lw.A_log = np.array([0.2, 1.1], dtype=np.float32)
+    lw.D = np.array([0.7, 1.3], dtype=np.float32)
+    st = S.zero_state(d)
+    st.conv[:] = rng.normal(size=st.conv.shape)
+    st.ssm[:] = rng.normal(size=st.ssm.shape)
+    res = rng.normal(size=(1, 32)).astype(np.float32)
+    return d, lw, st, res
+
+
+def _hand_layer_expected(d, lw, st, res):
+    """The layer written out with scalar loops and explicit index ranges.
+
+    in_proj rows, Mamba-2 order: z = [0, E), x = [E, 2E), B = [2E, 2E+N),
+    C = [2E+N, 2E+2N), dt_raw = [2E+2N, 2E+2N+H).  The conv runs over x, B and C
+    (window = three stored inputs, oldest first, then the new one; tap 3 = newest).
+    State update h' = dA h + (x dt) B[n]; read-out y = sum_n C[n] h'[n] + D x.
+    Gate z: g = y silu(z), stored fp32; xo = fp16(rmsnorm(g) w_g); res += out_proj(xo).
+    """
+    E, N, H, P, Dm = d.d_inner, d.d_state, d.nheads, d.headdim, d.d_model
+    r = [float(v) for v in res[0]]
+    x_in = [float(np.float16(v)) for v in _scalar_rmsnorm(r, lw.prenorm_w)]
+    sin = O.unpack_signs(lw.inp.bits, Dm)
+    zx = [float(lw.inp.alpha[o]) * sum(int(sin[o, k]) * x_in[k] for k in range(Dm)) for o in range(d.in_rows)]
+    z = zx[0:E]
+    xBC = zx[E:2 * E + 2 * N]
+    dt_raw = zx[2 * E + 2 * N:2 * E + 2 * N + H]
+    xc, conv_new = [], []
+    for c in range(E + 2 * N):
+        win = [float(st.conv[0, 0, c]), float(st.conv[0, 1, c]), float(st.conv[0, 2, c]), xBC[c]]
+        pre = float(lw.conv_b[c]) + sum(float(lw.conv_w[c, j]) * win[j] for j in range(4))
+        xc.append(_scalar_silu(pre))
+        conv_new.append(win[1:])
+    xs, Bv, Cv = xc[0:E], xc[E:E + N], xc[E + N:E + 2 * N]
+    y = [0.0] * E
+    hnew = np.zeros((H, P, N))
+    for h in range(H):
+        v = dt_raw[h] + float(lw.dt_bias[h])
+        dt = v if v > 20 else math.log1p(math.exp(v))
+        dA = math.exp(dt * -math.exp(float(lw.A_log[h])))
+        for p in range(P):
+            e = h * P + p
+            acc = 0.0
+            for n in range(N):
+                hv = dA * float(st.ssm[0, h, p, n]) + (xs[e] * dt) * Bv[n]
+                hnew[h, p, n] = hv
+                acc += Cv[n] * hv
+            y[e] = acc + float(lw.D[h]) * xs[e]
+    g = [float(np.float32(y[e] * _scalar_silu(z[e]))) for e in range(E)]
+    xo = [float(np.float16(v)) for v in _scalar_rmsnorm(g, lw.gnorm_w)]
+    sout = O.unpack_signs(lw.out.bits, E)
+    res_new = [float(np.float32(r[o] + float(lw.out.alpha[o]) * sum(int(sout[o, k]) * xo[k] for k in range(E))))
+               for o in range(Dm)]
+    return dict(x_in=x_in, zx=zx, xc=xc, conv=conv_new, y=y, ssm=hnew, g=g, xo=xo, res=res_new)
+
+
+@pytest.mark.parametrize("seed", [32, 33])
+def test_layer_wiring_by_hand(seed):
+    """Every intermediate of one layer step against the scalar-loop restatement above:
+    a B <-> C swap, x used as the gate instead of z, a wrong dt slice, a dropped or
+    misplaced norm weight, or a wrong conv window each change these values."""
+    d, lw, st, res = _hand_layer(seed)
+    t = O.layer_step(res, lw, st, d)
+    ex = _hand_layer_expected(d, lw, st, res)
+    close = dict(rel=1e-11, abs=1e-12)
+    assert [float(v) for v in t.x_in[0]] == ex["x_in"]
+    for o in range(d.in_rows):
+        assert t.zxbcdt[0, o] == pytest.approx(ex["zx"][o], **close)
+    for c in range(len(ex["xc"])):
+        assert t.xc[0, c] == pytest.approx(ex["xc"][c], **close)
+        for j in range(3):
+            assert float(t.conv[0, j, c]) == pytest.approx(float(np.float32(ex["conv"][c][j])), rel=1e-6)
+    for e in range(d.d_inner):
+        assert t.y[0, e] == pytest.approx(ex["y"][e], **close)
+        assert t.g[0, e] == pytest.approx(ex["g"][e], rel=1e-6, abs=1e-9)
+    np.testing.assert_allclose(t.ssm[0].astype(np.float64), ex["ssm"], rtol=1e-6, atol=1e-7)
+    assert [float(v) for v in t.x_out[0]] == ex["xo"]
+    np.testing.assert_allclose(t.res[0].astype(np.float64), ex["res"], rtol=1e-6, atol=1e-7)
