@@ -233,33 +233,58 @@ int pick_bt(int batch, int K, int rank) {
   return bt;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) ==
-        cudaSuccess && v > 0)
-      n = v;
-    else
-      n = 148;
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = 0;
   }
-  return n;
+  return dev;
+}
+
+// SM count of the current device, cached per device.
+int sm_count() {
+  static std::mutex mu;
+  static std::vector<std::array<int, 2>> cache;   // device, SMs
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& c : cache)
+    if (c[0] == dev) return c[1];
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+    cudaGetLastError();
+    v = 148;
+  }
+  cache.push_back({dev, v});
+  return v;
+}
+
+// Resident blocks per SM of `kernel` with `threads` threads and `smem` bytes of
+// dynamic shared memory on the current device, cached per (kernel, device, smem);
+// the kernel's dynamic shared-memory limit is raised on that device first.
+int occupancy(const void* kernel, int threads, int smem) {
+  struct Entry { const void* k; int dev, smem, blocks; };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& c : cache)
+    if (c.k == kernel && c.dev == dev && c.smem == smem) return c.blocks;
+  int nb = 0;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, size_t(smem)) != cudaSuccess || nb < 1) {
+    cudaGetLastError();
+    nb = 1;
+  }
+  cache.push_back({kernel, dev, smem, nb});
+  return nb;
 }
 
 template <int EPI, int BT>
 int launch_proj_bt(const ProjArgs& a, cudaStream_t st) {
   const size_t smem = proj_smem_bytes(a.K, a.rank, BT);
-  cudaFuncSetAttribute(k_proj<EPI, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   // one wave of resident blocks; each reuses its staged digit planes over several tiles
-  static int occ_smem = -1, occ_blocks = 1;
-  if (occ_smem != int(smem)) {
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_proj<EPI, BT>, kProjThreads, smem) != cudaSuccess ||
-        nb < 1)
-      nb = 1;
-    occ_smem = int(smem);
-    occ_blocks = nb;
-  }
+  const int occ_blocks = occupancy(reinterpret_cast<const void*>(k_proj<EPI, BT>), kProjThreads, int(smem));
   const int ntiles = (a.rows + kTileRows - 1) / kTileRows, gy = (a.batch + BT - 1) / BT;
   const int wave = std::max(1, occ_blocks * sm_count() / gy);
   const int gx = std::max(1, std::min((ntiles + kProjWarps - 1) / kProjWarps, wave));
@@ -295,17 +320,7 @@ size_t head_tc_smem(int D, int nb) { return size_t(2) * 8 * nb * (D + 4) * 2; }
 template <int NB, bool Q8>
 int launch_head_tc(const HeadArgs& h, cudaStream_t st, int* nparts) {
   const size_t smem = head_tc_smem(h.D, NB);
-  static int occ_smem = -1, occ_blocks = 1;
-  if (occ_smem != int(smem)) {
-    cudaFuncSetAttribute(k_lmhead_tc<NB, Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_lmhead_tc<NB, Q8>, kHeadWarps * 32, smem) !=
-            cudaSuccess ||
-        nb < 1)
-      nb = 1;
-    occ_smem = int(smem);
-    occ_blocks = nb;
-  }
+  const int occ_blocks = occupancy(reinterpret_cast<const void*>(k_lmhead_tc<NB, Q8>), kHeadWarps * 32, int(smem));
   const int gx = (h.batch + 8 * NB - 1) / (8 * NB);
   const int tiles = (h.vocab + 15) / 16;
   int gy = std::max(1, occ_blocks * sm_count() / gx);
@@ -340,16 +355,7 @@ constexpr int kSsmStreamSmemCap = 96 * 1024;
 
 template <int NCH, typename ST>
 int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
-  static int occ_smem = -1, occ_blocks = 1;
-  if (occ_smem != smem) {
-    cudaFuncSetAttribute(k_ssm_stream<NCH, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_ssm_stream<NCH, ST>, kSsmStreamThreads, smem) !=
-            cudaSuccess || nb < 1)
-      nb = 1;
-    occ_smem = smem;
-    occ_blocks = nb;
-  }
+  const int occ_blocks = occupancy(reinterpret_cast<const void*>(k_ssm_stream<NCH, ST>), kSsmStreamThreads, smem);
   const int items = sa.batch * sa.H;
   const int grid = std::max(1, std::min(items, occ_blocks * sm_count()));
   k_ssm_stream<NCH, ST><<<grid, kSsmStreamThreads, smem, st>>>(sa);

@@ -653,7 +653,9 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  int issued[2] = {0, 0}, landed[2] = {0, 0};   // thread 0: copy phases per buffer
   auto issue = [&](int item, int buf) {
+    ++issued[buf];
     const int b = item / H, h = item % H;
     unsigned char* base = sbuf + buf * bufb;
     mbar_expect_tx(&bar[buf], unsigned(it.bytes));
@@ -679,15 +681,24 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
       while (!mbar_try_wait(&bar[buf], par))
         if (++spins > (1 << 22)) { ok = false; break; }
       s_ok = ok ? 1 : 0;
-      if (!ok) atomicOr(a.status, 32768u);
+      if (ok) {
+        ++landed[buf];
+      } else {
+        atomicOr(a.status, 32768u);
+        // Before the block exits, let every copy still in flight towards its shared
+        // memory land: each buffer has at most one outstanding phase, whose parity is
+        // that of its last issue (bounded again; the status already marks the outputs
+        // invalid).
+        for (int bb = 0; bb < 2; ++bb) {
+          if (issued[bb] == landed[bb]) continue;
+          const unsigned pp = unsigned(issued[bb] - 1) & 1u;
+          long long s2 = 0;
+          while (!mbar_try_wait(&bar[bb], pp) && ++s2 < (1LL << 24)) __nanosleep(64);
+        }
+      }
     }
     __syncthreads();
-    if (!s_ok) {
-      // give copies that may still be in flight time to land, then leave
-      const long long t0 = clock64();
-      while (clock64() - t0 < 200000) __nanosleep(1000);
-      return;
-    }
+    if (!s_ok) return;
     (void)mbar_try_wait(&bar[buf], par);   // every thread acquires the copies' writes
     const unsigned char* base = sbuf + buf * bufb;
     const ST* st = reinterpret_cast<const ST*>(base + it.st);

@@ -846,13 +846,19 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   uint64_t* empty_cd = &bars[3];
   uint64_t* full_h = &bars[4];
   uint64_t* empty_h = &bars[4 + kHeadRingMax];
+  __shared__ int s_stale;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4 + 2 * kHeadRingMax; ++i) mbar_init(&bars[i], 1);
     for (int i = 0; i < EX_N; ++i) mbar_init(&xbars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // An abort flag left by an earlier call means its exchange words may still carry
+    // this launch's epoch: do nothing and say so (the caller zero-fills the workspace).
+    s_stale = aborted(pa.ctl) ? 1 : 0;
+    if (s_stale) atomicOr(pa.status, 1u);
   }
   // every CTA's barriers exist before any CTA of the cluster copies into it
   cluster_sync_all();
+  const bool stale = s_stale != 0;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.grid;
@@ -870,7 +876,9 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   const int NH = PSM(head_slots);
   const int chunk_bytes = kHeadChunkRows * 2 * D;
   auto head_slot = [&](int b) { return sm + b * chunk_bytes; };
-  if (warp == kPWarps) {
+  if (stale) {
+    // nothing issued, nothing to wait for
+  } else if (warp == kPWarps) {
     // ============================================================== copy warp
     bool ok = true;
     unsigned ab_issued = 0, cd_issued = 0, h_issued[kHeadRingMax] = {};

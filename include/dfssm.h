@@ -130,7 +130,9 @@ typedef struct dfssm_layer_state {
  * the scaffold product is computed exactly from these planes. */
 typedef struct dfssm_ws_layout {
   size_t total_bytes;
-  size_t status;     /* uint32 status word, 0 = ok.  Value 2: a token id was out of range
+  size_t status;     /* uint32 status word, 0 = ok.  Value 1: the batch-1 token kernel found
+                        the abort flag of an earlier failed call set and did nothing (zero
+                        the workspace).  Value 2: a token id was out of range
                         (clamped).  Values 4 .. 16384: a bounded wait of the batch-1 token
                         kernel gave up (each wait has its own value) and the call's outputs
                         are invalid.  Value 32768: a streamed SSM-state copy did not land
@@ -177,7 +179,10 @@ DFSSM_API int dfssm_repack_bits(const uint32_t* rowmajor, int rows, int cols, ui
 
 DFSSM_API size_t dfssm_proj_workspace_bytes(int rows, int cols, int rank, int batch);
 
-/* y [batch][rows] fp32 = projection of x [batch][cols] fp16 (finite values).  The
+/* Eq. 3 (Section 3.2), one scaffold + int8 LoRA projection, Section 4.1's "bits
+ * expanded on the fly" done in registers (the packed words are never expanded in
+ * memory).
+ * y [batch][rows] fp32 = projection of x [batch][cols] fp16 (finite values).  The
  * scaffold sum is exact (integer arithmetic on the activation's digit planes), the
  * LoRA stage 2 and scaling are fp64, y is rounded once to fp32.  The workspace
  * receives xq_in, sx_in, acc_in, u_in, xd_in and xdsum_in (see dfssm_ws_layout)
@@ -192,7 +197,9 @@ DFSSM_API int dfssm_proj_forward(const dfssm_proj* p, int rank, int batch, const
  * whose dfssm_proj_workspace_bytes exceeds 4 MiB returns
  * DFSSM_ERR_WORKSPACE_TOO_SMALL without enqueueing anything.  The first call on
  * a device looks up that device's address of the array, so make it before any
- * stream capture.  All calls on a device share the one array, which keeps the
+ * stream capture.  That address is kept for the life of the process: after a
+ * cudaDeviceReset (or any other reset of the device's primary context) do not call
+ * this entry point on that device again.  All calls on a device share the one array, which keeps the
  * last call's contents: calls whose kernels may overlap on the GPU (different
  * streams without ordering) race on it.  Nothing in it needs to start at zero. */
 DFSSM_API int dfssm_proj_forward_noalloc(const dfssm_proj* p, int rank, int batch, const uint16_t* x,
@@ -203,13 +210,23 @@ DFSSM_API int dfssm_proj_workspace_layout(int rows, int cols, int rank, int batc
 /* ---- decode step -------------------------------------------------------- */
 
 /* Workspace for dfssm_layer_step (n_layer == 0, vocab == 0) or for
- * dfssm_model_decode (n_layer >= 1, vocab >= 1).  The workspace must be
- * zero-filled once before its first use; the library leaves its control words
- * consistent after every successful call. */
+ * dfssm_model_decode (n_layer >= 1, vocab >= 1).  Section 4.1 preallocates all
+ * decode buffers once so that the token step can be a graph replay; this is that
+ * preallocation, owned by the caller.  The workspace must be zero-filled once
+ * before its first use; the library leaves its control words consistent after
+ * every call whose status word (dfssm_ws_layout.status) stays 0.  After a call that
+ * left a nonzero status in values 4 .. 16384 (a bounded wait gave up), every later
+ * call on the same workspace returns at once with status value 1 or-ed in, until
+ * the caller zero-fills the workspace again. */
 DFSSM_API size_t dfssm_workspace_bytes(const dfssm_dims* d, int n_layer, int vocab);
 DFSSM_API int dfssm_workspace_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* out);
 
-/* One decode token through one layer, residual add included:
+/* One decode token through one layer, residual add included ("Density Field State
+ * Space Models", Section 4.1: the decode step runs the conv1d step as a stateful
+ * shift register and the SSM step as a stateful recurrence over preallocated
+ * persistent state, the whole step replayed as a CUDA graph; Appendix B, Table 12:
+ * h = A h + (x * dt) (outer) B and the gate before the norm, norm(y * silu(z));
+ * Section 3.2, Eq. 3 and Table 1 for the two projections):
  *   x = fp16(rmsnorm(residual) * prenorm_w); [z|xBC|dt] = in_proj(x);
  *   xc = silu(conv1d_step(xBC)); SSM update of ssm_state; g = y * silu(z);
  *   xo = fp16(rmsnorm(g) * gnorm_w); residual += out_proj(xo).
@@ -217,7 +234,10 @@ DFSSM_API int dfssm_workspace_layout(const dfssm_dims* d, int n_layer, int vocab
 DFSSM_API int dfssm_layer_step(const dfssm_dims* d, const dfssm_layer_weights* w, const dfssm_layer_state* s,
                      float* residual, void* ws, size_t ws_bytes, void* stream);
 
-/* One greedy decode token for all batch rows through the whole model:
+/* One greedy decode token for all batch rows through the whole model ("Density
+ * Field State Space Models", Section 4.1: the batch-1 decode path, one graph per
+ * token; Section 4.3 and Table 2: batch-1 and batched decode throughput; Section 3.3
+ * and Table 1: tied embedding / LM head; Appendix B, Table 12 for each layer):
  *   residual = embed[tok_in]; n_layer layer steps; xf = rmsnorm(residual) * normf_w;
  *   logits = embed . xf (tied LM head, fp32 accumulation); tok_out = argmax
  *   (lowest token id wins ties).
