@@ -163,22 +163,47 @@ def oracle_slice(m, tok, n_layers: int, vocab_rows: int):
     return int(np.argmax(logits[0]))
 
 
-def _blas_threads():
+def _cpu_model() -> str:
     try:
-        from threadpoolctl import threadpool_info
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class _OneThread:
+    """The oracle runs single-threaded on one host core: BLAS limited to one thread
+    (numpy's own loops are single-threaded) and the process pinned to one core for the
+    duration.  Reports the threads the BLAS pools actually had inside the region."""
+
+    def __enter__(self):
+        from threadpoolctl import threadpool_limits, threadpool_info
+        self._lim = threadpool_limits(limits=1)
+        self._aff = None
+        if hasattr(os, "sched_getaffinity"):
+            self._aff = os.sched_getaffinity(0)
+            os.sched_setaffinity(0, {min(self._aff)})
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
+        self.threads = max(n) if n else 1
+        return self
+
+    def __exit__(self, *exc):
+        if self._aff is not None:
+            os.sched_setaffinity(0, self._aff)
+        self._lim.restore_original_limits()
 
 
 def time_oracle(m, tok, n_layers: int, vocab_rows: int, reps: int):
-    """Seconds per repetition of the slice; the slice is 1/frac of a token."""
-    oracle_slice(m, tok, 1, 16)      # import + first-touch outside the timing
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        oracle_slice(m, tok, n_layers, vocab_rows)
-    return (time.perf_counter() - t0) / reps
+    """(seconds per repetition of the slice, threads used); one thread, one core."""
+    with _OneThread() as one:
+        oracle_slice(m, tok, 1, 16)      # import + first-touch outside the timing
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle_slice(m, tok, n_layers, vocab_rows)
+        return (time.perf_counter() - t0) / reps, one.threads
 
 
 def slice_fraction(m, n_layers: int, vocab_rows: int) -> float:
@@ -304,12 +329,14 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         nl, vr = 1, m.vocab // 48
         reps = 3
-        sec = time_oracle(m, tok0, nl, vr, reps)
+        sec, threads = time_oracle(m, tok0, nl, vr, reps)
         frac = slice_fraction(m, nl, vr)
         line["cpu_baseline"] = {"value": round(frac / sec * d.batch, 5), "unit": "tokens/s",
-                                "cores": _blas_threads(), "kind": "oracle",
+                                "cores": threads, "kind": "oracle", "cpu_model": _cpu_model(),
+                                "host_cpus": os.cpu_count(),
                                 "sample": f"{reps} x (1 of 48 layers + {vr} of {m.vocab} LM-head rows), "
-                                          f"= {frac:.4f} token each by algorithmic bytes"}
+                                          f"= {frac:.4f} token each by algorithmic bytes; single thread "
+                                          f"on one core, extrapolated to a token"}
     return line
 
 
@@ -393,12 +420,14 @@ def run_reference(args, rank, world):
     m, tok0 = S.model_workload(args.workload)
     nl, vr = 1, m.vocab // 48
     frac = slice_fraction(m, nl, vr)
-    for _ in range(args.warmup):
-        oracle_slice(m, tok0, nl, vr)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_slice(m, tok0, nl, vr)
-    sec = time.perf_counter() - t0
+    with _OneThread() as one:
+        for _ in range(args.warmup):
+            oracle_slice(m, tok0, nl, vr)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_slice(m, tok0, nl, vr)
+        sec = time.perf_counter() - t0
+        threads = one.threads
     d = m.dims
     value = args.steps * frac * d.batch / sec
     return {
@@ -408,9 +437,10 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded random-init weights, random 1-token prompt)",
         "config": {"workload": args.workload, "batch": d.batch, "n_layer": len(m.layers), "vocab": m.vocab},
-        "cpu_baseline": {"value": round(value, 5), "unit": "tokens/s", "cores": _blas_threads(),
-                         "kind": "oracle",
-                         "sample": f"each step = 1 of 48 layers + {vr} LM-head rows = {frac:.4f} token"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle", "cpu_model": _cpu_model(), "host_cpus": os.cpu_count(),
+                         "sample": f"each step = 1 of 48 layers + {vr} LM-head rows = {frac:.4f} token, "
+                                   f"single thread on one core"},
         "e2e": {"value": round(value, 5), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

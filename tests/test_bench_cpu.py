@@ -20,7 +20,8 @@ def test_reference_arm_json_line():
         assert k in j, k
     assert j["impl"] == "reference" and j["steps"] == 1 and j["warmup"] == 3
     assert j["unit"] == "tokens/s" and j["value"] > 0 and j["higher_is_better"] is True
-    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
+    assert j["cpu_baseline"]["cpu_model"]
     assert j["cpu_baseline"]["value"] == j["value"]
     assert j["e2e"] == {"value": j["value"], "unit": j["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert j["config"]["workload"] == "model_48x2048_v50280_b1_greedy512"

@@ -331,7 +331,7 @@ def test_state_checkpoint_resume_bit_identical():
 
 # ---------------------------------------------------------------- model decode
 
-def _teacher_forced(m, tok0, steps, n_check_tokens=True, head="fp16"):
+def _teacher_forced(m, tok0, steps, n_check_tokens=True, head="fp16", all_layers=False):
     d = m.dims
     dm = F.DeviceModel.from_host(m, head=head)
     emb_q = None
@@ -358,9 +358,9 @@ def _teacher_forced(m, tok0, steps, n_check_tokens=True, head="fp16"):
         tr = O.model_step(tok, m, ost, emb_q=emb_q)
         e = rel_err(to_np(logits), tr.logits)
         assert e <= TOL, (t, e)
-        for l in (0, len(m.layers) - 1):
-            assert rel_err(to_np(states[l].ssm), tr.states[l].ssm) <= TOL
-            assert rel_err(to_np(states[l].conv), tr.states[l].conv) <= TOL
+        for l in (range(len(m.layers)) if all_layers else (0, len(m.layers) - 1)):
+            assert rel_err(to_np(states[l].ssm), tr.states[l].ssm) <= TOL, (t, l)
+            assert rel_err(to_np(states[l].conv), tr.states[l].conv) <= TOL, (t, l)
         got = to_np(tok_out)
         gl = to_np(logits)
         assert np.array_equal(got, np.argmax(gl, axis=-1))          # argmax of its own logits
@@ -433,7 +433,32 @@ def test_model_decode_1p3b_int8_head_parity():
 
 
 def test_model_decode_1p3b_parity():
+    """The benchmark's own launch configuration (48 layers, batch 1, the single-launch
+    token kernel) over 8 teacher-forced tokens, every layer's SSM and conv state
+    compared after every token."""
     m, tok = S.model_workload("model_48x2048_v50280_b1_greedy512")
     # the benchmark shape must take the single-launch persistent kernel
     assert F.launches_per_decode_step(m.dims, len(m.layers), m.vocab) == 1
-    _teacher_forced(m, tok, 2)
+    _teacher_forced(m, tok, 8, all_layers=True)
+
+
+def test_model_decode_1p3b_b16_parity():
+    """The batched decode workload at its own shape ("Density Field State Space
+    Models", Section 4.3, Table 2: batched decode): 48 layers, d_model 2048, batch 16,
+    random token ids as the prompt, the multi-launch path with the 16-row tensor-core
+    LM head; every layer's state after every step."""
+    m, tok = S.model_workload("model_48x2048_v50280_b16_256steps")
+    assert m.dims.batch == 16
+    assert F.launches_per_decode_step(m.dims, len(m.layers), m.vocab) == 1 + 5 * 48 + 2
+    _teacher_forced(m, tok, 2, all_layers=True)
+
+
+def test_model_decode_1p3b_b64_parity():
+    """Batch 64 at the 1.3B layer shape and the full vocabulary (the batch-64 decode
+    workload's kernels: the 2 x 16-row tensor-core LM head, the streamed SSM grid over
+    64 x 64 items), with 4 of its 48 layers to keep the oracle's time bounded."""
+    w = S.WORKLOADS["model_48x2048_v50280_b64_256steps"]
+    rng = np.random.default_rng(w["seed"])
+    m = S.gen_model(rng, w["dims"], 4, w["vocab"])
+    tok = S.gen_tokens(rng, 64, w["vocab"])
+    _teacher_forced(m, tok, 2, all_layers=True)
