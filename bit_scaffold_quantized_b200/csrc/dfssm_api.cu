@@ -260,9 +260,13 @@ int sm_count() {
 }
 
 // Resident blocks per SM of `kernel` with `threads` threads and `smem` bytes of
-// dynamic shared memory on the current device, cached per (kernel, device, smem);
-// the kernel's dynamic shared-memory limit is raised on that device first.
+// dynamic shared memory on the current device, cached per (kernel, device, smem).
+// The kernel's dynamic shared-memory limit is set to `smem` on every call (a cheap
+// host call): the same kernel runs with several sizes, and a launch needs the
+// limit at its own size.
 int occupancy(const void* kernel, int threads, int smem) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    cudaGetLastError();
   struct Entry { const void* k; int dev, smem, blocks; };
   static std::mutex mu;
   static std::vector<Entry> cache;
@@ -271,8 +275,7 @@ int occupancy(const void* kernel, int threads, int smem) {
   for (const auto& c : cache)
     if (c.k == kernel && c.dev == dev && c.smem == smem) return c.blocks;
   int nb = 0;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, size_t(smem)) != cudaSuccess || nb < 1) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, size_t(smem)) != cudaSuccess || nb < 1) {
     cudaGetLastError();
     nb = 1;
   }
