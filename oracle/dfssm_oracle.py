@@ -23,6 +23,8 @@ Sources ("Density Field State Space Models", C. Shinde):
   Section 4.1           bits expanded on the fly; conv step is a stateful shift register;
                         SSM step is a stateful recurrence; preallocated persistent state
   Appendix B, Table 12  h = A h + (x dt) (x) B; d_state = 128 at 1.3B; norm(y * silu(z))
+  Section 2, Appendix B the chunked (SSD) form of the scan over a prompt, block_len 64:
+                        the prompt pass (conv_seq, ssd_scan, layer_prefill, model_prefill)
 Where the pages are silent (the [z|x|B|C|dt] split, softplus, eps, conv tap order,
 activation quantiser, the per-row scaffold scale alpha) the standard Mamba-2
 block and the decode-step description this package implements fix the reading;
@@ -294,6 +296,28 @@ def ssd_scan(h0: np.ndarray, x: np.ndarray, Bm: np.ndarray, Cm: np.ndarray, dt_r
     return y, h
 
 
+def conv_seq(conv_state: np.ndarray, xBC: np.ndarray, w: np.ndarray, b: np.ndarray):
+    """Causal depthwise conv1d over a whole prompt (Section 4.1's conv step, applied to
+    T tokens at once, as the prompt pass of a Mamba-2 layer does).
+
+    conv_state [B, W-1, C] holds the W-1 inputs before the prompt, oldest first;
+    xBC [B, T, C] are the prompt's inputs.  Over the concatenation s = [state, xBC],
+    output t is silu(bias + sum_j w[:, j] * s[t + j]) (tap W-1 multiplies token t's own
+    input); the new state is the last W-1 entries of s, stored as fp32.  Inputs inside
+    the prompt enter the window at full precision.  Returns (xc fp64 [B, T, C], new
+    state fp32 [B, W-1, C])."""
+    cs = np.asarray(conv_state, dtype=np.float64)
+    x = np.asarray(xBC, dtype=np.float64)
+    W = cs.shape[1] + 1
+    T = x.shape[1]
+    seq = np.concatenate([cs, x], axis=1)                          # [B, W-1+T, C]
+    wt = np.asarray(w, dtype=np.float64)                            # [C, W]
+    pre = np.broadcast_to(np.asarray(b, dtype=np.float64), x.shape).copy()
+    for j in range(W):
+        pre += wt[:, j][None, None, :] * seq[:, j:j + T, :]
+    return silu(pre), seq[:, T:T + W - 1, :].astype(np.float32)
+
+
 @dataclass
 class LayerTrace:
     res: np.ndarray          # fp32 [B, D] residual after the layer
@@ -364,6 +388,52 @@ def layer_step(res: np.ndarray, lw, st, d) -> LayerTrace:
 
 
 @dataclass
+class PrefillTrace:
+    res: np.ndarray          # fp32 [B, T, D] residual after the layer, every prompt token
+    conv: np.ndarray         # fp32 conv state after the prompt
+    ssm: np.ndarray          # SSM state after the prompt (the fp64 final state rounded once)
+    x_in: np.ndarray         # fp16 [B, T, D]
+    zxbcdt: np.ndarray       # fp64 [B, T, in_rows]
+    xc: np.ndarray           # fp64 [B, T, conv_dim]
+    y: np.ndarray            # fp64 [B, T, d_inner]
+    g: np.ndarray            # [B, T, d_inner] gated value, stored as fp32 (held in fp64)
+    x_out: np.ndarray        # fp16 [B, T, d_inner]
+
+
+def layer_prefill(res: np.ndarray, lw, st, d, chunk: int = 64) -> PrefillTrace:
+    """A whole prompt of T tokens through one layer in one pass (the prompt step
+    before decode): the projections over all B*T token rows, the causal conv over the
+    sequence (conv_seq), the selective SSM as the chunked SSD scan (ssd_scan, Section
+    2; block_len 64, Appendix B), gate, gated RMSNorm and out_proj per token.  Each
+    token row goes through the same per-token arithmetic as layer_step; the SSM state
+    is carried in fp64 through the prompt and stored once at the end.
+    res fp32 [B, T, D].  Returns the per-token residuals and the states after the
+    prompt."""
+    check_layer_shapes(d, lw, st)
+    E, N, G, H, P = d.d_inner, d.d_state, d.ngroups, d.nheads, d.headdim
+    C = E + 2 * G * N
+    if G != 1:
+        raise ValueError("layer_prefill follows one group")
+    res = np.asarray(res, dtype=np.float32)
+    Bsz, T, Dm = res.shape
+    if T < 1:
+        raise ValueError("a prompt has at least one token")
+    x_in = rmsnorm(res, lw.prenorm_w).astype(np.float16)
+    zx = project(x_in.reshape(Bsz * T, Dm), lw.inp).y.reshape(Bsz, T, -1)
+    z = zx[..., :E]
+    xc, conv_new = conv_seq(st.conv, zx[..., E:E + C], lw.conv_w, lw.conv_b)
+    xs = xc[..., :E].reshape(Bsz, T, H, P)
+    y, hT = ssd_scan(st.ssm, xs, xc[..., E:E + N], xc[..., E + N:E + 2 * N], zx[..., E + C:],
+                     lw.dt_bias, lw.A_log, lw.D, chunk=chunk)
+    y = y.reshape(Bsz, T, E)
+    g = (y * silu(z)).astype(np.float32).astype(np.float64)
+    x_out = rmsnorm(g, lw.gnorm_w).astype(np.float16)
+    out = project(x_out.reshape(Bsz * T, E), lw.out).y.reshape(Bsz, T, Dm)
+    res_new = (res.astype(np.float64) + out).astype(np.float32)
+    return PrefillTrace(res_new, conv_new, hT.astype(st.ssm.dtype), x_in, zx, xc, y, g, x_out)
+
+
+@dataclass
 class State:
     conv: np.ndarray         # fp32 [B, W-1, conv_dim]
     ssm: np.ndarray          # fp32 [B, H, P, N]
@@ -385,6 +455,25 @@ def quantize_embedding(embed16: np.ndarray):
     [-127, 127], both decided in fp32; an all-zero row gets codes 0 and scale 1.
     Returns (int8 codes [V, D], fp32 scales [V])."""
     return quantize_act(embed16)
+
+
+def model_prefill(tokens: np.ndarray, m, states, chunk: int = 64) -> ModelTrace:
+    """A whole prompt tokens [B, T] through the model in one pass (layer_prefill per
+    layer), then the final RMSNorm, tied LM head and greedy argmax of the LAST prompt
+    token.  Returns the logits and token of that position, the last token's residual
+    and every layer's state after the prompt."""
+    d = m.dims
+    tok = np.asarray(tokens, dtype=np.int64)
+    res = m.embed[tok].astype(np.float32)                            # [B, T, D]
+    new_states = []
+    for lw, st in zip(m.layers, states):
+        t = layer_prefill(res, lw, st, d, chunk=chunk)
+        res = t.res
+        new_states.append(State(t.conv, t.ssm))
+    last = res[:, -1, :]
+    xf = rmsnorm(last, m.normf_w)
+    logits = xf @ m.embed.astype(np.float64).T
+    return ModelTrace(logits, np.argmax(logits, axis=-1).astype(np.int32), last, new_states)
 
 
 def model_step(tokens: np.ndarray, m, states, emb_q=None) -> ModelTrace:

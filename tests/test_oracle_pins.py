@@ -719,3 +719,88 @@ def test_layer_wiring_by_hand(seed):
     np.testing.assert_allclose(t.ssm[0].astype(np.float64), ex["ssm"], rtol=1e-6, atol=1e-7)
     assert [float(v) for v in t.x_out[0]] == ex["xo"]
     np.testing.assert_allclose(t.res[0].astype(np.float64), ex["res"], rtol=1e-6, atol=1e-7)
+
+
+# ---------------------------------------------------------------- prompt pass (prefill)
+
+def test_conv_seq_matches_np_convolve_and_steps():
+    """The sequence conv against np.convolve per channel (zero initial state) and
+    against token-by-token conv_step with a nonzero initial state (inputs exactly
+    representable in fp32, so the step's fp32 state storage rounds nothing)."""
+    rng = np.random.default_rng(40)
+    T, Cc, W = 13, 6, 4
+    u = rng.normal(size=(1, T, Cc)).astype(np.float32).astype(np.float64)
+    w = rng.uniform(-0.5, 0.5, size=(Cc, W)).astype(np.float16)
+    b = rng.uniform(-0.5, 0.5, size=Cc).astype(np.float16)
+    xc, st = O.conv_seq(np.zeros((1, W - 1, Cc), np.float32), u, w, b)
+    for c in range(Cc):
+        pre = np.convolve(u[0, :, c], w[c, ::-1].astype(np.float64))[:T] + float(b[c])
+        np.testing.assert_allclose(xc[0, :, c], pre / (1 + np.exp(-pre)), rtol=1e-12, atol=1e-14)
+    assert np.array_equal(st[0], u[0, T - 3:].astype(np.float32))
+    st0 = rng.normal(size=(2, W - 1, Cc)).astype(np.float32)
+    u2 = rng.normal(size=(2, T, Cc)).astype(np.float32).astype(np.float64)
+    xs, sN = O.conv_seq(st0, u2, w, b)
+    s = st0
+    for t in range(T):
+        y, s = O.conv_step(s, u2[:, t], w, b)
+        np.testing.assert_allclose(xs[:, t], y, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(sN, s)
+    # a one-token prompt is exactly one conv step
+    y1, s1 = O.conv_seq(st0, u2[:, :1], w, b)
+    ys, ss = O.conv_step(st0, u2[:, 0], w, b)
+    assert np.array_equal(y1[:, 0], ys) and np.array_equal(s1, ss)
+
+
+def _prefill_layer(seed, T, batch=2, rank=8):
+    d = S.Dims(batch=batch, d_model=256, d_inner=512, nheads=8, headdim=64, d_state=16, rank=rank)
+    rng = np.random.default_rng(seed)
+    lw = S.gen_layer(rng, d)
+    st = S.zero_state(d)
+    st.conv[:] = rng.normal(size=st.conv.shape)
+    st.ssm[:] = rng.normal(size=st.ssm.shape)
+    res = rng.normal(size=(batch, T, d.d_model)).astype(np.float16).astype(np.float32)
+    return d, lw, st, res
+
+
+def test_layer_prefill_one_token_is_one_layer_step():
+    d, lw, st, res = _prefill_layer(41, 1)
+    p = O.layer_prefill(res, lw, st, d)
+    t = O.layer_step(res[:, 0], lw, st, d)
+    assert np.array_equal(p.res[:, 0], t.res)
+    assert np.array_equal(p.conv, t.conv) and np.array_equal(p.ssm, t.ssm)
+    assert np.array_equal(p.x_out[:, 0], t.x_out)
+
+
+@pytest.mark.parametrize("T,chunk", [(5, 64), (9, 4), (20, 8)])
+def test_layer_prefill_tracks_token_steps(T, chunk):
+    """A prompt in one pass against T layer steps: the only difference is where the
+    states are rounded (fp32 after every token step, once after the prompt), so the
+    two agree to fp32 rounding, far inside the 2e-3 bar; the chunk length does not
+    matter beyond rounding."""
+    d, lw, st, res = _prefill_layer(42 + T, T)
+    p = O.layer_prefill(res, lw, st, d, chunk=chunk)
+    s = st
+    for t in range(T):
+        tr = O.layer_step(res[:, t], lw, s, d)
+        s = O.State(tr.conv, tr.ssm)
+        assert np.max(np.abs(p.res[:, t] - tr.res)) <= 1e-4 * max(1.0, np.max(np.abs(tr.res)))
+    np.testing.assert_allclose(p.ssm, s.ssm, rtol=1e-4, atol=1e-5)
+    np.testing.assert_allclose(p.conv, s.conv, rtol=1e-6, atol=1e-6)
+
+
+def test_model_prefill_last_logits_track_token_steps():
+    d = S.LAYER_SMALL.with_batch(2)
+    rng = np.random.default_rng(43)
+    m = S.gen_model(rng, d, 2, 300)
+    toks = rng.integers(0, 300, size=(2, 7)).astype(np.int32)
+    p = O.model_prefill(toks, m, [O.State(*(lambda z: (z.conv, z.ssm))(S.zero_state(d))) for _ in m.layers])
+    states = [O.State(*(lambda z: (z.conv, z.ssm))(S.zero_state(d))) for _ in m.layers]
+    for t in range(7):
+        tr = O.model_step(toks[:, t], m, states)
+        states = tr.states
+    rms = np.sqrt(np.mean(tr.logits ** 2))
+    assert np.max(np.abs(p.logits - tr.logits)) <= 1e-4 * rms
+    for a, b in zip(p.states, states):
+        np.testing.assert_allclose(a.ssm, b.ssm, rtol=1e-4, atol=1e-5)
+    with pytest.raises(ValueError):
+        O.layer_prefill(np.zeros((2, 0, d.d_model), np.float32), m.layers[0], S.zero_state(d), d)
