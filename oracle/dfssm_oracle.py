@@ -284,8 +284,9 @@ def ssd_scan(h0: np.ndarray, x: np.ndarray, Bm: np.ndarray, Cm: np.ndarray, dt_r
         c1 = min(c0 + chunk, T)
         cs = np.cumsum(a[:, c0:c1], axis=1)                         # [B, L, H]
         L = c1 - c0
-        seg = np.exp(cs[:, :, None, :] - cs[:, None, :, :])         # [B, t, s, H]
-        seg = seg * np.tril(np.ones((L, L)))[None, :, :, None]
+        # decay from s+1 to t, only where s <= t (the upper triangle would overflow exp)
+        low = np.tril(np.ones((L, L), dtype=bool))[None, :, :, None]
+        seg = np.exp(np.where(low, cs[:, :, None, :] - cs[:, None, :, :], -np.inf))   # [B, t, s, H]
         CB = np.einsum("btn,bsn->bts", Cm[:, c0:c1], Bm[:, c0:c1])   # [B, t, s]
         xdt = x[:, c0:c1] * dt[:, c0:c1, :, None]                   # [B, L, H, P]
         y[:, c0:c1] = np.einsum("bts,btsh,bshp->bthp", CB, seg, xdt)

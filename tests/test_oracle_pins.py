@@ -804,3 +804,25 @@ def test_model_prefill_last_logits_track_token_steps():
         np.testing.assert_allclose(a.ssm, b.ssm, rtol=1e-4, atol=1e-5)
     with pytest.raises(ValueError):
         O.layer_prefill(np.zeros((2, 0, d.d_model), np.float32), m.layers[0], S.zero_state(d), d)
+
+
+def test_ssd_scan_strong_decay_stays_finite():
+    """A strongly decaying head over a 64-token chunk (cumulative log-decay near -10^3):
+    the scan must stay finite and equal the token recurrence (the state forgets its
+    start, the output follows the last tokens)."""
+    rng = np.random.default_rng(44)
+    Bsz, T, H, P, N = 1, 64, 2, 3, 4
+    h0 = rng.normal(size=(Bsz, H, P, N))
+    x = rng.normal(size=(Bsz, T, H, P))
+    Bm, Cm = rng.normal(size=(Bsz, T, N)), rng.normal(size=(Bsz, T, N))
+    dt_raw = np.full((Bsz, T, H), 3.0)
+    dt_bias = np.zeros(H, dtype=np.float32)
+    A_log = np.array([np.log(16.0), 0.0], dtype=np.float32)
+    D = np.ones(H, dtype=np.float32)
+    y, hT = O.ssd_scan(h0, x, Bm, Cm, dt_raw, dt_bias, A_log, D, chunk=64)
+    assert np.all(np.isfinite(y)) and np.all(np.isfinite(hT))
+    h = h0.copy()
+    for t in range(T):
+        yt, h = O.ssm_step(h, x[:, t], Bm[:, t], Cm[:, t], dt_raw[:, t], dt_bias, A_log, D, state_dtype=np.float64)
+        assert np.max(np.abs(y[:, t] - yt)) <= 1e-10 * max(1.0, np.max(np.abs(yt)))
+    assert np.max(np.abs(hT - h)) <= 1e-10 * max(1.0, np.max(np.abs(h)))
