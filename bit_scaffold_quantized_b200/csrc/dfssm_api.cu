@@ -412,6 +412,68 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   return launch_proj<EPI_RESID>(po, st);
 }
 
+// ---- prompt pass (prefill) --------------------------------------------------------
+
+// Workspace of a prompt pass: the decode layout for B*T token rows, then the
+// last-token residual rows [B][D] fp32 (model prefill).  `base` is the token-row
+// layout (its total marks where the extra region starts).
+struct PrefillLayout {
+  dfssm_dims rows;          // dims with batch = B * T
+  dfssm_ws_layout base;     // layout of the B*T token rows
+  size_t last;              // [B][D] fp32
+  size_t total;
+};
+
+PrefillLayout prefill_layout(const dfssm_dims* d, int T, int n_layer, int vocab) {
+  PrefillLayout P;
+  P.rows = *d;
+  P.rows.batch = d->batch * T;
+  layer_layout(&P.rows, n_layer, vocab, &P.base);
+  P.last = P.base.total_bytes;
+  P.total = align256(P.last + size_t(4) * d->batch * d->d_model);
+  return P;
+}
+
+int check_prefill(const dfssm_dims* d, int T) {
+  REQUIRE(T >= 1, DFSSM_ERR_INVALID_ARG, "prompt length T (%d) must be >= 1", T);
+  REQUIRE(size_t(d->batch) * T <= 65535, DFSSM_ERR_UNSUPPORTED_SHAPE, "batch * T (%lld) > 65535",
+          (long long)d->batch * T);
+  REQUIRE(ssd_smem_bytes(d->headdim, d->d_state) <= 200 * 1024, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "headdim * d_state (%d x %d) too large for the prompt-pass scan", d->headdim, d->d_state);
+  return DFSSM_OK;
+}
+
+// One layer over the prompt: six launches on one stream.
+int layer_prefill_launch(const dfssm_dims* d, int T, const dfssm_layer_weights* w, const dfssm_layer_state* s,
+                         float* res, const Bufs& b, cudaStream_t st) {
+  const int BT = d->batch * T, D = d->d_model, E = d->d_inner, r = d->rank, C = conv_dim(d);
+  int rc = launch_prologue<0>(D, r, BT, res, nullptr, w->prenorm_w, b.in, &w->in, st);
+  if (rc) return rc;
+  ProjArgs pa = proj_args(&w->in, r, BT, b.in);
+  pa.zx = b.zxbcdt;
+  if ((rc = launch_proj<EPI_ZX>(pa, st))) return rc;
+  PrefillArgs fa{};
+  fa.B = d->batch; fa.T = T; fa.H = d->nheads; fa.P = d->headdim; fa.N = d->d_state; fa.E = E; fa.C = C;
+  fa.in_rows = in_rows(d); fa.zx = b.zxbcdt; fa.conv_w = w->conv_w; fa.conv_b = w->conv_b;
+  fa.conv_state = s->conv_state; fa.xc = b.xc; fa.dt_bias = w->dt_bias; fa.A_log = w->A_log; fa.D = w->D;
+  fa.state = s->ssm_state; fa.state16 = d->ssm_state_dtype == 1; fa.g = b.g;
+  k_conv_seq<<<dim3((C + 255) / 256, d->batch), 256, 0, st>>>(fa);
+  CHECK_LAUNCH("k_conv_seq");
+  const int smem = int(ssd_smem_bytes(fa.P, fa.N));
+  if (fa.state16) {
+    cudaFuncSetAttribute(k_ssd<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    k_ssd<__half><<<dim3(fa.H, d->batch), kSsdThreads, smem, st>>>(fa);
+  } else {
+    cudaFuncSetAttribute(k_ssd<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    k_ssd<float><<<dim3(fa.H, d->batch), kSsdThreads, smem, st>>>(fa);
+  }
+  CHECK_LAUNCH("k_ssd");
+  if ((rc = launch_prologue<0>(E, r, BT, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
+  ProjArgs po = proj_args(&w->out, r, BT, b.out);
+  po.out = res;
+  return launch_proj<EPI_RESID>(po, st);
+}
+
 // ---- persistent whole-token kernel (batch 1) ------------------------------------
 
 
@@ -466,7 +528,6 @@ int max_active_clusters(int dev, int Q, int smem, bool spec) {
 }
 
 bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
-int ilog2(int v) { int l = 0; while ((1 << l) < v) ++l; return l; }
 
 // Whether (and how) one token of these dims runs as the persistent kernel.
 PPlan plan_persistent(const dfssm_dims* d) {
@@ -483,9 +544,7 @@ PPlan plan_persistent(const dfssm_dims* d) {
   if (N % 16 || H % 16) return no("d_state and nheads must be multiples of 16");
   if (R != 0 && (!pow2(R) || R < 8 || R > kPThreads)) return no("rank must be 0 or a power of two in [8, 512]");
   const int Q = kPMaxCluster;
-  const int SD = D / Q, SE = E / Q;
-  if (D % Q || E % Q || !pow2(SD) || !pow2(SE) || SD < 32 || SE < 32 || SD > 2 * kPThreads || SE > 2 * kPThreads)
-    return no("d_model / 8 and d_inner / 8 must be powers of two in [32, 512]");
+  if (D > kPMaxK || E > kPMaxK) return no("d_model and d_inner must be <= 4096");
   const int units = E / 16, out_tiles = D / 16, nbc = 2 * N / 16;
   p.sm = plan_smem(D, E, H, N, R, Q);
   const PSmem& m = p.sm;
@@ -531,6 +590,28 @@ struct EmbedRef {
   const float* s = nullptr;
 };
 
+#ifdef DFSSM_PHASE_TIMERS
+// Phase-timer build: per-CTA cycle sums of the token kernel in a file-scope device
+// array (the address is looked up per device and cached).
+static __device__ unsigned long long g_phase_cycles[kPlanSMs * kPhaseSlots];
+std::mutex g_phase_mu;
+void* g_phase_addr[64] = {};
+
+int phase_buffer(unsigned long long** out) {
+  const int dev = current_device();
+  REQUIRE(dev >= 0 && dev < 64, DFSSM_ERR_DEVICE, "device %d beyond the 64 supported", dev);
+  std::lock_guard<std::mutex> lock(g_phase_mu);
+  if (g_phase_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_phase_cycles);
+    if (e != cudaSuccess || p == nullptr) return fail(DFSSM_ERR_CUDA, "phase timers: %s", cudaGetErrorString(e));
+    g_phase_addr[dev] = p;
+  }
+  *out = static_cast<unsigned long long*>(g_phase_addr[dev]);
+  return DFSSM_OK;
+}
+#endif
+
 int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int vocab,
                       const dfssm_layer_weights* layers, const dfssm_layer_state* states, const EmbedRef& emb,
                       const uint16_t* normf_w, const int32_t* tok_in, int32_t* tok_out, float* logits,
@@ -544,8 +625,7 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.kg_in = D / kTileCols; a.kg_out = E / kTileCols;
   a.units = E / 16; a.grid = plan.grid; a.Q = plan.Q;
   a.n_bc_tiles = 2 * N / 16; a.dt_tile0 = (2 * E + 2 * N) / 16; a.out_tiles = D / 16;
-  a.SD = D / plan.Q; a.SE = E / plan.Q; a.lgSD = ilog2(a.SD); a.lgSE = ilog2(a.SE);
-  a.BSD = kDigits * (a.SD + 16) + 16; a.BSE = kDigits * (a.SE + 16) + 16;
+  a.SD = D / plan.Q; a.SE = E / plan.Q;
   a.layer_mode = residual != nullptr;
   a.sm = plan.sm;
   a.embed = emb.f16; a.embed_q = emb.q; a.embed_s = emb.s;
@@ -567,6 +647,12 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.d_x_out = b.out.x; a.d_xq_out = b.out.xq; a.d_sx_out = b.out.sx; a.d_acc_out = b.out.acc;
   a.d_u_out = b.out.u; a.d_xd_out = b.out.xd; a.d_xdsum_out = b.out.xdsum; a.d_res = b.res;
   for (int l = 0; l < n_layer; ++l) a.L[l] = player(layers[l], states[l]);
+#ifdef DFSSM_PHASE_TIMERS
+  {
+    int rc = phase_buffer(&a.phase);
+    if (rc) return rc;
+  }
+#endif
   const PKernel kfn = persistent_kernel(plan.spec, emb.q != nullptr);
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.sm.total);
   if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "persistent smem attribute: %s", cudaGetErrorString(e));
@@ -595,7 +681,31 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
 
 extern "C" {
 
-int dfssm_version(void) { return 100; }
+int dfssm_version(void) { return 200; }
+
+int dfssm_phase_timers(uint64_t* out, int max_entries, int reset) {
+#ifdef DFSSM_PHASE_TIMERS
+  REQUIRE(max_entries >= 0, DFSSM_ERR_INVALID_ARG, "max_entries must be >= 0");
+  unsigned long long* dev = nullptr;
+  int rc = phase_buffer(&dev);
+  if (rc) return rc;
+  const int n = std::min(max_entries, kPlanSMs * kPhaseSlots);
+  if (n > 0) {
+    REQUIRE(out != nullptr, DFSSM_ERR_INVALID_ARG, "out is NULL");
+    const cudaError_t e = cudaMemcpy(out, dev, sizeof(uint64_t) * n, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "phase timers: %s", cudaGetErrorString(e));
+  }
+  if (reset) {
+    const cudaError_t e = cudaMemset(dev, 0, sizeof(uint64_t) * kPlanSMs * kPhaseSlots);
+    if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "phase timers: %s", cudaGetErrorString(e));
+  }
+  ok();
+  return n;
+#else
+  (void)out; (void)max_entries; (void)reset;
+  return fail(DFSSM_ERR_NOT_BUILT, "this library was built without DFSSM_PHASE_TIMERS");
+#endif
+}
 
 int dfssm_model_decode_launches(const dfssm_dims* d, int n_layer, int vocab) {
   if (check_dims(d) || n_layer < 1 || n_layer > kMaxLayers || vocab < 1) return 0;
@@ -885,3 +995,86 @@ extern "C" int dfssm_proj_forward_noalloc(const dfssm_proj* p, int rank, int bat
   // nothing left by an earlier call needs clearing.
   return dfssm_proj_forward(p, rank, batch, x, y, ws, kNoAllocScratchBytes, stream);
 }
+
+// ---- prompt pass (prefill) ----------------------------------------------------------
+
+extern "C" {
+
+int dfssm_prefill_workspace_layout(const dfssm_dims* d, int T, int n_layer, int vocab, dfssm_ws_layout* out) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if ((rc = check_prefill(d, T))) return rc;
+  REQUIRE(out != nullptr, DFSSM_ERR_INVALID_ARG, "layout is NULL");
+  REQUIRE(n_layer >= 0 && vocab >= 0 && (n_layer == 0) == (vocab == 0), DFSSM_ERR_INVALID_ARG,
+          "n_layer and vocab must both be 0 (layer prefill) or both positive (model prefill)");
+  const PrefillLayout P = prefill_layout(d, T, n_layer, vocab);
+  *out = P.base;
+  out->total_bytes = P.total;
+  return ok();
+}
+
+size_t dfssm_prefill_workspace_bytes(const dfssm_dims* d, int T, int n_layer, int vocab) {
+  dfssm_ws_layout L;
+  if (dfssm_prefill_workspace_layout(d, T, n_layer, vocab, &L)) return 0;
+  return L.total_bytes;
+}
+
+int dfssm_layer_prefill(const dfssm_dims* d, int T, const dfssm_layer_weights* w, const dfssm_layer_state* s,
+                        float* residual, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if ((rc = check_prefill(d, T))) return rc;
+  if ((rc = check_layer(d, w, s, 0))) return rc;
+  REQUIRE_PTR(residual);
+  REQUIRE_PTR(ws);
+  const PrefillLayout P = prefill_layout(d, T, 0, 0);
+  REQUIRE(ws_bytes >= P.total, DFSSM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, P.total);
+  const Bufs b = bind(ws, P.base, &P.rows);
+  if ((rc = layer_prefill_launch(d, T, w, s, residual, b, static_cast<cudaStream_t>(stream)))) return rc;
+  return ok();
+}
+
+int dfssm_model_prefill(const dfssm_dims* d, int n_layer, int vocab, const uint16_t* embed,
+                        const dfssm_layer_weights* layers, const dfssm_layer_state* states, const uint16_t* normf_w,
+                        int T, const int32_t* tokens, int32_t* tok_out, float* logits, void* ws, size_t ws_bytes,
+                        void* stream) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  if ((rc = check_prefill(d, T))) return rc;
+  REQUIRE(n_layer >= 1 && n_layer <= kMaxLayers, DFSSM_ERR_INVALID_ARG, "n_layer (%d) must be in [1, %d]",
+          n_layer, kMaxLayers);
+  REQUIRE(vocab >= 1, DFSSM_ERR_INVALID_ARG, "vocab must be positive");
+  REQUIRE(layers != nullptr && states != nullptr, DFSSM_ERR_INVALID_ARG, "layers/states NULL");
+  for (int l = 0; l < n_layer; ++l)
+    if ((rc = check_layer(d, &layers[l], &states[l], l))) return rc;
+  REQUIRE_PTR(embed);
+  REQUIRE_PTR(normf_w);
+  REQUIRE_PTR(tokens);
+  REQUIRE_PTR(tok_out);
+  REQUIRE(logits == nullptr || aligned16(logits), DFSSM_ERR_MISALIGNED, "logits not 16-byte aligned");
+  REQUIRE_PTR(ws);
+  const PrefillLayout P = prefill_layout(d, T, n_layer, vocab);
+  REQUIRE(ws_bytes >= P.total, DFSSM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, P.total);
+  const Bufs b = bind(ws, P.base, &P.rows);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int B = d->batch, D = d->d_model;
+  k_embed<<<B * T, 256, 0, st>>>(embed, nullptr, nullptr, tokens, vocab, D, b.res, b.status);
+  CHECK_LAUNCH("k_embed");
+  for (int l = 0; l < n_layer; ++l)
+    if ((rc = layer_prefill_launch(d, T, &layers[l], &states[l], b.res, b, st))) return rc;
+  float* last = at<float>(ws, P.last);
+  k_last_rows<<<B, 256, 0, st>>>(b.res, T, D, last);
+  CHECK_LAUNCH("k_last_rows");
+  float* part_val = reinterpret_cast<float*>(b.scratch);
+  int* part_idx = reinterpret_cast<int*>(b.scratch + size_t(4) * B * kHeadBlocks);
+  HeadArgs h{};
+  h.D = D; h.vocab = vocab; h.batch = B; h.res = last; h.normf_w = normf_w;
+  h.embed = embed; h.logits = logits; h.part_val = part_val; h.part_idx = part_idx;
+  int nparts = kHeadBlocks;
+  if ((rc = launch_head(h, st, &nparts))) return rc;
+  k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, nparts, tok_out);
+  CHECK_LAUNCH("k_argmax");
+  return ok();
+}
+
+}  // extern "C"

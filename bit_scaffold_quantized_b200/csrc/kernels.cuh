@@ -273,7 +273,7 @@ __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueC
 
 // ------------------------------------------------------------------ projection
 
-enum { EPI_STORE = 0, EPI_RESID = 1, EPI_INPROJ = 2 };
+enum { EPI_STORE = 0, EPI_RESID = 1, EPI_INPROJ = 2, EPI_ZX = 3 };
 
 struct ProjArgs {
   int rows, K, rank, batch;
@@ -285,7 +285,7 @@ struct ProjArgs {
   const int* xdsum;       // int32 [batch][kDigits]
   const double* u;        // fp64 [batch][rank]
   float* out;             // EPI_STORE: fp32 [batch][rows]; EPI_RESID: fp32 residual [batch][rows]
-  double* zx;             // EPI_INPROJ: fp64 [batch][rows]
+  double* zx;             // EPI_INPROJ, EPI_ZX: fp64 [batch][rows]
   // EPI_INPROJ conv step over rows [conv_lo, conv_lo + conv_dim)
   int conv_lo, conv_dim;
   const uint16_t* conv_w;  // [conv_dim][4]
@@ -427,6 +427,8 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
           a.out[oi] = float(double(a.out[oi]) + y);
         } else if (EPI == EPI_STORE) {
           a.out[oi] = float(y);
+        } else if (EPI == EPI_ZX) {
+          a.zx[oi] = y;
         } else {
           a.zx[oi] = y;
           const int c = o - a.conv_lo;
@@ -757,6 +759,176 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     __syncthreads();   // buffer consumed
     if (tid == 0 && item + 2 * int(gridDim.x) < nitems) issue(item + 2 * int(gridDim.x), buf);
   }
+}
+
+// ------------------------------------------------------------------ prompt pass (prefill)
+//
+// A prompt of T tokens per batch row goes through a layer in one pass: the
+// projections run on all B*T token rows at once (k_prologue_cl, k_proj), the conv
+// runs along the sequence (k_conv_seq) and the selective SSM as the chunked scan of
+// Mamba-2's state space duality form ("Density Field State Space Models", Section 2;
+// block_len 64 as in Appendix B) in k_ssd.
+
+struct PrefillArgs {
+  int B, T, H, P, N, E, C, in_rows;   // batch, prompt length, heads, headdim, d_state, d_inner, conv_dim, in_proj rows
+  const double* zx;         // fp64 [B*T][in_rows]: [z | x B C | dt] of every prompt token
+  const uint16_t* conv_w;   // fp16 [C][4]
+  const uint16_t* conv_b;   // fp16 [C]
+  float* conv_state;        // fp32 [B][3][C], in/out
+  double* xc;               // fp64 [B*T][C] conv outputs after SiLU
+  const float* dt_bias;     // [H]
+  const float* A_log;       // [H]
+  const float* D;           // [H]
+  void* state;              // [B][H][P][N], fp32 or (state16) fp16, in/out
+  bool state16;
+  float* g;                 // fp32 [B*T][E] gated value y * silu(z)
+};
+
+// grid (ceil(C / 256), B), 256 threads: one thread per conv channel walks the prompt
+// with the three stored inputs in registers (the prompt's own inputs enter the
+// window at full precision; the state is stored back as fp32 at the end).
+__global__ void __launch_bounds__(256) k_conv_seq(PrefillArgs a) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x, b = blockIdx.y;
+  if (c >= a.C) return;
+  float* cs = a.conv_state + size_t(b) * 3 * a.C;
+  double s0 = cs[c], s1 = cs[a.C + c], s2 = cs[2 * a.C + c];
+  const uint2 wv = *reinterpret_cast<const uint2*>(a.conv_w + size_t(c) * 4);
+  const double w0 = h2d(uint16_t(wv.x & 0xffff)), w1 = h2d(uint16_t(wv.x >> 16));
+  const double w2 = h2d(uint16_t(wv.y & 0xffff)), w3 = h2d(uint16_t(wv.y >> 16));
+  const double bias = h2d(a.conv_b[c]);
+  for (int t = 0; t < a.T; ++t) {
+    const size_t row = size_t(b) * a.T + t;
+    const double x = a.zx[row * a.in_rows + a.E + c];   // conv rows follow the E z rows
+    double pre = bias;
+    pre = fma(w0, s0, pre);
+    pre = fma(w1, s1, pre);
+    pre = fma(w2, s2, pre);
+    pre = fma(w3, x, pre);
+    a.xc[row * a.C + c] = silu_d(pre);
+    s0 = s1;
+    s1 = s2;
+    s2 = x;
+  }
+  cs[c] = float(s0);
+  cs[a.C + c] = float(s1);
+  cs[2 * a.C + c] = float(s2);
+}
+
+constexpr int kSsdL = 64;             // chunk length (block_len)
+constexpr int kSsdThreads = 256;
+
+// Shared memory of k_ssd: the state (transposed, [N][P] fp64), the chunk's x [L][P]
+// fp64, B transposed [N][L] and C [L][N] (fp32 copies of the fp64 conv outputs),
+// M [L][L] fp64, and per-token step sizes, cumulative log-decays and weights.
+__host__ __device__ inline size_t ssd_smem_bytes(int P, int N) {
+  return size_t(8) * P * N + size_t(8) * kSsdL * P + size_t(4) * 2 * kSsdL * N + size_t(8) * kSsdL * kSsdL +
+         size_t(8) * 4 * kSsdL;
+}
+
+DFSSM_DEV double ld_state(const float* p) { return double(*p); }
+DFSSM_DEV double ld_state(const __half* p) { return h2d(__half_as_ushort(*p)); }
+DFSSM_DEV void st_state(float* p, double v) { *p = float(v); }
+DFSSM_DEV void st_state(__half* p, double v) { *p = __ushort_as_half(d2h(v)); }
+
+// grid (H, B), 256 threads: one CTA per (batch row, head) walks the prompt in chunks
+// of up to 64 tokens, the state carried in fp64 in shared memory.  Per chunk, with
+// dt_t = softplus(dt_raw_t + dt_bias), cs_t = sum_{r <= t} dt_r A (A = -exp(A_log)):
+//   M[t][s] = (C_t . B_s) exp(cs_t - cs_s) dt_s  (s <= t),
+//   y_t[p]  = sum_s M[t][s] x_s[p] + exp(cs_t) (C_t . h[p]) + D x_t[p],
+//   h[p][n] <- exp(cs_end) h[p][n] + sum_s exp(cs_end - cs_s) dt_s x_s[p] B_s[n],
+// and g = y silu(z) is stored in fp32.  The state is read once and written once
+// (rounded to its storage type).
+template <typename ST>
+__global__ void __launch_bounds__(kSsdThreads) k_ssd(PrefillArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int P = a.P, N = a.N, T = a.T, E = a.E, C = a.C;
+  double* hs = reinterpret_cast<double*>(smem);            // [N][P]
+  double* xs = hs + P * N;                                  // [L][P]
+  float* BsT = reinterpret_cast<float*>(xs + kSsdL * P);    // [N][L]
+  float* Cs = BsT + kSsdL * N;                              // [L][N]
+  double* M = reinterpret_cast<double*>(Cs + kSsdL * N);    // [L][L]
+  double* dts = M + kSsdL * kSsdL;                          // [L]
+  double* cs = dts + kSsdL;                                 // [L]
+  double* ecs = cs + kSsdL;                                 // [L] exp(cs_t)
+  double* wend = ecs + kSsdL;                               // [L] exp(cs_end - cs_s) dt_s
+  ST* gst = static_cast<ST*>(a.state) + (size_t(b) * a.H + h) * P * N;
+  for (int i = tid; i < P * N; i += blockDim.x) {
+    const int p = i / N, n = i % N;
+    hs[n * P + p] = ld_state(gst + i);
+  }
+  const double A = -exp(double(a.A_log[h])), Dh = double(a.D[h]), dtb = double(a.dt_bias[h]);
+  for (int c0 = 0; c0 < T; c0 += kSsdL) {
+    const int L = min(kSsdL, T - c0);
+    __syncthreads();   // the previous chunk is done with the buffers
+    for (int i = tid; i < L * P; i += blockDim.x) {
+      const int t = i / P, p = i % P;
+      xs[i] = a.xc[(size_t(b) * T + c0 + t) * C + h * P + p];
+    }
+    for (int i = tid; i < L * N; i += blockDim.x) {
+      const int t = i / N, n = i % N;
+      const double* row = a.xc + (size_t(b) * T + c0 + t) * C + E;
+      BsT[n * kSsdL + t] = float(row[n]);
+      Cs[t * N + n] = float(row[N + n]);
+    }
+    if (tid < L)
+      dts[tid] = softplus_d(a.zx[(size_t(b) * T + c0 + tid) * a.in_rows + E + C + h] + dtb);
+    __syncthreads();
+    if (tid == 0) {                 // cumulative log-decay, left to right
+      double acc = 0.0;
+      for (int t = 0; t < L; ++t) {
+        acc += dts[t] * A;
+        cs[t] = acc;
+      }
+    }
+    __syncthreads();
+    if (tid < L) {
+      ecs[tid] = exp(cs[tid]);
+      wend[tid] = exp(cs[L - 1] - cs[tid]) * dts[tid];
+    }
+    for (int i = tid; i < L * L; i += blockDim.x) {
+      const int t = i / L, s = i % L;
+      double v = 0.0;
+      if (s <= t) {
+        double cb = 0.0;
+        for (int n = 0; n < N; ++n) cb = fma(double(Cs[t * N + n]), double(BsT[n * kSsdL + s]), cb);
+        v = cb * exp(cs[t] - cs[s]) * dts[s];
+      }
+      M[t * kSsdL + s] = v;
+    }
+    __syncthreads();
+    for (int i = tid; i < L * P; i += blockDim.x) {
+      const int t = i / P, p = i % P;
+      double y = 0.0;
+      for (int s = 0; s <= t; ++s) y = fma(M[t * kSsdL + s], xs[s * P + p], y);
+      double yi = 0.0;
+      for (int n = 0; n < N; ++n) yi = fma(double(Cs[t * N + n]), hs[n * P + p], yi);
+      y = fma(ecs[t], yi, y);
+      y = fma(Dh, xs[t * P + p], y);
+      const size_t row = size_t(b) * T + c0 + t;
+      const double z = a.zx[row * a.in_rows + h * P + p];
+      a.g[row * E + h * P + p] = float(y * silu_d(z));
+    }
+    __syncthreads();
+    const double eend = exp(cs[L - 1]);
+    for (int i = tid; i < P * N; i += blockDim.x) {
+      const int n = i / P, p = i % P;
+      double acc = 0.0;
+      for (int s = 0; s < L; ++s) acc = fma(wend[s] * xs[s * P + p], double(BsT[n * kSsdL + s]), acc);
+      hs[i] = fma(eend, hs[i], acc);
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < P * N; i += blockDim.x) {
+    const int p = i / N, n = i % N;
+    st_state(gst + i, hs[n * P + p]);
+  }
+}
+
+// grid (B), 256 threads: dst[b] = src[b * T + T - 1] (rows of D floats).
+__global__ void k_last_rows(const float* __restrict__ src, int T, int D, float* __restrict__ dst) {
+  const int b = blockIdx.x;
+  for (int k = threadIdx.x; k < D; k += blockDim.x) dst[size_t(b) * D + k] = src[(size_t(b) * T + T - 1) * D + k];
 }
 
 // ------------------------------------------------------------------ embedding / LM head

@@ -9,44 +9,62 @@
 //     shared-memory traffic).  Full/empty mbarrier pairs hand the buffers over.
 // 16 warps, not 17, so that each thread may hold 128 registers.
 //
-// The layer is instruction-bound, so no CTA repeats work that its cluster can
-// split: every activation vector is prepared in Q slices (CTA of rank r owns
-// columns [r S, (r+1) S)), and the cluster all-gathers the slices' scaffold digit
-// planes, their integer sums and their max |x| with bulk copies from shared memory
-// into the other CTAs' shared memory (completion counted in bytes on the
-// receiver's mbarrier).  LoRA stage 1 is split the same way (each CTA multiplies
-// its slice of the int8 codes with its slice of every A row; the int32 partials
-// are all-gathered and summed in a fixed order, so the result is exact).
-//
-// Grid-wide exchanges (two per layer) go through "tagged words" in global memory:
-// 64-bit words holding 32 data bits and a 32-bit tag (launch epoch, layer,
-// exchange kind), stored and polled without fences; a word is valid exactly when
-// its tag matches.  Besides the values, each producer publishes the fp64 sum of
-// squares of its values, so a consumer of a slice still gets the full RMSNorm.
+// A layer is a chain of dependent steps whose cost is latency, not bytes (a layer
+// moves 8 MB, 1.25 us of HBM time on the whole chip).  Measured on the B200: a
+// grid-wide all-gather of tagged words costs ~1.5-1.8 us whether a CTA gathers a
+// slice or the whole vector, and a cluster all-to-all ~0.6 us.  So:
+//   * Two grid-wide exchanges per layer, the minimum for row-split projections (every
+//     output row needs the whole input vector): the residual after out_proj and the
+//     gated value after the SSM.  Every CTA gathers the WHOLE vector and prepares the
+//     projection's activation itself (RMSNorm, fp16 rounding, six digit planes, exact
+//     integer sum, max |x|): no slice all-gathers inside the cluster.
+//   * Grid-wide words are "tagged words": 64-bit words holding 32 data bits and a
+//     32-bit tag (launch epoch, layer, exchange kind), stored and polled without
+//     fences; a word is valid exactly when its tag matches.  Each thread keeps all of
+//     its words' loads in flight.  Producers also publish the fp64 sum of squares of
+//     their values, so every consumer gets the RMSNorm without another reduction.
+//   * Three cluster exchanges per layer, by st.async into every CTA of the cluster
+//     (completion counted in bytes on the receiver's mbarrier), each overlapped with
+//     tensor-core work: the int32 LoRA stage-1 partials of the in_proj (split over the
+//     cluster by columns) behind the in_proj's shared tiles, the shared rows (B and C
+//     after conv + SiLU, step sizes and decays, computed by every cluster for itself)
+//     behind the z/x tiles, the out_proj's LoRA partials behind the out_proj tiles.
 //
 // Per layer (B = 1), CTA c of cluster k, rank r:
-//   R    gather slice r of the residual and the sum-of-squares partials
-//   A    x = fp16(rmsnorm(res) w) on the slice: digit planes, sum, max -> cluster
-//   B    int8 codes of the slice, LoRA partials of all rows -> cluster
-//   -    exact int8 scaffold MMA on its in_proj tiles: the z and x rows of its own
-//        SSM channels plus its share of the cluster's "shared" tiles (all B/C rows
-//        and the dt rows of the cluster's heads; every cluster computes them)
-//   C    LoRA stage 2, conv step of its x channels; shared rows (B/C after conv +
-//        SiLU, raw dt) -> cluster
-//   G    SSM update of its own state rows, g = y silu(z) and its sum of squares
-//        published as fp32 / fp64 tagged words
-//   A'B' the gated RMSNorm, codes and LoRA stage 1 of the out_proj on slice r of g
-//   R'   out_proj rows of its tiles added to the residual and published
+//   R   gather the residual (all D words) and the sums of squares
+//   A   x = fp16(rmsnorm(res) w): six digit planes of all D columns, sum, max
+//   L   int8 codes of slice r, LoRA partials of all rows -> the cluster
+//   S   exact int8 scaffold MMA of this CTA's share of the cluster's shared tiles
+//       (all B/C rows and the dt rows of the cluster's heads); LoRA stage 2, conv
+//       step + SiLU (B/C), softplus and decay (dt) -> the cluster
+//   Z   scaffold MMA of the z and x rows of its own SSM channels, LoRA stage 2, conv
+//       step of its x channels, silu(z)
+//   G   SSM update of its own state rows, g = y silu(z) and its sum of squares
+//       published; gather all E gated values
+//   A'L' the gated RMSNorm, codes and LoRA stage 1 of the out_proj
+//   O   out_proj rows of its tiles added to the residual and published
 // Final: gather the residual, final RMSNorm, stream this CTA's LM-head rows,
 // publish (best logit, id); CTA 0 reduces to the greedy token.
 //
 // Every spin is bounded: a wait that gives up sets a status bit and an abort flag
 // that makes every CTA leave the token early; all CTAs of a cluster meet at a
 // final cluster barrier (after an abort, only once in-flight copies have had time
-// to land), so none exits while another may still write into it.
+// to land), so none exits while another may still write into it.  A launch that
+// finds the abort flag of an earlier call set does nothing (status value 1).
+//
+// Built with DFSSM_PHASE_TIMERS, thread 0 of every CTA adds the clock64 cycles of
+// each phase (summed over the layers) into PParams::phase[CTA][slot].
 #pragma once
 
 #include "common.cuh"
+
+// Built with DFSSM_NOINLINE, the large per-phase helpers are real calls (one copy
+// of each in the kernel's code) instead of being inlined at every use.
+#ifdef DFSSM_NOINLINE
+#define DFSSM_BIG __device__ __noinline__
+#else
+#define DFSSM_BIG DFSSM_DEV
+#endif
 
 namespace dfssm {
 
@@ -62,15 +80,24 @@ constexpr int kPMaxSharedRows = 16 * kPMaxSharedTiles;
 constexpr int kPMaxOutTiles = 2;                  // out_proj tiles per CTA
 constexpr int kPMaxCluster = 8;
 constexpr int kPMaxHeads = 4;                     // heads touched by one CTA's SSM rows
+constexpr int kPMaxK = 4096;                      // largest d_model / d_inner of the token kernel
 constexpr int kPSsmRows = (kPMaxUnits * 16 + kPWarps - 1) / kPWarps;   // SSM rows per compute warp
 constexpr long long kSpinLimit = 1LL << 22;       // polls before a wait gives up (seconds)
-constexpr int kHeadChunkRows = 7;                  // LM-head rows per chunk: 14 warps = 7 rows x 2 halves
+constexpr int kHeadChunkRows = 7;                 // LM-head rows per chunk: 14 warps = 7 rows x 2 halves
 constexpr int kHeadRingMax = 8;                   // LM-head chunk slots (all buffers free after the last layer)
+constexpr int kPhaseSlots = 32;                   // phase-timer slots per CTA (the last counts calls)
+constexpr int kPlanSMs = 256;                     // upper bound on CTAs of one launch (sizes the exchange scratch)
 
 // tagged-word exchange kinds
 enum { XR = 0, XG = 1, XHEAD = 2 };
 // cluster exchanges (one mbarrier each, one phase per layer)
-enum { EX_A_IN = 0, EX_B_IN = 1, EX_C = 2, EX_A_OUT = 3, EX_B_OUT = 4, EX_N = 5 };
+enum { EX_LIN = 0, EX_SH = 1, EX_LOUT = 2, EX_N = 3 };
+// phase-timer slots (cycles of thread 0, summed over the layers)
+enum {
+  PH_GATHER_R = 0, PH_WAIT_AB, PH_PREP_IN, PH_LORA_IN, PH_MMA_SH, PH_WAIT_LIN, PH_SHARED, PH_MMA_ZX, PH_ZX_EPI,
+  PH_WAIT_SH, PH_SSM, PH_GATHER_G, PH_WAIT_CD, PH_PREP_OUT, PH_LORA_OUT, PH_MMA_OUT, PH_WAIT_LOUT, PH_RESID,
+  PH_HEAD, PH_N
+};
 
 struct PLayer {
   const uint16_t* prenorm_w;
@@ -94,7 +121,7 @@ struct PSmem {
   int out_tiles, out_bq, out_alpha, out_sb, a_out, gnorm, sa_out;
   int cd_end;
   // working
-  int vs, xs, xqs, stg_a, asm_a, stg_b, rcv_b, yin, shr, stg_c, shst, u, resown;
+  int vfull, planes, xs, xqs, rcv, yin, shr, shst, u, resown;
   int ring_end, head_slots;       // LM-head chunk slots [0, head_slots) tile [0, ring_end)
   int part, full, misc;
   int total;
@@ -107,8 +134,7 @@ struct __align__(16) PParams {
   int units, grid, Q;            // SSM row units (E/16), CTAs, CTAs per cluster
   int n_bc_tiles, dt_tile0;      // 2N/16 and first dt tile index
   int out_tiles;                 // D/16
-  int SD, SE, lgSD, lgSE;        // slice widths (D/Q, E/Q, powers of two) and their log2
-  int BSD, BSE;                  // bytes of one slice block: 6 digit planes (+16 pad each) + sum + max
+  int SD, SE;                    // LoRA stage-1 column slices (D/Q, E/Q)
   int layer_mode;                // 1: residual in/out from `residual`, no embedding / head
   PSmem sm;
   // io
@@ -124,6 +150,7 @@ struct __align__(16) PParams {
   unsigned long long* x_g;       // E gated-value words
   unsigned long long* x_gs;      // 2 grid words: fp64 sum of squares of each CTA's gated values
   unsigned long long* x_head;    // 2 grid words
+  unsigned long long* phase;     // [grid][kPhaseSlots] phase cycles (timer builds), or null
   // diagnostics of the last layer (workspace regions of dfssm_ws_layout)
   uint16_t* d_x_in; int8_t* d_xq_in; float* d_sx_in; int* d_acc_in; double* d_u_in; int8_t* d_xd_in;
   int* d_xdsum_in; double* d_zx; double* d_xc; float* d_g; uint16_t* d_x_out; int8_t* d_xq_out;
@@ -131,23 +158,24 @@ struct __align__(16) PParams {
   PLayer L[kMaxLayers];
 };
 
-
-// Shared-memory plan of one shape (byte offsets); the host plans launches with the
-// same function, and the compile-time shape below bakes its result into the code.
-constexpr int kPlanSMs = 256;   // upper bound on CTAs of one launch (sizes the exchange scratch)
-
 __host__ __device__ constexpr int ptake(int& off, int bytes) {
   const int at = off;
   off = (off + (bytes > 16 ? bytes : 16) + 15) & ~15;
   return at;
 }
 
+// Digit-plane stride of a K-column activation: K + 64 bytes, so that the 16-byte
+// B-fragment loads of one quarter-warp (planes g, g + 1 at 16-byte offsets 0..48)
+// fall in 8 distinct 16-byte bank groups.
+__host__ __device__ constexpr int plane_stride(int K) { return K + 64; }
+
+// Shared-memory plan of one shape (byte offsets); the host plans launches with the
+// same function, and the compile-time shape below bakes its result into the code.
 __host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R, int Q) {
   PSmem m{};
   const int kg_in = D / kTileCols, kg_out = E / kTileCols;
   const int SD = D / Q, SE = E / Q;
-  const int BSD = kDigits * (SD + 16) + 16, BSE = kDigits * (SE + 16) + 16;
-  const int Smax = SD > SE ? SD : SE, BSmax = BSD > BSE ? BSD : BSE, R4 = R > 4 ? R : 4, R1 = R > 1 ? R : 1;
+  const int K = D > E ? D : E, Smax = SD > SE ? SD : SE, R4 = R > 4 ? R : 4, R1 = R > 1 ? R : 1;
   int off = 0;
   m.in_tiles = ptake(off, kPMaxInTiles * kg_in * 512);
   m.in_bq = ptake(off, kPMaxInTiles * 16 * R);
@@ -160,7 +188,7 @@ __host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R,
   m.sh_convb = ptake(off, kPMaxShared * 32);
   m.sh_cst = ptake(off, 3 * kPMaxShared * 64);
   m.a_in = ptake(off, R * SD);
-  m.prenorm = ptake(off, 2 * SD);
+  m.prenorm = ptake(off, 2 * D);
   m.sa_in = ptake(off, 2 * R);
   m.hd_dtb = ptake(off, 4 * H);
   m.hd_alog = ptake(off, 4 * H);
@@ -172,31 +200,28 @@ __host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R,
   m.out_alpha = ptake(off, kPMaxOutTiles * 32);
   m.out_sb = ptake(off, kPMaxOutTiles * 32);
   m.a_out = ptake(off, R * SE);
-  m.gnorm = ptake(off, 2 * SE);
+  m.gnorm = ptake(off, 2 * E);
   m.sa_out = ptake(off, 2 * R);
   m.cd_end = off;
-  m.vs = ptake(off, 4 * Smax);
+  m.vfull = ptake(off, 4 * K);
+  m.planes = ptake(off, kDigits * plane_stride(K));
   m.xs = ptake(off, 2 * Smax);
   m.xqs = ptake(off, Smax);
-  m.stg_a = ptake(off, BSmax);
-  m.asm_a = ptake(off, Q * BSmax);
-  m.stg_b = ptake(off, 4 * R4);
-  m.rcv_b = ptake(off, Q * 4 * R4);
+  m.rcv = ptake(off, 2 * Q * 4 * R4);          // [2][Q][R]: in_proj and out_proj LoRA partials
   m.yin = ptake(off, kPMaxInTiles * 16 * 8);
   m.shr = ptake(off, 2 * kPMaxSharedRows * 8);
-  m.stg_c = ptake(off, 2 * kPMaxShared * 16 * 8);
   m.shst = ptake(off, 3 * kPMaxShared * 16 * 4);
   m.u = ptake(off, 8 * R1);
   m.resown = ptake(off, kPMaxOutTiles * 16 * 4);
   // everything above is free once the last layer is done: the LM-head chunk ring
   // (grown to five chunks when that still leaves room for the rest)
   const int chunk = kHeadChunkRows * 2 * D;
-  if (off < 5 * chunk && 5 * chunk + 4 * (2 * kPlanSMs + 2 * D) + 8 * 1024 <= 200 * 1024) off = 5 * chunk;
+  if (off < 5 * chunk && 5 * chunk + 4 * (2 * kPlanSMs + D) + 8 * 1024 <= 200 * 1024) off = 5 * chunk;
   m.ring_end = off;
   m.head_slots = off / chunk;
   if (m.head_slots > kHeadRingMax) m.head_slots = kHeadRingMax;
   m.part = ptake(off, 16 * 16 * kDigits * 4);
-  m.full = ptake(off, 4 * (2 * kPlanSMs + 2 * D));
+  m.full = ptake(off, 4 * (2 * kPlanSMs + D));
   m.misc = ptake(off, kPMaxInTiles * 16 * 8);
   m.total = off;
   return m;
@@ -208,7 +233,7 @@ __host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R,
 struct ShapeAny {
   static constexpr bool kConst = false;
   static constexpr int D = 0, E = 0, H = 0, P = 0, N = 0, R = 0, Q = 0, C = 0, kg_in = 0, kg_out = 0;
-  static constexpr int SD = 0, SE = 0, lgSD = 0, lgSE = 0, BSD = 0, BSE = 0;
+  static constexpr int SD = 0, SE = 0;
   static constexpr int units = 0, n_bc_tiles = 0, dt_tile0 = 0, out_tiles = 0;
   static constexpr PSmem kPlan{};
 };
@@ -216,12 +241,10 @@ struct Shape2048 {
   static constexpr bool kConst = true;
   static constexpr int D = 2048, E = 4096, H = 64, P = 64, N = 128, R = 32, Q = 8, C = E + 2 * N;
   static constexpr int kg_in = D / kTileCols, kg_out = E / kTileCols;
-  static constexpr int SD = D / Q, SE = E / Q, lgSD = 8, lgSE = 9;
-  static constexpr int BSD = kDigits * (SD + 16) + 16, BSE = kDigits * (SE + 16) + 16;
+  static constexpr int SD = D / Q, SE = E / Q;
   static constexpr int units = E / 16, n_bc_tiles = 2 * N / 16, dt_tile0 = (2 * E + 2 * N) / 16, out_tiles = D / 16;
   static constexpr PSmem kPlan = plan_smem(D, E, H, N, R, Q);
 };
-static_assert((1 << Shape2048::lgSD) == Shape2048::SD && (1 << Shape2048::lgSE) == Shape2048::SE, "slice widths");
 
 // ------------------------------------------------------------------ primitives
 
@@ -233,14 +256,17 @@ DFSSM_DEV bool mbar_try_wait_cluster(uint64_t* bar, unsigned parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// Shared memory of this CTA -> shared memory of a CTA of the cluster (addresses
-// from cluster_map), completion counted on that CTA's mbarrier.
-DFSSM_DEV void bulk_s2c(uint32_t dst, const void* src, unsigned bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      :: "r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(bar) : "memory");
+// 4 / 8 bytes into the shared memory of a CTA of the cluster (addresses from
+// cluster_map), completion counted on that CTA's mbarrier.
+DFSSM_DEV void st_async_b32(uint32_t dst, uint32_t v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               :: "r"(dst), "r"(v), "r"(bar) : "memory");
 }
-// Named barrier 1 over the CTA's 16 warps.
+DFSSM_DEV void st_async_b64(uint32_t dst, unsigned long long v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];"
+               :: "r"(dst), "l"(v), "r"(bar) : "memory");
+}
+// Named barrier 1 over the CTA's 15 compute warps.
 DFSSM_DEV void csync() { asm volatile("bar.sync 1, %0;" :: "n"(kPThreads) : "memory"); }
 DFSSM_DEV bool csync_and(bool v) {
   unsigned r;
@@ -276,32 +302,35 @@ DFSSM_DEV void give_up(unsigned* status, unsigned* ctl, unsigned bit) {
 }
 
 // Compute warps: gather n1 tagged words from src1 into dst1 and n2 from src2 into
-// dst2 (32-bit payloads).  Returns false (after flagging) if a word did not arrive
-// within the spin limit.
-DFSSM_DEV bool tw_gather2(unsigned* status, unsigned* ctl, const unsigned long long* src1, int n1, uint32_t* dst1,
-                          const unsigned long long* src2, int n2, uint32_t* dst2, uint32_t tag, unsigned bit) {
+// dst2 (32-bit payloads).  Each thread keeps its (up to GW per pass) words' loads in
+// flight and re-polls only the missing ones.  Returns false (after flagging) if a
+// word did not arrive within the spin limit.
+template <int GW>
+DFSSM_BIG bool tw_gather(unsigned* status, unsigned* ctl, const unsigned long long* src1, int n1, uint32_t* dst1,
+                         const unsigned long long* src2, int n2, uint32_t* dst2, uint32_t tag, unsigned bit) {
   bool ok = true;
   const int n = n1 + n2;
-  for (int base = 0; base < n && ok; base += 4 * kPThreads) {
-    unsigned long long w[4];
-    int idx[4];
+  for (int base = 0; base < n && ok; base += GW * kPThreads) {
     unsigned pending = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      idx[i] = base + i * kPThreads + int(threadIdx.x);
-      if (idx[i] < n) pending |= 1u << i;
-    }
+    for (int i = 0; i < GW; ++i)
+      if (base + i * kPThreads + int(threadIdx.x) < n) pending |= 1u << i;
     long long spins = 0;
     while (pending) {
+      unsigned long long w[GW];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (pending & (1u << i)) w[i] = tw_load(idx[i] < n1 ? src1 + idx[i] : src2 + (idx[i] - n1));
+      for (int i = 0; i < GW; ++i) {
+        const int idx = base + i * kPThreads + int(threadIdx.x);
+        if (pending & (1u << i)) w[i] = tw_load(idx < n1 ? src1 + idx : src2 + (idx - n1));
+      }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < GW; ++i) {
+        const int idx = base + i * kPThreads + int(threadIdx.x);
         if ((pending & (1u << i)) && uint32_t(w[i] >> 32) == tag) {
-          *(idx[i] < n1 ? dst1 + idx[i] : dst2 + (idx[i] - n1)) = uint32_t(w[i]);
+          *(idx < n1 ? dst1 + idx : dst2 + (idx - n1)) = uint32_t(w[i]);
           pending &= ~(1u << i);
         }
+      }
       if (pending && ((++spins & 255) == 0) && (spins > kSpinLimit || aborted(ctl))) {
         give_up(status, ctl, bit);
         ok = false;
@@ -330,7 +359,8 @@ DFSSM_DEV bool mbar_wait_compute(unsigned* status, unsigned* ctl, uint64_t* bar,
   return csync_and(ok);
 }
 // Cluster exchange: thread 0 arms the barrier with the bytes the cluster sends to
-// this CTA and waits (bounded) for the phase, the compute warps agree, then every
+// this CTA (the sends may already have landed: the transaction count may run ahead
+// of the arm) and waits (bounded) for the phase, the compute warps agree, then every
 // thread takes the phase once more to acquire the cluster's writes for itself.
 DFSSM_DEV bool xwait(unsigned* status, unsigned* ctl, uint64_t* bar, unsigned bytes, unsigned parity, unsigned bit) {
   bool ok = true;
@@ -349,14 +379,6 @@ DFSSM_DEV bool xwait(unsigned* status, unsigned* ctl, uint64_t* bar, unsigned by
   if (ok) (void)mbar_try_wait_cluster(bar, parity);
   return ok;
 }
-// Send `bytes` of this CTA's staging buffer to offset `dst` (same layout in every
-// CTA) of every CTA of the cluster.  The writing threads have already fenced their
-// stores for the async proxy; the compute warps meet once so the copies see them.
-DFSSM_DEV void xsend(const void* stage, void* dst, unsigned bytes, uint64_t* bar, int Q) {
-  csync();
-  if (int(threadIdx.x) < Q && bytes > 0)
-    bulk_s2c(cluster_map(smem_u32(dst), threadIdx.x), stage, bytes, cluster_map(smem_u32(bar), threadIdx.x));
-}
 
 // Compute-warp reductions (fixed order, identical in every CTA).
 DFSSM_DEV double csum_d(double v, double* red) {
@@ -364,25 +386,22 @@ DFSSM_DEV double csum_d(double v, double* red) {
   v = warp_sum_d(v);
   if (lane == 0) red[warp] = v;
   csync();
-  double t = 0.0;
-#pragma unroll
-  for (int w = 0; w < kPWarps; ++w) t += red[w];
+  double t = lane < kPWarps ? red[lane] : 0.0;
+  t = warp_sum_d(t);
   csync();
   return t;
 }
-// Sum of the fp64 partials published by the grid's CTAs (word pairs), in CTA order,
-// by warp 0; every compute thread gets the result.
-DFSSM_DEV double sum_partials(const uint32_t* words, int G, double* red) {
+// Sum of the fp64 partials published by the grid's CTAs (word pairs), by every warp
+// for itself (a fixed butterfly: every lane of every warp gets the same value).
+DFSSM_DEV double sum_partials(const uint32_t* words, int G) {
   const int lane = threadIdx.x & 31;
-  if ((threadIdx.x >> 5) == 0) {
-    double t = 0.0;
-    for (int c = lane; c < G; c += 32) t += f64_of(words + 2 * c);
-    t = warp_sum_d(t);
-    if (lane == 0) red[0] = t;
-  }
-  csync();
-  const double v = red[0];
-  csync();
+  double t = 0.0;
+  for (int c = lane; c < G; c += 32) t += f64_of(words + 2 * c);
+  return warp_sum_d(t);
+}
+DFSSM_DEV long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
@@ -524,9 +543,9 @@ DFSSM_DEV void issue_group(unsigned char* sm, uint64_t* bar, F&& list) {
 }
 
 // The AB group of layer l: this CTA's in_proj tiles, their LoRA B rows and scales,
-// its slice of every LoRA A row and of the pre-norm weight, its SSM state rows and
+// its slice of every LoRA A row, the whole pre-norm weight, its SSM state rows and
 // the conv weights and state of its x channels and B/C rows.
-DFSSM_DEV void produce_ab(const PParams& a, const PWork& w, const PLayer& L, unsigned char* sm, uint64_t* full) {
+DFSSM_BIG void produce_ab(const PParams& a, const PWork& w, const PLayer& L, unsigned char* sm, uint64_t* full) {
   const PSmem& s = a.sm;
   issue_group(sm, full, [&](CopyList& c) {
     const int tile_bytes = a.kg_in * 512;
@@ -541,7 +560,7 @@ DFSSM_DEV void produce_ab(const PParams& a, const PWork& w, const PLayer& L, uns
       c.put(s.in_sb + slot * 32, (L.in_sB ? L.in_sB : L.in_alpha) + size_t(t0) * 16, n * 32);
       slot += n;
     }
-    c.put(s.prenorm, L.prenorm_w + size_t(w.r) * a.SD, 2 * a.SD);
+    c.put(s.prenorm, L.prenorm_w, 2 * a.D);
     c.put(s.state, L.ssm_state + size_t(16 * w.u0) * a.N, w.nu * 16 * a.N * 4);
     const int ch = 16 * w.u0;
     c.put(s.convw_x, L.conv_w + size_t(ch) * 4, w.nu * 128);
@@ -562,12 +581,12 @@ DFSSM_DEV void produce_ab(const PParams& a, const PWork& w, const PLayer& L, uns
 }
 
 // The CD group of layer l: this CTA's out_proj tiles with their LoRA B rows and
-// scales, its slice of every LoRA A row and of the gated-norm weight.
-DFSSM_DEV void produce_cd(const PParams& a, const PWork& w, const PLayer& L, unsigned char* sm, uint64_t* full) {
+// scales, its slice of every LoRA A row and the whole gated-norm weight.
+DFSSM_BIG void produce_cd(const PParams& a, const PWork& w, const PLayer& L, unsigned char* sm, uint64_t* full) {
   const PSmem& s = a.sm;
   issue_group(sm, full, [&](CopyList& c) {
     const int tile_bytes = a.kg_out * 512;
-    c.put(s.gnorm, L.gnorm_w + size_t(w.r) * a.SE, 2 * a.SE);
+    c.put(s.gnorm, L.gnorm_w, 2 * a.E);
     c.put(s.out_tiles, L.out_bits + size_t(w.o0) * a.kg_out * 128, w.no * tile_bytes);
     if (a.R) {
       c.put(s.out_bq, L.out_B + size_t(w.o0) * 16 * a.R, w.no * 16 * a.R);
@@ -581,42 +600,60 @@ DFSSM_DEV void produce_cd(const PParams& a, const PWork& w, const PLayer& L, uns
 
 // ------------------------------------------------------------------ activation prep
 
-// Slice preparation (elements tid, tid + kPThreads, ...): x = fp16((v rs) w) into
-// xs, its six digit planes into the staging block (plane stride S + 16), and the
-// block tail: the exact sum of the slice's X = x 2^24 (int64) and max |x| (fp16 bits).
-DFSSM_DEV void prep_slice(const float* v, const uint16_t* w, int S, double rs, unsigned char* stage, int* red,
-                          uint16_t* xs, uint16_t* x_diag, int8_t* xd_diag, int K_diag) {
+// Whole-vector preparation by the compute threads: x = fp16((v rs) w) for all K
+// columns, their six digit planes (plane stride PS), the fp16 bits of the LoRA slice
+// [s0, s0 + S) into xs, and -- identical in every thread -- the exact sum of X = x 2^24
+// and max |x| (fp16 bits).  Four consecutive columns per thread and pass, so each
+// plane gets one 32-bit store.  `red` holds 3 ints per warp; it is read after the
+// block barrier here, so the caller puts a barrier before its next use.
+DFSSM_BIG void prep_full(const float* v, const uint16_t* w, int K, double rs, unsigned char* planes, int PS, int s0,
+                         int S, uint16_t* xs, int* red, long long* xsum, unsigned* amax, uint16_t* x_diag,
+                         int8_t* xd_diag) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int PS = S + 16;
   const float rs32 = float(rs);
   int xh = 0, xl = 0;
   unsigned am = 0;
-  for (int i = tid; i < S; i += kPThreads) {
-    const uint32_t h = norm_fp16(v[i], rs, rs32, half_to_float_bits(w[i]));
-    uint32_t lo, hi;
-    digits_of(h, &lo, &hi);
-    xs[i] = uint16_t(h);
-    stage[i] = uint8_t(lo);
-    stage[PS + i] = uint8_t(lo >> 8);
-    stage[2 * PS + i] = uint8_t(lo >> 16);
-    stage[3 * PS + i] = uint8_t(lo >> 24);
-    stage[4 * PS + i] = uint8_t(hi);
-    stage[5 * PS + i] = uint8_t(hi >> 8);
-    const long long X = half_times_2p24_64(h);
-    xh += int(X >> 20);                      // X = xh 2^20 + xl, 0 <= xl < 2^20
-    xl += int(X & 0xfffff);
-    am = max(am, h & 0x7fffu);
+  for (int g = tid; g < K / 4; g += kPThreads) {
+    const float4 v4 = reinterpret_cast<const float4*>(v)[g];
+    const uint2 w4 = reinterpret_cast<const uint2*>(w)[g];
+    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+    const uint32_t ww[4] = {w4.x & 0xffffu, w4.x >> 16, w4.y & 0xffffu, w4.y >> 16};
+    uint32_t lo[4], hi[4], h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      h[e] = norm_fp16(vv[e], rs, rs32, half_to_float_bits(ww[e]));
+      digits_of(h[e], &lo[e], &hi[e]);
+      const long long X = half_times_2p24_64(h[e]);
+      xh += int(X >> 20);                    // X = xh 2^20 + xl, 0 <= xl < 2^20
+      xl += int(X & 0xfffff);
+      am = max(am, h[e] & 0x7fffu);
+    }
+    // plane d, columns 4g..4g+3: byte d of lo (d < 4) or of hi (d = 4, 5) of each column
+    const uint32_t p0 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0040), __byte_perm(lo[2], lo[3], 0x0040), 0x5410);
+    const uint32_t p1 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0051), __byte_perm(lo[2], lo[3], 0x0051), 0x5410);
+    const uint32_t p2 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0062), __byte_perm(lo[2], lo[3], 0x0062), 0x5410);
+    const uint32_t p3 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0073), __byte_perm(lo[2], lo[3], 0x0073), 0x5410);
+    const uint32_t p4 = __byte_perm(__byte_perm(hi[0], hi[1], 0x0040), __byte_perm(hi[2], hi[3], 0x0040), 0x5410);
+    const uint32_t p5 = __byte_perm(__byte_perm(hi[0], hi[1], 0x0051), __byte_perm(hi[2], hi[3], 0x0051), 0x5410);
+    uint32_t* pw = reinterpret_cast<uint32_t*>(planes) + g;
+    const int PW = PS / 4;
+    pw[0] = p0;
+    pw[PW] = p1;
+    pw[2 * PW] = p2;
+    pw[3 * PW] = p3;
+    pw[4 * PW] = p4;
+    pw[5 * PW] = p5;
+    const int c0 = 4 * g - s0;
+    if (c0 >= 0 && c0 < S)
+      *reinterpret_cast<uint2*>(xs + c0) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
     if (x_diag) {
-      x_diag[i] = uint16_t(h);
-      xd_diag[i] = int8_t(lo);
-      xd_diag[K_diag + i] = int8_t(lo >> 8);
-      xd_diag[2 * K_diag + i] = int8_t(lo >> 16);
-      xd_diag[3 * K_diag + i] = int8_t(lo >> 24);
-      xd_diag[4 * K_diag + i] = int8_t(hi);
-      xd_diag[5 * K_diag + i] = int8_t(hi >> 8);
+      *reinterpret_cast<uint2*>(x_diag + 4 * g) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+      const uint32_t pp[6] = {p0, p1, p2, p3, p4, p5};
+#pragma unroll
+      for (int d = 0; d < kDigits; ++d) *reinterpret_cast<uint32_t*>(xd_diag + size_t(d) * K + 4 * g) = pp[d];
     }
   }
-  // per thread |xh|, xl < 2^21: 32-lane sums fit int32; the warps' sums are combined in int64
+  // per thread |xh|, xl < 2^24: 32-lane sums fit int32; the warps' sums are combined in int64
   const int sh = __reduce_add_sync(0xffffffffu, xh);
   const int sl = __reduce_add_sync(0xffffffffu, xl);
   const unsigned amw = __reduce_max_sync(0xffffffffu, am);
@@ -626,40 +663,22 @@ DFSSM_DEV void prep_slice(const float* v, const uint16_t* w, int S, double rs, u
     red[3 * warp + 2] = int(amw);
   }
   csync();
-  if (tid == 0) {
-    long long sum = 0;
-    unsigned mx = 0;
-    for (int i = 0; i < kPWarps; ++i) {
-      sum += (static_cast<long long>(red[3 * i]) << 20) + red[3 * i + 1];
-      mx = max(mx, unsigned(red[3 * i + 2]));
-    }
-    *reinterpret_cast<long long*>(stage + kDigits * PS) = sum;
-    *reinterpret_cast<unsigned*>(stage + kDigits * PS + 8) = mx;
-  }
-  fence_async_smem();
-}
-
-// After the cluster's slice blocks arrived: exact sum of X over the whole vector
-// and its max |x| (fp16 bits), in a fixed order.
-DFSSM_DEV void slice_totals(const unsigned char* asmb, int Q, int S, int BS, long long* xsum, unsigned* amax) {
   long long s = 0;
   unsigned m = 0;
-  for (int q = 0; q < Q; ++q) {
-    const unsigned char* t = asmb + q * BS + kDigits * (S + 16);
-    s += *reinterpret_cast<const long long*>(t);
-    m = max(m, *reinterpret_cast<const unsigned*>(t + 8));
+  if (lane < kPWarps) {
+    s = (static_cast<long long>(red[3 * lane]) << 20) + red[3 * lane + 1];
+    m = unsigned(red[3 * lane + 2]);
   }
-  *xsum = s;
-  *amax = m;
+  *xsum = warp_sum_ll(s);
+  *amax = __reduce_max_sync(0xffffffffu, m);
 }
 
-// Digit-plane sums of the whole vector from the cluster's blocks (diagnostics only),
-// by all compute threads.
-DFSSM_DEV void plane_sums(const unsigned char* asmb, int Q, int S, int BS, int* red, int* out) {
+// Digit-plane sums of the whole vector (diagnostics only), by all compute threads.
+DFSSM_BIG void plane_sums(const unsigned char* planes, int PS, int K, int* red, int* out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int d = 0; d < kDigits; ++d) {
     int t = 0;
-    for (int i = tid; i < Q * S; i += kPThreads) t += int(int8_t(asmb[(i / S) * BS + d * (S + 16) + i % S]));
+    for (int i = tid; i < K; i += kPThreads) t += int(int8_t(planes[d * PS + i]));
     t = __reduce_add_sync(0xffffffffu, t);
     if (lane == 0) red[warp] = t;
     csync();
@@ -672,11 +691,12 @@ DFSSM_DEV void plane_sums(const unsigned char* asmb, int Q, int S, int BS, int* 
   }
 }
 
-// int8 codes of the slice (from its fp16 bits), then LoRA stage-1 partials of the
-// slice for all R rows: stage[j] = sum_k A[j][k] q[k] over the slice, fenced for the
-// async proxy.
-DFSSM_DEV void codes_and_lora_partials(const uint16_t* xs, int S, float sx, float rcp, bool nonzero, int8_t* xqs,
-                                       const int8_t* Aslice, int R, int* stage, int8_t* xq_diag) {
+// int8 codes of the LoRA slice (from its fp16 bits), then the slice's LoRA stage-1
+// partials of all R rows, sum_k A[j][k] q[k], sent by st.async to slot r of every
+// CTA of the cluster (Q x R int32 land on each CTA's barrier `bar`).
+DFSSM_BIG void codes_and_lora_send(const uint16_t* xs, int S, float sx, float rcp, bool nonzero, int8_t* xqs,
+                                   const int8_t* Aslice, int R, int r, int Q, int* rcv, uint64_t* bar,
+                                   int8_t* xq_diag) {
   const int tid = threadIdx.x;
   for (int i = tid; i < S; i += kPThreads) {
     const int q = nonzero ? quant_code_bits(half_to_float_bits(xs[i]), sx, rcp) : 0;
@@ -686,8 +706,9 @@ DFSSM_DEV void codes_and_lora_partials(const uint16_t* xs, int S, float sx, floa
   csync();
   if (R > 0) {
     // 16 lanes per row, two rows per warp; rows beyond the first pass of the warps
-    // come round again
+    // come round again (R is even, so both halves of a warp run the same passes)
     const int half = (tid & 31) >> 4, sub = tid & 15;
+    const uint32_t dst0 = smem_u32(rcv + r * R), bar0 = smem_u32(bar);
     for (int j = 2 * (tid >> 5) + half; j < R; j += 2 * kPWarps) {
       const int* A4 = reinterpret_cast<const int*>(Aslice + j * S);
       const int* q4 = reinterpret_cast<const int*>(xqs);
@@ -695,16 +716,14 @@ DFSSM_DEV void codes_and_lora_partials(const uint16_t* xs, int S, float sx, floa
       for (int i = sub; i < S / 4; i += 16) acc = __dp4a(A4[i], q4[i], acc);
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (sub == 0) {
-        stage[j] = acc;
-        fence_async_smem();
-      }
+      // lanes 0..Q-1 of the half-warp each send the row's partial to one CTA
+      if (sub < Q) st_async_b32(cluster_map(dst0 + 4 * j, sub), uint32_t(acc), cluster_map(bar0, sub));
     }
   }
 }
 
 // Sum of the cluster's LoRA partials (fixed order) -> u[j] = acc sA[j] sx in fp64.
-DFSSM_DEV void lora_finish(const int* rcv, int Q, int R, const uint16_t* sA, float sx, double* u, int* acc_diag,
+DFSSM_BIG void lora_finish(const int* rcv, int Q, int R, const uint16_t* sA, float sx, double* u, int* acc_diag,
                            double* u_diag) {
   const int j = threadIdx.x;
   if (j < R) {
@@ -720,42 +739,38 @@ DFSSM_DEV void lora_finish(const int* rcv, int Q, int R, const uint16_t* sA, flo
   csync();
 }
 
-// LoRA stage 2 for `nrows` rows: out[r] = sum_j B[r][j] u[j] in fp64, one thread
-// per row with four interleaved partial sums (R is a multiple of 8).
-DFSSM_DEV void lora2_rows(const int8_t* Bq, int nrows, const double* u, int R, double* out) {
-  for (int r = threadIdx.x; r < nrows; r += kPThreads) {
-    const int* b4 = reinterpret_cast<const int*>(Bq + r * R);
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int j4 = 0; j4 < R / 4; ++j4) {
-      const int v = b4[j4];
+// LoRA stage 2 of one row: sum_j B[j] u[j] in fp64, four interleaved partial sums
+// (R is a multiple of 8).
+DFSSM_DEV double lora2_row(const int8_t* Brow, const double* u, int R) {
+  const int* b4 = reinterpret_cast<const int*>(Brow);
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int j4 = 0; j4 < R / 4; ++j4) {
+    const int v = b4[j4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[e] = fma(double(int8_t(v >> (8 * e))), u[4 * j4 + e], acc[e]);
-    }
-    out[r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    for (int e = 0; e < 4; ++e) acc[e] = fma(double(int8_t(v >> (8 * e))), u[4 * j4 + e], acc[e]);
   }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 // Exact scaffold MMA over `ntile` tiles (smem, kg groups each), split into units
 // (tile, kgroup chunk); int32 partials to part[unit][16][kDigits].  The activation
-// digit planes come from the cluster's slice blocks: column k lies in block
-// k >> lgS at offset k & (S - 1) of each plane (stride S + 16).  Register q of the
-// A fragment of product s is word q of the lane's sign vector masked to bits
-// s, s + 8, s + 16, s + 24: unsigned bytes 0 or 2^s, one instruction per register.
-// Product s accumulates into its own set, 2^s times its 0/1 sums (|sum| < 2^27),
-// and the sets are recombined exactly with right shifts.  One 16-byte load per
-// plane row gives the B fragments of products 2m and 2m + 1.  Returns the chunks
-// per tile.
-DFSSM_DEV int scaffold_mma(const unsigned char* tiles, int ntile, int kg, const unsigned char* asmb, int lgS, int BS,
+// digit planes are whole-vector planes (stride PS).  Register q of the A fragment of
+// product s is word q of the lane's sign vector masked to bits s, s + 8, s + 16,
+// s + 24: unsigned bytes 0 or 2^s, one instruction per register.  Product s
+// accumulates into its own set, 2^s times its 0/1 sums (|sum| < 2^27), and the sets
+// are recombined exactly with right shifts.  One 16-byte load per plane row gives
+// the B fragments of products 2m and 2m + 1; the next k-group's words and planes are
+// loaded while the current one's products issue.  Returns the chunks per tile.
+DFSSM_BIG int scaffold_mma(const unsigned char* tiles, int ntile, int kg, const unsigned char* planes, int PS,
                            int* part) {
   constexpr int nw = kPWarps;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  int nchunk = nw / ntile;
+  int nchunk = nw / max(ntile, 1);
   if (nchunk < 1) nchunk = 1;
   if (nchunk > kg) nchunk = kg;
-  const int S = 1 << lgS;
   const int nunits = ntile * nchunk;
-  const unsigned char* dbase = asmb + (g < kDigits ? g : 0) * (S + 16);
+  const unsigned char* dbase = planes + (g < kDigits ? g : 0) * PS + 16 * t;
   for (int unit = warp; unit < nunits; unit += nw) {
     const int ti = unit / nchunk, ci = unit % nchunk;
     const int kg_lo = ci * kg / nchunk, kg_hi = (ci + 1) * kg / nchunk;
@@ -763,22 +778,32 @@ DFSSM_DEV int scaffold_mma(const unsigned char* tiles, int ntile, int kg, const 
 #pragma unroll
     for (int s = 0; s < 8; ++s) acc[s][0] = acc[s][1] = acc[s][2] = acc[s][3] = 0;
     const uint4* tw = reinterpret_cast<const uint4*>(tiles + size_t(ti) * kg * 512);
+    uint4 wv = tw[kg_lo * 32 + lane];
+    uint4 bq[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      bq[m] = g < kDigits ? *reinterpret_cast<const uint4*>(dbase + kg_lo * kTileCols + 64 * m) : make_uint4(0, 0, 0, 0);
     for (int kgi = kg_lo; kgi < kg_hi; ++kgi) {
-      const uint4 wv = tw[kgi * 32 + lane];
+      uint4 wn = wv, bn[4] = {bq[0], bq[1], bq[2], bq[3]};
+      if (kgi + 1 < kg_hi) {
+        wn = tw[(kgi + 1) * 32 + lane];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          if (g < kDigits) bn[m] = *reinterpret_cast<const uint4*>(dbase + (kgi + 1) * kTileCols + 64 * m);
+      }
       const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        // 16 aligned columns never straddle a slice block (S >= 16)
-        const int k0 = kgi * kTileCols + 64 * m + 16 * t;
-        uint4 bq = make_uint4(0, 0, 0, 0);
-        if (g < kDigits) bq = *reinterpret_cast<const uint4*>(dbase + (k0 >> lgS) * BS + (k0 & (S - 1)));
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const uint32_t mask = 0x01010101u << (2 * m + e);
           const uint32_t af[4] = {words[0] & mask, words[1] & mask, words[2] & mask, words[3] & mask};
-          mma_u8s8_16832(acc[2 * m + e], af, e ? bq.z : bq.x, e ? bq.w : bq.y);
+          mma_u8s8_16832(acc[2 * m + e], af, e ? bq[m].z : bq[m].x, e ? bq[m].w : bq[m].y);
         }
       }
+      wv = wn;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) bq[m] = bn[m];
     }
     int tot[4];
 #pragma unroll
@@ -803,7 +828,7 @@ DFSSM_DEV int scaffold_mma(const unsigned char* tiles, int ntile, int kg, const 
 
 // Scaffold value (without alpha) of row r of tile ti from the unit partials:
 // sum_k s_k x_k = 2^-24 (2 sum_d 256^d Q_d - sum_k X_k), exact in int64.
-DFSSM_DEV double tile_row_value(const int* part, int ti, int nchunk, int r, long long xsum) {
+DFSSM_BIG double tile_row_value(const int* part, int ti, int nchunk, int r, long long xsum) {
   long long S = 0;
 #pragma unroll
   for (int d = kDigits - 1; d >= 0; --d) {
@@ -812,6 +837,17 @@ DFSSM_DEV double tile_row_value(const int* part, int ti, int nchunk, int r, long
     S = S * 256 + s;
   }
   return double(2 * S - xsum) * (1.0 / 16777216.0);
+}
+
+// Pre-activation of one conv channel: bias + taps 0..2 on the stored inputs (oldest
+// first) + tap 3 on the new input, in fp64.
+DFSSM_DEV double conv_step_d(const uint16_t* cw, double cb, float c0, float c1, float c2, double xv) {
+  double pre = cb;
+  pre = fma(h2d(cw[0]), double(c0), pre);
+  pre = fma(h2d(cw[1]), double(c1), pre);
+  pre = fma(h2d(cw[2]), double(c2), pre);
+  pre = fma(h2d(cw[3]), xv, pre);
+  return pre;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -827,7 +863,9 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   __shared__ __align__(8) uint64_t xbars[EX_N];
   __shared__ double redd[kPWarps];
   __shared__ int redi[3 * kPWarps];
+  __shared__ int redo[3 * kPWarps];
   __shared__ double ssw[kPWarps * kPSsmRows];
+  __shared__ int s_stale;
   for (int i = threadIdx.x; i < int(sizeof(PParams) / 16); i += blockDim.x)
     reinterpret_cast<uint4*>(pbuf)[i] = reinterpret_cast<const uint4*>(&pa)[i];
   const PParams& a = *reinterpret_cast<const PParams*>(pbuf);
@@ -837,8 +875,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   const int D = kC ? SH::D : pa.D, E = kC ? SH::E : pa.E, P = kC ? SH::P : pa.P, N = kC ? SH::N : pa.N;
   const int R = kC ? SH::R : pa.R, C = kC ? SH::C : pa.C, Q = kC ? SH::Q : pa.Q;
   const int kg_in = kC ? SH::kg_in : pa.kg_in, kg_out = kC ? SH::kg_out : pa.kg_out;
-  const int SD = kC ? SH::SD : pa.SD, SE = kC ? SH::SE : pa.SE, lgSD = kC ? SH::lgSD : pa.lgSD;
-  const int lgSE = kC ? SH::lgSE : pa.lgSE, BSD = kC ? SH::BSD : pa.BSD, BSE = kC ? SH::BSE : pa.BSE;
+  const int SD = kC ? SH::SD : pa.SD, SE = kC ? SH::SE : pa.SE;
 #define PSM(f) (kC ? SH::kPlan.f : pa.sm.f)
   uint64_t* full_ab = &bars[0];
   uint64_t* empty_ab = &bars[1];
@@ -846,7 +883,6 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   uint64_t* empty_cd = &bars[3];
   uint64_t* full_h = &bars[4];
   uint64_t* empty_h = &bars[4 + kHeadRingMax];
-  __shared__ int s_stale;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4 + 2 * kHeadRingMax; ++i) mbar_init(&bars[i], 1);
     for (int i = 0; i < EX_N; ++i) mbar_init(&xbars[i], 1);
@@ -935,28 +971,49 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
     auto tag = [&](int l, int kind) { return tagbase + uint32_t(l * 8 + kind + 1); };
     unsigned* status = a.status;
     unsigned* ctl = a.ctl;
+#ifdef DFSSM_PHASE_TIMERS
+    // slots PH_N, PH_N + 1: the in-side preparation and the z/x MMA repeated with
+    // their code already cached; PH_N + 2: the barriers around the repeat (excluded)
+    long long ptime[PH_N + 3];
+#pragma unroll
+    for (int i = 0; i < PH_N + 3; ++i) ptime[i] = 0;
+    long long tlast = clock64();
+#define PT(k)                              \
+  do {                                     \
+    if (tid == 0) {                        \
+      const long long t_ = clock64();      \
+      ptime[k] += t_ - tlast;              \
+      tlast = t_;                          \
+    }                                      \
+  } while (0)
+#else
+#define PT(k) \
+  do {        \
+  } while (0)
+#endif
 
-    float* vs = sp<float>(sm, PSM(vs));                 // this CTA's slice of the residual / gated value
-    uint16_t* xs = sp<uint16_t>(sm, PSM(xs));          // fp16 bits of this CTA's slice
+    float* vfull = sp<float>(sm, PSM(vfull));          // the whole residual / gated value
+    unsigned char* planes = sm + PSM(planes);          // six digit planes of the activation
+    uint16_t* xs = sp<uint16_t>(sm, PSM(xs));          // fp16 bits of this CTA's LoRA slice
     int8_t* xqs = sp<int8_t>(sm, PSM(xqs));
-    unsigned char* stg_a = sm + PSM(stg_a);            // own slice block
-    unsigned char* asm_a = sm + PSM(asm_a);            // the cluster's slice blocks
-    int* stg_b = sp<int>(sm, PSM(stg_b));              // own LoRA partials
-    int* rcv_b = sp<int>(sm, PSM(rcv_b));              // the cluster's LoRA partials
+    int* rcv_in = sp<int>(sm, PSM(rcv));               // [Q][R] the cluster's in_proj LoRA partials
+    int* rcv_out = rcv_in + Q * (R > 4 ? R : 4);       // [Q][R] the cluster's out_proj LoRA partials
     int* part = sp<int>(sm, PSM(part));
     double* yin = sp<double>(sm, PSM(yin));            // [kPMaxInTiles * 16] in_proj outputs of own tiles (slot order)
     double* shr = sp<double>(sm, PSM(shr));            // [kPMaxSharedRows] the cluster's shared rows
-    double* stg_c = sp<double>(sm, PSM(stg_c));        // own shared rows
     float* shst = sp<float>(sm, PSM(shst));            // [3][kPMaxShared * 16] new conv state of own B/C rows
     double* u = sp<double>(sm, PSM(u));                // [R] LoRA stage-1 outputs
     float* resown = sp<float>(sm, PSM(resown));        // residual of own out_proj rows
-    double* lo = sp<double>(sm, PSM(misc));            // LoRA stage-2 sums of own rows
-    uint32_t* scratch32 = sp<uint32_t>(sm, PSM(full));
+    uint32_t* scratch32 = sp<uint32_t>(sm, PSM(full)); // gathered partial words, then the head's residual
     const int zslot = 0, xslot = w.nu, shslot = 2 * w.nu;
     const int SHR = kPMaxShared * 16;
-    const int r0D = w.r * SD, r0E = w.r * SE;   // this CTA's slices
+    const int PSD = plane_stride(D), PSE = plane_stride(E);
+    const int tile_in = kg_in * 512;
+    const uint32_t shr_s = smem_u32(shr), xsh_s = smem_u32(&xbars[EX_SH]);
+    // this CTA's shared rows start at cluster shared row 16 s0 + 16 (s0 - nbc)+
+    const int shr_own = 16 * w.s0 + 16 * max(w.s0 - w.nbc, 0);
 
-    // ---- layer-0 residual: own slice, own out rows, sum of squares (every CTA)
+    // ---- layer-0 residual: the whole vector and its sum of squares (every CTA)
     double ss;
     {
       int t = 0;
@@ -970,17 +1027,14 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       const uint16_t* erow = a.embed + size_t(t) * D;
       const int8_t* eqrow = q8 ? a.embed_q + size_t(t) * D : nullptr;
       const float es = q8 ? a.embed_s[t] : 0.f;
-      auto res0 = [&](int k) {
-        return a.layer_mode ? a.residual[k] : q8 ? es * float(eqrow[k]) : h2f(erow[k]);
-      };
       double acc = 0.0;
       for (int k = tid; k < D; k += kPThreads) {
-        const double v = double(res0(k));
-        acc = fma(v, v, acc);
+        const float v = a.layer_mode ? a.residual[k] : q8 ? es * float(eqrow[k]) : h2f(erow[k]);
+        vfull[k] = v;
+        acc = fma(double(v), double(v), acc);
       }
-      for (int k = tid; k < SD; k += kPThreads) vs[k] = res0(r0D + k);
-      if (tid < w.no * 16) resown[tid] = res0(w.o0 * 16 + tid);
       ss = csum_d(acc, redd);
+      if (tid < w.no * 16) resown[tid] = vfull[w.o0 * 16 + tid];
     }
 
     bool alive = true;
@@ -991,111 +1045,135 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       const bool wdiag = diag && w.c == 0;
       const unsigned par = unsigned(l) & 1u;
 
-      // ---- R: own slice of the residual and the sums of squares
+      // ---- R: the whole residual and the sums of squares
       if (l > 0) {
-        if (!tw_gather2(status, ctl, a.x_r + r0D, SD, reinterpret_cast<uint32_t*>(vs), a.x_rs, 2 * G, scratch32,
-                        tag(l, XR), 4u)) {
+        if (!tw_gather<(2048 + 2 * 128 + kPThreads - 1) / kPThreads>(
+                status, ctl, a.x_r, D, reinterpret_cast<uint32_t*>(vfull), a.x_rs, 2 * G, scratch32, tag(l, XR),
+                4u)) {
           alive = false;
           break;
         }
-        ss = sum_partials(scratch32, G, redd);
+        ss = sum_partials(scratch32, G);
       }
+      PT(PH_GATHER_R);
       if (!mbar_wait_compute(status, ctl, full_ab, par, 8u)) { alive = false; break; }
+      PT(PH_WAIT_AB);
 
-      // ---- A: pre-norm on the slice -> the cluster
+      // ---- A: pre-norm of the whole vector, digit planes, sum, max
       const double rs_in = 1.0 / sqrt(ss / double(D) + kEpsD);
-      prep_slice(vs, sp<uint16_t>(sm, PSM(prenorm)), SD, rs_in, stg_a, redi, xs, cdiag ? a.d_x_in + r0D : nullptr,
-                 cdiag ? a.d_xd_in + r0D : nullptr, D);
-      xsend(stg_a, asm_a + w.r * BSD, unsigned(BSD), &xbars[EX_A_IN], Q);
-      if (!xwait(status, ctl, &xbars[EX_A_IN], unsigned(Q * BSD), par, 16u)) { alive = false; break; }
       long long xsum_in;
       unsigned amax_in;
-      slice_totals(asm_a, Q, SD, BSD, &xsum_in, &amax_in);
+      prep_full(vfull, sp<uint16_t>(sm, PSM(prenorm)), D, rs_in, planes, PSD, w.r * SD, SD, xs, redi, &xsum_in,
+                &amax_in, wdiag ? a.d_x_in : nullptr, a.d_xd_in);
       const float am_in = half_to_float_bits(amax_in);
       const float sx_in = am_in > 0.f ? __fdiv_rn(am_in, 127.f) : 1.f;
+      PT(PH_PREP_IN);
+#ifdef DFSSM_PHASE_TIMERS
+      // the same preparation once more, its code now in the instruction caches
+      // (idempotent: same inputs, same outputs)
+      csync();
+      PT(PH_N + 2);
+      prep_full(vfull, sp<uint16_t>(sm, PSM(prenorm)), D, rs_in, planes, PSD, w.r * SD, SD, xs, redi, &xsum_in,
+                &amax_in, nullptr, nullptr);
+      PT(PH_N);
+      csync();
+      PT(PH_N + 2);
+#endif
+      // ---- L: codes and LoRA partials of the slice -> the cluster
+      codes_and_lora_send(xs, SD, sx_in, __frcp_rn(sx_in), am_in > 0.f, xqs, sp<int8_t>(sm, PSM(a_in)), R, w.r, Q,
+                          rcv_in, &xbars[EX_LIN], cdiag ? a.d_xq_in + w.r * SD : nullptr);
       if (wdiag) {
         if (tid == 0) *a.d_sx_in = sx_in;
-        plane_sums(asm_a, Q, SD, BSD, redi, a.d_xdsum_in);
+        plane_sums(planes, PSD, D, redi, a.d_xdsum_in);
       }
-      // ---- B: codes and LoRA partials of the slice -> the cluster
-      codes_and_lora_partials(xs, SD, sx_in, __frcp_rn(sx_in), am_in > 0.f, xqs, sp<int8_t>(sm, PSM(a_in)), R,
-                              stg_b, cdiag ? a.d_xq_in + r0D : nullptr);
-      if (R) xsend(stg_b, rcv_b + w.r * R, unsigned(4 * R), &xbars[EX_B_IN], Q);
-      // ---- in_proj scaffold on own tiles
-      const int nch_in = scaffold_mma(sm + PSM(in_tiles), w.ntile, kg_in, asm_a, lgSD, BSD, part);
-      if (tid < w.ntile * 16)
-        yin[tid] = h2d(sp<uint16_t>(sm, PSM(in_alpha))[tid]) * tile_row_value(part, tid / 16, nch_in, tid % 16, xsum_in);
-      // ---- u_in, LoRA stage 2 of own rows
+      PT(PH_LORA_IN);
+      // ---- S: the shared tiles (B/C rows, dt rows) first: the cluster waits for them
+      int nch = 1;
+      if (w.ns > 0) nch = scaffold_mma(sm + PSM(in_tiles) + shslot * tile_in, w.ns, kg_in, planes, PSD, part);
+      if (tid < w.ns * 16)
+        yin[shslot * 16 + tid] = h2d(sp<uint16_t>(sm, PSM(in_alpha))[shslot * 16 + tid]) *
+                                 tile_row_value(part, tid / 16, nch, tid % 16, xsum_in);
+      PT(PH_MMA_SH);
       if (R) {
-        if (!xwait(status, ctl, &xbars[EX_B_IN], unsigned(Q * 4 * R), par, 32u)) { alive = false; break; }
-        lora_finish(rcv_b, Q, R, sp<uint16_t>(sm, PSM(sa_in)), sx_in, u, wdiag ? a.d_acc_in : nullptr, a.d_u_in);
-        lora2_rows(sp<int8_t>(sm, PSM(in_bq)), w.ntile * 16, u, R, lo);
+        if (!xwait(status, ctl, &xbars[EX_LIN], unsigned(Q * 4 * R), par, 16u)) { alive = false; break; }
+        lora_finish(rcv_in, Q, R, sp<uint16_t>(sm, PSM(sa_in)), sx_in, u, wdiag ? a.d_acc_in : nullptr, a.d_u_in);
       }
-      csync();
-      if (tid < w.ntile * 16) {
-        double y = yin[tid];
-        if (R) y = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[tid]), lo[tid], y);
-        yin[tid] = y;
-        if (diag) a.d_zx[slot_tile(a, w, tid / 16) * 16 + tid % 16] = y;
-      }
-      csync();
-      // ---- C: conv step of own x channels, gate, shared rows -> the cluster
-      if (tid < w.nu * 16) {
-        const int uu = tid / 16, r = tid % 16;
-        const double xv = yin[(xslot + uu) * 16 + r];
-        const uint16_t* cw = sp<uint16_t>(sm, PSM(convw_x)) + (uu * 16 + r) * 4;
-        const float c0 = sp<float>(sm, PSM(cst_x))[(0 * kPMaxUnits + uu) * 16 + r];
-        const float c1 = sp<float>(sm, PSM(cst_x))[(1 * kPMaxUnits + uu) * 16 + r];
-        const float c2 = sp<float>(sm, PSM(cst_x))[(2 * kPMaxUnits + uu) * 16 + r];
-        double pre = h2d(sp<uint16_t>(sm, PSM(convb_x))[uu * 16 + r]);
-        pre = fma(h2d(cw[0]), double(c0), pre);
-        pre = fma(h2d(cw[1]), double(c1), pre);
-        pre = fma(h2d(cw[2]), double(c2), pre);
-        pre = fma(h2d(cw[3]), xv, pre);
-        const int ch = 16 * (w.u0 + uu) + r;
-        float* gcs = L.conv_state;
-        gcs[ch] = c1;
-        gcs[C + ch] = c2;
-        gcs[2 * C + ch] = float(xv);
-        const double xc = silu_d(pre);
-        yin[(xslot + uu) * 16 + r] = xc;
-        if (diag) a.d_xc[ch] = xc;
-      } else if (tid >= 64 && tid < 64 + w.nu * 16) {   // gate silu(z), in place of z
-        const int rr = tid - 64;
-        yin[(zslot + rr / 16) * 16 + rr % 16] = silu_d(yin[(zslot + rr / 16) * 16 + rr % 16]);
-      } else if (tid >= 128 && tid < 128 + w.ns * 16) {   // own shared rows
-        const int i = tid - 128;
+      PT(PH_WAIT_LIN);
+      // own shared rows: LoRA stage 2, then conv + SiLU (B/C) or step size + decay (dt),
+      // each value sent to every CTA of the cluster
+      if (tid < w.ns * 16) {
+        const int i = tid;
         const int si = w.s0 + i / 16, r = i % 16;        // shared tile of the cluster, row in it
-        double v = yin[(shslot + i / 16) * 16 + r];
+        double v = yin[shslot * 16 + i];
+        if (R) v = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[shslot * 16 + i]),
+                       lora2_row(sp<int8_t>(sm, PSM(in_bq)) + (shslot * 16 + i) * R, u, R), v);
+        if (diag) a.d_zx[slot_tile(a, w, shslot + i / 16) * 16 + r] = v;
         if (si < w.nbc) {                                 // a B/C row: conv step + SiLU
-          const uint16_t* cw = sp<uint16_t>(sm, PSM(sh_convw)) + i * 4;
           const float* cst = sp<float>(sm, PSM(sh_cst));
           const float c0 = cst[i], c1 = cst[SHR + i], c2 = cst[2 * SHR + i];
-          double pre = h2d(sp<uint16_t>(sm, PSM(sh_convb))[i]);
-          pre = fma(h2d(cw[0]), double(c0), pre);
-          pre = fma(h2d(cw[1]), double(c1), pre);
-          pre = fma(h2d(cw[2]), double(c2), pre);
-          pre = fma(h2d(cw[3]), v, pre);
+          const double pre = conv_step_d(sp<uint16_t>(sm, PSM(sh_convw)) + i * 4,
+                                         h2d(sp<uint16_t>(sm, PSM(sh_convb))[i]), c0, c1, c2, v);
           shst[i] = c1;
           shst[SHR + i] = c2;
           shst[2 * SHR + i] = float(v);
-          v = silu_d(pre);
-          if (diag) a.d_xc[E + 16 * si + r] = v;
-          stg_c[i] = v;
+          const double xc = silu_d(pre);
+          if (diag) a.d_xc[E + 16 * si + r] = xc;
+          const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(xc));
+          for (int q = 0; q < Q; ++q)
+            st_async_b64(cluster_map(shr_s + 8 * (shr_own + i), q), bits, cluster_map(xsh_s, q));
         } else {                                          // a dt row: step size and decay of its head
           const int h = 16 * (w.cdt0 + si - w.nbc) + r;
           const double dt = softplus_d(v + double(sp<float>(sm, PSM(hd_dtb))[h]));
-          const int o = 16 * w.nsbc + 32 * (si - w.s0 - w.nsbc) + r;   // dt tile: 16 steps, then 16 decays
-          stg_c[o] = dt;
-          stg_c[o + 16] = exp(dt * -exp(double(sp<float>(sm, PSM(hd_alog))[h])));
+          const double dA = exp(dt * -exp(double(sp<float>(sm, PSM(hd_alog))[h])));
+          const int o = shr_own + 16 * w.nsbc + 32 * (i / 16 - w.nsbc) + r;   // dt tile: 16 steps, 16 decays
+          const unsigned long long b0 = static_cast<unsigned long long>(__double_as_longlong(dt));
+          const unsigned long long b1 = static_cast<unsigned long long>(__double_as_longlong(dA));
+          for (int q = 0; q < Q; ++q) {
+            st_async_b64(cluster_map(shr_s + 8 * o, q), b0, cluster_map(xsh_s, q));
+            st_async_b64(cluster_map(shr_s + 8 * (o + 16), q), b1, cluster_map(xsh_s, q));
+          }
         }
-        fence_async_smem();
       }
-      // shared rows of the cluster: B/C rows (16 per tile), then per dt tile 16 steps
-      // and 16 decays; this CTA's tiles are contiguous from shared row 16 s0 + 16 (s0 - nbc)+
-      xsend(stg_c, shr + 16 * w.s0 + 16 * max(w.s0 - w.nbc, 0),
-            unsigned((16 * w.nsbc + 32 * (w.ns - w.nsbc)) * 8), &xbars[EX_C], Q);
-      if (!xwait(status, ctl, &xbars[EX_C], unsigned((2 * w.NS - w.nbc) * 16 * 8), par, 64u)) { alive = false; break; }
+      PT(PH_SHARED);
+      // ---- Z: the z and x tiles of own SSM channels
+      nch = scaffold_mma(sm + PSM(in_tiles), 2 * w.nu, kg_in, planes, PSD, part);
+      PT(PH_MMA_ZX);
+#ifdef DFSSM_PHASE_TIMERS
+      nch = scaffold_mma(sm + PSM(in_tiles), 2 * w.nu, kg_in, planes, PSD, part);
+      PT(PH_N + 1);
+#endif
+      if (tid < 2 * w.nu * 16) {
+        const int i = tid;
+        double v = h2d(sp<uint16_t>(sm, PSM(in_alpha))[i]) * tile_row_value(part, i / 16, nch, i % 16, xsum_in);
+        if (R) v = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[i]), lora2_row(sp<int8_t>(sm, PSM(in_bq)) + i * R, u, R), v);
+        if (diag) a.d_zx[slot_tile(a, w, i / 16) * 16 + i % 16] = v;
+        if (i < w.nu * 16) {                              // z row: the gate silu(z)
+          yin[i] = silu_d(v);
+        } else {                                          // x row: conv step + SiLU
+          const int j = i - w.nu * 16;                    // channel within the CTA's units
+          const int uu = j / 16, r = j % 16;
+          const float* cst = sp<float>(sm, PSM(cst_x));
+          const float c0 = cst[(0 * kPMaxUnits + uu) * 16 + r];
+          const float c1 = cst[(1 * kPMaxUnits + uu) * 16 + r];
+          const float c2 = cst[(2 * kPMaxUnits + uu) * 16 + r];
+          const double pre = conv_step_d(sp<uint16_t>(sm, PSM(convw_x)) + j * 4,
+                                         h2d(sp<uint16_t>(sm, PSM(convb_x))[j]), c0, c1, c2, v);
+          const int ch = 16 * w.u0 + j;
+          float* gcs = L.conv_state;
+          gcs[ch] = c1;
+          gcs[C + ch] = c2;
+          gcs[2 * C + ch] = float(v);
+          const double xc = silu_d(pre);
+          yin[i] = xc;
+          if (diag) a.d_xc[ch] = xc;
+        }
+      }
+      PT(PH_ZX_EPI);
+      if (!xwait(status, ctl, &xbars[EX_SH], unsigned((2 * w.NS - w.nbc) * 16 * 8), par, 32u)) {
+        alive = false;
+        break;
+      }
+      PT(PH_WAIT_SH);
       // ---- G: SSM update of own rows (warp per row, 4 states per lane per step);
       // publish g and the sum of its squares
       {
@@ -1164,54 +1242,57 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         if (lane == 0) tw_put_f64(a.x_gs + 2 * w.c, t, tag(l, XG));
       }
       if (tid == 0) mbar_arrive(empty_ab);      // AB group consumed: the copy warp may refill it
-      // ---- G: own slice of the gated value and the sums of squares
-      if (!tw_gather2(status, ctl, a.x_g + r0E, SE, reinterpret_cast<uint32_t*>(vs), a.x_gs, 2 * G, scratch32,
-                      tag(l, XG), 64u)) {
+      PT(PH_SSM);
+      // ---- G: the whole gated value and the sums of squares
+      if (!tw_gather<(4096 + 2 * 128 + kPThreads - 1) / kPThreads>(
+              status, ctl, a.x_g, E, reinterpret_cast<uint32_t*>(vfull), a.x_gs, 2 * G, scratch32, tag(l, XG),
+              64u)) {
         alive = false;
         break;
       }
-      const double ssg = sum_partials(scratch32, G, redd);
+      const double ssg = sum_partials(scratch32, G);
       if (w.k == 0) {   // B/C conv state of this layer: every CTA has finished reading it
         for (int i = tid; i < w.nsbc * 16; i += kPThreads) {
           const int ch = E + 16 * w.s0 + i;
           for (int r = 0; r < 3; ++r) L.conv_state[size_t(r) * C + ch] = shst[r * SHR + i];
         }
       }
+      PT(PH_GATHER_G);
       if (!mbar_wait_compute(status, ctl, full_cd, par, 128u)) { alive = false; break; }
-      // ---- A': gated RMSNorm on the slice -> the cluster
+      PT(PH_WAIT_CD);
+      // ---- A': gated RMSNorm of the whole vector
       const double rs_out = 1.0 / sqrt(ssg / double(E) + kEpsD);
-      prep_slice(vs, sp<uint16_t>(sm, PSM(gnorm)), SE, rs_out, stg_a, redi, xs, cdiag ? a.d_x_out + r0E : nullptr,
-                 cdiag ? a.d_xd_out + r0E : nullptr, E);
-      xsend(stg_a, asm_a + w.r * BSE, unsigned(BSE), &xbars[EX_A_OUT], Q);
-      if (!xwait(status, ctl, &xbars[EX_A_OUT], unsigned(Q * BSE), par, 128u)) { alive = false; break; }
       long long xsum_out;
       unsigned amax_out;
-      slice_totals(asm_a, Q, SE, BSE, &xsum_out, &amax_out);
+      prep_full(vfull, sp<uint16_t>(sm, PSM(gnorm)), E, rs_out, planes, PSE, w.r * SE, SE, xs, redo, &xsum_out,
+                &amax_out, wdiag ? a.d_x_out : nullptr, a.d_xd_out);
       const float am_out = half_to_float_bits(amax_out);
       const float sx_out = am_out > 0.f ? __fdiv_rn(am_out, 127.f) : 1.f;
+      PT(PH_PREP_OUT);
+      // ---- L': codes and LoRA partials of the slice -> the cluster
+      codes_and_lora_send(xs, SE, sx_out, __frcp_rn(sx_out), am_out > 0.f, xqs, sp<int8_t>(sm, PSM(a_out)), R,
+                          w.r, Q, rcv_out, &xbars[EX_LOUT], cdiag ? a.d_xq_out + w.r * SE : nullptr);
       if (wdiag) {
         if (tid == 0) *a.d_sx_out = sx_out;
-        plane_sums(asm_a, Q, SE, BSE, redi, a.d_xdsum_out);
+        plane_sums(planes, PSE, E, redo, a.d_xdsum_out);
       }
-      // ---- B': codes and LoRA partials of the slice -> the cluster
-      codes_and_lora_partials(xs, SE, sx_out, __frcp_rn(sx_out), am_out > 0.f, xqs, sp<int8_t>(sm, PSM(a_out)), R,
-                              stg_b, cdiag ? a.d_xq_out + r0E : nullptr);
-      if (R) xsend(stg_b, rcv_b + w.r * R, unsigned(4 * R), &xbars[EX_B_OUT], Q);
-      // ---- out_proj scaffold on own tiles
+      PT(PH_LORA_OUT);
+      // ---- O: out_proj scaffold on own tiles
       int nch_out = 1;
-      if (w.no > 0) nch_out = scaffold_mma(sm + PSM(out_tiles), w.no, kg_out, asm_a, lgSE, BSE, part);
+      if (w.no > 0) nch_out = scaffold_mma(sm + PSM(out_tiles), w.no, kg_out, planes, PSE, part);
+      PT(PH_MMA_OUT);
       if (R) {
-        if (!xwait(status, ctl, &xbars[EX_B_OUT], unsigned(Q * 4 * R), par, 256u)) { alive = false; break; }
-        lora_finish(rcv_b, Q, R, sp<uint16_t>(sm, PSM(sa_out)), sx_out, u, wdiag ? a.d_acc_out : nullptr, a.d_u_out);
-        lora2_rows(sp<int8_t>(sm, PSM(out_bq)), w.no * 16, u, R, lo);
-        csync();
+        if (!xwait(status, ctl, &xbars[EX_LOUT], unsigned(Q * 4 * R), par, 256u)) { alive = false; break; }
+        lora_finish(rcv_out, Q, R, sp<uint16_t>(sm, PSM(sa_out)), sx_out, u, wdiag ? a.d_acc_out : nullptr,
+                    a.d_u_out);
       }
-      // ---- R': residual rows and their sum of squares, published for the next layer
+      PT(PH_WAIT_LOUT);
+      // ---- residual rows and their sum of squares, published for the next layer
       const bool last = (l + 1 == a.n_layer);
       if (tid < w.no * 16) {
         const int o = w.o0 * 16 + tid;
         double y = h2d(sp<uint16_t>(sm, PSM(out_alpha))[tid]) * tile_row_value(part, tid / 16, nch_out, tid % 16, xsum_out);
-        if (R) y = fma(h2d(sp<uint16_t>(sm, PSM(out_sb))[tid]), lo[tid], y);
+        if (R) y = fma(h2d(sp<uint16_t>(sm, PSM(out_sb))[tid]), lora2_row(sp<int8_t>(sm, PSM(out_bq)) + tid * R, u, R), y);
         const float rn = float(double(resown[tid]) + y);
         resown[tid] = rn;
         if (!(last && a.layer_mode)) tw_put(a.x_r + o, __float_as_uint(rn), tag(l + 1, XR));
@@ -1228,17 +1309,20 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         if (lane == 0 && !(last && a.layer_mode)) tw_put_f64(a.x_rs + 2 * w.c, t, tag(l + 1, XR));
       }
       if (tid == 0) mbar_arrive(empty_cd);      // CD group consumed
+      PT(PH_RESID);
     }
 
     // ---- LM head
     if (alive && !a.layer_mode) {
       const int L = a.n_layer;
-      float* fres = sp<float>(sm, PSM(full)) + 2 * G;     // [D] residual, then [D] normalised
-      float* xn = fres + D;
-      if (tw_gather2(status, ctl, a.x_r, D, reinterpret_cast<uint32_t*>(fres), a.x_rs, 2 * G, scratch32, tag(L, XR),
-                     512u)) {
-        const double rs = 1.0 / sqrt(sum_partials(scratch32, G, redd) / double(D) + kEpsD);
-        for (int k = tid; k < D; k += kPThreads) xn[k] = float((double(fres[k]) * rs) * h2d(a.normf_w[k]));
+      // the final residual lands beyond the ring (the copy warp is already filling
+      // chunk slots over the working buffers) and is normalised in place
+      float* xn = reinterpret_cast<float*>(scratch32 + 2 * G);     // [D] residual, then normalised
+      if (tw_gather<(2048 + 2 * 128 + kPThreads - 1) / kPThreads>(
+              status, ctl, a.x_r, D, reinterpret_cast<uint32_t*>(xn), a.x_rs, 2 * G, scratch32, tag(L, XR),
+              512u)) {
+        const double rs = 1.0 / sqrt(sum_partials(scratch32, G) / double(D) + kEpsD);
+        for (int k = tid; k < D; k += kPThreads) xn[k] = float((double(xn[k]) * rs) * h2d(a.normf_w[k]));
         csync();
         float best = -INFINITY;
         int besti = 0x7fffffff;
@@ -1327,7 +1411,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         }
         csync();
         if (w.c == 0 && alive) {
-          if (tw_gather2(status, ctl, a.x_head, 2 * G, scratch32, a.x_head, 0, scratch32, tag(L, XHEAD), 2048u) &&
+          if (tw_gather<1>(status, ctl, a.x_head, 2 * G, scratch32, a.x_head, 0, scratch32, tag(L, XHEAD), 2048u) &&
               tid == 0) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
@@ -1340,7 +1424,15 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
           }
         }
       }
+      PT(PH_HEAD);
     }
+#ifdef DFSSM_PHASE_TIMERS
+    if (tid == 0 && a.phase) {
+      for (int i = 0; i < PH_N + 2; ++i) a.phase[size_t(w.c) * kPhaseSlots + i] += ptime[i];
+      a.phase[size_t(w.c) * kPhaseSlots + kPhaseSlots - 1] += 1;   // calls
+    }
+#endif
+#undef PT
     // ---- end of token: CTA 0 advances the launch epoch once every CTA has
     // published into the last exchange (so all have read the epoch)
     if (w.c == 0 && tid == 0 && !aborted(ctl)) ctl[0] = ctl[0] + 1;

@@ -15,7 +15,12 @@ from typing import List, Optional, Sequence
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libdfssm.so")
+# DFSSM_VARIANT=phases loads the build with the token kernel's phase timers
+# (libdfssm_phases.so, see build.py); DFSSM_LIBRARY names any other build of the
+# same library by path; the default is the product build.
+VARIANT = os.environ.get("DFSSM_VARIANT", "")
+LIB_PATH = os.environ.get("DFSSM_LIBRARY") or os.path.join(
+    _PKG, "libdfssm_phases.so" if VARIANT == "phases" else "libdfssm.so")
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -23,6 +28,8 @@ ERR_UNSUPPORTED_SHAPE = -2
 ERR_MISALIGNED = -3
 ERR_WORKSPACE_TOO_SMALL = -4
 ERR_CUDA = -5
+ERR_DEVICE = -6
+ERR_NOT_BUILT = -7
 DTYPE_F16, DTYPE_F32 = 0, 1
 LAYOUT_ROWMAJOR, LAYOUT_TILED = 0, 1
 
@@ -32,7 +39,9 @@ EXPORTS = [
     "dfssm_proj_workspace_layout",
     "dfssm_workspace_bytes", "dfssm_workspace_layout", "dfssm_layer_step",
     "dfssm_model_decode", "dfssm_model_decode_launches", "dfssm_last_error", "dfssm_version",
-    "dfssm_model_decode_q8", "dfssm_quantize_rows_int8",
+    "dfssm_model_decode_q8", "dfssm_quantize_rows_int8", "dfssm_phase_timers",
+    "dfssm_prefill_workspace_bytes", "dfssm_prefill_workspace_layout", "dfssm_layer_prefill",
+    "dfssm_model_prefill",
 ]
 
 
@@ -80,7 +89,7 @@ def lib() -> C.CDLL:
         return _lib
     if not os.path.exists(LIB_PATH):
         from . import build
-        build.build()
+        build.build(variant=VARIANT)
     L = C.CDLL(LIB_PATH)
     vp, i, sz = C.c_void_p, C.c_int, C.c_size_t
     L.dfssm_packed_words.argtypes = [i, i, i]
@@ -103,6 +112,14 @@ def lib() -> C.CDLL:
     L.dfssm_model_decode_q8.argtypes = [C.POINTER(CDims), i, i, vp, vp, C.POINTER(CLayerWeights),
                                         C.POINTER(CLayerState), vp, vp, vp, vp, vp, sz, vp]
     L.dfssm_quantize_rows_int8.argtypes = [vp, i, i, vp, vp, vp]
+    L.dfssm_phase_timers.argtypes = [vp, i, i]
+    L.dfssm_prefill_workspace_bytes.argtypes = [C.POINTER(CDims), i, i, i]
+    L.dfssm_prefill_workspace_bytes.restype = sz
+    L.dfssm_prefill_workspace_layout.argtypes = [C.POINTER(CDims), i, i, i, C.POINTER(CWsLayout)]
+    L.dfssm_layer_prefill.argtypes = [C.POINTER(CDims), i, C.POINTER(CLayerWeights), C.POINTER(CLayerState),
+                                      vp, vp, sz, vp]
+    L.dfssm_model_prefill.argtypes = [C.POINTER(CDims), i, i, vp, C.POINTER(CLayerWeights),
+                                      C.POINTER(CLayerState), vp, i, vp, vp, vp, vp, sz, vp]
     L.dfssm_last_error.restype = C.c_char_p
     L.dfssm_version.restype = C.c_int
     for name in EXPORTS:
@@ -351,3 +368,38 @@ def ws_view(ws, offset: int, dtype, shape):
     n = int(np.prod(shape))
     nbytes = n * torch.empty((), dtype=dtype).element_size()
     return ws[offset:offset + nbytes].view(dtype).view(*shape)
+
+
+# ------------------------------------------------------------------ prompt pass
+
+def prefill_workspace_layout(d, T: int, n_layer: int = 0, vocab: int = 0) -> CWsLayout:
+    L = CWsLayout()
+    cd = cdims(d)
+    _check(lib().dfssm_prefill_workspace_layout(C.byref(cd), T, n_layer, vocab, C.byref(L)))
+    return L
+
+
+def prefill_workspace(d, T: int, n_layer: int = 0, vocab: int = 0, device="cuda"):
+    import torch
+    return torch.zeros(prefill_workspace_layout(d, T, n_layer, vocab).total_bytes, dtype=torch.uint8,
+                       device=device)
+
+
+def layer_prefill(d, T: int, w: DeviceLayer, s: DeviceState, residual, ws, stream=None) -> None:
+    """One layer over a prompt: residual fp32 [batch, T, d_model] in/out (dfssm_layer_prefill)."""
+    cd, cw, cs = cdims(d), w.c(), s.c()
+    _check(lib().dfssm_layer_prefill(C.byref(cd), T, C.byref(cw), C.byref(cs), _ptr(residual), _ptr(ws),
+                                     ws.numel(), _stream(stream)))
+
+
+def model_prefill(m: DeviceModel, states: Sequence[DeviceState], tokens, tok_out, ws, logits=None,
+                  stream=None) -> None:
+    """The model over prompts tokens int32 [batch, T] (dfssm_model_prefill): states
+    updated in place, logits / greedy token of the last prompt token."""
+    n = len(m.layers)
+    cd = cdims(m.dims)
+    cw = (CLayerWeights * n)(*[lw.c() for lw in m.layers])
+    cs = (CLayerState * n)(*[s.c() for s in states])
+    _check(lib().dfssm_model_prefill(C.byref(cd), n, m.vocab, _ptr(m.embed), cw, cs, _ptr(m.normf_w),
+                                     int(tokens.shape[1]), _ptr(tokens), _ptr(tok_out), _ptr(logits), _ptr(ws),
+                                     ws.numel(), _stream(stream)))

@@ -44,7 +44,8 @@ enum {
   DFSSM_ERR_MISALIGNED = -3,         /* a pointer is not 16-byte aligned */
   DFSSM_ERR_WORKSPACE_TOO_SMALL = -4,
   DFSSM_ERR_CUDA = -5,               /* a CUDA runtime call or launch failed */
-  DFSSM_ERR_DEVICE = -6              /* no usable sm_100 device */
+  DFSSM_ERR_DEVICE = -6,             /* no usable sm_100 device */
+  DFSSM_ERR_NOT_BUILT = -7           /* a facility this build of the library leaves out */
 };
 
 enum { DFSSM_DTYPE_F16 = 0, DFSSM_DTYPE_F32 = 1 };
@@ -271,9 +272,56 @@ DFSSM_API int dfssm_model_decode_q8(const dfssm_dims* d, int n_layer, int vocab,
 DFSSM_API int dfssm_quantize_rows_int8(const uint16_t* w, int rows, int cols, int8_t* q, float* scale,
                                        void* stream);
 
+/* ---- prompt pass (prefill) ---------------------------------------------- */
+
+/* The step before decode: a prompt of T tokens per batch row goes through a layer
+ * (or the model) in one pass ("Density Field State Space Models", Section 2: the
+ * chunked state space duality (SSD) form of the Mamba-2 scan; Appendix B: chunks of
+ * block_len 64).  Every token row gets the same per-token arithmetic as the decode
+ * step (pre-norm, both projections with their exact scaffold, LoRA, gate, gated
+ * norm); the conv runs along the sequence from the stored conv state, and the SSM
+ * runs as the chunked scan from the stored SSM state, carried in fp64 through the
+ * prompt and stored once at the end.  On return the states are those after the
+ * last prompt token, ready for dfssm_model_decode.  Limits: T >= 1, batch * T <=
+ * 65535, headdim * d_state <= 8192 (the scan keeps a head's state in shared memory).
+ *
+ * Workspace: dfssm_prefill_workspace_bytes(d, T, 0, 0) for a layer,
+ * (d, T, n_layer, vocab) for the model; no zero-fill needed.  Its layout (the
+ * dfssm_ws_layout regions for batch * T token rows, token-major: row b * T + t)
+ * holds the last layer's intermediates of every prompt token. */
+DFSSM_API size_t dfssm_prefill_workspace_bytes(const dfssm_dims* d, int T, int n_layer, int vocab);
+DFSSM_API int dfssm_prefill_workspace_layout(const dfssm_dims* d, int T, int n_layer, int vocab,
+                                             dfssm_ws_layout* out);
+
+/* One layer over the prompt: residual fp32 [batch][T][d_model] in/out (every token's
+ * residual after the layer), state updated in place. */
+DFSSM_API int dfssm_layer_prefill(const dfssm_dims* d, int T, const dfssm_layer_weights* w,
+                                  const dfssm_layer_state* s, float* residual, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/* The model over the prompt: tokens int32 [batch][T] (device); every layer's state
+ * updated in place; logits fp32 [batch][vocab] (or NULL) and tok_out int32 [batch]
+ * (greedy, lowest id on ties) of the LAST prompt token, so that tok_out is the first
+ * decode input.  fp16 tied embedding / LM head. */
+DFSSM_API int dfssm_model_prefill(const dfssm_dims* d, int n_layer, int vocab, const uint16_t* embed,
+                                  const dfssm_layer_weights* layers, const dfssm_layer_state* states,
+                                  const uint16_t* normf_w, int T, const int32_t* tokens, int32_t* tok_out,
+                                  float* logits, void* ws, size_t ws_bytes, void* stream);
+
 /* Number of kernel launches one dfssm_model_decode call enqueues for these
  * arguments (0 if they are invalid). */
 DFSSM_API int dfssm_model_decode_launches(const dfssm_dims* d, int n_layer, int vocab);
+
+/* Per-phase cycle counters of the batch-1 token kernel (a measurement facility,
+ * not part of the method; the paper reports a per-layer time breakdown in Table 13
+ * and this is the same kind of breakdown for the fused kernel).  Only a library
+ * built with -DDFSSM_PHASE_TIMERS records them; the default build returns
+ * DFSSM_ERR_NOT_BUILT.  Entry [cta * 32 + slot] is the sum over the calls since the
+ * last reset of the clock64 cycles thread 0 of that CTA spent in phase `slot`
+ * (slots 0..18 in the kernel's phase order; slot 31 counts calls).  Copies
+ * min(max_entries, 256 * 32) entries to the host buffer `out` (synchronous), then
+ * zeroes the counters if `reset` is nonzero.  Returns the number of entries copied. */
+DFSSM_API int dfssm_phase_timers(uint64_t* out, int max_entries, int reset);
 
 /* Message describing the calling thread's last nonzero return ("" if none). */
 DFSSM_API const char* dfssm_last_error(void);

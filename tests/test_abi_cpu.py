@@ -23,7 +23,13 @@ def _declared():
 def test_library_builds_and_loads():
     build.build()
     L = F.lib()
-    assert L.dfssm_version() == 100
+    assert L.dfssm_version() == 200
+
+
+def test_phase_timers_absent_from_the_product_build():
+    buf = (C.c_uint64 * 64)()
+    assert F.lib().dfssm_phase_timers(buf, 64, 1) == F.ERR_NOT_BUILT
+    assert "DFSSM_PHASE_TIMERS" in F.last_error()
 
 
 def test_exports_every_declared_symbol():
