@@ -4,6 +4,7 @@
 #include <array>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -170,6 +171,8 @@ void layer_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* 
     L->res = kNone;
     L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), 0) + dta);
   }
+  // the batch-1 token kernel's control words follow the LM-head partials in the scratch
+  L->control = L->scratch + align256(size_t(8) * B * (n_layer > 0 ? kHeadBlocks : 1));
   L->total_bytes = align256(bp.off);
 }
 
@@ -297,8 +300,34 @@ int launch_proj_bt(const ProjArgs& a, cudaStream_t st) {
   return DFSSM_OK;
 }
 
+// Which scaffold kernel a batched projection takes: the register-fragment mma.sync
+// kernel (k_proj, the default: measured faster end to end so far), or the tcgen05
+// tile kernel (k_proj_tc) when DFSSM_PROJ_PATH=tc is set in the environment (read at
+// every call, so a caller can switch between calls); DFSSM_PROJ_PATH=mma forces k_proj.
+int proj_path_override() {
+  const char* e = getenv("DFSSM_PROJ_PATH");
+  if (e && strcmp(e, "mma") == 0) return 1;
+  if (e && strcmp(e, "tc") == 0) return 2;
+  return 0;
+}
+constexpr int kTcMinBatch = 1 << 30;   // the automatic choice never takes the tcgen05 kernel yet
+
+template <int EPI, int BG>
+int launch_proj_tc_bg(const ProjArgs& a, cudaStream_t st) {
+  const int smem = int(proj_tc_smem_bytes(BG, a.rank));
+  cudaError_t e = cudaFuncSetAttribute(k_proj_tc<EPI, BG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "k_proj_tc smem attribute: %s", cudaGetErrorString(e));
+  const dim3 grid((a.rows + kTcM - 1) / kTcM, (a.batch + BG - 1) / BG);
+  k_proj_tc<EPI, BG><<<grid, kTcThreads, smem, st>>>(a);
+  CHECK_LAUNCH("k_proj_tc");
+  return DFSSM_OK;
+}
+
 template <int EPI>
 int launch_proj(const ProjArgs& a, cudaStream_t st) {
+  const int path = proj_path_override();
+  if (path == 2 || (path == 0 && a.batch >= kTcMinBatch))
+    return a.batch >= 32 ? launch_proj_tc_bg<EPI, 32>(a, st) : launch_proj_tc_bg<EPI, 16>(a, st);
   switch (pick_bt(a.batch, a.K, a.rank)) {
     case 1: return launch_proj_bt<EPI, 1>(a, st);
     case 2: return launch_proj_bt<EPI, 2>(a, st);
@@ -395,6 +424,7 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   int rc = launch_prologue<0>(D, r, B, res, nullptr, w->prenorm_w, b.in, &w->in, st);
   if (rc) return rc;
   ProjArgs pa = proj_args(&w->in, r, B, b.in);
+  pa.status = b.status;
   pa.zx = b.zxbcdt;
   pa.conv_lo = E; pa.conv_dim = C; pa.conv_w = w->conv_w; pa.conv_b = w->conv_b;
   pa.conv_state = s->conv_state; pa.xc = b.xc;
@@ -408,6 +438,7 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   if ((rc = launch_ssm(sa, st))) return rc;
   if ((rc = launch_prologue<0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, B, b.out);
+  po.status = b.status;
   po.out = res;
   return launch_proj<EPI_RESID>(po, st);
 }
@@ -450,6 +481,7 @@ int layer_prefill_launch(const dfssm_dims* d, int T, const dfssm_layer_weights* 
   int rc = launch_prologue<0>(D, r, BT, res, nullptr, w->prenorm_w, b.in, &w->in, st);
   if (rc) return rc;
   ProjArgs pa = proj_args(&w->in, r, BT, b.in);
+  pa.status = b.status;
   pa.zx = b.zxbcdt;
   if ((rc = launch_proj<EPI_ZX>(pa, st))) return rc;
   PrefillArgs fa{};
@@ -470,6 +502,7 @@ int layer_prefill_launch(const dfssm_dims* d, int T, const dfssm_layer_weights* 
   CHECK_LAUNCH("k_ssd");
   if ((rc = launch_prologue<0>(E, r, BT, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, BT, b.out);
+  po.status = b.status;
   po.out = res;
   return launch_proj<EPI_RESID>(po, st);
 }
@@ -543,19 +576,40 @@ PPlan plan_persistent(const dfssm_dims* d) {
   if (d->ssm_state_dtype != 0) return no("the token kernel holds fp32 SSM state");
   if (N % 16 || H % 16) return no("d_state and nheads must be multiples of 16");
   if (R != 0 && (!pow2(R) || R < 8 || R > kPThreads)) return no("rank must be 0 or a power of two in [8, 512]");
-  const int Q = kPMaxCluster;
   if (D > kPMaxK || E > kPMaxK) return no("d_model and d_inner must be <= 4096");
   const int units = E / 16, out_tiles = D / 16, nbc = 2 * N / 16;
-  p.sm = plan_smem(D, E, H, N, R, Q);
+  // Clusters of 4 or 8 CTAs: the larger co-resident grid wins (clusters of 4 first on a
+  // tie), so that every CTA gets as few SSM units and out_proj tiles as possible.
+  int best_grid = 0, best_Q = 0, best_U = 0;
+  for (int Q : {4, 8}) {
+    int U = 0;
+    const int probe = std::min(kPlanSMs / Q, std::min(units, out_tiles) / Q) * Q;
+    if (probe < Q) continue;
+    for (int c = 0; c < probe; ++c) U = std::max(U, assign_cta(c, probe, Q, units, P, nbc, out_tiles).nu);
+    const PSmem m = plan_smem(D, E, H, N, R, Q, U);
+    if (m.total + int(sizeof(PParams)) + 1024 > optin || m.head_slots < 2) continue;
+    const bool spec = D == Shape2048::D && E == Shape2048::E && H == Shape2048::H && P == Shape2048::P &&
+                      N == Shape2048::N && R == Shape2048::R && Q == Shape2048::Q && U == Shape2048::U;
+    const int maxc = max_active_clusters(dev, Q, m.total, spec);
+    const int grid = std::min(std::min(maxc, kPlanSMs / Q), std::min(units, out_tiles) / Q) * Q;
+    if (grid > best_grid) {
+      best_grid = grid;
+      best_Q = Q;
+      int U2 = 0;
+      for (int c = 0; c < grid; ++c) U2 = std::max(U2, assign_cta(c, grid, Q, units, P, nbc, out_tiles).nu);
+      best_U = U2;
+    }
+  }
+  if (best_grid < 4) return no("no co-resident cluster of persistent CTAs");
+  const int Q = best_Q, grid = best_grid;
+  p.sm = plan_smem(D, E, H, N, R, Q, best_U);
   const PSmem& m = p.sm;
   p.spec = D == Shape2048::D && E == Shape2048::E && H == Shape2048::H && P == Shape2048::P && N == Shape2048::N &&
-           R == Shape2048::R && Q == Shape2048::Q;
+           R == Shape2048::R && Q == Shape2048::Q && best_U == Shape2048::U;
   if (p.spec && std::memcmp(&p.sm, &Shape2048::kPlan, sizeof(PSmem)) != 0) return no("compile-time plan mismatch");
   if (m.total + int(sizeof(PParams)) + 1024 > optin) return no("shared memory plan exceeds the per-block limit");
   if (m.head_slots < 2) return no("fewer than two LM-head chunk slots fit in shared memory");
-  const int maxc = max_active_clusters(dev, Q, m.total, p.spec);
-  const int grid = std::min(std::min(maxc, kPlanSMs / Q), std::min(units, out_tiles) / Q) * Q;
-  if (grid < Q) return no("no co-resident cluster of persistent CTAs");
+  if (max_active_clusters(dev, Q, m.total, p.spec) * Q < grid) return no("the final plan does not stay co-resident");
   for (int c = 0; c < grid; ++c) {
     const PWork w = assign_cta(c, grid, Q, units, P, nbc, out_tiles);
     if (w.nu < 1 || w.nu > kPMaxUnits) return no("SSM row units per CTA out of range");
@@ -631,8 +685,8 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
   a.embed = emb.f16; a.embed_q = emb.q; a.embed_s = emb.s;
   a.normf_w = normf_w; a.tok_in = tok_in; a.tok_out = tok_out; a.logits = logits;
   a.residual = residual;
-  unsigned char* scratch = at<unsigned char>(ws, WL.scratch);
-  unsigned char* pbase = scratch + align256(size_t(8) * d->batch * std::max(head_blocks, 1));
+  (void)head_blocks;
+  unsigned char* pbase = at<unsigned char>(ws, WL.control);
   a.status = at<unsigned>(ws, WL.status);
   a.ctl = reinterpret_cast<unsigned*>(pbase);
   unsigned long long* wd = reinterpret_cast<unsigned long long*>(pbase + 256);
@@ -795,6 +849,7 @@ int dfssm_proj_forward(const dfssm_proj* p, int rank, int batch, const uint16_t*
           at<double>(ws, L.u_in), at<int8_t>(ws, L.xd_in), at<int>(ws, L.xdsum_in)};
   if ((rc = launch_prologue<1>(p->cols, rank, batch, nullptr, x, nullptr, act, p, st))) return rc;
   ProjArgs a = proj_args(p, rank, batch, act);
+  a.status = at<unsigned>(ws, L.status);
   a.out = y;
   if ((rc = launch_proj<EPI_STORE>(a, st))) return rc;
   return ok();

@@ -297,6 +297,7 @@ struct ProjArgs {
   const float* dt_bias;    // [nheads]
   const float* A_log;      // [nheads]
   double* dta;             // fp64 [batch][nheads][2]: dt = softplus(dt_raw + dt_bias), dA = exp(-dt exp(A_log))
+  unsigned* status;        // workspace status word (value 65536: a tensor-core wait gave up), may be null
 };
 
 constexpr int kProjWarps = 16;
@@ -310,6 +311,43 @@ __host__ __device__ __forceinline__ size_t proj_smem_bytes(int K, int rank, int 
          + size_t(8) * bt * (rank > 0 ? rank : 1)                 // u (fp64)
          + size_t(4) * kProjWarps * 16 * proj_pstride(bt)         // per-warp int32 tile sums
          + size_t(4) * bt * kDigits;                              // digit sums
+}
+
+// Output (batch row b, projection row o) with value y: store, residual add, or the
+// in_proj epilogue (fp64 store, conv step + SiLU of the conv rows, step size and
+// decay of the dt rows).
+template <int EPI>
+DFSSM_DEV void proj_epilogue(const ProjArgs& a, int b, int o, double y) {
+  const size_t oi = size_t(b) * a.rows + o;
+  if (EPI == EPI_RESID) {
+    a.out[oi] = float(double(a.out[oi]) + y);
+  } else if (EPI == EPI_STORE) {
+    a.out[oi] = float(y);
+  } else if (EPI == EPI_ZX) {
+    a.zx[oi] = y;
+  } else {
+    a.zx[oi] = y;
+    const int c = o - a.conv_lo;
+    if (c >= 0 && c < a.conv_dim) {
+      float* cs = a.conv_state + size_t(b) * 3 * a.conv_dim;
+      const uint2 wv = *reinterpret_cast<const uint2*>(a.conv_w + size_t(c) * 4);
+      const double s0 = cs[c], s1 = cs[a.conv_dim + c], s2 = cs[2 * a.conv_dim + c];
+      double pre = h2d(a.conv_b[c]);
+      pre = fma(h2d(uint16_t(wv.x & 0xffff)), s0, pre);
+      pre = fma(h2d(uint16_t(wv.x >> 16)), s1, pre);
+      pre = fma(h2d(uint16_t(wv.y & 0xffff)), s2, pre);
+      pre = fma(h2d(uint16_t(wv.y >> 16)), y, pre);
+      a.xc[size_t(b) * a.conv_dim + c] = silu_d(pre);
+      cs[c] = float(s1);
+      cs[a.conv_dim + c] = float(s2);
+      cs[2 * a.conv_dim + c] = float(y);
+    } else if (o >= a.dt_lo && o < a.dt_lo + a.nheads) {
+      const int hh = o - a.dt_lo;
+      const double dt = softplus_d(y + double(a.dt_bias[hh]));
+      a.dta[(size_t(b) * a.nheads + hh) * 2] = dt;
+      a.dta[(size_t(b) * a.nheads + hh) * 2 + 1] = exp(dt * -exp(double(a.A_log[hh])));
+    }
+  }
 }
 
 // Scaffold value of one row from its per-plane 0/1 sums q[d] = sum_k bit * D_d[k]:
@@ -422,40 +460,230 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
           }
           y = fma(sb, l, y);
         }
-        const size_t oi = size_t(b) * a.rows + o;
-        if (EPI == EPI_RESID) {
-          a.out[oi] = float(double(a.out[oi]) + y);
-        } else if (EPI == EPI_STORE) {
-          a.out[oi] = float(y);
-        } else if (EPI == EPI_ZX) {
-          a.zx[oi] = y;
-        } else {
-          a.zx[oi] = y;
-          const int c = o - a.conv_lo;
-          if (c >= 0 && c < a.conv_dim) {
-            float* cs = a.conv_state + size_t(b) * 3 * a.conv_dim;
-            const uint2 wv = *reinterpret_cast<const uint2*>(a.conv_w + size_t(c) * 4);
-            const double s0 = cs[c], s1 = cs[a.conv_dim + c], s2 = cs[2 * a.conv_dim + c];
-            double pre = h2d(a.conv_b[c]);
-            pre = fma(h2d(uint16_t(wv.x & 0xffff)), s0, pre);
-            pre = fma(h2d(uint16_t(wv.x >> 16)), s1, pre);
-            pre = fma(h2d(uint16_t(wv.y & 0xffff)), s2, pre);
-            pre = fma(h2d(uint16_t(wv.y >> 16)), y, pre);
-            a.xc[size_t(b) * a.conv_dim + c] = silu_d(pre);
-            cs[c] = float(s1);
-            cs[a.conv_dim + c] = float(s2);
-            cs[2 * a.conv_dim + c] = float(y);
-          } else if (o >= a.dt_lo && o < a.dt_lo + a.nheads) {
-            const int hh = o - a.dt_lo;
-            const double dt = softplus_d(y + double(a.dt_bias[hh]));
-            a.dta[(size_t(b) * a.nheads + hh) * 2] = dt;
-            a.dta[(size_t(b) * a.nheads + hh) * 2 + 1] = exp(dt * -exp(double(a.A_log[hh])));
-          }
-        }
+        proj_epilogue<EPI>(a, b, o, y);
       }
     }
     __syncwarp();   // the warp's tile sums are consumed before its next tile's
   }
+}
+
+// ------------------------------------------------------------------ projection on tcgen05
+//
+// The batched scaffold on the 5th-generation tensor cores: tcgen05.mma kind::i8
+// (0/1 sign bytes times signed digit-plane bytes, int32 accumulators in tensor
+// memory).  A CTA owns one M = 128 tile of projection rows and a group of BG
+// batch rows (N = 6 BG digit-plane columns).  Per 256-column k-block its 128 threads
+// (a) expand the k-block's tiled sign words into 0/1 bytes in natural column order
+// and (b) copy the batch rows' digit planes (cp.async), both into the no-swizzle
+// K-major UMMA layout: 16-byte column chunks c, each holding its rows in 8-row core
+// matrices of 128 bytes, so a K = 32 instruction takes two chunks (leading byte
+// offset = rows x 16) of 8-row groups 128 bytes apart (stride byte offset).  One
+// thread then issues the eight K = 32 MMAs and commits them to the stage's mbarrier;
+// two stages let the next k-block's staging overlap the MMAs.  Every integer sum is
+// exact (|sum| <= 2^20 for K <= 8192); the epilogue reads the accumulators with
+// tcgen05.ld (warp w: TMEM lanes 32w..32w+31 = tile rows) and finishes each (row,
+// batch row) exactly as k_proj does.
+
+constexpr int kTcThreads = 256;      // two warpgroups: both stage; each finishes half the batch rows
+constexpr int kTcM = 128;              // projection rows per CTA (one UMMA M tile)
+constexpr int kTcStages = 2;
+
+template <int BG>
+struct TcShape {
+  static constexpr int N = kDigits * BG;                 // digit-plane columns (a multiple of 16)
+  static constexpr int A_BYTES = kTcM * kTileCols;       // 32 KB per k-block
+  static constexpr int B_BYTES = N * kTileCols;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  static_assert(N % 16 == 0 && N <= 256, "UMMA N");
+};
+
+__host__ __device__ inline size_t proj_tc_smem_bytes(int bg, int rank) {
+  return size_t(kTcStages) * (size_t(kTcM) * kTileCols + size_t(kDigits) * bg * kTileCols) +
+         size_t(8) * bg * (rank > 0 ? rank : 1) + size_t(4) * bg * kDigits + 1024;
+}
+
+DFSSM_DEV uint64_t umma_desc_kmajor(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  // start address, leading / stride byte offsets (16-byte units), version 1, no swizzle
+  return uint64_t((saddr >> 4) & 0x3fffu) | (uint64_t((lbo >> 4) & 0x3fffu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3fffu) << 32) | (uint64_t(1) << 46);
+}
+
+// Instruction descriptor of kind::i8: D s32 (c_format 2), A and B both signed 8-bit
+// (format 1; the 0/1 sign bytes are valid s8 values, and A and B keep one type),
+// both K-major, N >> 3, M = 128 >> 4.
+template <int N>
+DFSSM_DEV constexpr uint32_t umma_idesc_s8() {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(kTcM >> 4) << 24);
+}
+
+DFSSM_DEV void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+template <int EPI, int BG>
+__global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(ProjArgs a) {
+  using SH = TcShape<BG>;
+  constexpr int N = SH::N;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ __align__(8) uint64_t mbar[kTcStages];
+  __shared__ uint32_t tmem_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * kTcM, b0 = blockIdx.y * BG;
+  const int K = a.K, kgroups = K / kTileCols;
+  const int ntiles = (a.rows + kTileRows - 1) / kTileRows;
+  const int nb = min(BG, a.batch - b0);
+  const int rk = a.rank > 0 ? a.rank : 1;
+  unsigned char* stages = smem;
+  double* us = reinterpret_cast<double*>(smem + kTcStages * SH::STAGE);      // [BG][rank]
+  int* T = reinterpret_cast<int*>(us + BG * rk);                              // [BG][kDigits]
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(&tmem_s)), "n"(SH::TMEM_COLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kTcStages; ++i) mbar_init(&mbar[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = tid; i < BG * a.rank; i += kTcThreads) {
+    const int bb = i / a.rank, j = i % a.rank;
+    us[i] = bb < nb ? a.u[size_t(b0 + bb) * a.rank + j] : 0.0;
+  }
+  for (int i = tid; i < BG * kDigits; i += kTcThreads) T[i] = i / kDigits < nb ? a.xdsum[size_t(b0) * kDigits + i] : 0;
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = tmem_s;
+  bool ok = true;
+
+  for (int kb = 0; kb < kgroups; ++kb) {
+    const int st = kb % kTcStages;
+    unsigned char* As = stages + st * SH::STAGE;
+    unsigned char* Bs = As + SH::A_BYTES;
+    if (kb >= kTcStages) {        // the MMAs that last read this stage have completed
+      if (tid == 0) {
+        long long spins = 0;
+        const unsigned par = unsigned(kb / kTcStages - 1) & 1u;
+        while (!mbar_try_wait(&mbar[st], par))
+          if (++spins > (1LL << 24)) { if (a.status) atomicOr(a.status, 65536u); ok = false; break; }
+      }
+      __syncthreads();
+    }
+    // digit planes of the batch rows: row n = 6 bb + d, chunk c at c (N 16) + (n / 8) 128 + (n % 8) 16
+    for (int i = tid; i < nb * kDigits * 16; i += kTcThreads) {
+      const int n = i >> 4, c = i & 15;
+      cp_async16(Bs + c * (N * 16) + (n >> 3) * 128 + (n & 7) * 16,
+                 a.xd + (size_t(b0) * kDigits + n) * K + size_t(kb) * kTileCols + c * 16);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // sign bytes of the 8 row tiles: lane (g, t) of a tile holds rows g and g + 8, and for
+    // m = 0..3 the 16 columns 64 m + 16 t .. + 15 of each: byte 8 e + 4 h + i is bit
+    // 2 m + e + 8 i of word r / 8 + 2 h
+    {
+      const int g = lane >> 2, t = lane & 3;
+      for (int tt = warp; tt < kTcM / kTileRows; tt += kTcThreads / 32) {
+        const int rt = m0 / kTileRows + tt;
+        uint4 wv = make_uint4(0, 0, 0, 0);
+        if (rt < ntiles) wv = __ldg(reinterpret_cast<const uint4*>(a.bits) + (size_t(rt) * kgroups + kb) * 32 + lane);
+        const uint32_t wq[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t W0 = wq[half], W1 = wq[half + 2];
+          const int row = tt * kTileRows + g + 8 * half;
+          unsigned char* rb = As + (row >> 3) * 128 + (row & 7) * 16;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint4 v = make_uint4((W0 >> (2 * m)) & 0x01010101u, (W1 >> (2 * m)) & 0x01010101u,
+                                       (W0 >> (2 * m + 1)) & 0x01010101u, (W1 >> (2 * m + 1)) & 0x01010101u);
+            *reinterpret_cast<uint4*>(rb + (4 * m + t) * (kTcM * 16)) = v;
+          }
+        }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t as = smem_u32(As), bs = smem_u32(Bs);
+      constexpr uint32_t idesc = umma_idesc_s8<N>();
+#pragma unroll
+      for (int kk = 0; kk < kTileCols / 32; ++kk) {
+        const uint64_t ad = umma_desc_kmajor(as + kk * 2 * (kTcM * 16), kTcM * 16, 128);
+        const uint64_t bd = umma_desc_kmajor(bs + kk * 2 * (N * 16), N * 16, 128);
+        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n"
+            :: "r"(tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc) : "memory");
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                   :: "r"(smem_u32(&mbar[st])) : "memory");
+    }
+  }
+  // all MMAs done (the last commit tracks every earlier one)
+  if (tid == 0) {
+    const int kb = kgroups - 1;
+    long long spins = 0;
+    while (!mbar_try_wait(&mbar[kb % kTcStages], unsigned(kb / kTcStages) & 1u))
+      if (++spins > (1LL << 24)) { if (a.status) atomicOr(a.status, 65536u); ok = false; break; }
+  }
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+
+  // epilogue: thread = tile row (TMEM lane quarter = warp % 4); warpgroup wg finishes
+  // the batch-row octets wg, wg + 2, ... (48 accumulator columns at a time).  The
+  // row's LoRA B bytes are read once; u comes from shared memory.
+  const int quarter = warp & 3, wg = warp >> 2;
+  const int r = 32 * quarter + lane, o = m0 + r;
+  const double al = o < a.rows ? h2d(a.alpha[o]) : 0.0;
+  const double sb = (o < a.rows && a.rank > 0) ? h2d(a.sB[o]) : 0.0;
+  const int8_t* Br = a.B + size_t(o < a.rows ? o : 0) * a.rank;
+  for (int g8 = 8 * wg; g8 < BG; g8 += 16) {
+    uint32_t q[48];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const uint32_t taddr = tmem + (uint32_t(32 * quarter) << 16) + uint32_t(g8 * kDigits + 16 * j);
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+          : "=r"(q[16 * j + 0]), "=r"(q[16 * j + 1]), "=r"(q[16 * j + 2]), "=r"(q[16 * j + 3]),
+            "=r"(q[16 * j + 4]), "=r"(q[16 * j + 5]), "=r"(q[16 * j + 6]), "=r"(q[16 * j + 7]),
+            "=r"(q[16 * j + 8]), "=r"(q[16 * j + 9]), "=r"(q[16 * j + 10]), "=r"(q[16 * j + 11]),
+            "=r"(q[16 * j + 12]), "=r"(q[16 * j + 13]), "=r"(q[16 * j + 14]), "=r"(q[16 * j + 15])
+          : "r"(taddr));
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    if (o < a.rows && ok) {
+#pragma unroll
+      for (int bi = 0; bi < 8; ++bi) {
+        const int bb = g8 + bi;
+        if (bb < nb) {
+          long long S = 0;
+#pragma unroll
+          for (int d = kDigits - 1; d >= 0; --d) S = S * 256 + (2LL * int(q[bi * kDigits + d]) - T[bb * kDigits + d]);
+          double y = al * (double(S) * (1.0 / 16777216.0));
+          if (a.rank > 0) {
+            const double* ur = us + bb * a.rank;
+            const int* b4 = reinterpret_cast<const int*>(Br);
+            double l[4] = {0.0, 0.0, 0.0, 0.0};
+            for (int j4 = 0; j4 < a.rank / 4; ++j4) {
+              const int v = __ldg(b4 + j4);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) l[e] = fma(double(int8_t(v >> (8 * e))), ur[4 * j4 + e], l[e]);
+            }
+            y = fma(sb, (l[0] + l[1]) + (l[2] + l[3]), y);
+          }
+          proj_epilogue<EPI>(a, b0 + bb, o, y);
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "n"(SH::TMEM_COLS) : "memory");
 }
 
 // ------------------------------------------------------------------ SSM step

@@ -73,8 +73,8 @@ constexpr int kPWarps = 15;                       // compute warps
 constexpr int kPThreads = 32 * kPWarps;           // compute threads
 constexpr int kPBlock = kPThreads + 32;           // + the copy warp: 16 warps, 128 registers each
 constexpr int kPMaxUnits = 3;                     // SSM row units (16 channels) per CTA
-constexpr int kPMaxShared = 4;                    // shared (B/C, dt) tiles per CTA
-constexpr int kPMaxInTiles = 8;                   // z, x and shared tiles per CTA
+constexpr int kPMaxShared = 5;                    // shared (B/C, dt) tiles per CTA
+constexpr int kPMaxInTiles = 9;                   // z, x and shared tiles per CTA
 constexpr int kPMaxSharedTiles = 20;              // shared tiles of one cluster
 constexpr int kPMaxSharedRows = 16 * kPMaxSharedTiles;
 constexpr int kPMaxOutTiles = 2;                  // out_proj tiles per CTA
@@ -83,7 +83,7 @@ constexpr int kPMaxHeads = 4;                     // heads touched by one CTA's 
 constexpr int kPMaxK = 4096;                      // largest d_model / d_inner of the token kernel
 constexpr int kPSsmRows = (kPMaxUnits * 16 + kPWarps - 1) / kPWarps;   // SSM rows per compute warp
 constexpr long long kSpinLimit = 1LL << 22;       // polls before a wait gives up (seconds)
-constexpr int kHeadChunkRows = 7;                 // LM-head rows per chunk: 14 warps = 7 rows x 2 halves
+constexpr int kHeadChunkRows = 15;                // LM-head fp16 rows per chunk: one per compute warp
 constexpr int kHeadRingMax = 8;                   // LM-head chunk slots (all buffers free after the last layer)
 constexpr int kPhaseSlots = 32;                   // phase-timer slots per CTA (the last counts calls)
 constexpr int kPlanSMs = 256;                     // upper bound on CTAs of one launch (sizes the exchange scratch)
@@ -123,7 +123,7 @@ struct PSmem {
   // working
   int vfull, planes, xs, xqs, rcv, yin, shr, shst, u, resown;
   int ring_end, head_slots;       // LM-head chunk slots [0, head_slots) tile [0, ring_end)
-  int part, full, misc;
+  int part, full, misc, lo2;
   int total;
 };
 
@@ -144,7 +144,8 @@ struct __align__(16) PParams {
   float* residual;               // layer mode: [D] in/out
   // workspace
   unsigned* status;              // status word
-  unsigned* ctl;                 // [0] launch epoch, [1] abort flag
+  unsigned* ctl;                 // [0] launch epoch, [1] abort flag, [2] test: CTA + 1 that withholds its
+                                 // layer-0 residual words, [3] test: polls before a wait gives up
   unsigned long long* x_r;       // D residual words
   unsigned long long* x_rs;      // 2 grid words: fp64 sum of squares of each CTA's residual rows
   unsigned long long* x_g;       // E gated-value words
@@ -169,9 +170,10 @@ __host__ __device__ constexpr int ptake(int& off, int bytes) {
 // fall in 8 distinct 16-byte bank groups.
 __host__ __device__ constexpr int plane_stride(int K) { return K + 64; }
 
-// Shared-memory plan of one shape (byte offsets); the host plans launches with the
-// same function, and the compile-time shape below bakes its result into the code.
-__host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R, int Q) {
+// Shared-memory plan of one shape (byte offsets) for clusters of Q CTAs holding at
+// most U SSM units each; the host plans launches with the same function, and the
+// compile-time shape below bakes its result into the code.
+__host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R, int Q, int U) {
   PSmem m{};
   const int kg_in = D / kTileCols, kg_out = E / kTileCols;
   const int SD = D / Q, SE = E / Q;
@@ -193,7 +195,7 @@ __host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R,
   m.hd_dtb = ptake(off, 4 * H);
   m.hd_alog = ptake(off, 4 * H);
   m.hd_d = ptake(off, 4 * H);
-  m.state = ptake(off, kPMaxUnits * 16 * N * 4);
+  m.state = ptake(off, U * 16 * N * 4);
   m.ab_end = off;
   m.out_tiles = ptake(off, kPMaxOutTiles * kg_out * 512);
   m.out_bq = ptake(off, kPMaxOutTiles * 16 * R);
@@ -222,7 +224,8 @@ __host__ __device__ constexpr PSmem plan_smem(int D, int E, int H, int N, int R,
   if (m.head_slots > kHeadRingMax) m.head_slots = kHeadRingMax;
   m.part = ptake(off, 16 * 16 * kDigits * 4);
   m.full = ptake(off, 4 * (2 * kPlanSMs + D));
-  m.misc = ptake(off, kPMaxInTiles * 16 * 8);
+  m.misc = ptake(off, kPMaxInTiles * 16 * kDigits * 4);
+  m.lo2 = ptake(off, kPMaxInTiles * 16 * 8);
   m.total = off;
   return m;
 }
@@ -239,11 +242,11 @@ struct ShapeAny {
 };
 struct Shape2048 {
   static constexpr bool kConst = true;
-  static constexpr int D = 2048, E = 4096, H = 64, P = 64, N = 128, R = 32, Q = 8, C = E + 2 * N;
+  static constexpr int D = 2048, E = 4096, H = 64, P = 64, N = 128, R = 32, Q = 4, U = 2, C = E + 2 * N;
   static constexpr int kg_in = D / kTileCols, kg_out = E / kTileCols;
   static constexpr int SD = D / Q, SE = E / Q;
   static constexpr int units = E / 16, n_bc_tiles = 2 * N / 16, dt_tile0 = (2 * E + 2 * N) / 16, out_tiles = D / 16;
-  static constexpr PSmem kPlan = plan_smem(D, E, H, N, R, Q);
+  static constexpr PSmem kPlan = plan_smem(D, E, H, N, R, Q, U);
 };
 
 // ------------------------------------------------------------------ primitives
@@ -296,6 +299,14 @@ DFSSM_DEV double f64_of(const uint32_t* w2) {
 
 DFSSM_DEV bool aborted(const unsigned* ctl) { return *reinterpret_cast<volatile const unsigned*>(ctl + 1) != 0; }
 
+// Polls a wait makes before it gives up: control word 3 when a test sets it (so that a
+// wait made to run out ends within milliseconds), else kSpinLimit.  Read only every
+// 256 polls.
+DFSSM_DEV long long spin_limit(const unsigned* ctl) {
+  const unsigned v = *reinterpret_cast<volatile const unsigned*>(ctl + 3);
+  return v ? static_cast<long long>(v) : kSpinLimit;
+}
+
 DFSSM_DEV void give_up(unsigned* status, unsigned* ctl, unsigned bit) {
   atomicOr(status, bit);
   atomicExch(ctl + 1, 1u);
@@ -331,10 +342,15 @@ DFSSM_BIG bool tw_gather(unsigned* status, unsigned* ctl, const unsigned long lo
           pending &= ~(1u << i);
         }
       }
-      if (pending && ((++spins & 255) == 0) && (spins > kSpinLimit || aborted(ctl))) {
-        give_up(status, ctl, bit);
-        ok = false;
-        break;
+      if (pending) {
+        if (((++spins & 255) == 0) && (spins > spin_limit(ctl) || aborted(ctl))) {
+          give_up(status, ctl, bit);
+          ok = false;
+          break;
+        }
+        // a short pause between polls keeps the waiting CTAs' loads from crowding
+        // the L2 that the producers are still writing through
+        __nanosleep(64);
       }
     }
   }
@@ -345,7 +361,7 @@ DFSSM_BIG bool tw_gather(unsigned* status, unsigned* ctl, const unsigned long lo
 DFSSM_DEV bool mbar_wait(unsigned* status, unsigned* ctl, uint64_t* bar, unsigned parity, unsigned bit) {
   long long spins = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if (((++spins & 255) == 0) && (spins > kSpinLimit || aborted(ctl))) {
+    if (((++spins & 255) == 0) && (spins > spin_limit(ctl) || aborted(ctl))) {
       give_up(status, ctl, bit);
       return false;
     }
@@ -368,7 +384,7 @@ DFSSM_DEV bool xwait(unsigned* status, unsigned* ctl, uint64_t* bar, unsigned by
     mbar_expect_tx(bar, bytes);
     long long spins = 0;
     while (!mbar_try_wait_cluster(bar, parity)) {
-      if (((++spins & 255) == 0) && (spins > kSpinLimit || aborted(ctl))) {
+      if (((++spins & 255) == 0) && (spins > spin_limit(ctl) || aborted(ctl))) {
         give_up(status, ctl, bit);
         ok = false;
         break;
@@ -600,12 +616,48 @@ DFSSM_BIG void produce_cd(const PParams& a, const PWork& w, const PLayer& L, uns
 
 // ------------------------------------------------------------------ activation prep
 
+// fp16 bits of z = (v * rs) * w correctly rounded from the fp64 product: the fp32
+// product lies within 4 fp32 ulps of it, so when its low 13 mantissa bits are more
+// than 4 away from the fp16 rounding midpoint (0x1000) and z is in the fp16 normal
+// range, the hardware fp32 -> fp16 rounding of it is already the answer; otherwise
+// fp64 decides.
+DFSSM_DEV uint32_t norm_half(float v, double rs, float rs32, float wf) {
+  const float z = (v * rs32) * wf;
+  const float az = fabsf(z);
+  const int low13 = int(__float_as_uint(z) & 0x1fffu);
+  if (az >= 6.103515625e-05f && az < 65504.f && abs(low13 - 0x1000) > 4) return __half_as_ushort(__float2half_rn(z));
+  return d2h((double(v) * rs) * double(wf));
+}
+
+// X = x 2^24 of one fp16 value as balanced base-256 digits (planes 0-3 in lo, 4-5 in
+// the low bytes of hi), and its contribution to the exact sum split as X = xh 2^20 + xl.
+// For |x| <= 127 (the usual case) X fits int32 and the four digits come from one add
+// and one xor; larger values take the 64-bit path.
+DFSSM_DEV void digits_and_sum(uint32_t h, uint32_t* lo, uint32_t* hi, int* xh, int* xl) {
+  const uint32_t ha = h & 0x7fffu;
+  if (ha <= 0x57f0u) {
+    const uint32_t e = ha >> 10, m = ha & 0x3ffu;
+    int X = e ? int((m | 0x400u) << (e - 1u)) : int(m);
+    X = (h & 0x8000u) ? -X : X;
+    *lo = (uint32_t(X) + 0x80808080u) ^ 0x80808080u;
+    *hi = 0u;
+    *xh += X >> 20;
+    *xl += X & 0xfffff;
+    return;
+  }
+  digits_of(h, lo, hi);
+  const long long X = half_times_2p24_64(h);
+  *xh += int(X >> 20);
+  *xl += int(X & 0xfffff);
+}
+
 // Whole-vector preparation by the compute threads: x = fp16((v rs) w) for all K
 // columns, their six digit planes (plane stride PS), the fp16 bits of the LoRA slice
 // [s0, s0 + S) into xs, and -- identical in every thread -- the exact sum of X = x 2^24
-// and max |x| (fp16 bits).  Four consecutive columns per thread and pass, so each
-// plane gets one 32-bit store.  `red` holds 3 ints per warp; it is read after the
-// block barrier here, so the caller puts a barrier before its next use.
+// and max |x| (fp16 bits).  Four consecutive columns per thread and pass: the four
+// digit words are transposed into one word per plane with eight byte permutes.
+// `red` holds 3 ints per warp; it is read after the block barrier here, so the
+// caller puts a barrier before its next use.
 DFSSM_BIG void prep_full(const float* v, const uint16_t* w, int K, double rs, unsigned char* planes, int PS, int s0,
                          int S, uint16_t* xs, int* red, long long* xsum, unsigned* amax, uint16_t* x_diag,
                          int8_t* xd_diag) {
@@ -613,41 +665,42 @@ DFSSM_BIG void prep_full(const float* v, const uint16_t* w, int K, double rs, un
   const float rs32 = float(rs);
   int xh = 0, xl = 0;
   unsigned am = 0;
+  const int PW = PS / 4;
   for (int g = tid; g < K / 4; g += kPThreads) {
     const float4 v4 = reinterpret_cast<const float4*>(v)[g];
     const uint2 w4 = reinterpret_cast<const uint2*>(w)[g];
-    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-    const uint32_t ww[4] = {w4.x & 0xffffu, w4.x >> 16, w4.y & 0xffffu, w4.y >> 16};
-    uint32_t lo[4], hi[4], h[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      h[e] = norm_fp16(vv[e], rs, rs32, half_to_float_bits(ww[e]));
-      digits_of(h[e], &lo[e], &hi[e]);
-      const long long X = half_times_2p24_64(h[e]);
-      xh += int(X >> 20);                    // X = xh 2^20 + xl, 0 <= xl < 2^20
-      xl += int(X & 0xfffff);
-      am = max(am, h[e] & 0x7fffu);
-    }
-    // plane d, columns 4g..4g+3: byte d of lo (d < 4) or of hi (d = 4, 5) of each column
-    const uint32_t p0 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0040), __byte_perm(lo[2], lo[3], 0x0040), 0x5410);
-    const uint32_t p1 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0051), __byte_perm(lo[2], lo[3], 0x0051), 0x5410);
-    const uint32_t p2 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0062), __byte_perm(lo[2], lo[3], 0x0062), 0x5410);
-    const uint32_t p3 = __byte_perm(__byte_perm(lo[0], lo[1], 0x0073), __byte_perm(lo[2], lo[3], 0x0073), 0x5410);
-    const uint32_t p4 = __byte_perm(__byte_perm(hi[0], hi[1], 0x0040), __byte_perm(hi[2], hi[3], 0x0040), 0x5410);
-    const uint32_t p5 = __byte_perm(__byte_perm(hi[0], hi[1], 0x0051), __byte_perm(hi[2], hi[3], 0x0051), 0x5410);
+    const float2 wa = __half22float2(*reinterpret_cast<const __half2*>(&w4.x));
+    const float2 wb = __half22float2(*reinterpret_cast<const __half2*>(&w4.y));
+    const uint32_t h0 = norm_half(v4.x, rs, rs32, wa.x), h1 = norm_half(v4.y, rs, rs32, wa.y);
+    const uint32_t h2 = norm_half(v4.z, rs, rs32, wb.x), h3 = norm_half(v4.w, rs, rs32, wb.y);
+    uint32_t l0, l1, l2, l3, i0, i1, i2, i3;
+    digits_and_sum(h0, &l0, &i0, &xh, &xl);
+    digits_and_sum(h1, &l1, &i1, &xh, &xl);
+    digits_and_sum(h2, &l2, &i2, &xh, &xl);
+    digits_and_sum(h3, &l3, &i3, &xh, &xl);
+    am = max(max(am, max(h0 & 0x7fffu, h1 & 0x7fffu)), max(h2 & 0x7fffu, h3 & 0x7fffu));
+    // 4 x 4 byte transpose: plane d gets byte d of each column's digit word
+    const uint32_t t0 = __byte_perm(l0, l1, 0x5140), t1 = __byte_perm(l0, l1, 0x7362);
+    const uint32_t t2 = __byte_perm(l2, l3, 0x5140), t3 = __byte_perm(l2, l3, 0x7362);
     uint32_t* pw = reinterpret_cast<uint32_t*>(planes) + g;
-    const int PW = PS / 4;
+    const uint32_t p0 = __byte_perm(t0, t2, 0x5410), p1 = __byte_perm(t0, t2, 0x7632);
+    const uint32_t p2 = __byte_perm(t1, t3, 0x5410), p3 = __byte_perm(t1, t3, 0x7632);
+    uint32_t p4 = 0u, p5 = 0u;
+    if ((i0 | i1 | i2 | i3) != 0u) {
+      p4 = __byte_perm(__byte_perm(i0, i1, 0x0040), __byte_perm(i2, i3, 0x0040), 0x5410);
+      p5 = __byte_perm(__byte_perm(i0, i1, 0x0051), __byte_perm(i2, i3, 0x0051), 0x5410);
+    }
     pw[0] = p0;
     pw[PW] = p1;
     pw[2 * PW] = p2;
     pw[3 * PW] = p3;
     pw[4 * PW] = p4;
     pw[5 * PW] = p5;
+    const uint2 hh = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
     const int c0 = 4 * g - s0;
-    if (c0 >= 0 && c0 < S)
-      *reinterpret_cast<uint2*>(xs + c0) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+    if (c0 >= 0 && c0 < S) *reinterpret_cast<uint2*>(xs + c0) = hh;
     if (x_diag) {
-      *reinterpret_cast<uint2*>(x_diag + 4 * g) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+      *reinterpret_cast<uint2*>(x_diag + 4 * g) = hh;
       const uint32_t pp[6] = {p0, p1, p2, p3, p4, p5};
 #pragma unroll
       for (int d = 0; d < kDigits; ++d) *reinterpret_cast<uint32_t*>(xd_diag + size_t(d) * K + 4 * g) = pp[d];
@@ -739,19 +792,6 @@ DFSSM_BIG void lora_finish(const int* rcv, int Q, int R, const uint16_t* sA, flo
   csync();
 }
 
-// LoRA stage 2 of one row: sum_j B[j] u[j] in fp64, four interleaved partial sums
-// (R is a multiple of 8).
-DFSSM_DEV double lora2_row(const int8_t* Brow, const double* u, int R) {
-  const int* b4 = reinterpret_cast<const int*>(Brow);
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int j4 = 0; j4 < R / 4; ++j4) {
-    const int v = b4[j4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[e] = fma(double(int8_t(v >> (8 * e))), u[4 * j4 + e], acc[e]);
-  }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
 // Exact scaffold MMA over `ntile` tiles (smem, kg groups each), split into units
 // (tile, kgroup chunk); int32 partials to part[unit][16][kDigits].  The activation
 // digit planes are whole-vector planes (stride PS).  Register q of the A fragment of
@@ -826,17 +866,40 @@ DFSSM_BIG int scaffold_mma(const unsigned char* tiles, int ntile, int kg, const 
   return nchunk;
 }
 
-// Scaffold value (without alpha) of row r of tile ti from the unit partials:
-// sum_k s_k x_k = 2^-24 (2 sum_d 256^d Q_d - sum_k X_k), exact in int64.
-DFSSM_BIG double tile_row_value(const int* part, int ti, int nchunk, int r, long long xsum) {
+// The unit partials of `ntile` tiles summed over their chunks into a [ntile][16][6]
+// table, one compute thread per (tile, row, digit), in chunk order.
+DFSSM_DEV void combine_parts(const int* part, int ntile, int nchunk, int* tbl) {
+  for (int i = threadIdx.x; i < ntile * 16 * kDigits; i += kPThreads) {
+    const int ti = i / (16 * kDigits), rd = i % (16 * kDigits);
+    int s = 0;
+    for (int c = 0; c < nchunk; ++c) s += part[(ti * nchunk + c) * 16 * kDigits + rd];
+    tbl[i] = s;
+  }
+  csync();
+}
+// Scaffold value (without alpha) of table row i: 2^-24 (2 sum_d 256^d Q_d - sum_k X_k).
+DFSSM_DEV double table_row_value(const int* tbl, int i, long long xsum) {
   long long S = 0;
 #pragma unroll
-  for (int d = kDigits - 1; d >= 0; --d) {
-    int s = 0;
-    for (int c = 0; c < nchunk; ++c) s += part[((ti * nchunk + c) * 16 + r) * kDigits + d];
-    S = S * 256 + s;
-  }
+  for (int d = kDigits - 1; d >= 0; --d) S = S * 256 + tbl[i * kDigits + d];
   return double(2 * S - xsum) * (1.0 / 16777216.0);
+}
+// LoRA stage 2 of `nrows` rows, out[r] = sum_j B[r][j] u[j] in fp64, four lanes per row
+// (lane q takes the terms j = q mod 4), combined as (q0 + q1) + (q2 + q3).
+DFSSM_DEV void lora2_all(const int8_t* Bq, int nrows, const double* u, int R, double* out) {
+  const int q = threadIdx.x & 3;
+  for (int base = 0; base < nrows * 4; base += kPThreads) {
+    const int i = base + int(threadIdx.x), r = i >> 2;
+    double acc = 0.0;
+    if (r < nrows) {
+      const int8_t* br = Bq + r * R;
+      for (int j = q; j < R; j += 4) acc = fma(double(br[j]), u[j], acc);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (q == 0 && r < nrows) out[r] = acc;
+  }
+  csync();
 }
 
 // Pre-activation of one conv channel: bias + taps 0..2 on the stored inputs (oldest
@@ -865,7 +928,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   __shared__ int redi[3 * kPWarps];
   __shared__ int redo[3 * kPWarps];
   __shared__ double ssw[kPWarps * kPSsmRows];
-  __shared__ int s_stale;
+  __shared__ int s_stale, s_withhold;
   for (int i = threadIdx.x; i < int(sizeof(PParams) / 16); i += blockDim.x)
     reinterpret_cast<uint4*>(pbuf)[i] = reinterpret_cast<const uint4*>(&pa)[i];
   const PParams& a = *reinterpret_cast<const PParams*>(pbuf);
@@ -884,13 +947,15 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   uint64_t* full_h = &bars[4];
   uint64_t* empty_h = &bars[4 + kHeadRingMax];
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 4 + 2 * kHeadRingMax; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 4 + kHeadRingMax; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < kHeadRingMax; ++i) mbar_init(&bars[4 + kHeadRingMax + i], kPWarps);   // head slots: one arrival per compute warp
     for (int i = 0; i < EX_N; ++i) mbar_init(&xbars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     // An abort flag left by an earlier call means its exchange words may still carry
     // this launch's epoch: do nothing and say so (the caller zero-fills the workspace).
     s_stale = aborted(pa.ctl) ? 1 : 0;
     if (s_stale) atomicOr(pa.status, 1u);
+    s_withhold = int(*reinterpret_cast<volatile const unsigned*>(pa.ctl + 2));
   }
   // every CTA's barriers exist before any CTA of the cluster copies into it
   cluster_sync_all();
@@ -900,7 +965,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
   const int G = a.grid;
   const int v0 = int((long long)w.c * a.vocab / G), v1 = int((long long)(w.c + 1) * a.vocab / G);
   // LM-head rows: fp16, or (Q8) int8 codes with a per-row scale.  Slots are spaced for
-  // 7 fp16 rows, which is 14 int8 rows: an int8 chunk is 14 rows (half the chunks).
+  // 15 fp16 rows, which is 30 int8 rows: an int8 chunk is 30 rows (half the chunks).
   // A compile-time choice keeps the fp16 kernel's registers as they were.
   constexpr bool q8 = Q8;
   constexpr int CR = Q8 ? 2 * kHeadChunkRows : kHeadChunkRows;
@@ -972,11 +1037,9 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
     unsigned* status = a.status;
     unsigned* ctl = a.ctl;
 #ifdef DFSSM_PHASE_TIMERS
-    // slots PH_N, PH_N + 1: the in-side preparation and the z/x MMA repeated with
-    // their code already cached; PH_N + 2: the barriers around the repeat (excluded)
-    long long ptime[PH_N + 3];
+    long long ptime[PH_N];
 #pragma unroll
-    for (int i = 0; i < PH_N + 3; ++i) ptime[i] = 0;
+    for (int i = 0; i < PH_N; ++i) ptime[i] = 0;
     long long tlast = clock64();
 #define PT(k)                              \
   do {                                     \
@@ -1068,17 +1131,6 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       const float am_in = half_to_float_bits(amax_in);
       const float sx_in = am_in > 0.f ? __fdiv_rn(am_in, 127.f) : 1.f;
       PT(PH_PREP_IN);
-#ifdef DFSSM_PHASE_TIMERS
-      // the same preparation once more, its code now in the instruction caches
-      // (idempotent: same inputs, same outputs)
-      csync();
-      PT(PH_N + 2);
-      prep_full(vfull, sp<uint16_t>(sm, PSM(prenorm)), D, rs_in, planes, PSD, w.r * SD, SD, xs, redi, &xsum_in,
-                &amax_in, nullptr, nullptr);
-      PT(PH_N);
-      csync();
-      PT(PH_N + 2);
-#endif
       // ---- L: codes and LoRA partials of the slice -> the cluster
       codes_and_lora_send(xs, SD, sx_in, __frcp_rn(sx_in), am_in > 0.f, xqs, sp<int8_t>(sm, PSM(a_in)), R, w.r, Q,
                           rcv_in, &xbars[EX_LIN], cdiag ? a.d_xq_in + w.r * SD : nullptr);
@@ -1088,15 +1140,21 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       }
       PT(PH_LORA_IN);
       // ---- S: the shared tiles (B/C rows, dt rows) first: the cluster waits for them
+      int* tbl = sp<int>(sm, PSM(misc));                 // [tiles][16][6] chunk-summed digit sums
+      double* lo = sp<double>(sm, PSM(lo2));            // LoRA stage-2 sums of own in_proj rows (slot order)
       int nch = 1;
-      if (w.ns > 0) nch = scaffold_mma(sm + PSM(in_tiles) + shslot * tile_in, w.ns, kg_in, planes, PSD, part);
+      if (w.ns > 0) {
+        nch = scaffold_mma(sm + PSM(in_tiles) + shslot * tile_in, w.ns, kg_in, planes, PSD, part);
+        combine_parts(part, w.ns, nch, tbl);
+      }
       if (tid < w.ns * 16)
-        yin[shslot * 16 + tid] = h2d(sp<uint16_t>(sm, PSM(in_alpha))[shslot * 16 + tid]) *
-                                 tile_row_value(part, tid / 16, nch, tid % 16, xsum_in);
+        yin[shslot * 16 + tid] = h2d(sp<uint16_t>(sm, PSM(in_alpha))[shslot * 16 + tid]) * table_row_value(tbl, tid, xsum_in);
       PT(PH_MMA_SH);
       if (R) {
         if (!xwait(status, ctl, &xbars[EX_LIN], unsigned(Q * 4 * R), par, 16u)) { alive = false; break; }
         lora_finish(rcv_in, Q, R, sp<uint16_t>(sm, PSM(sa_in)), sx_in, u, wdiag ? a.d_acc_in : nullptr, a.d_u_in);
+        // the shared rows first (the cluster waits for them); the z/x rows' after the send
+        lora2_all(sp<int8_t>(sm, PSM(in_bq)) + shslot * 16 * R, w.ns * 16, u, R, lo + shslot * 16);
       }
       PT(PH_WAIT_LIN);
       // own shared rows: LoRA stage 2, then conv + SiLU (B/C) or step size + decay (dt),
@@ -1105,8 +1163,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         const int i = tid;
         const int si = w.s0 + i / 16, r = i % 16;        // shared tile of the cluster, row in it
         double v = yin[shslot * 16 + i];
-        if (R) v = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[shslot * 16 + i]),
-                       lora2_row(sp<int8_t>(sm, PSM(in_bq)) + (shslot * 16 + i) * R, u, R), v);
+        if (R) v = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[shslot * 16 + i]), lo[shslot * 16 + i], v);
         if (diag) a.d_zx[slot_tile(a, w, shslot + i / 16) * 16 + r] = v;
         if (si < w.nbc) {                                 // a B/C row: conv step + SiLU
           const float* cst = sp<float>(sm, PSM(sh_cst));
@@ -1137,15 +1194,13 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       PT(PH_SHARED);
       // ---- Z: the z and x tiles of own SSM channels
       nch = scaffold_mma(sm + PSM(in_tiles), 2 * w.nu, kg_in, planes, PSD, part);
+      combine_parts(part, 2 * w.nu, nch, tbl);
+      if (R) lora2_all(sp<int8_t>(sm, PSM(in_bq)), 2 * w.nu * 16, u, R, lo);
       PT(PH_MMA_ZX);
-#ifdef DFSSM_PHASE_TIMERS
-      nch = scaffold_mma(sm + PSM(in_tiles), 2 * w.nu, kg_in, planes, PSD, part);
-      PT(PH_N + 1);
-#endif
       if (tid < 2 * w.nu * 16) {
         const int i = tid;
-        double v = h2d(sp<uint16_t>(sm, PSM(in_alpha))[i]) * tile_row_value(part, i / 16, nch, i % 16, xsum_in);
-        if (R) v = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[i]), lora2_row(sp<int8_t>(sm, PSM(in_bq)) + i * R, u, R), v);
+        double v = h2d(sp<uint16_t>(sm, PSM(in_alpha))[i]) * table_row_value(tbl, i, xsum_in);
+        if (R) v = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[i]), lo[i], v);
         if (diag) a.d_zx[slot_tile(a, w, i / 16) * 16 + i % 16] = v;
         if (i < w.nu * 16) {                              // z row: the gate silu(z)
           yin[i] = silu_d(v);
@@ -1278,24 +1333,31 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       }
       PT(PH_LORA_OUT);
       // ---- O: out_proj scaffold on own tiles
-      int nch_out = 1;
-      if (w.no > 0) nch_out = scaffold_mma(sm + PSM(out_tiles), w.no, kg_out, planes, PSE, part);
+      int* tbl_o = sp<int>(sm, PSM(misc));
+      double* lo_o = sp<double>(sm, PSM(lo2));
+      if (w.no > 0) {
+        const int nch_out = scaffold_mma(sm + PSM(out_tiles), w.no, kg_out, planes, PSE, part);
+        combine_parts(part, w.no, nch_out, tbl_o);
+      }
       PT(PH_MMA_OUT);
       if (R) {
         if (!xwait(status, ctl, &xbars[EX_LOUT], unsigned(Q * 4 * R), par, 256u)) { alive = false; break; }
         lora_finish(rcv_out, Q, R, sp<uint16_t>(sm, PSM(sa_out)), sx_out, u, wdiag ? a.d_acc_out : nullptr,
                     a.d_u_out);
+        lora2_all(sp<int8_t>(sm, PSM(out_bq)), w.no * 16, u, R, lo_o);
       }
       PT(PH_WAIT_LOUT);
-      // ---- residual rows and their sum of squares, published for the next layer
+      // ---- residual rows and their sum of squares, published for the next layer (a
+      // test can make one CTA withhold its layer-0 words so that the next gather runs out)
       const bool last = (l + 1 == a.n_layer);
+      const bool publish = !(last && a.layer_mode) && !(l == 0 && s_withhold == w.c + 1);
       if (tid < w.no * 16) {
         const int o = w.o0 * 16 + tid;
-        double y = h2d(sp<uint16_t>(sm, PSM(out_alpha))[tid]) * tile_row_value(part, tid / 16, nch_out, tid % 16, xsum_out);
-        if (R) y = fma(h2d(sp<uint16_t>(sm, PSM(out_sb))[tid]), lora2_row(sp<int8_t>(sm, PSM(out_bq)) + tid * R, u, R), y);
+        double y = h2d(sp<uint16_t>(sm, PSM(out_alpha))[tid]) * table_row_value(tbl_o, tid, xsum_out);
+        if (R) y = fma(h2d(sp<uint16_t>(sm, PSM(out_sb))[tid]), lo_o[tid], y);
         const float rn = float(double(resown[tid]) + y);
         resown[tid] = rn;
-        if (!(last && a.layer_mode)) tw_put(a.x_r + o, __float_as_uint(rn), tag(l + 1, XR));
+        if (publish) tw_put(a.x_r + o, __float_as_uint(rn), tag(l + 1, XR));
         if (last) {
           if (a.layer_mode) a.residual[o] = rn;
           else a.d_res[o] = rn;
@@ -1306,7 +1368,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         double t = 0.0;
         for (int i = lane; i < w.no * 16; i += 32) t = fma(double(resown[i]), double(resown[i]), t);
         t = warp_sum_d(t);
-        if (lane == 0 && !(last && a.layer_mode)) tw_put_f64(a.x_rs + 2 * w.c, t, tag(l + 1, XR));
+        if (lane == 0 && publish) tw_put_f64(a.x_rs + 2 * w.c, t, tag(l + 1, XR));
       }
       if (tid == 0) mbar_arrive(empty_cd);      // CD group consumed
       PT(PH_RESID);
@@ -1324,84 +1386,96 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         const double rs = 1.0 / sqrt(sum_partials(scratch32, G) / double(D) + kEpsD);
         for (int k = tid; k < D; k += kPThreads) xn[k] = float((double(xn[k]) * rs) * h2d(a.normf_w[k]));
         csync();
-        float best = -INFINITY;
-        int besti = 0x7fffffff;
-        float* hsum = sp<float>(sm, PSM(part));     // [2][CR][2]
-        // warp 2 r + h takes half h of row r of every chunk; its lanes keep their
-        // columns of the normalised residual in registers (kHV 8-column groups each)
-        constexpr int kHV = 4;
-        const int hrow = warp >> 1, hhalf = warp & 1;
-        const int hn = D / 16, hb = hhalf * hn;      // 8-column groups per half row, first group of this half
+        // Every compute warp takes whole rows -- row `warp` of each 15-row group of a
+        // chunk (one group per fp16 chunk, two per int8 chunk) -- waits on the chunk's
+        // slot itself and releases it with its own arrival (the empty barriers count
+        // one arrival per compute warp), so no block barrier runs per chunk.  A lane
+        // keeps its kHV 8-column groups of the normalised residual in registers.
+        constexpr int kHV = 8;
+        const int hn = D / 8;                        // 8-column groups per row
         float xr[kHV][8];
 #pragma unroll
         for (int m = 0; m < kHV; ++m)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xr[m][e] = lane + 32 * m < hn ? xn[(hb + lane + 32 * m) * 8 + e] : 0.f;
-        for (int ci = 0; ci < head_chunks && alive; ++ci) {
+          for (int e = 0; e < 8; ++e) xr[m][e] = lane + 32 * m < hn ? xn[(lane + 32 * m) * 8 + e] : 0.f;
+        auto f16x8 = [](const uint4& wv, float (&f)[8]) {
+          const __half2* wh = reinterpret_cast<const __half2*>(&wv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 t2 = __half22float2(wh[i]);
+            f[2 * i] = t2.x;
+            f[2 * i + 1] = t2.y;
+          }
+        };
+        float best = -INFINITY;
+        int besti = 0x7fffffff;
+        bool hok = true;
+        for (int ci = 0; ci < head_chunks; ++ci) {
           const int b = ci % NH;
-          if (!mbar_wait_compute(status, ctl, full_h + b, unsigned(ci / NH) & 1u, 1024u)) { alive = false; break; }
+          {   // every lane takes the slot's phase (bounded; lane 0 flags a timeout)
+            long long spins = 0;
+            while (!mbar_try_wait(full_h + b, unsigned(ci / NH) & 1u)) {
+              if (((++spins & 255) == 0) && (spins > spin_limit(ctl) || aborted(ctl))) {
+                if (lane == 0) give_up(status, ctl, 1024u);
+                hok = false;
+                break;
+              }
+            }
+            hok = __all_sync(0xffffffffu, hok);
+          }
+          if (!hok) break;
           const int r0 = v0 + ci * CR, nr = min(CR, v1 - r0);
-          float* hs = hsum + (ci & 1) * 2 * CR;
 #pragma unroll
-          for (int rsub = 0; rsub < CR / kHeadChunkRows; ++rsub) {
-          const int row = hrow + kHeadChunkRows * rsub;
-          if (row < nr) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            auto acc8 = [&](const float (&f)[8], const float* x) {
-              acc[0] = fmaf(f[0], x[0], acc[0]); acc[1] = fmaf(f[1], x[1], acc[1]);
-              acc[2] = fmaf(f[2], x[2], acc[2]); acc[3] = fmaf(f[3], x[3], acc[3]);
-              acc[0] = fmaf(f[4], x[4], acc[0]); acc[1] = fmaf(f[5], x[5], acc[1]);
-              acc[2] = fmaf(f[6], x[6], acc[2]); acc[3] = fmaf(f[7], x[7], acc[3]);
-            };
-            auto f16x8 = [](const uint4& wv, float (&f)[8]) {
-              const __half2* wh = reinterpret_cast<const __half2*>(&wv);
+          for (int rsub = 0; rsub < CR / kPWarps; ++rsub) {
+            const int row = warp + kPWarps * rsub;
+            if (row < nr) {
+              const unsigned char* wrow = head_slot(b) + size_t(row) * head_row_bytes;
+              float acc[4] = {0.f, 0.f, 0.f, 0.f};
+              auto acc8 = [&](const float (&f)[8], const float* x) {
+                acc[0] = fmaf(f[0], x[0], acc[0]); acc[1] = fmaf(f[1], x[1], acc[1]);
+                acc[2] = fmaf(f[2], x[2], acc[2]); acc[3] = fmaf(f[3], x[3], acc[3]);
+                acc[0] = fmaf(f[4], x[4], acc[0]); acc[1] = fmaf(f[5], x[5], acc[1]);
+                acc[2] = fmaf(f[6], x[6], acc[2]); acc[3] = fmaf(f[7], x[7], acc[3]);
+              };
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 t2 = __half22float2(wh[i]);
-                f[2 * i] = t2.x;
-                f[2 * i + 1] = t2.y;
+              for (int m = 0; m < kHV; ++m) {
+                if (lane + 32 * m < hn) {
+                  float f[8];
+                  if (q8) i8x8_to_float(reinterpret_cast<const uint2*>(wrow)[lane + 32 * m], f);
+                  else f16x8(reinterpret_cast<const uint4*>(wrow)[lane + 32 * m], f);
+                  acc8(f, xr[m]);
+                }
               }
-            };
-            const unsigned char* wrow = head_slot(b) + size_t(row) * head_row_bytes;
-#pragma unroll
-            for (int m = 0; m < kHV; ++m) {
-              if (lane + 32 * m < hn) {
+              for (int c = lane + 32 * kHV; c < hn; c += 32) {   // rows wider than kHV groups per lane
                 float f[8];
-                if (q8) i8x8_to_float(reinterpret_cast<const uint2*>(wrow)[hb + lane + 32 * m], f);
-                else f16x8(reinterpret_cast<const uint4*>(wrow)[hb + lane + 32 * m], f);
-                acc8(f, xr[m]);
+                if (q8) i8x8_to_float(reinterpret_cast<const uint2*>(wrow)[c], f);
+                else f16x8(reinterpret_cast<const uint4*>(wrow)[c], f);
+                acc8(f, xn + c * 8);
+              }
+              float lg = warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
+              if (lane == 0) {
+                if (q8) lg *= a.embed_s[r0 + row];
+                if (a.logits) a.logits[r0 + row] = lg;
+                if (lg > best || (lg == best && r0 + row < besti)) {
+                  best = lg;
+                  besti = r0 + row;
+                }
               }
             }
-            for (int c = lane + 32 * kHV; c < hn; c += 32) {   // half rows wider than kHV groups per lane
-              float f[8];
-              if (q8) i8x8_to_float(reinterpret_cast<const uint2*>(wrow)[hb + c], f);
-              else f16x8(reinterpret_cast<const uint4*>(wrow)[hb + c], f);
-              acc8(f, xn + (hb + c) * 8);
-            }
-            const float v = warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
-            if (lane == 0) hs[row * 2 + hhalf] = v;
           }
-          }
-          csync();
-          if (tid == 0) mbar_arrive(empty_h + b);      // the slot may be refilled
-          if (tid < nr) {
-            float lg = hs[tid * 2] + hs[tid * 2 + 1];
-            if (q8) lg *= a.embed_s[r0 + tid];
-            if (a.logits) a.logits[r0 + tid] = lg;
-            if (lg > best || (lg == best && r0 + tid < besti)) { best = lg; besti = r0 + tid; }
-          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty_h + b);      // this warp is done with the slot
         }
-        csync();
-        // best over the threads that held rows
-        if (tid < CR) {
-          scratch32[2 * tid] = __float_as_uint(best);
-          scratch32[2 * tid + 1] = uint32_t(besti);
+        // best of each warp, then of the CTA
+        if (lane == 0) {
+          scratch32[2 * warp] = __float_as_uint(best);
+          scratch32[2 * warp + 1] = uint32_t(besti);
         }
-        csync();
+        alive = csync_and(hok) && alive;
         if (tid == 0) {
           float bv = -INFINITY;
           int bi = 0x7fffffff;
-          for (int i = 0; i < CR; ++i) {
+          for (int i = 0; i < kPWarps; ++i) {
             const float v = __uint_as_float(scratch32[2 * i]);
             const int id = int(scratch32[2 * i + 1]);
             if (v > bv || (v == bv && id < bi)) { bv = v; bi = id; }
@@ -1428,7 +1502,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
     }
 #ifdef DFSSM_PHASE_TIMERS
     if (tid == 0 && a.phase) {
-      for (int i = 0; i < PH_N + 2; ++i) a.phase[size_t(w.c) * kPhaseSlots + i] += ptime[i];
+      for (int i = 0; i < PH_N; ++i) a.phase[size_t(w.c) * kPhaseSlots + i] += ptime[i];
       a.phase[size_t(w.c) * kPhaseSlots + kPhaseSlots - 1] += 1;   // calls
     }
 #endif

@@ -76,7 +76,7 @@ class CWsLayout(C.Structure):
     _fields_ = [(n, C.c_size_t) for n in
                 ("total_bytes", "status", "x_in", "xq_in", "sx_in", "acc_in", "u_in", "xd_in", "xdsum_in",
                  "zxbcdt", "xc", "g", "x_out", "xq_out", "sx_out", "acc_out", "u_out", "xd_out", "xdsum_out",
-                 "res", "scratch")]
+                 "res", "scratch", "control")]
 
 
 _lib = None

@@ -158,6 +158,12 @@ typedef struct dfssm_ws_layout {
   size_t xdsum_out;  /* int32 [batch][6] */
   size_t res;        /* fp32  [batch][d_model]    residual stream (model decode only) */
   size_t scratch;    /* internal */
+  size_t control;    /* uint32 [4] control words of the batch-1 token kernel: [0] launch epoch,
+                        [1] abort flag (both zero in a fresh workspace, kept by the library);
+                        [2], [3] test hooks, zero in normal use: [2] = c + 1 makes CTA c
+                        withhold its layer-0 residual words and [3] = n bounds every wait at
+                        n polls, so that a test can make a bounded wait run out without any
+                        GPU fault (the call then returns with a status value in 4 .. 16384). */
 } dfssm_ws_layout;
 
 /* ---- weight packing (not on the timed path) ------------------------------ */

@@ -1,6 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same
 seeded inputs.  Bit-exact for packing and for the int8 x int8 -> int32 low-rank
 partials; max relative error <= 2e-3 for fp outputs and states."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -462,3 +464,72 @@ def test_model_decode_1p3b_b64_parity():
     m = S.gen_model(rng, w["dims"], 4, w["vocab"])
     tok = S.gen_tokens(rng, 64, w["vocab"])
     _teacher_forced(m, tok, 2, all_layers=True)
+
+
+def test_bounded_wait_runs_out_and_is_reported():
+    """Failure detection without a GPU fault: the workspace's test hooks make CTA 0
+    withhold its layer-0 residual words and bound every wait at 4096 polls.  The next
+    layer's gather runs out: the call returns promptly with status value 4 (the
+    residual gather) and the abort flag set, every CTA having left the token; a later
+    call on the same workspace refuses to run (status value 1); a fresh workspace and
+    state decode oracle-exact again."""
+    rng = np.random.default_rng(37)
+    m = S.gen_model(rng, LAYER_SMALL_P, 3, 1000)
+    d = m.dims
+    assert F.launches_per_decode_step(d, 3, 1000) == 1
+    dm = F.DeviceModel.from_host(m)
+    states = [F.DeviceState.zeros(d) for _ in m.layers]
+    call = F.ModelCall(dm, states)
+    ws = F.workspace(d, 3, 1000)
+    L = F.workspace_layout(d, 3, 1000)
+    ctl = F.ws_view(ws, L.control, torch.int32, (4,))
+    ctl[2] = 1
+    ctl[3] = 4096
+    tok = torch.from_numpy(S.gen_tokens(rng, 1, 1000)).to(DEV)
+    out = torch.zeros(1, dtype=torch.int32, device=DEV)
+    t0 = time.time()
+    call(tok, out, ws, None)
+    _sync()
+    assert time.time() - t0 < 60
+    status = int(to_np(F.ws_view(ws, L.status, torch.int32, (1,)))[0])
+    assert status & 4, status
+    assert int(to_np(ctl)[1]) == 1
+    ctl[2] = 0
+    ctl[3] = 0
+    call(tok, out, ws, None)
+    _sync()
+    assert int(to_np(F.ws_view(ws, L.status, torch.int32, (1,)))[0]) & 1
+    _teacher_forced(m, S.gen_tokens(rng, 1, 1000), 2)
+
+
+@pytest.fixture
+def tc_path(monkeypatch):
+    """Batched projections on the tcgen05 kernel (k_proj_tc) for the test's calls."""
+    monkeypatch.setenv("DFSSM_PROJ_PATH", "tc")
+
+
+@pytest.mark.parametrize("d_in,d_out,rank,batch", [(2048, 8512, 32, 16), (4096, 2048, 32, 64), (256, 1064, 8, 40),
+                                                   (2048, 8512, 64, 256), (256, 48, 0, 3)])
+def test_proj_tcgen05_parity(tc_path, d_in, d_out, rank, batch):
+    """The tcgen05 tile kernel against the oracle: int8 codes / partials bit-exact, the
+    projection to fp32 rounding; ragged M tiles (1064, 48 rows) and batch groups."""
+    if rank:
+        p, x = S.proj_workload(d_in, d_out, rank, batch)
+    else:
+        rng = np.random.default_rng(7)
+        p = S.gen_proj(rng, d_out, d_in, 0)
+        x = rng.normal(size=(batch, d_in)).astype(np.float16)
+    _proj_case(p, x, rank)
+
+
+def test_model_decode_tcgen05_batched_parity(tc_path):
+    """A 3-layer small model at batch 12 and a 2-layer 1.3B-shaped one at batch 16,
+    decoded with every projection on the tcgen05 kernel."""
+    d = S.LAYER_SMALL.with_batch(12)
+    rng = np.random.default_rng(38)
+    m = S.gen_model(rng, d, 3, 1000)
+    _teacher_forced(m, S.gen_tokens(rng, 12, 1000), 3)
+    w = S.WORKLOADS["model_48x2048_v50280_b16_256steps"]
+    rng = np.random.default_rng(w["seed"])
+    m = S.gen_model(rng, w["dims"], 2, w["vocab"])
+    _teacher_forced(m, S.gen_tokens(rng, 16, w["vocab"]), 2, all_layers=True)
