@@ -47,11 +47,11 @@ THROTTLE_BITS = {
 
 
 def profiled_traffic():
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary.
-
-    Returns None when the kernel source has changed since those counters were taken.
-    """
-    path = os.path.join(ROOT, "profiles", "k_decode_persistent_model_48x2048_v50280_b1_launches.md")
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, or
+    None with the reason.  Returns None when the kernel source has changed since those
+    counters were taken, or when the summary records that the kernel could not be
+    captured."""
+    path = os.path.join(ROOT, "profiles", "k_decode_persistent_model_48x2048_b1.md")
     src = os.path.join(ROOT, "bit_scaffold_quantized_b200", "csrc", "persistent.cuh")
     try:
         with open(path) as f:
@@ -65,6 +65,13 @@ def profiled_traffic():
     if not t or not h or h.group(1) != sha:
         return None
     return int(t.group(1))
+
+
+def traffic_note(traffic):
+    if traffic is not None:
+        return "dram__bytes_read.sum + dram__bytes_write.sum per launch, profiles/k_decode_persistent_model_48x2048_b1.md"
+    return ("not measured: ncu cannot launch the cooperative cluster token kernel (LaunchFailed under the "
+            "profiler, even for the one-pass launch list); see profiles/k_decode_persistent_model_48x2048_b1.md")
 
 
 def load_peaks():
@@ -318,6 +325,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"no flush: each step streams {bytes_tok / 1e6:.1f} MB > 126 MB L2"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+                     "traffic_source": traffic_note(profiled_traffic()),
                      "kernel": "whole decode step (graph replay)",
                      "algorithmic_bytes_per_step": bytes_tok, "peak_source": peak_kind},
         "roofline_tokens_per_s": round(peak * 1e9 / bytes_tok * d.batch, 1),   # one step = batch tokens

@@ -581,6 +581,10 @@ PPlan plan_persistent(const dfssm_dims* d) {
   // Clusters of 4 or 8 CTAs: the larger co-resident grid wins (clusters of 4 first on a
   // tie), so that every CTA gets as few SSM units and out_proj tiles as possible.
   int best_grid = 0, best_Q = 0, best_U = 0;
+  // DFSSM_TOKEN_MAX_CTAS caps the grid (a diagnostic: a smaller co-resident grid can
+  // be launched under a profiler); unset, the largest co-resident grid is used.
+  int cap = kPlanSMs;
+  if (const char* e = getenv("DFSSM_TOKEN_MAX_CTAS")) cap = std::max(4, std::min(kPlanSMs, atoi(e)));
   for (int Q : {4, 8}) {
     int U = 0;
     const int probe = std::min(kPlanSMs / Q, std::min(units, out_tiles) / Q) * Q;
@@ -591,7 +595,7 @@ PPlan plan_persistent(const dfssm_dims* d) {
     const bool spec = D == Shape2048::D && E == Shape2048::E && H == Shape2048::H && P == Shape2048::P &&
                       N == Shape2048::N && R == Shape2048::R && Q == Shape2048::Q && U == Shape2048::U;
     const int maxc = max_active_clusters(dev, Q, m.total, spec);
-    const int grid = std::min(std::min(maxc, kPlanSMs / Q), std::min(units, out_tiles) / Q) * Q;
+    const int grid = std::min(std::min(maxc, cap / Q), std::min(units, out_tiles) / Q) * Q;
     if (grid > best_grid) {
       best_grid = grid;
       best_Q = Q;
