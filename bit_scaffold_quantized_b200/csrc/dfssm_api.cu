@@ -1,5 +1,7 @@
 // C ABI of libdfssm.so: host-side argument validation, workspace layout and the
 // launch sequences of the DF-SSM decode step.  Declarations and semantics: dfssm.h.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <array>
 #include <cstdarg>
@@ -300,26 +302,94 @@ int launch_proj_bt(const ProjArgs& a, cudaStream_t st) {
   return DFSSM_OK;
 }
 
-// Which scaffold kernel a batched projection takes: the register-fragment mma.sync
-// kernel (k_proj, the default: measured faster end to end so far), or the tcgen05
-// tile kernel (k_proj_tc) when DFSSM_PROJ_PATH=tc is set in the environment (read at
-// every call, so a caller can switch between calls); DFSSM_PROJ_PATH=mma forces k_proj.
+// Which scaffold kernel a batched projection takes: from batch 16 on the tcgen05
+// tile kernel (k_proj_tc), below it the register-fragment mma.sync kernel (k_proj),
+// whose per-row work suits a few batch rows.  DFSSM_PROJ_PATH=tc or =mma in the
+// environment (read at every call) forces one of them, e.g. to compare the two.
 int proj_path_override() {
   const char* e = getenv("DFSSM_PROJ_PATH");
   if (e && strcmp(e, "mma") == 0) return 1;
   if (e && strcmp(e, "tc") == 0) return 2;
   return 0;
 }
-constexpr int kTcMinBatch = 1 << 30;   // the automatic choice never takes the tcgen05 kernel yet
+constexpr int kTcMinBatch = 16;
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against
+// the driver library), looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// The two TMA maps of k_proj_tc: the tiled sign words as [row tiles][K/256 x 128
+// words] (box: 8 tiles x 128 words, no swizzle) and the digit planes as
+// [batch x 6][K] bytes (box: N = 6 BG rows x 128 bytes, 128-byte swizzle).  Rows past
+// the ends read as zeros.
+int proj_tc_maps(const ProjArgs& a, int bg, CUtensorMap* bits, CUtensorMap* planes) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(DFSSM_ERR_CUDA, "k_proj_tc: cuTensorMapEncodeTiled is not available");
+  REQUIRE(aligned16(a.bits) && aligned16(a.xd), DFSSM_ERR_MISALIGNED,
+          "k_proj_tc: sign words and digit planes must be 16-byte aligned");
+  const int kgroups = a.K / kTileCols, ntiles = (a.rows + kTileRows - 1) / kTileRows;
+  const cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t bdim[2] = {cuuint64_t(kgroups) * kTileWords, cuuint64_t(ntiles)};
+  const cuuint64_t bstride[1] = {cuuint64_t(kgroups) * kTileWords * 4};
+  const cuuint32_t bbox[2] = {cuuint32_t(kTileWords), cuuint32_t(kTcTiles)};
+  CUresult r = enc(bits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(a.bits), bdim, bstride, bbox,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DFSSM_ERR_CUDA, "k_proj_tc: sign-word tensor map (%d)", int(r));
+  const cuuint64_t pdim[2] = {cuuint64_t(a.K), cuuint64_t(a.batch) * kDigits};
+  const cuuint64_t pstride[1] = {cuuint64_t(a.K)};
+  const cuuint32_t pbox[2] = {128u, cuuint32_t(kDigits * bg)};
+  r = enc(planes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(a.xd), pdim, pstride, pbox, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DFSSM_ERR_CUDA, "k_proj_tc: digit-plane tensor map (%d)", int(r));
+  return DFSSM_OK;
+}
+
+// K split of a tcgen05 projection: double the CTAs sharing K (a cluster along z)
+// while the grid still fits one wave of the SMs and every CTA keeps >= 2 k-blocks.
+int proj_tc_split(int tiles, int kgroups) {
+  int ks = 1;
+  while (ks < kTcMaxSplit && tiles * ks * 2 <= sm_count() && kgroups % (ks * 2) == 0 && kgroups / (ks * 2) >= 2)
+    ks *= 2;
+  return ks;
+}
 
 template <int EPI, int BG>
 int launch_proj_tc_bg(const ProjArgs& a, cudaStream_t st) {
-  const int smem = int(proj_tc_smem_bytes(BG, a.rank));
+  constexpr int smem = int(proj_tc_smem_bytes(BG));
   cudaError_t e = cudaFuncSetAttribute(k_proj_tc<EPI, BG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "k_proj_tc smem attribute: %s", cudaGetErrorString(e));
-  const dim3 grid((a.rows + kTcM - 1) / kTcM, (a.batch + BG - 1) / BG);
-  k_proj_tc<EPI, BG><<<grid, kTcThreads, smem, st>>>(a);
-  CHECK_LAUNCH("k_proj_tc");
+  REQUIRE(a.rank % 4 == 0, DFSSM_ERR_UNSUPPORTED_SHAPE, "k_proj_tc: rank %d", a.rank);
+  CUtensorMap tb, tp;
+  if (int rc = proj_tc_maps(a, BG, &tb, &tp)) return rc;
+  const int mt = (a.rows + kTcM - 1) / kTcM, gb = (a.batch + BG - 1) / BG;
+  const int ks = proj_tc_split(mt * gb, a.K / kTileCols);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = unsigned(ks);
+  cfg.gridDim = dim3(mt, gb, ks);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = size_t(smem);
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_proj_tc<EPI, BG>, a, tb, tp);
+  if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "k_proj_tc launch: %s", cudaGetErrorString(e));
   return DFSSM_OK;
 }
 

@@ -13,6 +13,8 @@
 //   k_embed, k_quant_rows, k_pack_*   embedding gather, int8 row quantiser, sign packing
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace dfssm {
@@ -471,42 +473,76 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
 //
 // The batched scaffold on the 5th-generation tensor cores: tcgen05.mma kind::i8
 // (0/1 sign bytes times signed digit-plane bytes, int32 accumulators in tensor
-// memory).  A CTA owns one M = 128 tile of projection rows and a group of BG
-// batch rows (N = 6 BG digit-plane columns).  Per 256-column k-block its 128 threads
-// (a) expand the k-block's tiled sign words into 0/1 bytes in natural column order
-// and (b) copy the batch rows' digit planes (cp.async), both into the no-swizzle
-// K-major UMMA layout: 16-byte column chunks c, each holding its rows in 8-row core
-// matrices of 128 bytes, so a K = 32 instruction takes two chunks (leading byte
-// offset = rows x 16) of 8-row groups 128 bytes apart (stride byte offset).  One
-// thread then issues the eight K = 32 MMAs and commits them to the stage's mbarrier;
-// two stages let the next k-block's staging overlap the MMAs.  Every integer sum is
-// exact (|sum| <= 2^20 for K <= 8192); the epilogue reads the accumulators with
-// tcgen05.ld (warp w: TMEM lanes 32w..32w+31 = tile rows) and finishes each (row,
-// batch row) exactly as k_proj does.
+// memory).  A CTA owns one M = 128 tile of projection rows, a group of BG batch rows
+// (N = 6 BG digit-plane columns) and a share of K: gridDim.z CTAs of one cluster
+// split K and add their integer sums over distributed shared memory.  The warps
+// specialise:
+//   warp 0       TMA producer: per 256-column k-block, the 8 row tiles' packed sign
+//                words (one 2D box of 8 x 512 bytes) and the batch rows' digit planes
+//                (two 2D boxes of 128 K-bytes x N rows, 128-byte swizzle) into a ring
+//                of shared-memory stages;
+//   warp 1       MMA issuer (one thread): eight K = 32 MMAs per k-block, A read from
+//                tensor memory and B from the stage, committed to the stage's and the
+//                A buffer's `empty` barriers, the last also to `done`;
+//   warps 2..5   expanders: thread = one tile row (TMEM lane); it gathers the row's
+//                256 sign bits of the k-block from the stage and writes them as 0/1
+//                bytes into one of four A buffers in tensor memory (64 columns each,
+//                4 K-bytes per column);
+//   warps 6..11  LoRA stage 2 while the MMAs run: l[row][b] = sum_j B_q[row][j] u[b][j]
+//                for the rows this CTA finishes, as fp64 tensor-core MMAs (m16n8k4),
+//                into shared memory;
+//   warps 0..7   the epilogue: tcgen05.ld of the accumulators (warp w: TMEM lanes
+//                32 (w mod 4) .. + 31 = tile rows) and each (row, batch row) finished
+//                exactly as k_proj does; with a K split, each CTA folds its plane
+//                sums into one int64 partial per (row, batch row) and stores it
+//                (st.async) into CTA z of the cluster, which adds them for rows
+//                [128 z / Z, 128 (z+1) / Z) and finishes those rows.
+// Keeping A in tensor memory leaves shared memory to the TMA ring and its bandwidth
+// to the B reads.  B uses the canonical 128-byte-swizzle K-major layout: 8-row atoms
+// of 8 x 128 bytes (stride byte offset 1024), the 16-byte chunk of row r at chunk
+// index XOR (r mod 8); a K = 32 instruction starts 32 bytes further into its
+// 128-column slab.  Every integer sum is exact (|sum| <= 2^20 for K <= 8192).  Every
+// wait on an mbarrier is bounded: one that runs out sets status bit 65536 and the
+// roles fall through to the common exit; the one cluster barrier (every CTA arrives at
+// the start and waits before its sends) is reached by every CTA.
 
-constexpr int kTcThreads = 256;      // two warpgroups: both stage; each finishes half the batch rows
-constexpr int kTcM = 128;              // projection rows per CTA (one UMMA M tile)
-constexpr int kTcStages = 2;
+constexpr int kTcWarps = 12;
+constexpr int kTcThreads = kTcWarps * 32;
+constexpr int kTcEpiThreads = 256;              // warps 0..7
+constexpr int kTcLoraThreads = 192;             // warps 6..11
+constexpr int kTcM = 128;                       // projection rows per CTA (one UMMA M tile)
+constexpr int kTcTiles = kTcM / kTileRows;      // 8 sign tiles per CTA
+constexpr int kTcMaxStages = 6;
+constexpr int kTcABufs = 4;                     // A buffers in tensor memory
+constexpr int kTcACol = 256;                    // first TMEM column of the A buffers
+constexpr int kTcTmemCols = 512;
+constexpr int kTcMaxSplit = 8;                  // CTAs of one cluster sharing K
+constexpr long long kTcSpinLimit = 1LL << 24;
+constexpr size_t kTcSmemCap = 225 * 1024;
 
-template <int BG>
-struct TcShape {
-  static constexpr int N = kDigits * BG;                 // digit-plane columns (a multiple of 16)
-  static constexpr int A_BYTES = kTcM * kTileCols;       // 32 KB per k-block
-  static constexpr int B_BYTES = N * kTileCols;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
-  static_assert(N % 16 == 0 && N <= 256, "UMMA N");
-};
-
-__host__ __device__ inline size_t proj_tc_smem_bytes(int bg, int rank) {
-  return size_t(kTcStages) * (size_t(kTcM) * kTileCols + size_t(kDigits) * bg * kTileCols) +
-         size_t(8) * bg * (rank > 0 ? rank : 1) + size_t(4) * bg * kDigits + 1024;
+__host__ __device__ constexpr int tc_stage_bytes(int bg) {
+  return 2 * (kDigits * bg) * 128 + kTcTiles * kTileWords * 4;
+}
+// LoRA sums [128][BG + 1] fp64, the digit-sum terms [BG] int64, the K-split partial
+// scaffold sums [128][BG] int64 (the cluster's CTAs x this CTA's rows), alignment slack.
+__host__ __device__ constexpr size_t tc_tail_bytes(int bg) {
+  return size_t(8) * kTcM * (bg + 1) + size_t(8) * bg + size_t(8) * kTcM * bg + 1024 + 16;
+}
+// Stages of the TMA ring that fit (at least 2).
+__host__ __device__ constexpr int tc_stages(int bg) {
+  return (long long)(kTcSmemCap - tc_tail_bytes(bg)) / tc_stage_bytes(bg) > kTcMaxStages
+             ? kTcMaxStages
+             : int((long long)(kTcSmemCap - tc_tail_bytes(bg)) / tc_stage_bytes(bg));
+}
+__host__ __device__ constexpr size_t proj_tc_smem_bytes(int bg) {
+  return size_t(tc_stages(bg)) * tc_stage_bytes(bg) + tc_tail_bytes(bg);
 }
 
-DFSSM_DEV uint64_t umma_desc_kmajor(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  // start address, leading / stride byte offsets (16-byte units), version 1, no swizzle
-  return uint64_t((saddr >> 4) & 0x3fffu) | (uint64_t((lbo >> 4) & 0x3fffu) << 16) |
-         (uint64_t((sbo >> 4) & 0x3fffu) << 32) | (uint64_t(1) << 46);
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: start address, leading
+// byte offset 16 (unused by this layout), stride byte offset 1024, version 1.
+DFSSM_DEV uint64_t umma_desc_sw128(uint32_t saddr) {
+  return uint64_t((saddr >> 4) & 0x3fffu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
 // Instruction descriptor of kind::i8: D s32 (c_format 2), A and B both signed 8-bit
@@ -517,173 +553,327 @@ DFSSM_DEV constexpr uint32_t umma_idesc_s8() {
   return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(kTcM >> 4) << 24);
 }
 
-DFSSM_DEV void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
+DFSSM_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
+}
+
+DFSSM_DEV bool tc_wait(uint64_t* bar, unsigned parity, unsigned* status, int* fail) {
+  long long spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if (++spins > kTcSpinLimit || *reinterpret_cast<volatile int*>(fail)) {
+      if (spins > kTcSpinLimit && status) atomicOr(status, 65536u);
+      *reinterpret_cast<volatile int*>(fail) = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+DFSSM_DEV void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               :: "r"(smem_u32(bar)) : "memory");
+}
+
+// 48 accumulator columns (one batch-row octet) of this warp's 32 TMEM lanes.
+DFSSM_DEV void tc_load48(uint32_t taddr, uint32_t (&q)[48]) {
+#pragma unroll
+  for (int j = 0; j < 3; ++j)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(q[16 * j + 0]), "=r"(q[16 * j + 1]), "=r"(q[16 * j + 2]), "=r"(q[16 * j + 3]),
+          "=r"(q[16 * j + 4]), "=r"(q[16 * j + 5]), "=r"(q[16 * j + 6]), "=r"(q[16 * j + 7]),
+          "=r"(q[16 * j + 8]), "=r"(q[16 * j + 9]), "=r"(q[16 * j + 10]), "=r"(q[16 * j + 11]),
+          "=r"(q[16 * j + 12]), "=r"(q[16 * j + 13]), "=r"(q[16 * j + 14]), "=r"(q[16 * j + 15])
+        : "r"(taddr + uint32_t(16 * j)));
+}
+
+// Finish one (row, batch-row octet) from its 48 plane sums: sum_d 256^d (2 q_d - T_d)
+// is exact in int64 (|q_d| <= 2^20, so q_4 + 256 q_5 fits 32 bits); al 2^-24 is exact,
+// so al2 * S rounds once, as al * (S 2^-24) does; then the LoRA term and the store.
+template <int EPI, int BG>
+DFSSM_DEV void tc_finish(const ProjArgs& a, const uint32_t (&q)[48], int o, int g8, int nb, int b0, double al2,
+                         double sb, const long long* Ts, const double* lrow) {
+#pragma unroll
+  for (int bi = 0; bi < 8; ++bi) {
+    const int* qd = reinterpret_cast<const int*>(&q[bi * kDigits]);
+    const long long sq = (long long)qd[0] + (long long)qd[1] * 256 + (long long)qd[2] * 65536 +
+                         (long long)qd[3] * 16777216 + (long long)(qd[4] + qd[5] * 256) * 4294967296LL;
+    double y = al2 * double(2 * sq - Ts[g8 + bi]);
+    if (a.rank > 0) y = fma(sb, lrow[g8 + bi], y);
+    if (g8 + bi < nb) proj_epilogue<EPI>(a, b0 + g8 + bi, o, y);
+  }
 }
 
 template <int EPI, int BG>
-__global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(ProjArgs a) {
-  using SH = TcShape<BG>;
-  constexpr int N = SH::N;
-  extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t mbar[kTcStages];
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_proj_tc(ProjArgs a, const __grid_constant__ CUtensorMap tm_bits, const __grid_constant__ CUtensorMap tm_planes) {
+  constexpr int N = kDigits * BG, B_SLAB = N * 128, BITS = kTcTiles * kTileWords * 4;
+  constexpr int STAGE = tc_stage_bytes(BG), S = tc_stages(BG), LS = BG + 1;
+  static_assert(N % 16 == 0 && N <= kTcACol, "UMMA N and the accumulator columns");
+  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(S >= 2, "two stages at least");
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full[kTcMaxStages], empty[kTcMaxStages], aready[kTcABufs], aempty[kTcABufs];
+  __shared__ __align__(8) uint64_t done, rbar;
   __shared__ uint32_t tmem_s;
+  __shared__ int fail;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.x * kTcM, b0 = blockIdx.y * BG;
-  const int K = a.K, kgroups = K / kTileCols;
-  const int ntiles = (a.rows + kTileRows - 1) / kTileRows;
+  const int ks = gridDim.z, kz = blockIdx.z;                 // K split: cluster (1, 1, ks)
+  const int kpc = a.K / kTileCols / ks, kb0 = kz * kpc;      // k-blocks of this CTA
   const int nb = min(BG, a.batch - b0);
-  const int rk = a.rank > 0 ? a.rank : 1;
-  unsigned char* stages = smem;
-  double* us = reinterpret_cast<double*>(smem + kTcStages * SH::STAGE);      // [BG][rank]
-  int* T = reinterpret_cast<int*>(us + BG * rk);                              // [BG][kDigits]
+  const int LR = kTcM / ks, lr0 = kz * LR;                   // rows this CTA finishes
+  const uint32_t raw = smem_u32(smem_raw);
+  unsigned char* stages = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sbase = smem_u32(stages);
+  double* Ls = reinterpret_cast<double*>(stages + S * STAGE);           // [128][BG + 1] LoRA sums
+  long long* Ts = reinterpret_cast<long long*>(Ls + kTcM * LS);         // [BG]: sum_d 256^d T[d]
+  long long* rcv = reinterpret_cast<long long*>(                        // [ks][LR][BG] K-split partials
+      (reinterpret_cast<uintptr_t>(Ts + BG) + 15) & ~uintptr_t(15));
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 :: "r"(smem_u32(&tmem_s)), "n"(SH::TMEM_COLS) : "memory");
+                 :: "r"(smem_u32(&tmem_s)), "n"(kTcTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (tid == 0) {
-    for (int i = 0; i < kTcStages; ++i) mbar_init(&mbar[i], 1);
+  if (tid == 32) {
+    for (int i = 0; i < kTcMaxStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < kTcABufs; ++i) {
+      mbar_init(&aready[i], 4);
+      mbar_init(&aempty[i], 1);
+    }
+    mbar_init(&done, 1);
+    mbar_init(&rbar, 1);
+    fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int i = tid; i < BG * a.rank; i += kTcThreads) {
-    const int bb = i / a.rank, j = i % a.rank;
-    us[i] = bb < nb ? a.u[size_t(b0 + bb) * a.rank + j] : 0.0;
-  }
-  for (int i = tid; i < BG * kDigits; i += kTcThreads) T[i] = i / kDigits < nb ? a.xdsum[size_t(b0) * kDigits + i] : 0;
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = tmem_s;
-  bool ok = true;
+  if (ks > 1) {
+    // the cluster's barriers are initialised before any CTA sends (the matching
+    // wait comes just before the sends); rbar expects every CTA's partials
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    if (tid == 0) mbar_expect_tx(&rbar, unsigned(ks * LR * BG * 8));
+  }
 
-  for (int kb = 0; kb < kgroups; ++kb) {
-    const int st = kb % kTcStages;
-    unsigned char* As = stages + st * SH::STAGE;
-    unsigned char* Bs = As + SH::A_BYTES;
-    if (kb >= kTcStages) {        // the MMAs that last read this stage have completed
-      if (tid == 0) {
-        long long spins = 0;
-        const unsigned par = unsigned(kb / kTcStages - 1) & 1u;
-        while (!mbar_try_wait(&mbar[st], par))
-          if (++spins > (1LL << 24)) { if (a.status) atomicOr(a.status, 65536u); ok = false; break; }
+  if (warp == 0) {
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tm_bits)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tm_planes)) : "memory");
+      int issued = 0;
+      for (int kb = 0; kb < kpc; ++kb) {
+        const int st = kb % S, kg = kb0 + kb;
+        if (kb >= S && !tc_wait(&empty[st], unsigned(kb / S - 1) & 1u, a.status, &fail)) break;
+        const uint32_t sg = sbase + st * STAGE;
+        mbar_expect_tx(&full[st], BITS + 2 * B_SLAB);
+        tma_load_2d(sg + 2 * B_SLAB, &tm_bits, kg * kTileWords, m0 / kTileRows, &full[st]);
+        tma_load_2d(sg, &tm_planes, kg * kTileCols, b0 * kDigits, &full[st]);
+        tma_load_2d(sg + B_SLAB, &tm_planes, kg * kTileCols + 128, b0 * kDigits, &full[st]);
+        issued = kb + 1;
       }
-      __syncthreads();
-    }
-    // digit planes of the batch rows: row n = 6 bb + d, chunk c at c (N 16) + (n / 8) 128 + (n % 8) 16
-    for (int i = tid; i < nb * kDigits * 16; i += kTcThreads) {
-      const int n = i >> 4, c = i & 15;
-      cp_async16(Bs + c * (N * 16) + (n >> 3) * 128 + (n & 7) * 16,
-                 a.xd + (size_t(b0) * kDigits + n) * K + size_t(kb) * kTileCols + c * 16);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    // sign bytes of the 8 row tiles: lane (g, t) of a tile holds rows g and g + 8, and for
-    // m = 0..3 the 16 columns 64 m + 16 t .. + 15 of each: byte 8 e + 4 h + i is bit
-    // 2 m + e + 8 i of word r / 8 + 2 h
-    {
-      const int g = lane >> 2, t = lane & 3;
-      for (int tt = warp; tt < kTcM / kTileRows; tt += kTcThreads / 32) {
-        const int rt = m0 / kTileRows + tt;
-        uint4 wv = make_uint4(0, 0, 0, 0);
-        if (rt < ntiles) wv = __ldg(reinterpret_cast<const uint4*>(a.bits) + (size_t(rt) * kgroups + kb) * 32 + lane);
-        const uint32_t wq[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t W0 = wq[half], W1 = wq[half + 2];
-          const int row = tt * kTileRows + g + 8 * half;
-          unsigned char* rb = As + (row >> 3) * 128 + (row & 7) * 16;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint4 v = make_uint4((W0 >> (2 * m)) & 0x01010101u, (W1 >> (2 * m)) & 0x01010101u,
-                                       (W0 >> (2 * m + 1)) & 0x01010101u, (W1 >> (2 * m + 1)) & 0x01010101u);
-            *reinterpret_cast<uint4*>(rb + (4 * m + t) * (kTcM * 16)) = v;
-          }
+      // no copy may still be landing when the stages are reused or the CTA leaves
+      for (int kb = max(0, issued - S); kb < issued; ++kb) {
+        long long spins = 0;
+        while (!mbar_try_wait(&full[kb % S], unsigned(kb / S) & 1u) && ++spins < kTcSpinLimit) {
         }
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t as = smem_u32(As), bs = smem_u32(Bs);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_s8<N>();
+      for (int kb = 0; kb < kpc; ++kb) {
+        const int st = kb % S, ab = kb % kTcABufs;
+        if (!tc_wait(&full[st], unsigned(kb / S) & 1u, a.status, &fail) ||
+            !tc_wait(&aready[ab], unsigned(kb / kTcABufs) & 1u, a.status, &fail))
+          break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t bs = sbase + st * STAGE;
+        const uint32_t ta = tmem + uint32_t(kTcACol + 64 * ab);
 #pragma unroll
-      for (int kk = 0; kk < kTileCols / 32; ++kk) {
-        const uint64_t ad = umma_desc_kmajor(as + kk * 2 * (kTcM * 16), kTcM * 16, 128);
-        const uint64_t bd = umma_desc_kmajor(bs + kk * 2 * (N * 16), N * 16, 128);
-        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-        asm volatile(
-            "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
-            " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n"
-            :: "r"(tmem), "l"(ad), "l"(bd), "r"(idesc), "r"(acc) : "memory");
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = umma_desc_sw128(bs + (kk >> 2) * B_SLAB + (kk & 3) * 32);
+          const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+          asm volatile(
+              "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+              " tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}\n"
+              :: "r"(tmem), "r"(ta + 8 * kk), "l"(bd), "r"(idesc), "r"(acc) : "memory");
+        }
+        tc_commit(&empty[st]);
+        tc_commit(&aempty[ab]);
       }
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                   :: "r"(smem_u32(&mbar[st])) : "memory");
+      tc_commit(&done);   // tracks every MMA issued above (also after a wait gave up)
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // expander: thread = tile row r (TMEM lane).  Row r = 16 tt + 8 hf + g of tile tt
+    // lives in the 16-byte words of lanes 4 g + t (t = 0..3): word hf holds, for
+    // m = 0..3, bits 2 m (+ 8 i) of columns 64 m + 16 t + i (i = 0..3) and bits 2 m + 1
+    // of columns 64 m + 16 t + 8 + i; word hf + 2 the next four columns of each.  The
+    // 16-byte K chunk c = 4 m + t of the row is then
+    // {w_hf >> 2m, w_hf+2 >> 2m, w_hf >> 2m+1, w_hf+2 >> 2m+1} & 0x01010101.
+    const int r = 32 * (warp & 3) + lane, tt = r >> 4, hf = (r >> 3) & 1, g = r & 7;
+    const uint32_t trow = tmem + (uint32_t(32 * (warp & 3)) << 16);
+    for (int kb = 0; kb < kpc; ++kb) {
+      const int st = kb % S, ab = kb % kTcABufs;
+      if (kb >= kTcABufs && !tc_wait(&aempty[ab], unsigned(kb / kTcABufs - 1) & 1u, a.status, &fail)) break;
+      if (!tc_wait(&full[st], unsigned(kb / S) & 1u, a.status, &fail)) break;
+      const unsigned char* wb = stages + st * STAGE + 2 * B_SLAB + tt * 512 + g * 64;
+      uint32_t w0[4], w1[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint4 v = *reinterpret_cast<const uint4*>(wb + 16 * t);
+        w0[t] = hf ? v.y : v.x;
+        w1[t] = hf ? v.w : v.z;
+      }
+      uint32_t o[64];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int m = c >> 2, t = c & 3;
+        o[4 * c + 0] = (w0[t] >> (2 * m)) & 0x01010101u;
+        o[4 * c + 1] = (w1[t] >> (2 * m)) & 0x01010101u;
+        o[4 * c + 2] = (w0[t] >> (2 * m + 1)) & 0x01010101u;
+        o[4 * c + 3] = (w1[t] >> (2 * m + 1)) & 0x01010101u;
+      }
+      asm volatile(
+          "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+          "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,"
+          "%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};"
+          :: "r"(trow + uint32_t(kTcACol + 64 * ab)),
+             "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7]),
+             "r"(o[8]), "r"(o[9]), "r"(o[10]), "r"(o[11]), "r"(o[12]), "r"(o[13]), "r"(o[14]), "r"(o[15]),
+             "r"(o[16]), "r"(o[17]), "r"(o[18]), "r"(o[19]), "r"(o[20]), "r"(o[21]), "r"(o[22]), "r"(o[23]),
+             "r"(o[24]), "r"(o[25]), "r"(o[26]), "r"(o[27]), "r"(o[28]), "r"(o[29]), "r"(o[30]), "r"(o[31]),
+             "r"(o[32]), "r"(o[33]), "r"(o[34]), "r"(o[35]), "r"(o[36]), "r"(o[37]), "r"(o[38]), "r"(o[39]),
+             "r"(o[40]), "r"(o[41]), "r"(o[42]), "r"(o[43]), "r"(o[44]), "r"(o[45]), "r"(o[46]), "r"(o[47]),
+             "r"(o[48]), "r"(o[49]), "r"(o[50]), "r"(o[51]), "r"(o[52]), "r"(o[53]), "r"(o[54]), "r"(o[55]),
+             "r"(o[56]), "r"(o[57]), "r"(o[58]), "r"(o[59]), "r"(o[60]), "r"(o[61]), "r"(o[62]), "r"(o[63])
+          : "memory");
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aready[ab]);
     }
   }
-  // all MMAs done (the last commit tracks every earlier one)
-  if (tid == 0) {
-    const int kb = kgroups - 1;
-    long long spins = 0;
-    while (!mbar_try_wait(&mbar[kb % kTcStages], unsigned(kb / kTcStages) & 1u))
-      if (++spins > (1LL << 24)) { if (a.status) atomicOr(a.status, 65536u); ok = false; break; }
+  if (warp >= 6) {
+    // LoRA stage 2 of rows [lr0, lr0 + LR) on the fp64 tensor cores: L = B_q u^T as
+    // m16n8k4 MMAs (rows x batch rows x ranks).  In k-step 4 G + s the fragment column
+    // t (thread t of a quad) stands for rank 16 G + 4 t + s, for A (B_q bytes, four
+    // ranks per 32-bit load) and B (u, four ranks per two 16-byte loads) alike.
+    const int lw = warp - 6, g = lane >> 2, t = lane & 3;
+    for (int i = tid - 192; i < BG; i += kTcLoraThreads) {
+      long long sum = 0;
+      if (i < nb)
+        for (int d = kDigits - 1; d >= 0; --d) sum = sum * 256 + a.xdsum[size_t(b0 + i) * kDigits + d];
+      Ts[i] = sum;
+    }
+    const int MT = LR / 16, NT = BG / 8;
+    for (int item = lw; item < MT * NT && a.rank > 0; item += kTcLoraThreads / 32) {
+      const int mt = lr0 / 16 + item / NT, nt = item % NT;
+      const int r0 = 16 * mt + g, r1 = r0 + 8, o0 = m0 + r0, o1 = m0 + r1, bq = b0 + 8 * nt + g;
+      double c[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int G = 0; G < (a.rank + 15) / 16; ++G) {
+        const int j = 16 * G + 4 * t;                      // rank % 4 == 0: j < rank covers j .. j + 3
+        const bool jv = j < a.rank;
+        const int w0 = (jv && o0 < a.rows) ? __ldg(reinterpret_cast<const int*>(a.B + size_t(o0) * a.rank + j)) : 0;
+        const int w1 = (jv && o1 < a.rows) ? __ldg(reinterpret_cast<const int*>(a.B + size_t(o1) * a.rank + j)) : 0;
+        double2 ua = make_double2(0.0, 0.0), ub = ua;
+        if (jv && 8 * nt + g < nb) {
+          const double2* up = reinterpret_cast<const double2*>(a.u + size_t(bq) * a.rank + j);
+          ua = up[0];
+          ub = up[1];
+        }
+        const double uv[4] = {ua.x, ua.y, ub.x, ub.y};
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+          const double a0 = double(int8_t(w0 >> (8 * s4))), a1 = double(int8_t(w1 >> (8 * s4)));
+          asm volatile("mma.sync.aligned.m16n8k4.row.col.f64.f64.f64.f64 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+                       : "+d"(c[0]), "+d"(c[1]), "+d"(c[2]), "+d"(c[3]) : "d"(a0), "d"(a1), "d"(uv[s4]));
+        }
+      }
+      // D fragment: (r0, 2t), (r0, 2t + 1), (r1, 2t), (r1, 2t + 1) of the 16 x 8 tile
+      Ls[r0 * LS + 8 * nt + 2 * t] = c[0];
+      Ls[r0 * LS + 8 * nt + 2 * t + 1] = c[1];
+      Ls[r1 * LS + 8 * nt + 2 * t] = c[2];
+      Ls[r1 * LS + 8 * nt + 2 * t + 1] = c[3];
+    }
+  }
+  // the epilogue warps wait for the MMAs; everyone then sees Ls and Ts
+  bool ok = true;
+  if (warp < 8) {
+    ok = tc_wait(&done, 0u, a.status, &fail);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   }
   __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-
-  // epilogue: thread = tile row (TMEM lane quarter = warp % 4); warpgroup wg finishes
-  // the batch-row octets wg, wg + 2, ... (48 accumulator columns at a time).  The
-  // row's LoRA B bytes are read once; u comes from shared memory.
-  const int quarter = warp & 3, wg = warp >> 2;
-  const int r = 32 * quarter + lane, o = m0 + r;
-  const double al = o < a.rows ? h2d(a.alpha[o]) : 0.0;
-  const double sb = (o < a.rows && a.rank > 0) ? h2d(a.sB[o]) : 0.0;
-  const int8_t* Br = a.B + size_t(o < a.rows ? o : 0) * a.rank;
-  for (int g8 = 8 * wg; g8 < BG; g8 += 16) {
-    uint32_t q[48];
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      const uint32_t taddr = tmem + (uint32_t(32 * quarter) << 16) + uint32_t(g8 * kDigits + 16 * j);
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-          : "=r"(q[16 * j + 0]), "=r"(q[16 * j + 1]), "=r"(q[16 * j + 2]), "=r"(q[16 * j + 3]),
-            "=r"(q[16 * j + 4]), "=r"(q[16 * j + 5]), "=r"(q[16 * j + 6]), "=r"(q[16 * j + 7]),
-            "=r"(q[16 * j + 8]), "=r"(q[16 * j + 9]), "=r"(q[16 * j + 10]), "=r"(q[16 * j + 11]),
-            "=r"(q[16 * j + 12]), "=r"(q[16 * j + 13]), "=r"(q[16 * j + 14]), "=r"(q[16 * j + 15])
-          : "r"(taddr));
+  ok = ok && !*reinterpret_cast<volatile int*>(&fail);
+  const int quarter = warp & 3, h = (warp >> 2) & 1;
+  if (ks == 1) {
+    if (warp < 8) {
+      // warp w: TMEM lanes 32 (w mod 4) .. + 31, batch-row octets w / 4, + 2, ...
+      const int r = 32 * quarter + lane, o = m0 + r;
+      const double al2 = o < a.rows ? h2d(a.alpha[o]) * (1.0 / 16777216.0) : 0.0;
+      const double sb = (o < a.rows && a.rank > 0) ? h2d(a.sB[o]) : 0.0;
+      for (int g8 = 8 * h; g8 < BG; g8 += 16) {
+        uint32_t q[48];
+        tc_load48(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(g8 * kDigits), q);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (ok && o < a.rows) tc_finish<EPI, BG>(a, q, o, g8, nb, b0, al2, sb, Ts, Ls + r * LS);
+      }
     }
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-    if (o < a.rows && ok) {
+  } else {
+    // K split: each epilogue thread folds its row's plane sums into one exact int64
+    // partial sum_d 256^d q_d per batch row and stores it (st.async) into the CTA
+    // that finishes the row, slot [kz][row - its first row][batch row]; that CTA adds
+    // the cluster's partials once its barrier has counted all of them
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if (warp < 8) {
+      const int r = 32 * quarter + lane, p = r / LR, rl = r % LR;
+      const uint32_t dst = cluster_map(smem_u32(rcv + (kz * LR + rl) * BG), unsigned(p));
+      const uint32_t bar = cluster_map(smem_u32(&rbar), unsigned(p));
+      for (int g8 = 8 * h; g8 < BG; g8 += 16) {
+        uint32_t q[48];
+        tc_load48(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(g8 * kDigits), q);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-      for (int bi = 0; bi < 8; ++bi) {
-        const int bb = g8 + bi;
-        if (bb < nb) {
-          long long S = 0;
+        for (int bi = 0; bi < 8; bi += 2) {
+          long long sq[2];
 #pragma unroll
-          for (int d = kDigits - 1; d >= 0; --d) S = S * 256 + (2LL * int(q[bi * kDigits + d]) - T[bb * kDigits + d]);
-          double y = al * (double(S) * (1.0 / 16777216.0));
-          if (a.rank > 0) {
-            const double* ur = us + bb * a.rank;
-            const int* b4 = reinterpret_cast<const int*>(Br);
-            double l[4] = {0.0, 0.0, 0.0, 0.0};
-            for (int j4 = 0; j4 < a.rank / 4; ++j4) {
-              const int v = __ldg(b4 + j4);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) l[e] = fma(double(int8_t(v >> (8 * e))), ur[4 * j4 + e], l[e]);
-            }
-            y = fma(sb, (l[0] + l[1]) + (l[2] + l[3]), y);
+          for (int e = 0; e < 2; ++e) {
+            const int* qd = reinterpret_cast<const int*>(&q[(bi + e) * kDigits]);
+            sq[e] = (long long)qd[0] + (long long)qd[1] * 256 + (long long)qd[2] * 65536 +
+                    (long long)qd[3] * 16777216 + (long long)(qd[4] + qd[5] * 256) * 4294967296LL;
           }
-          proj_epilogue<EPI>(a, b0 + bb, o, y);
+          asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.s64 [%0], {%1, %2}, [%3];"
+                       :: "r"(dst + uint32_t(8 * (g8 + bi))), "l"(sq[0]), "l"(sq[1]), "r"(bar) : "memory");
         }
+      }
+    }
+    if (tid < kTcEpiThreads) {
+      const bool got = tc_wait(&rbar, 0u, a.status, &fail);
+      const int rl = tid % LR, slot = tid / LR, nslot = kTcEpiThreads / LR;
+      const int r = lr0 + rl, o = m0 + r;
+      const double al2 = o < a.rows ? h2d(a.alpha[o]) * (1.0 / 16777216.0) : 0.0;
+      const double sb = (o < a.rows && a.rank > 0) ? h2d(a.sB[o]) : 0.0;
+      for (int b8 = slot; b8 < BG && got && ok && o < a.rows; b8 += nslot) {
+        long long sq = 0;
+        for (int p = 0; p < ks; ++p) sq += rcv[(p * LR + rl) * BG + b8];
+        double y = al2 * double(2 * sq - Ts[b8]);
+        if (a.rank > 0) y = fma(sb, Ls[r * LS + b8], y);
+        if (b8 < nb) proj_epilogue<EPI>(a, b0 + b8, o, y);
       }
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "n"(SH::TMEM_COLS) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "n"(kTcTmemCols) : "memory");
 }
 
 // ------------------------------------------------------------------ SSM step

@@ -509,10 +509,13 @@ def tc_path(monkeypatch):
 
 
 @pytest.mark.parametrize("d_in,d_out,rank,batch", [(2048, 8512, 32, 16), (4096, 2048, 32, 64), (256, 1064, 8, 40),
-                                                   (2048, 8512, 64, 256), (256, 48, 0, 3)])
+                                                   (2048, 8512, 64, 256), (256, 48, 0, 3), (1024, 48, 16, 5),
+                                                   (8192, 256, 128, 33)])
 def test_proj_tcgen05_parity(tc_path, d_in, d_out, rank, batch):
     """The tcgen05 tile kernel against the oracle: int8 codes / partials bit-exact, the
-    projection to fp32 rounding; ragged M tiles (1064, 48 rows) and batch groups."""
+    projection to fp32 rounding; ragged M tiles (1064, 48 rows) and batch groups (40,
+    33 rows), K split over clusters of 2, 4 and 8 CTAs (8512 rows at batch 16, 2048 at
+    64, 48 rows at K 1024, 256 rows at K 8192), LoRA ranks 0 to 128."""
     if rank:
         p, x = S.proj_workload(d_in, d_out, rank, batch)
     else:
