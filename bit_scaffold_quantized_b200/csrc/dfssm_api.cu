@@ -163,15 +163,13 @@ void layer_layout(const dfssm_dims* d, int n_layer, int vocab, dfssm_ws_layout* 
   L->u_out = bp.take(8 * B * r);
   L->xd_out = bp.take(B * kDigits * E);
   L->xdsum_out = bp.take(4 * B * kDigits);
-  // internal scratch: persistent-kernel / LM-head words, then the multi-launch
-  // path's per-(batch, head) step size and decay (fp64 pairs)
-  const size_t dta = 16 * B * size_t(d->nheads);
+  // internal scratch: persistent-kernel / LM-head words
   if (n_layer > 0) {
     L->res = bp.take(4 * B * D);
-    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), kHeadBlocks) + dta);
+    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), kHeadBlocks));
   } else {
     L->res = kNone;
-    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), 0) + dta);
+    L->scratch = bp.take(persistent_scratch_bytes(d->batch, d->d_model, d->d_inner, in_rows(d), 0));
   }
   // the batch-1 token kernel's control words follow the LM-head partials in the scratch
   L->control = L->scratch + align256(size_t(8) * B * (n_layer > 0 ? kHeadBlocks : 1));
@@ -190,7 +188,6 @@ struct Bufs {
   Act in, out;
   double* zxbcdt; double* xc; float* g;
   float* res; unsigned char* scratch;
-  double* dta;     // [batch][nheads][2] step size and decay (multi-launch path)
 };
 
 Bufs bind(void* ws, const dfssm_ws_layout& L, const dfssm_dims* d) {
@@ -206,7 +203,6 @@ Bufs bind(void* ws, const dfssm_ws_layout& L, const dfssm_dims* d) {
   b.g = at<float>(ws, L.g);
   b.res = L.res == kNone ? nullptr : at<float>(ws, L.res);
   b.scratch = at<unsigned char>(ws, L.scratch);
-  b.dta = at<double>(ws, L.total_bytes) - 2 * size_t(d->batch) * d->nheads;
   return b;
 }
 
@@ -219,11 +215,28 @@ int launch_prologue(int K, int rank, int batch, const float* src, const uint16_t
   a.K = K; a.rank = rank; a.src = src; a.src16 = src16; a.w = w;
   a.x = o.x; a.xq = o.xq; a.sx = o.sx; a.xd = o.xd; a.xdsum = o.xdsum;
   a.A = p->A; a.sA = p->sA; a.acc = o.acc; a.u = o.u;
-  // the API limits (K a multiple of 256 and <= 8192, rank <= 128) are the kernel's
+  // the API limits (K a multiple of 256 and <= 8192, rank <= 128) are the kernels'
   REQUIRE(K % (16 * kPrologueCQ) == 0 && K <= kPrologueCQ * kPrologueClThreads * kPrologueClVals &&
-              rank <= kPrologueMaxRank,
+              K <= 4 * kPrologueRowThreads * kPrologueRowGroups && rank <= kPrologueMaxRank,
           DFSSM_ERR_UNSUPPORTED_SHAPE, "prologue: K (%d) or rank (%d) out of range", K, rank);
-  k_prologue_cl<MODE><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a);
+  if (batch >= kPrologueRowMinBatch) {
+    const int g = (K + 4 * kPrologueRowThreads - 1) / (4 * kPrologueRowThreads);
+    switch (g) {
+      case 1: k_prologue_row<MODE, 1><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
+      case 2: k_prologue_row<MODE, 2><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
+      case 3: k_prologue_row<MODE, 3><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
+      default: k_prologue_row<MODE, 4><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
+    }
+    CHECK_LAUNCH("k_prologue_row");
+    return DFSSM_OK;
+  }
+  const int v = (K / kPrologueCQ + kPrologueClThreads - 1) / kPrologueClThreads;
+  switch (v) {
+    case 1: k_prologue_cl<MODE, 1><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
+    case 2: k_prologue_cl<MODE, 2><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
+    case 3: k_prologue_cl<MODE, 3><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
+    default: k_prologue_cl<MODE, 4><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
+  }
   CHECK_LAUNCH("k_prologue_cl");
   return DFSSM_OK;
 }
@@ -459,7 +472,9 @@ template <int NCH, typename ST>
 int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
   const int occ_blocks = occupancy(reinterpret_cast<const void*>(k_ssm_stream<NCH, ST>), kSsmStreamThreads, smem);
   const int items = sa.batch * sa.H;
-  const int grid = std::max(1, std::min(items, occ_blocks * sm_count()));
+  // every block's items fit its step-size table
+  const int grid = std::max((items + kSsmStreamMaxItems - 1) / kSsmStreamMaxItems,
+                            std::max(1, std::min(items, occ_blocks * sm_count())));
   k_ssm_stream<NCH, ST><<<grid, kSsmStreamThreads, smem, st>>>(sa);
   CHECK_LAUNCH("k_ssm_stream");
   return DFSSM_OK;
@@ -472,7 +487,7 @@ int launch_ssm_t(const SsmArgs& sa, cudaStream_t st) {
   const bool aligned = (size_t(sa.conv_dim) * 8) % 16 == 0 && (size_t(sa.in_rows) * 8) % 16 == 0 &&
                        (size_t(sa.E) * 8) % 16 == 0 && (size_t(sa.P) * 8) % 16 == 0 &&
                        (size_t(sa.P) * sa.N * sizeof(ST)) % 16 == 0 &&
-                       aligned16(sa.state) && aligned16(sa.xc) && aligned16(sa.zx) && aligned16(sa.dta);
+                       aligned16(sa.state) && aligned16(sa.xc) && aligned16(sa.zx);
   if (aligned && smem <= kSsmStreamSmemCap) {
     if (sa.N <= 128) return launch_ssm_stream<1, ST>(sa, smem, st);
     return launch_ssm_stream<2, ST>(sa, smem, st);
@@ -498,13 +513,12 @@ int layer_multikernel(const dfssm_dims* d, const dfssm_layer_weights* w, const d
   pa.zx = b.zxbcdt;
   pa.conv_lo = E; pa.conv_dim = C; pa.conv_w = w->conv_w; pa.conv_b = w->conv_b;
   pa.conv_state = s->conv_state; pa.xc = b.xc;
-  pa.dt_lo = E + C; pa.nheads = d->nheads; pa.dt_bias = w->dt_bias; pa.A_log = w->A_log; pa.dta = b.dta;
   if ((rc = launch_proj<EPI_INPROJ>(pa, st))) return rc;
   SsmArgs sa{};
   sa.H = d->nheads; sa.P = d->headdim; sa.N = d->d_state; sa.E = E; sa.conv_dim = C; sa.in_rows = in_rows(d);
   sa.zx = b.zxbcdt; sa.xc = b.xc; sa.dt_bias = w->dt_bias; sa.A_log = w->A_log; sa.D = w->D;
   sa.state = s->ssm_state; sa.state16 = d->ssm_state_dtype == 1;
-  sa.g = b.g; sa.dta = b.dta; sa.batch = B; sa.status = b.status;
+  sa.g = b.g; sa.dt_lo = E + C; sa.batch = B; sa.status = b.status;
   if ((rc = launch_ssm(sa, st))) return rc;
   if ((rc = launch_prologue<0>(E, r, B, b.g, nullptr, w->gnorm_w, b.out, &w->out, st))) return rc;
   ProjArgs po = proj_args(&w->out, r, B, b.out);

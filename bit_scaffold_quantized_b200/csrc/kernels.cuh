@@ -122,7 +122,9 @@ constexpr int kPrologueClThreads = 512;  // two CTAs per SM (64 registers): a ba
 constexpr int kPrologueClVals = 4;      // K / CQ / 512 <= 4: K <= 8192
 constexpr int kPrologueMaxRank = 128;
 
-template <int MODE>
+// V = ceil(K / CQ / 512) values per thread (no padding values through the
+// normalisation's slow path).
+template <int MODE, int V>
 __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueClThreads, 2)
     k_prologue_cl(PrologueArgs a) {
   constexpr int CQ = kPrologueCQ, NW = kPrologueClThreads / 32;
@@ -148,21 +150,21 @@ __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueC
       av[rr][m] = (j < a.rank && c < nvq) ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K + k0) + c)
                                           : make_uint4(0, 0, 0, 0);
     }
-  uint32_t h[kPrologueClVals];
+  uint32_t h[V];
   float am = 0.f;
   if (MODE == 0) {
     const float* v = a.src + size_t(b) * K + k0;
-    float vf[kPrologueClVals];
-    uint16_t wh[kPrologueClVals];
+    float vf[V];
+    uint16_t wh[V];
 #pragma unroll
-    for (int i = 0; i < kPrologueClVals; ++i) {
+    for (int i = 0; i < V; ++i) {
       const int k = tid + i * kPrologueClThreads;
       vf[i] = k < Kq ? v[k] : 0.f;
       wh[i] = k < Kq ? a.w[k0 + k] : uint16_t(0);
     }
     double ss = 0.0;
 #pragma unroll
-    for (int i = 0; i < kPrologueClVals; ++i) ss = fma(double(vf[i]), double(vf[i]), ss);
+    for (int i = 0; i < V; ++i) ss = fma(double(vf[i]), double(vf[i]), ss);
     ss = block_sum_d(ss, redd);
     cluster_sync_all();                    // every CTA of the cluster runs: remote stores allowed
     if (tid < CQ) st_cluster_f64(cluster_map(smem_u32(&xss[q]), tid), ss);
@@ -173,15 +175,17 @@ __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueC
     const double rs = 1.0 / sqrt(sst / double(K) + kEpsD);
     const float rs32 = float(rs);
 #pragma unroll
-    for (int i = 0; i < kPrologueClVals; ++i) {
+    for (int i = 0; i < V; ++i) {
       const int k = tid + i * kPrologueClThreads;
-      h[i] = k < Kq ? norm_fp16(vf[i], rs, rs32, half_to_float_bits(wh[i])) : 0u;
+      h[i] = 0u;
+      if (k >= Kq) continue;
+      h[i] = norm_fp16(vf[i], rs, rs32, half_to_float_bits(wh[i]));
       am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
-      if (k < Kq && a.x) a.x[size_t(b) * K + k0 + k] = uint16_t(h[i]);
+      if (a.x) a.x[size_t(b) * K + k0 + k] = uint16_t(h[i]);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < kPrologueClVals; ++i) {
+    for (int i = 0; i < V; ++i) {
       const int k = tid + i * kPrologueClThreads;
       h[i] = k < Kq ? a.src16[size_t(b) * K + k0 + k] : 0u;
       am = fmaxf(am, fabsf(half_to_float_bits(h[i])));
@@ -200,7 +204,7 @@ __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueC
 #pragma unroll
   for (int d = 0; d < kDigits; ++d) dsum[d] = 0;
 #pragma unroll
-  for (int i = 0; i < kPrologueClVals; ++i) {
+  for (int i = 0; i < V; ++i) {
     const int k = tid + i * kPrologueClThreads;
     if (k < Kq) {
       const int8_t c = amt > 0.f ? int8_t(quant_code_bits(half_to_float_bits(h[i]), sx, rcp)) : int8_t(0);
@@ -273,6 +277,161 @@ __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueC
   }
 }
 
+// Row prologue: the same outputs as k_prologue_cl from one 512-thread CTA per batch
+// row (grid (B)), for batches that fill the GPU with rows: no cluster exchange, three
+// block barriers.  Thread t owns the 4-column groups t, t + 512, ... (16-byte loads,
+// one word per group and output plane); warp w takes LoRA rows w, w + 16, ... (the
+// first one's slice loaded up front).  The sum of squares and max |x| are reduced by
+// every warp from the 16 warp partials in a fixed order.
+constexpr int kPrologueRowThreads = 512;
+constexpr int kPrologueRowGroups = 4;    // 4-column groups per thread: K <= 8192
+constexpr int kPrologueRowMinBatch = 16;
+
+// G = ceil(K / 2048) groups per thread, so that no thread carries padding columns
+// through the normalisation (a zero takes the slow exact-rounding path).
+template <int MODE, int G>
+__global__ void __launch_bounds__(kPrologueRowThreads, 1) k_prologue_row(PrologueArgs a) {
+  constexpr int NW = kPrologueRowThreads / 32, PRE = 4;
+  __shared__ double redd[NW];
+  __shared__ float redf[NW];
+  __shared__ int red6[NW][kDigits];
+  __shared__ __align__(16) int8_t qs[8192];
+  const int K = a.K, b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nvq = K / 16;                                   // 16-byte chunks of a row
+  uint4 av[PRE];
+#pragma unroll
+  for (int m = 0; m < PRE; ++m) {
+    const int c = lane + 32 * m;
+    av[m] = (warp < a.rank && c < nvq) ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(warp) * K) + c)
+                                       : make_uint4(0, 0, 0, 0);
+  }
+  uint32_t h[G][4];
+  float am = 0.f;
+  if (MODE == 0) {
+    float vf[G][4];
+    uint2 wh[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int k = 4 * (tid + kPrologueRowThreads * g);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      uint2 w = make_uint2(0u, 0u);
+      if (k < K) {
+        v = *reinterpret_cast<const float4*>(a.src + size_t(b) * K + k);
+        w = *reinterpret_cast<const uint2*>(a.w + k);
+      }
+      vf[g][0] = v.x; vf[g][1] = v.y; vf[g][2] = v.z; vf[g][3] = v.w;
+      wh[g] = w;
+    }
+    double ss = 0.0;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss = fma(double(vf[g][e]), double(vf[g][e]), ss);
+    ss = warp_sum_d(ss);
+    if (lane == 0) redd[warp] = ss;
+    __syncthreads();
+    const double sst = warp_sum_d(lane < NW ? redd[lane] : 0.0);
+    const double rs = 1.0 / sqrt(sst / double(K) + kEpsD);
+    const float rs32 = float(rs);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int k = 4 * (tid + kPrologueRowThreads * g);
+      const uint32_t wv[4] = {wh[g].x & 0xffffu, wh[g].x >> 16, wh[g].y & 0xffffu, wh[g].y >> 16};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) h[g][e] = 0u;
+      if (k >= K) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h[g][e] = norm_fp16(vf[g][e], rs, rs32, half_to_float_bits(wv[e]));
+        am = fmaxf(am, fabsf(half_to_float_bits(h[g][e])));
+      }
+      if (a.x)
+        *reinterpret_cast<uint2*>(a.x + size_t(b) * K + k) =
+            make_uint2(h[g][0] | (h[g][1] << 16), h[g][2] | (h[g][3] << 16));
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int k = 4 * (tid + kPrologueRowThreads * g);
+      uint2 v = make_uint2(0u, 0u);
+      if (k < K) v = *reinterpret_cast<const uint2*>(a.src16 + size_t(b) * K + k);
+      h[g][0] = v.x & 0xffffu; h[g][1] = v.x >> 16; h[g][2] = v.y & 0xffffu; h[g][3] = v.y >> 16;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(half_to_float_bits(h[g][e])));
+    }
+  }
+  am = warp_max(am);
+  if (lane == 0) redf[warp] = am;
+  __syncthreads();
+  const float amt = warp_max(lane < NW ? redf[lane] : 0.f);
+  const float sx = amt > 0.f ? __fdiv_rn(amt, 127.f) : 1.f;
+  const float rcp = __frcp_rn(sx);
+  int dsum[kDigits];
+#pragma unroll
+  for (int d = 0; d < kDigits; ++d) dsum[d] = 0;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int k = 4 * (tid + kPrologueRowThreads * g);
+    if (k < K) {
+      uint32_t cw = 0u, pw[kDigits] = {0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t c = amt > 0.f ? uint32_t(quant_code_bits(half_to_float_bits(h[g][e]), sx, rcp)) & 0xffu : 0u;
+        cw |= c << (8 * e);
+        uint32_t lo, hi;
+        digits_of(h[g][e], &lo, &hi);
+        const uint32_t w6[kDigits] = {lo, lo >> 8, lo >> 16, lo >> 24, hi, hi >> 8};
+#pragma unroll
+        for (int d = 0; d < kDigits; ++d) {
+          pw[d] |= (w6[d] & 0xffu) << (8 * e);
+          dsum[d] += int8_t(w6[d] & 0xffu);
+        }
+      }
+      *reinterpret_cast<uint32_t*>(qs + k) = cw;
+      *reinterpret_cast<uint32_t*>(a.xq + size_t(b) * K + k) = cw;
+#pragma unroll
+      for (int d = 0; d < kDigits; ++d)
+        *reinterpret_cast<uint32_t*>(a.xd + (size_t(b) * kDigits + d) * K + k) = pw[d];
+    }
+  }
+#pragma unroll
+  for (int d = 0; d < kDigits; ++d) {
+    const int t = __reduce_add_sync(0xffffffffu, dsum[d]);
+    if (lane == 0) red6[warp][d] = t;
+  }
+  __syncthreads();                         // codes and the warps' plane sums complete
+  if (tid < kDigits) {
+    int t = 0;
+    for (int w = 0; w < NW; ++w) t += red6[w][tid];
+    a.xdsum[b * kDigits + tid] = t;
+    if (tid == 0) a.sx[b] = sx;
+  }
+  const uint4* q16 = reinterpret_cast<const uint4*>(qs);
+  for (int j = warp; j < a.rank; j += NW) {
+    int acc = 0;
+    for (int c = lane, m = 0; c < nvq; c += 32, ++m) {
+      uint4 w4;
+      if (j == warp && m < PRE) {
+#pragma unroll
+        for (int mm = 0; mm < PRE; ++mm)
+          if (mm == m) w4 = av[mm];
+      } else {
+        w4 = __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K) + c);
+      }
+      const uint4 x4 = q16[c];
+      acc = __dp4a(int(w4.x), int(x4.x), acc);
+      acc = __dp4a(int(w4.y), int(x4.y), acc);
+      acc = __dp4a(int(w4.z), int(x4.z), acc);
+      acc = __dp4a(int(w4.w), int(x4.w), acc);
+    }
+    acc = warp_sum_i(acc);
+    if (lane == 0) {
+      a.acc[size_t(b) * a.rank + j] = acc;
+      a.u[size_t(b) * a.rank + j] = (double(acc) * h2d(a.sA[j])) * double(sx);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ projection
 
 enum { EPI_STORE = 0, EPI_RESID = 1, EPI_INPROJ = 2, EPI_ZX = 3 };
@@ -294,11 +453,6 @@ struct ProjArgs {
   const uint16_t* conv_b;  // [conv_dim]
   float* conv_state;       // fp32 [batch][3][conv_dim]
   double* xc;              // fp64 [batch][conv_dim]
-  // EPI_INPROJ step sizes: rows [dt_lo, dt_lo + nheads) are dt_raw of each head
-  int dt_lo, nheads;
-  const float* dt_bias;    // [nheads]
-  const float* A_log;      // [nheads]
-  double* dta;             // fp64 [batch][nheads][2]: dt = softplus(dt_raw + dt_bias), dA = exp(-dt exp(A_log))
   unsigned* status;        // workspace status word (value 65536: a tensor-core wait gave up), may be null
 };
 
@@ -343,12 +497,57 @@ DFSSM_DEV void proj_epilogue(const ProjArgs& a, int b, int o, double y) {
       cs[c] = float(s1);
       cs[a.conv_dim + c] = float(s2);
       cs[2 * a.conv_dim + c] = float(y);
-    } else if (o >= a.dt_lo && o < a.dt_lo + a.nheads) {
-      const int hh = o - a.dt_lo;
-      const double dt = softplus_d(y + double(a.dt_bias[hh]));
-      a.dta[(size_t(b) * a.nheads + hh) * 2] = dt;
-      a.dta[(size_t(b) * a.nheads + hh) * 2 + 1] = exp(dt * -exp(double(a.A_log[hh])));
     }
+  }
+}
+
+// proj_epilogue for up to M batch rows bs[0..n) of one projection row o, with every
+// load the stores could alias (the residual, the conv state) issued before the first
+// store, so that a thread waits for one round trip per group rather than per output.
+template <int EPI, int M>
+DFSSM_DEV void proj_epilogue_group(const ProjArgs& a, int o, const int (&bs)[M], const double (&ys)[M], int n) {
+  if (EPI == EPI_RESID) {
+    float r[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) r[i] = i < n ? a.out[size_t(bs[i]) * a.rows + o] : 0.f;
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+      if (i < n) a.out[size_t(bs[i]) * a.rows + o] = float(double(r[i]) + ys[i]);
+  } else if (EPI == EPI_INPROJ && o - a.conv_lo >= 0 && o - a.conv_lo < a.conv_dim) {
+    const int c = o - a.conv_lo, cd = a.conv_dim;
+    float s0[M], s1[M], s2[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+      const float* cs = a.conv_state + size_t(i < n ? bs[i] : 0) * 3 * cd;
+      s0[i] = i < n ? cs[c] : 0.f;
+      s1[i] = i < n ? cs[cd + c] : 0.f;
+      s2[i] = i < n ? cs[2 * cd + c] : 0.f;
+    }
+    const uint2 wv = *reinterpret_cast<const uint2*>(a.conv_w + size_t(c) * 4);
+    const double w0 = h2d(uint16_t(wv.x & 0xffff)), w1 = h2d(uint16_t(wv.x >> 16));
+    const double w2 = h2d(uint16_t(wv.y & 0xffff)), w3 = h2d(uint16_t(wv.y >> 16)), cb = h2d(a.conv_b[c]);
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+      if (i < n) {
+        const int b = bs[i];
+        const double y = ys[i];
+        a.zx[size_t(b) * a.rows + o] = y;
+        double pre = cb;
+        pre = fma(w0, double(s0[i]), pre);
+        pre = fma(w1, double(s1[i]), pre);
+        pre = fma(w2, double(s2[i]), pre);
+        pre = fma(w3, y, pre);
+        a.xc[size_t(b) * cd + c] = silu_d(pre);
+        float* cs = a.conv_state + size_t(b) * 3 * cd;
+        cs[c] = s1[i];
+        cs[cd + c] = s2[i];
+        cs[2 * cd + c] = float(y);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+      if (i < n) proj_epilogue<EPI>(a, bs[i], o, ys[i]);
   }
 }
 
@@ -595,6 +794,8 @@ DFSSM_DEV void tc_load48(uint32_t taddr, uint32_t (&q)[48]) {
 template <int EPI, int BG>
 DFSSM_DEV void tc_finish(const ProjArgs& a, const uint32_t (&q)[48], int o, int g8, int nb, int b0, double al2,
                          double sb, const long long* Ts, const double* lrow) {
+  int bs[8];
+  double ys[8];
 #pragma unroll
   for (int bi = 0; bi < 8; ++bi) {
     const int* qd = reinterpret_cast<const int*>(&q[bi * kDigits]);
@@ -602,8 +803,10 @@ DFSSM_DEV void tc_finish(const ProjArgs& a, const uint32_t (&q)[48], int o, int 
                          (long long)qd[3] * 16777216 + (long long)(qd[4] + qd[5] * 256) * 4294967296LL;
     double y = al2 * double(2 * sq - Ts[g8 + bi]);
     if (a.rank > 0) y = fma(sb, lrow[g8 + bi], y);
-    if (g8 + bi < nb) proj_epilogue<EPI>(a, b0 + g8 + bi, o, y);
+    bs[bi] = b0 + g8 + bi;
+    ys[bi] = y;
   }
+  proj_epilogue_group<EPI, 8>(a, o, bs, ys, min(8, nb - g8));
 }
 
 template <int EPI, int BG>
@@ -861,13 +1064,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int r = lr0 + rl, o = m0 + r;
       const double al2 = o < a.rows ? h2d(a.alpha[o]) * (1.0 / 16777216.0) : 0.0;
       const double sb = (o < a.rows && a.rank > 0) ? h2d(a.sB[o]) : 0.0;
-      for (int b8 = slot; b8 < BG && got && ok && o < a.rows; b8 += nslot) {
-        long long sq = 0;
-        for (int p = 0; p < ks; ++p) sq += rcv[(p * LR + rl) * BG + b8];
-        double y = al2 * double(2 * sq - Ts[b8]);
-        if (a.rank > 0) y = fma(sb, Ls[r * LS + b8], y);
-        if (b8 < nb) proj_epilogue<EPI>(a, b0 + b8, o, y);
+      // batch rows slot, slot + nslot, ... (at most 8: nslot >= 4 as LR <= 64)
+      int bs[8];
+      double ys[8];
+      int n = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int b8 = slot + i * nslot;
+        bs[i] = b0 + b8;
+        ys[i] = 0.0;
+        if (b8 < BG && b8 < nb) {
+          long long sq = 0;
+          for (int p = 0; p < ks; ++p) sq += rcv[(p * LR + rl) * BG + b8];
+          double y = al2 * double(2 * sq - Ts[b8]);
+          if (a.rank > 0) y = fma(sb, Ls[r * LS + b8], y);
+          ys[i] = y;
+          n = i + 1;
+        }
       }
+      if (got && ok && o < a.rows) proj_epilogue_group<EPI, 8>(a, o, bs, ys, n);
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -888,12 +1103,19 @@ struct SsmArgs {
   void* state;           // [B][H][P][N], fp32 or (state16) fp16
   bool state16;
   float* g;              // fp32 [B][E]
-  const double* dta;     // fp64 [B][H][2]: step size and decay (from the in_proj epilogue)
+  int dt_lo;             // zx row of head 0's raw step size (rows dt_lo .. dt_lo + H - 1)
   int batch;
   unsigned* status;      // value 32768 is or-ed in if a streamed copy did not land (k_ssm_stream)
 };
 
 constexpr int kSsmThreads = 256;
+
+// Step size and decay of (batch row b, head h) from the in_proj output:
+// dt = softplus(dt_raw + dt_bias), dA = exp(-dt exp(A_log)), in fp64.
+DFSSM_DEV double2 step_and_decay(const SsmArgs& a, int b, int h) {
+  const double dt = softplus_d(a.zx[size_t(b) * a.in_rows + a.dt_lo + h] + double(a.dt_bias[h]));
+  return make_double2(dt, exp(dt * -exp(double(a.A_log[h]))));
+}
 
 // Sum over the warp of R per-lane values, folded so that each shuffle level halves
 // the values a lane carries: afterwards every lane holds the full sum of value
@@ -921,9 +1143,9 @@ DFSSM_DEV double fold_rows(double (&y)[R], int lane, int* sel) {
 // grid (H, B): one block per head and batch row; warp w owns state rows w, w + 8, ...
 // A lane holds NCH float4 of a row (columns 4 (lane + 32 c)), and a warp keeps
 // 8 / NCH rows in flight: their state loads are issued before anything else (they
-// depend on nothing), then B, C, x and the step size and decay arrive (computed once
-// per head by the in_proj epilogue: dt = softplus(dt_raw + dt_bias),
-// dA = exp(-dt * exp(A_log))).  Arithmetic in fp64, state stored back in fp32 with
+// depend on nothing), then B, C, x and the step size and decay arrive (computed from
+// the raw step-size row: dt = softplus(dt_raw + dt_bias), dA = exp(-dt * exp(A_log))).
+// Arithmetic in fp64, state stored back in fp32 with
 // streaming hints (read and written once per step):
 //   h' = dA h + (x dt) B,  y = C . h' + D x,  g = y * silu(z) (stored fp32).
 // Four consecutive state values (16-byte aligned for fp32, 8-byte for fp16) as
@@ -977,7 +1199,8 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
     double xv[RW];
 #pragma unroll
     for (int i = 0; i < RW; ++i) xv[i] = r0 + i * kW < P ? xcb[h * P + r0 + i * kW] : 0.0;
-    const double dt = a.dta[(size_t(b) * a.H + h) * 2], dA = a.dta[(size_t(b) * a.H + h) * 2 + 1];
+    const double2 sd = step_and_decay(a, b, h);
+    const double dt = sd.x, dA = sd.y;
     double y[RW];
 #pragma unroll
     for (int i = 0; i < RW; ++i) {
@@ -1012,10 +1235,9 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
 }
 
 // Bytes of one (batch, head) item of k_ssm_stream and their offsets in a buffer:
-// state [P][N] (es bytes per value), then B and C [2N] fp64, x [P] fp64, z [P] fp64,
-// (dt, dA) fp64.
+// state [P][N] (es bytes per value), then B and C [2N] fp64, x [P] fp64, z [P] fp64.
 struct SsmItem {
-  int st, bc, x, z, dta, bytes;
+  int st, bc, x, z, bytes;
 };
 __host__ __device__ inline SsmItem ssm_item(int P, int N, int es) {
   SsmItem it;
@@ -1023,17 +1245,19 @@ __host__ __device__ inline SsmItem ssm_item(int P, int N, int es) {
   it.bc = ((es * P * N + 15) / 16) * 16;
   it.x = it.bc + 16 * N;
   it.z = it.x + 8 * P;
-  it.dta = it.z + 8 * P;
-  it.bytes = it.dta + 16;
+  it.bytes = it.z + 8 * P;
   return it;
 }
 constexpr int kSsmStreamThreads = 256;
+constexpr int kSsmStreamMaxItems = 256;   // items per block (a step-size table entry each)
 
 // Streaming SSM update: grid of resident blocks; block c takes the (batch, head)
-// items c, c + gridDim.x, ...  Each item's inputs (its P N values of state, the
-// batch row's B and C, the head's x and z, its step size and decay) arrive by bulk
+// items c, c + gridDim.x, ... (at most kSsmStreamMaxItems).  Each item's inputs (its
+// P N values of state, the batch row's B and C, the head's x and z) arrive by bulk
 // copies into one of two shared-memory buffers, the next item's while this one is
-// computed, so HBM always has a block's worth of state in flight per block.  Warp w
+// computed, so HBM always has a block's worth of state in flight per block.  The
+// block's step sizes and decays are computed up front, one item per thread, while
+// the first copies land.  Warp w
 // takes rows w, w + 8, ... four at a time; a lane holds NCH float4 of a row.  Same
 // arithmetic as k_ssm (fp64, state stored back in its own type with a streaming hint).
 // Four consecutive state values from shared memory, converted once to fp64 (fp16
@@ -1061,6 +1285,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
   extern __shared__ __align__(16) unsigned char sbuf[];
   __shared__ __align__(8) uint64_t bar[2];
   __shared__ int s_ok;
+  __shared__ double2 sdt[kSsmStreamMaxItems];
   constexpr int RW = 4, kW = kSsmStreamThreads / 32;
   const int P = a.P, N = a.N, H = a.H, N4 = N / 4;
   const SsmItem it = ssm_item(P, N, int(sizeof(ST)));
@@ -1084,11 +1309,14 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     bulk_g2s(base + it.bc, a.xc + size_t(b) * a.conv_dim + a.E, unsigned(16 * N), &bar[buf]);
     bulk_g2s(base + it.x, a.xc + size_t(b) * a.conv_dim + size_t(h) * P, unsigned(8 * P), &bar[buf]);
     bulk_g2s(base + it.z, a.zx + size_t(b) * a.in_rows + size_t(h) * P, unsigned(8 * P), &bar[buf]);
-    bulk_g2s(base + it.dta, a.dta + (size_t(b) * H + h) * 2, 16u, &bar[buf]);
   };
   if (tid == 0) {
     if (int(blockIdx.x) < nitems) issue(blockIdx.x, 0);
     if (int(blockIdx.x + gridDim.x) < nitems) issue(blockIdx.x + gridDim.x, 1);
+  }
+  for (int k = tid; k < kSsmStreamMaxItems; k += kSsmStreamThreads) {
+    const int item = int(blockIdx.x) + k * int(gridDim.x);
+    if (item < nitems) sdt[k] = step_and_decay(a, item / H, item % H);
   }
   for (int k = 0;; ++k) {
     const int item = int(blockIdx.x) + k * int(gridDim.x);
@@ -1126,8 +1354,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     const double* Cs = Bs + N;
     const double* xs = reinterpret_cast<const double*>(base + it.x);
     const double* zs = reinterpret_cast<const double*>(base + it.z);
-    const double dt = reinterpret_cast<const double*>(base + it.dta)[0];
-    const double dA = reinterpret_cast<const double*>(base + it.dta)[1];
+    const double dt = sdt[k].x, dA = sdt[k].y;
     const int b = item / H, h = item % H;
     ST* gst = static_cast<ST*>(a.state) + (size_t(b) * H + h) * P * N;
     double Bv[NCH][4], Cv[NCH][4];
