@@ -525,6 +525,27 @@ def test_proj_tcgen05_parity(tc_path, d_in, d_out, rank, batch):
     _proj_case(p, x, rank)
 
 
+@pytest.fixture
+def mma_path(monkeypatch):
+    """Batched projections on the mma.sync kernel (k_proj) for the test's calls."""
+    monkeypatch.setenv("DFSSM_PROJ_PATH", "mma")
+
+
+@pytest.mark.parametrize("d_in,d_out,rank,batch", [(2048, 8512, 32, 64), (4096, 2048, 64, 16)])
+def test_proj_mma_forced_parity(mma_path, d_in, d_out, rank, batch):
+    """The mma.sync kernel at batches where tcgen05 is the default."""
+    p, x = S.proj_workload(d_in, d_out, rank, batch)
+    _proj_case(p, x, rank)
+
+
+def test_model_decode_mma_batched_parity(mma_path):
+    """A 2-layer 1.3B-shaped model at batch 16 with every projection on k_proj."""
+    w = S.WORKLOADS["model_48x2048_v50280_b16_256steps"]
+    rng = np.random.default_rng(w["seed"] + 1)
+    m = S.gen_model(rng, w["dims"], 2, w["vocab"])
+    _teacher_forced(m, S.gen_tokens(rng, 16, w["vocab"]), 2, all_layers=True)
+
+
 def test_model_decode_tcgen05_batched_parity(tc_path):
     """A 3-layer small model at batch 12 and a 2-layer 1.3B-shaped one at batch 16,
     decoded with every projection on the tcgen05 kernel."""
