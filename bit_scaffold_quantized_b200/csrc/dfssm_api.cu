@@ -464,14 +464,14 @@ int launch_head(const HeadArgs& h, cudaStream_t st, int* nparts) {
   return h.embed_q ? launch_head_q<true>(h, st, nparts) : launch_head_q<false>(h, st, nparts);
 }
 
-// SSM update of the multi-launch path: the streaming kernel when an item's inputs
-// fit two shared-memory buffers and every bulk copy is 16-byte aligned, else k_ssm.
+// SSM update of the multi-launch path: the streaming kernel when kSsmBufs buffers of
+// an item's inputs fit and every bulk copy is 16-byte aligned, else k_ssm.
 constexpr int kSsmStreamSmemCap = 96 * 1024;
 
 template <int NCH, typename ST>
 int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
   const int occ_blocks = occupancy(reinterpret_cast<const void*>(k_ssm_stream<NCH, ST>), kSsmStreamThreads, smem);
-  const int items = sa.batch * sa.H;
+  const int items = sa.batch * sa.H * kSsmSplit;
   // every block's items fit its step-size table
   const int grid = std::max((items + kSsmStreamMaxItems - 1) / kSsmStreamMaxItems,
                             std::max(1, std::min(items, occ_blocks * sm_count())));
@@ -483,10 +483,11 @@ int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
 template <typename ST>
 int launch_ssm_t(const SsmArgs& sa, cudaStream_t st) {
   const SsmItem it = ssm_item(sa.P, sa.N, int(sizeof(ST)));
-  const int smem = 2 * ((it.bytes + 127) & ~127);
-  const bool aligned = (size_t(sa.conv_dim) * 8) % 16 == 0 && (size_t(sa.in_rows) * 8) % 16 == 0 &&
+  const int smem = kSsmBufs * ((it.bytes + 127) & ~127);
+  const bool aligned = sa.P % kSsmSplit == 0 && it.rows % 2 == 0 &&
+                       (size_t(sa.conv_dim) * 8) % 16 == 0 && (size_t(sa.in_rows) * 8) % 16 == 0 &&
                        (size_t(sa.E) * 8) % 16 == 0 && (size_t(sa.P) * 8) % 16 == 0 &&
-                       (size_t(sa.P) * sa.N * sizeof(ST)) % 16 == 0 &&
+                       (size_t(it.rows) * sa.N * sizeof(ST)) % 16 == 0 &&
                        aligned16(sa.state) && aligned16(sa.xc) && aligned16(sa.zx);
   if (aligned && smem <= kSsmStreamSmemCap) {
     if (sa.N <= 128) return launch_ssm_stream<1, ST>(sa, smem, st);

@@ -1234,31 +1234,46 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
   }
 }
 
-// Bytes of one (batch, head) item of k_ssm_stream and their offsets in a buffer:
-// state [P][N] (es bytes per value), then B and C [2N] fp64, x [P] fp64, z [P] fp64.
+// k_ssm_stream items: (batch row, head, part), the part being P / kSsmSplit state
+// rows (rows update independently given B, C, x and the step size).  Bytes of an item
+// and their offsets in a buffer: state [RP][N] (es bytes per value), then B and C
+// [2N] fp64, x [RP] fp64, z [RP] fp64.
+#ifndef DFSSM_SSM_SPLIT
+#define DFSSM_SSM_SPLIT 1
+#endif
+#ifndef DFSSM_SSM_BUFS
+#define DFSSM_SSM_BUFS 2
+#endif
+// Measured at batch 64 (ms per 48-layer step): whole items with 2 buffers 4.92;
+// halves with 2 / 3 / 4 buffers 5.29 / 5.43 / 6.07; quarters with 4 buffers 7.37 -- the
+// per-item fixed work (B and C into registers, two block barriers, the row folds), not
+// the bytes in flight, is what smaller items add.
+constexpr int kSsmSplit = DFSSM_SSM_SPLIT;   // parts per (batch, head)
+constexpr int kSsmBufs = DFSSM_SSM_BUFS;     // shared-memory buffers per block
 struct SsmItem {
-  int st, bc, x, z, bytes;
+  int rows, st, bc, x, z, bytes;
 };
 __host__ __device__ inline SsmItem ssm_item(int P, int N, int es) {
   SsmItem it;
+  it.rows = P / kSsmSplit;
   it.st = 0;
-  it.bc = ((es * P * N + 15) / 16) * 16;
+  it.bc = ((es * it.rows * N + 15) / 16) * 16;
   it.x = it.bc + 16 * N;
-  it.z = it.x + 8 * P;
-  it.bytes = it.z + 8 * P;
+  it.z = it.x + 8 * it.rows;
+  it.bytes = it.z + 8 * it.rows;
   return it;
 }
 constexpr int kSsmStreamThreads = 256;
 constexpr int kSsmStreamMaxItems = 256;   // items per block (a step-size table entry each)
 
-// Streaming SSM update: grid of resident blocks; block c takes the (batch, head)
-// items c, c + gridDim.x, ... (at most kSsmStreamMaxItems).  Each item's inputs (its
-// P N values of state, the batch row's B and C, the head's x and z) arrive by bulk
-// copies into one of two shared-memory buffers, the next item's while this one is
-// computed, so HBM always has a block's worth of state in flight per block.  The
-// block's step sizes and decays are computed up front, one item per thread, while
-// the first copies land.  Warp w
-// takes rows w, w + 8, ... four at a time; a lane holds NCH float4 of a row.  Same
+// Streaming SSM update: grid of resident blocks; block c takes the items c,
+// c + gridDim.x, ... (at most kSsmStreamMaxItems).  Each item's inputs (its RP N
+// values of state, the batch row's B and C, the rows' x and z) arrive by bulk copies
+// into one of kSsmBufs shared-memory buffers; a buffer is refilled with the item
+// kSsmBufs further on as soon as its item is computed, so a block keeps kSsmBufs - 1
+// items in flight while it computes one.  The block's step sizes and decays are
+// computed up front, one item per thread, while the first copies land.  Warp w takes
+// rows w, w + 8, ... four at a time; a lane holds NCH float4 of a row.  Same
 // arithmetic as k_ssm (fp64, state stored back in its own type with a streaming hint).
 // Four consecutive state values from shared memory, converted once to fp64 (fp16
 // goes straight to fp64: one exact conversion per value).
@@ -1283,46 +1298,50 @@ DFSSM_DEV D4 ld_smem_state4(const __half* p) {
 template <int NCH, typename ST>
 __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
   extern __shared__ __align__(16) unsigned char sbuf[];
-  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ __align__(8) uint64_t bar[kSsmBufs];
   __shared__ int s_ok;
   __shared__ double2 sdt[kSsmStreamMaxItems];
   constexpr int RW = 4, kW = kSsmStreamThreads / 32;
   const int P = a.P, N = a.N, H = a.H, N4 = N / 4;
   const SsmItem it = ssm_item(P, N, int(sizeof(ST)));
+  const int RP = it.rows;
   const int bufb = (it.bytes + 127) & ~127;
-  const int nitems = a.batch * H;
+  const int nitems = a.batch * H * kSsmSplit;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int j = 0; j < kSsmBufs; ++j) mbar_init(&bar[j], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  int issued[2] = {0, 0}, landed[2] = {0, 0};   // thread 0: copy phases per buffer
+  int issued[kSsmBufs], landed[kSsmBufs];   // thread 0: copy phases per buffer
+#pragma unroll
+  for (int j = 0; j < kSsmBufs; ++j) issued[j] = landed[j] = 0;
   auto issue = [&](int item, int buf) {
     ++issued[buf];
-    const int b = item / H, h = item % H;
+    const int bh = item / kSsmSplit, part = item % kSsmSplit, b = bh / H, h = bh % H, r0 = part * RP;
     unsigned char* base = sbuf + buf * bufb;
     mbar_expect_tx(&bar[buf], unsigned(it.bytes));
-    bulk_g2s(base + it.st, static_cast<const ST*>(a.state) + (size_t(b) * H + h) * P * N,
-             unsigned(sizeof(ST) * P * N), &bar[buf]);
+    bulk_g2s(base + it.st, static_cast<const ST*>(a.state) + ((size_t(b) * H + h) * P + r0) * N,
+             unsigned(sizeof(ST) * RP * N), &bar[buf]);
     bulk_g2s(base + it.bc, a.xc + size_t(b) * a.conv_dim + a.E, unsigned(16 * N), &bar[buf]);
-    bulk_g2s(base + it.x, a.xc + size_t(b) * a.conv_dim + size_t(h) * P, unsigned(8 * P), &bar[buf]);
-    bulk_g2s(base + it.z, a.zx + size_t(b) * a.in_rows + size_t(h) * P, unsigned(8 * P), &bar[buf]);
+    bulk_g2s(base + it.x, a.xc + size_t(b) * a.conv_dim + size_t(h) * P + r0, unsigned(8 * RP), &bar[buf]);
+    bulk_g2s(base + it.z, a.zx + size_t(b) * a.in_rows + size_t(h) * P + r0, unsigned(8 * RP), &bar[buf]);
   };
-  if (tid == 0) {
-    if (int(blockIdx.x) < nitems) issue(blockIdx.x, 0);
-    if (int(blockIdx.x + gridDim.x) < nitems) issue(blockIdx.x + gridDim.x, 1);
-  }
+  if (tid == 0)
+    for (int j = 0; j < kSsmBufs; ++j)
+      if (int(blockIdx.x + j * gridDim.x) < nitems) issue(blockIdx.x + j * gridDim.x, j);
   for (int k = tid; k < kSsmStreamMaxItems; k += kSsmStreamThreads) {
     const int item = int(blockIdx.x) + k * int(gridDim.x);
-    if (item < nitems) sdt[k] = step_and_decay(a, item / H, item % H);
+    if (item < nitems) {
+      const int bh = item / kSsmSplit;
+      sdt[k] = step_and_decay(a, bh / H, bh % H);
+    }
   }
   for (int k = 0;; ++k) {
     const int item = int(blockIdx.x) + k * int(gridDim.x);
     if (item >= nitems) break;
-    const int buf = k & 1;
-    const unsigned par = unsigned(k >> 1) & 1u;
+    const int buf = k % kSsmBufs;
+    const unsigned par = unsigned(k / kSsmBufs) & 1u;
     if (tid == 0) {
       long long spins = 0;
       bool ok = true;
@@ -1337,7 +1356,7 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
         // memory land: each buffer has at most one outstanding phase, whose parity is
         // that of its last issue (bounded again; the status already marks the outputs
         // invalid).
-        for (int bb = 0; bb < 2; ++bb) {
+        for (int bb = 0; bb < kSsmBufs; ++bb) {
           if (issued[bb] == landed[bb]) continue;
           const unsigned pp = unsigned(issued[bb] - 1) & 1u;
           long long s2 = 0;
@@ -1355,8 +1374,8 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
     const double* xs = reinterpret_cast<const double*>(base + it.x);
     const double* zs = reinterpret_cast<const double*>(base + it.z);
     const double dt = sdt[k].x, dA = sdt[k].y;
-    const int b = item / H, h = item % H;
-    ST* gst = static_cast<ST*>(a.state) + (size_t(b) * H + h) * P * N;
+    const int bh = item / kSsmSplit, b = bh / H, h = bh % H, rbase = (item % kSsmSplit) * RP;
+    ST* gst = static_cast<ST*>(a.state) + ((size_t(b) * H + h) * P + rbase) * N;
     double Bv[NCH][4], Cv[NCH][4];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
@@ -1367,17 +1386,17 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
         Cv[c][e] = n4 < N4 ? Cs[4 * n4 + e] : 0.0;
       }
     }
-    for (int r0 = warp; r0 < P; r0 += RW * kW) {
+    for (int r0 = warp; r0 < RP; r0 += RW * kW) {
       double y[RW];
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
         const int p = r0 + i * kW;
-        const double xdt = p < P ? xs[p] * dt : 0.0;
+        const double xdt = p < RP ? xs[p] * dt : 0.0;
         double acc = 0.0;
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           const int n4 = lane + 32 * c;
-          if (p < P && n4 < N4) {
+          if (p < RP && n4 < N4) {
             const D4 hv = ld_smem_state4(st + size_t(p) * N + 4 * n4);
             const double h0 = fma(dA, hv.x, xdt * Bv[c][0]);
             const double h1 = fma(dA, hv.y, xdt * Bv[c][1]);
@@ -1395,14 +1414,14 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
       int sel;
       const double ys = fold_rows<RW>(y, lane, &sel);
       const int p = r0 + sel * kW;
-      if ((lane & (32 / RW - 1)) == 0 && p < P) {
-        const int e = h * P + p;
+      if ((lane & (32 / RW - 1)) == 0 && p < RP) {
+        const int e = h * P + rbase + p;
         const double yy = fma(double(a.D[h]), xs[p], ys);
         a.g[size_t(b) * a.E + e] = float(yy * silu_d(zs[p]));
       }
     }
     __syncthreads();   // buffer consumed
-    if (tid == 0 && item + 2 * int(gridDim.x) < nitems) issue(item + 2 * int(gridDim.x), buf);
+    if (tid == 0 && item + kSsmBufs * int(gridDim.x) < nitems) issue(item + kSsmBufs * int(gridDim.x), buf);
   }
 }
 
