@@ -281,7 +281,8 @@ __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueC
 // row (grid (B)), for batches that fill the GPU with rows: no cluster exchange, three
 // block barriers.  Thread t owns the 4-column groups t, t + 512, ... (16-byte loads,
 // one word per group and output plane); warp w takes LoRA rows w, w + 16, ... (the
-// first one's slice loaded up front).  The sum of squares and max |x| are reduced by
+// first two rows' slices loaded up front, later rows' chunks all requested before
+// their products).  The sum of squares and max |x| are reduced by
 // every warp from the 16 warp partials in a fixed order.
 constexpr int kPrologueRowThreads = 512;
 constexpr int kPrologueRowGroups = 4;    // 4-column groups per thread: K <= 8192
@@ -291,20 +292,24 @@ constexpr int kPrologueRowMinBatch = 16;
 // through the normalisation (a zero takes the slow exact-rounding path).
 template <int MODE, int G>
 __global__ void __launch_bounds__(kPrologueRowThreads, 1) k_prologue_row(PrologueArgs a) {
-  constexpr int NW = kPrologueRowThreads / 32, PRE = 4;
+  constexpr int NW = kPrologueRowThreads / 32, PRE = G < 2 ? 4 : 8;   // chunks per lane of a row: K / 512
   __shared__ double redd[NW];
   __shared__ float redf[NW];
   __shared__ int red6[NW][kDigits];
   __shared__ __align__(16) int8_t qs[8192];
   const int K = a.K, b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nvq = K / 16;                                   // 16-byte chunks of a row
-  uint4 av[PRE];
+  // the warp's first two LoRA rows (all of them up to rank 32), up to K = 4096, are
+  // requested before any arithmetic
+  uint4 av[2][PRE];
 #pragma unroll
-  for (int m = 0; m < PRE; ++m) {
-    const int c = lane + 32 * m;
-    av[m] = (warp < a.rank && c < nvq) ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(warp) * K) + c)
-                                       : make_uint4(0, 0, 0, 0);
-  }
+  for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+    for (int m = 0; m < PRE; ++m) {
+      const int c = lane + 32 * m, j = warp + NW * rr;
+      av[rr][m] = (j < a.rank && c < nvq) ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K) + c)
+                                          : make_uint4(0, 0, 0, 0);
+    }
   uint32_t h[G][4];
   float am = 0.f;
   if (MODE == 0) {
@@ -407,22 +412,35 @@ __global__ void __launch_bounds__(kPrologueRowThreads, 1) k_prologue_row(Prologu
     if (tid == 0) a.sx[b] = sx;
   }
   const uint4* q16 = reinterpret_cast<const uint4*>(qs);
-  for (int j = warp; j < a.rank; j += NW) {
+  auto dot4 = [](const uint4& w4, const uint4& x4, int acc) {
+    acc = __dp4a(int(w4.x), int(x4.x), acc);
+    acc = __dp4a(int(w4.y), int(x4.y), acc);
+    acc = __dp4a(int(w4.z), int(x4.z), acc);
+    return __dp4a(int(w4.w), int(x4.w), acc);
+  };
+  for (int rr = 0, j = warp; j < a.rank; ++rr, j += NW) {
     int acc = 0;
-    for (int c = lane, m = 0; c < nvq; c += 32, ++m) {
-      uint4 w4;
-      if (j == warp && m < PRE) {
+    if (rr < 2) {
 #pragma unroll
-        for (int mm = 0; mm < PRE; ++mm)
-          if (mm == m) w4 = av[mm];
-      } else {
-        w4 = __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K) + c);
+      for (int m = 0; m < PRE; ++m) {
+        const int c = lane + 32 * m;
+        if (c < nvq) acc = dot4(rr == 0 ? av[0][m] : av[1][m], q16[c], acc);
       }
-      const uint4 x4 = q16[c];
-      acc = __dp4a(int(w4.x), int(x4.x), acc);
-      acc = __dp4a(int(w4.y), int(x4.y), acc);
-      acc = __dp4a(int(w4.z), int(x4.z), acc);
-      acc = __dp4a(int(w4.w), int(x4.w), acc);
+      for (int c = lane + 32 * PRE; c < nvq; c += 32)
+        acc = dot4(__ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K) + c), q16[c], acc);
+    } else {
+      // later rows (rank > 32): every chunk of the row requested before the products
+      uint4 w[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const int c = lane + 32 * m;
+        w[m] = c < nvq ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K) + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const int c = lane + 32 * m;
+        if (c < nvq) acc = dot4(w[m], q16[c], acc);
+      }
     }
     acc = warp_sum_i(acc);
     if (lane == 0) {
