@@ -25,6 +25,8 @@ Sources ("Density Field State Space Models", C. Shinde):
   Appendix B, Table 12  h = A h + (x dt) (x) B; d_state = 128 at 1.3B; norm(y * silu(z))
   Section 2, Appendix B the chunked (SSD) form of the scan over a prompt, block_len 64:
                         the prompt pass (conv_seq, ssd_scan, layer_prefill, model_prefill)
+  Section 3.4, App. D   the density-field state representation (df_field_size, df_encode,
+                        df_decode, df_roundtrip) and its use at chunk boundaries (DF-SSD)
 Where the pages are silent (the [z|x|B|C|dt] split, softplus, eps, conv tap order,
 activation quantiser, the per-row scaffold scale alpha) the standard Mamba-2
 block and the decode-step description this package implements fix the reading;
@@ -255,7 +257,7 @@ def gated_rmsnorm(y: np.ndarray, z: np.ndarray, w: np.ndarray, eps: float = EPS)
 
 
 def ssd_scan(h0: np.ndarray, x: np.ndarray, Bm: np.ndarray, Cm: np.ndarray, dt_raw: np.ndarray,
-             dt_bias: np.ndarray, A_log: np.ndarray, D: np.ndarray, chunk: int = 64):
+             dt_bias: np.ndarray, A_log: np.ndarray, D: np.ndarray, chunk: int = 64, df: bool = False):
     """Selective-SSM over a whole prompt of T tokens in the chunked (state space
     duality, "SSD") form of Mamba-2, which the pages name (Section 2) and use with
     block_len = 64 (Appendix B, DF-SSD).  One group.
@@ -270,7 +272,10 @@ def ssd_scan(h0: np.ndarray, x: np.ndarray, Bm: np.ndarray, Cm: np.ndarray, dt_r
       h_next = exp(cs[end]) h_prev + sum_s exp(cs[end] - cs[s]) dt_s x_s (outer) B_s.
     This is the recurrence h_t = dA_t h_{t-1} + (x_t dt_t) (outer) B_t, y_t = C_t . h_t
     + D x_t unrolled over a chunk, in fp64 throughout (no rounding of the state
-    between tokens).  Returns (y fp64 [B, T, H, P], final state fp64 [B, H, P, N])."""
+    between tokens).  With df (DF-SSD, Section 3.4 / Appendix D) the state carried
+    from one chunk to the next passes through the density-field encoding and readout
+    (df_roundtrip); the state after the last chunk is returned as computed.
+    Returns (y fp64 [B, T, H, P], final state fp64 [B, H, P, N])."""
     x = np.asarray(x, dtype=np.float64)
     Bm = np.asarray(Bm, dtype=np.float64)
     Cm = np.asarray(Cm, dtype=np.float64)
@@ -293,8 +298,89 @@ def ssd_scan(h0: np.ndarray, x: np.ndarray, Bm: np.ndarray, Cm: np.ndarray, dt_r
         y[:, c0:c1] += np.exp(cs)[..., None] * np.einsum("btn,bhpn->bthp", Cm[:, c0:c1], h)
         tail = np.exp(cs[:, -1:, :] - cs)                           # [B, L, H]: decay from s+1 to the end
         h = np.exp(cs[:, -1, :])[:, :, None, None] * h + np.einsum("bsh,bshp,bsn->bhpn", tail, xdt, Bm[:, c0:c1])
+        if df and c1 < T:
+            h = df_roundtrip(h)
     y += np.asarray(D, dtype=np.float64)[None, None, :, None] * x
     return y, h
+
+
+# --------------------------------------------------------------------------
+# Density-field state representation (Section 3.4, Appendix D)
+# --------------------------------------------------------------------------
+# Reading of the pages (Section 3.4: a K x K binary field with K^2 ~ 4 d_state, mean
+# +- 3 sigma normalisation to [0, 1], first-order sigma-delta with an 8-bit
+# accumulator, threshold 0.5, popcount readout; Appendix D: K = 23 at d_state 128):
+#   * one field per state row (the d_state values of one head row); K is the smallest
+#     integer with K^2 >= 4 d_state, each value owns 4 consecutive cells (raster
+#     order), the K^2 - 4 d_state spare cells stay 0;
+#   * mu and sigma are the row's mean and population standard deviation (fp64 sums
+#     left to right); the field keeps lo = mu - 3 sigma and span = 6 sigma as fp32;
+#   * the 8-bit input of value i is q_i = rint(255 clip((h_i - lo) / span, 0, 1))
+#     (q = 128 when span is 0);
+#   * the sigma-delta error e (signed 8-bit, 0 at the row's first cell, carried from
+#     value to value) gives cell = [e + q >= 128] (0.5 of full scale) and
+#     e <- e + q - 255 cell;
+#   * the readout is lo + span popcount / 4 over the value's cells (fp64).
+
+DF_CELLS = 4     # cells per state value
+
+
+def df_field_size(n: int) -> int:
+    """K of the K x K field of a row of n state values: the least K with K^2 >= 4 n."""
+    K = 1
+    while K * K < DF_CELLS * n:
+        K += 1
+    return K
+
+
+def df_encode(row: np.ndarray):
+    """Encode one state row (n values).  Returns (cells uint8 [K*K], lo fp32, span fp32)."""
+    h = np.asarray(row, dtype=np.float64)
+    n = h.shape[0]
+    total = 0.0
+    for v in h:                       # left to right
+        total = total + v
+    mu = total / n
+    ss = 0.0
+    for v in h:
+        d = v - mu
+        ss = ss + d * d
+    sigma = np.sqrt(ss / n)
+    lo = np.float32(mu - 3.0 * sigma)
+    span = np.float32(6.0 * sigma)
+    K = df_field_size(n)
+    cells = np.zeros(K * K, dtype=np.uint8)
+    e = 0
+    for i in range(n):
+        if span == 0:
+            q = 128
+        else:
+            t = (h[i] - np.float64(lo)) / np.float64(span)
+            q = int(np.rint(255.0 * min(1.0, max(0.0, t))))
+        for j in range(DF_CELLS):
+            s_ = e + q
+            bit = 1 if s_ >= 128 else 0
+            e = s_ - 255 * bit
+            cells[DF_CELLS * i + j] = bit
+    return cells, lo, span
+
+
+def df_decode(cells: np.ndarray, lo, span, n: int) -> np.ndarray:
+    """Readout of a field: value i = lo + span * (ones among its cells) / 4 (fp64)."""
+    c = np.asarray(cells, dtype=np.int64)[:DF_CELLS * n].reshape(n, DF_CELLS)
+    d = c.sum(axis=1) / float(DF_CELLS)
+    return np.float64(lo) + d * np.float64(span)
+
+
+def df_roundtrip(h: np.ndarray) -> np.ndarray:
+    """Encode and read out every row (last axis) of a state array; fp64 result."""
+    h = np.asarray(h, dtype=np.float64)
+    flat = h.reshape(-1, h.shape[-1])
+    out = np.empty_like(flat)
+    for r in range(flat.shape[0]):
+        cells, lo, span = df_encode(flat[r])
+        out[r] = df_decode(cells, lo, span, flat.shape[1])
+    return out.reshape(h.shape)
 
 
 def conv_seq(conv_state: np.ndarray, xBC: np.ndarray, w: np.ndarray, b: np.ndarray):
@@ -401,14 +487,15 @@ class PrefillTrace:
     x_out: np.ndarray        # fp16 [B, T, d_inner]
 
 
-def layer_prefill(res: np.ndarray, lw, st, d, chunk: int = 64) -> PrefillTrace:
+def layer_prefill(res: np.ndarray, lw, st, d, chunk: int = 64, df: bool = False) -> PrefillTrace:
     """A whole prompt of T tokens through one layer in one pass (the prompt step
     before decode): the projections over all B*T token rows, the causal conv over the
     sequence (conv_seq), the selective SSM as the chunked SSD scan (ssd_scan, Section
     2; block_len 64, Appendix B), gate, gated RMSNorm and out_proj per token.  Each
     token row goes through the same per-token arithmetic as layer_step; the SSM state
     is carried in fp64 through the prompt and stored once at the end.
-    res fp32 [B, T, D].  Returns the per-token residuals and the states after the
+    res fp32 [B, T, D].  df: the density-field state codec at the chunk boundaries of
+    the scan (ssd_scan).  Returns the per-token residuals and the states after the
     prompt."""
     check_layer_shapes(d, lw, st)
     E, N, G, H, P = d.d_inner, d.d_state, d.ngroups, d.nheads, d.headdim
@@ -425,7 +512,7 @@ def layer_prefill(res: np.ndarray, lw, st, d, chunk: int = 64) -> PrefillTrace:
     xc, conv_new = conv_seq(st.conv, zx[..., E:E + C], lw.conv_w, lw.conv_b)
     xs = xc[..., :E].reshape(Bsz, T, H, P)
     y, hT = ssd_scan(st.ssm, xs, xc[..., E:E + N], xc[..., E + N:E + 2 * N], zx[..., E + C:],
-                     lw.dt_bias, lw.A_log, lw.D, chunk=chunk)
+                     lw.dt_bias, lw.A_log, lw.D, chunk=chunk, df=df)
     y = y.reshape(Bsz, T, E)
     g = (y * silu(z)).astype(np.float32).astype(np.float64)
     x_out = rmsnorm(g, lw.gnorm_w).astype(np.float16)
@@ -458,7 +545,7 @@ def quantize_embedding(embed16: np.ndarray):
     return quantize_act(embed16)
 
 
-def model_prefill(tokens: np.ndarray, m, states, chunk: int = 64) -> ModelTrace:
+def model_prefill(tokens: np.ndarray, m, states, chunk: int = 64, df: bool = False) -> ModelTrace:
     """A whole prompt tokens [B, T] through the model in one pass (layer_prefill per
     layer), then the final RMSNorm, tied LM head and greedy argmax of the LAST prompt
     token.  Returns the logits and token of that position, the last token's residual
@@ -468,7 +555,7 @@ def model_prefill(tokens: np.ndarray, m, states, chunk: int = 64) -> ModelTrace:
     res = m.embed[tok].astype(np.float32)                            # [B, T, D]
     new_states = []
     for lw, st in zip(m.layers, states):
-        t = layer_prefill(res, lw, st, d, chunk=chunk)
+        t = layer_prefill(res, lw, st, d, chunk=chunk, df=df)
         res = t.res
         new_states.append(State(t.conv, t.ssm))
     last = res[:, -1, :]

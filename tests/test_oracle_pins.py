@@ -826,3 +826,80 @@ def test_ssd_scan_strong_decay_stays_finite():
         yt, h = O.ssm_step(h, x[:, t], Bm[:, t], Cm[:, t], dt_raw[:, t], dt_bias, A_log, D, state_dtype=np.float64)
         assert np.max(np.abs(y[:, t] - yt)) <= 1e-10 * max(1.0, np.max(np.abs(yt)))
     assert np.max(np.abs(hT - h)) <= 1e-10 * max(1.0, np.max(np.abs(h)))
+
+
+# ---------------------------------------------------------------- density-field state codec
+
+def test_df_field_size_matches_appendix_d():
+    """Appendix D: K = 23 for d_state = 128 (field 23 x 23 = 529); Section 3.4: K^2 ~ 4 d_state."""
+    assert O.df_field_size(128) == 23
+    for n in range(1, 300):
+        K = O.df_field_size(n)
+        assert K * K >= 4 * n > (K - 1) * (K - 1)
+
+
+def test_df_worked_example():
+    """A two-value row worked by hand (tests/golden/df_codec_worked_example.json)."""
+    g = json.load(open(os.path.join(GOLDEN, "df_codec_worked_example.json")))
+    cells, lo, span = O.df_encode(np.array(g["row"]))
+    assert O.df_field_size(len(g["row"])) == g["K"]
+    assert cells.tolist() == g["cells"]
+    assert float(lo) == g["lo"] and float(span) == g["span"]
+    assert O.df_decode(cells, lo, span, 2).tolist() == g["decoded"]
+
+
+def test_df_constant_row_is_exact():
+    """A constant row has sigma 0: the readout is the value itself."""
+    for c in (0.0, 1.5, -3.25, np.float32(0.1)):
+        row = np.full(128, np.float64(np.float32(c)))
+        assert np.array_equal(O.df_roundtrip(row), row)
+
+
+def test_df_total_density_tracks_the_input():
+    """First-order error feedback keeps the field's total density within half a cell
+    of the normalised input's (plus the 8-bit rounding): the ones over the row, B,
+    satisfy |B - 4 sum v| <= 0.5 + 4 n / 510.  Without the feedback (each cell
+    rounded alone) the error grows with n."""
+    rng = np.random.default_rng(11)
+    for n in (16, 128):
+        for _ in range(20):
+            row = rng.normal(0.0, rng.uniform(0.1, 3.0), size=n) + rng.normal()
+            cells, lo, span = O.df_encode(row)
+            v = np.clip((row - np.float64(lo)) / np.float64(span), 0.0, 1.0)
+            B = int(cells.sum())
+            assert abs(B - 4 * v.sum()) <= 0.5 + 4 * n / 510.0 + 1e-9
+            assert cells[4 * n:].sum() == 0          # spare cells stay empty
+
+
+def test_df_readout_levels_and_clipping():
+    """Every readout is lo + span k/4 (k = 0..4); values beyond mean +- 3 sigma clip
+    to the field's ends."""
+    rng = np.random.default_rng(12)
+    row = rng.normal(size=128)
+    row[5], row[77] = 50.0, -50.0                    # far outside mean +- 3 sigma
+    cells, lo, span = O.df_encode(row)
+    out = O.df_decode(cells, lo, span, 128)
+    k = (out - np.float64(lo)) / np.float64(span) * 4
+    assert np.allclose(k, np.rint(k), atol=1e-9) and k.min() >= 0 and k.max() <= 4
+    assert out[5] == np.float64(lo) + np.float64(span) and out[77] == np.float64(lo)
+
+
+def test_ssd_scan_df_only_at_interior_chunk_boundaries():
+    """DF-SSD: with one chunk there is no interior boundary (identical to the plain
+    scan); with two, the second chunk starts from the codec's readout of the first
+    chunk's state."""
+    rng = np.random.default_rng(13)
+    B_, T, H, P, N = 1, 12, 2, 3, 4
+    h0 = rng.normal(size=(B_, H, P, N))
+    x = rng.normal(size=(B_, T, H, P))
+    Bm, Cm = rng.normal(size=(B_, T, N)), rng.normal(size=(B_, T, N))
+    dt_raw = rng.normal(size=(B_, T, H))
+    dtb, Al, D = rng.normal(size=H), rng.uniform(0, 2, size=H), rng.normal(size=H)
+    y1, h1 = O.ssd_scan(h0, x, Bm, Cm, dt_raw, dtb, Al, D, chunk=T, df=True)
+    y0, h0_ = O.ssd_scan(h0, x, Bm, Cm, dt_raw, dtb, Al, D, chunk=T, df=False)
+    assert np.array_equal(y1, y0) and np.array_equal(h1, h0_)
+    ya, ha = O.ssd_scan(h0, x[:, :6], Bm[:, :6], Cm[:, :6], dt_raw[:, :6], dtb, Al, D, chunk=6)
+    yb, hb = O.ssd_scan(O.df_roundtrip(ha), x[:, 6:], Bm[:, 6:], Cm[:, 6:], dt_raw[:, 6:], dtb, Al, D, chunk=6)
+    y2, h2 = O.ssd_scan(h0, x, Bm, Cm, dt_raw, dtb, Al, D, chunk=6, df=True)
+    assert np.allclose(y2, np.concatenate([ya, yb], axis=1), rtol=1e-12, atol=1e-12)
+    assert np.allclose(h2, hb, rtol=1e-12, atol=1e-12)
