@@ -110,6 +110,8 @@ int check_dims(const dfssm_dims* d) {
           "headdim (%d) must be a multiple of 16 and <= 128", d->headdim);
   REQUIRE(d->ssm_state_dtype == 0 || d->ssm_state_dtype == 1, DFSSM_ERR_INVALID_ARG,
           "ssm_state_dtype (%d) must be 0 (fp32) or 1 (fp16)", d->ssm_state_dtype);
+  REQUIRE(d->df_chunk_codec == 0 || d->df_chunk_codec == 1, DFSSM_ERR_INVALID_ARG,
+          "df_chunk_codec (%d) must be 0 or 1", d->df_chunk_codec);
   REQUIRE(d->d_state % 4 == 0 && d->d_state <= 256, DFSSM_ERR_UNSUPPORTED_SHAPE,
           "d_state (%d) must be a multiple of 4 and <= 256", d->d_state);
   REQUIRE(d->rank >= 0 && d->rank <= 128 && d->rank % 4 == 0, DFSSM_ERR_UNSUPPORTED_SHAPE,
@@ -556,6 +558,8 @@ int check_prefill(const dfssm_dims* d, int T) {
           (long long)d->batch * T);
   REQUIRE(ssd_smem_bytes(d->headdim, d->d_state) <= 200 * 1024, DFSSM_ERR_UNSUPPORTED_SHAPE,
           "headdim * d_state (%d x %d) too large for the prompt-pass scan", d->headdim, d->d_state);
+  REQUIRE(!d->df_chunk_codec || d->headdim <= kSsdThreads, DFSSM_ERR_UNSUPPORTED_SHAPE,
+          "the chunk-boundary codec takes headdim <= %d (%d)", kSsdThreads, d->headdim);
   return DFSSM_OK;
 }
 
@@ -573,7 +577,7 @@ int layer_prefill_launch(const dfssm_dims* d, int T, const dfssm_layer_weights* 
   fa.B = d->batch; fa.T = T; fa.H = d->nheads; fa.P = d->headdim; fa.N = d->d_state; fa.E = E; fa.C = C;
   fa.in_rows = in_rows(d); fa.zx = b.zxbcdt; fa.conv_w = w->conv_w; fa.conv_b = w->conv_b;
   fa.conv_state = s->conv_state; fa.xc = b.xc; fa.dt_bias = w->dt_bias; fa.A_log = w->A_log; fa.D = w->D;
-  fa.state = s->ssm_state; fa.state16 = d->ssm_state_dtype == 1; fa.g = b.g;
+  fa.state = s->ssm_state; fa.state16 = d->ssm_state_dtype == 1; fa.g = b.g; fa.df = d->df_chunk_codec != 0;
   k_conv_seq<<<dim3((C + 255) / 256, d->batch), 256, 0, st>>>(fa);
   CHECK_LAUNCH("k_conv_seq");
   const int smem = int(ssd_smem_bytes(fa.P, fa.N));
@@ -824,7 +828,7 @@ int launch_persistent(const PPlan& plan, const dfssm_dims* d, int n_layer, int v
 
 extern "C" {
 
-int dfssm_version(void) { return 200; }
+int dfssm_version(void) { return 210; }
 
 int dfssm_phase_timers(uint64_t* out, int max_entries, int reset) {
 #ifdef DFSSM_PHASE_TIMERS
@@ -1218,6 +1222,36 @@ int dfssm_model_prefill(const dfssm_dims* d, int n_layer, int vocab, const uint1
   if ((rc = launch_head(h, st, &nparts))) return rc;
   k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, nparts, tok_out);
   CHECK_LAUNCH("k_argmax");
+  return ok();
+}
+
+
+// ---- density-field state codec -------------------------------------------------
+
+int dfssm_df_field_words(int d_state) {
+  REQUIRE(d_state >= 1, DFSSM_ERR_INVALID_ARG, "d_state (%d) must be >= 1", d_state);
+  return df_field_words(d_state);
+}
+
+int dfssm_df_encode(const float* rows, int n_rows, int d_state, uint32_t* cells, float* lo, float* span,
+                    float* rows_out, void* stream) {
+  REQUIRE(rows && cells && lo && span && n_rows >= 0 && d_state >= 1, DFSSM_ERR_INVALID_ARG,
+          "df_encode: null pointer or bad size (rows %d, d_state %d)", n_rows, d_state);
+  if (n_rows == 0) return ok();
+  k_df_encode<<<(n_rows + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(rows, n_rows, d_state, cells,
+                                                                                      lo, span, rows_out);
+  CHECK_LAUNCH("k_df_encode");
+  return ok();
+}
+
+int dfssm_df_decode(const uint32_t* cells, const float* lo, const float* span, int n_rows, int d_state,
+                    float* rows, void* stream) {
+  REQUIRE(rows && cells && lo && span && n_rows >= 0 && d_state >= 1, DFSSM_ERR_INVALID_ARG,
+          "df_decode: null pointer or bad size (rows %d, d_state %d)", n_rows, d_state);
+  if (n_rows == 0) return ok();
+  k_df_decode<<<(n_rows + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(cells, lo, span, n_rows,
+                                                                                      d_state, rows);
+  CHECK_LAUNCH("k_df_decode");
   return ok();
 }
 

@@ -1443,6 +1443,115 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
   }
 }
 
+// ------------------------------------------------------------------ density-field state codec
+//
+// "Density Field State Space Models", Section 3.4 and Appendix D: a state row of n
+// values is held as a K x K binary field (K^2 >= 4 n; K = 23 at d_state 128), four
+// cells per value in raster order, the spare cells 0.  The row's mean mu and
+// population standard deviation sigma (fp64, summed left to right) give
+// lo = mu - 3 sigma and span = 6 sigma, kept as fp32; value i's 8-bit code is
+// q = rint(255 clip((h - lo) / span, 0, 1)) (128 if span is 0); a first-order
+// sigma-delta with a signed 8-bit error e (0 at the row's first cell, carried along
+// the row) sets cell = [e + q >= 128] and e <- e + q - 255 cell; the readout is
+// lo + span (ones among the value's cells) / 4.  Every fp64 step is an explicitly
+// rounded intrinsic in a fixed order (no contraction), so the integer decisions are
+// the same as in any other IEEE evaluation of these formulas.
+
+constexpr int kDfCells = 4;   // cells per state value
+
+__host__ __device__ inline int df_field_k(int n) {
+  int K = 1;
+  while (K * K < kDfCells * n) ++K;
+  return K;
+}
+__host__ __device__ inline int df_field_words(int n) {
+  const int K = df_field_k(n);
+  return (K * K + 31) / 32;
+}
+
+// One row: get(i) reads value i, put(i, v) receives its readout (after get(i) has
+// been read for the last time); cells (may be null) receives the field, 32 cells a
+// word, low bit first; lo and span are returned.
+template <typename Get, typename Put>
+DFSSM_DEV void df_row(int n, Get get, Put put, uint32_t* cells, float* lo_out, float* span_out) {
+  double total = 0.0;
+  for (int i = 0; i < n; ++i) total = __dadd_rn(total, get(i));
+  const double mu = __ddiv_rn(total, double(n));
+  double ss = 0.0;
+  for (int i = 0; i < n; ++i) {
+    const double d = __dsub_rn(get(i), mu);
+    ss = __dadd_rn(ss, __dmul_rn(d, d));
+  }
+  const double sigma = __dsqrt_rn(__ddiv_rn(ss, double(n)));
+  const float lo = __double2float_rn(__dsub_rn(mu, __dmul_rn(3.0, sigma)));
+  const float span = __double2float_rn(__dmul_rn(6.0, sigma));
+  const double lod = double(lo), spand = double(span);
+  int e = 0;
+  uint32_t word = 0u;
+  for (int i = 0; i < n; ++i) {
+    int q = 128;
+    if (span != 0.f) {
+      const double t = __ddiv_rn(__dsub_rn(get(i), lod), spand);
+      q = int(rint(__dmul_rn(255.0, fmin(1.0, fmax(0.0, t)))));
+    }
+    int ones = 0;
+#pragma unroll
+    for (int j = 0; j < kDfCells; ++j) {
+      const int sum = e + q;
+      const int bit = sum >= 128 ? 1 : 0;
+      e = sum - 255 * bit;
+      ones += bit;
+      const int c = kDfCells * i + j;
+      word |= uint32_t(bit) << (c & 31);
+      if ((c & 31) == 31) {
+        if (cells) cells[c >> 5] = word;
+        word = 0u;
+      }
+    }
+    put(i, __dadd_rn(lod, __dmul_rn(double(ones) * (1.0 / kDfCells), spand)));
+  }
+  if (cells) {
+    const int K = df_field_k(n), words = (K * K + 31) / 32;
+    int w = (kDfCells * n) >> 5;
+    if ((kDfCells * n) & 31) cells[w++] = word;   // the last partial word, spare cells 0
+    for (; w < words; ++w) cells[w] = 0u;
+  }
+  if (lo_out) *lo_out = lo;
+  if (span_out) *span_out = span;
+}
+
+// grid (ceil(rows / 128)), 128 threads: thread = one row of n fp32 values -> its field
+// (words_per_row words), lo and span; rows_out (may be null, may alias rows) gets the
+// readout.
+__global__ void __launch_bounds__(128) k_df_encode(const float* rows, int n_rows, int n, uint32_t* cells,
+                                                    float* lo, float* span, float* rows_out) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= n_rows) return;
+  const float* src = rows + size_t(r) * n;
+  float* dst = rows_out ? rows_out + size_t(r) * n : nullptr;
+  const int words = df_field_words(n);
+  df_row(
+      n, [&](int i) { return double(src[i]); },
+      [&](int i, double v) {
+        if (dst) dst[i] = __double2float_rn(v);
+      },
+      cells + size_t(r) * words, lo + r, span + r);
+}
+
+// grid (ceil(rows / 128)), 128 threads: readout of each row's field into fp32.
+__global__ void __launch_bounds__(128) k_df_decode(const uint32_t* cells, const float* lo, const float* span,
+                                                    int n_rows, int n, float* rows) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= n_rows) return;
+  const uint32_t* f = cells + size_t(r) * df_field_words(n);
+  const double lod = double(lo[r]), spand = double(span[r]);
+  for (int i = 0; i < n; ++i) {
+    const int c = kDfCells * i;
+    const int ones = __popc((f[c >> 5] >> (c & 31)) & ((1u << kDfCells) - 1u));
+    rows[size_t(r) * n + i] = __double2float_rn(__dadd_rn(lod, __dmul_rn(double(ones) * (1.0 / kDfCells), spand)));
+  }
+}
+
 // ------------------------------------------------------------------ prompt pass (prefill)
 //
 // A prompt of T tokens per batch row goes through a layer in one pass: the
@@ -1464,6 +1573,7 @@ struct PrefillArgs {
   void* state;              // [B][H][P][N], fp32 or (state16) fp16, in/out
   bool state16;
   float* g;                 // fp32 [B*T][E] gated value y * silu(z)
+  bool df;                  // density-field codec on the state carried between chunks (DF-SSD)
 };
 
 // grid (ceil(C / 256), B), 256 threads: one thread per conv channel walks the prompt
@@ -1519,7 +1629,8 @@ DFSSM_DEV void st_state(__half* p, double v) { *p = __ushort_as_half(d2h(v)); }
 //   y_t[p]  = sum_s M[t][s] x_s[p] + exp(cs_t) (C_t . h[p]) + D x_t[p],
 //   h[p][n] <- exp(cs_end) h[p][n] + sum_s exp(cs_end - cs_s) dt_s x_s[p] B_s[n],
 // and g = y silu(z) is stored in fp32.  The state is read once and written once
-// (rounded to its storage type).
+// (rounded to its storage type).  With a.df the state carried into each next chunk
+// passes through the density-field codec (df_row); the final state does not.
 template <typename ST>
 __global__ void __launch_bounds__(kSsdThreads) k_ssd(PrefillArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -1598,6 +1709,15 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd(PrefillArgs a) {
       double acc = 0.0;
       for (int s = 0; s < L; ++s) acc = fma(wend[s] * xs[s * P + p], double(BsT[n * kSsdL + s]), acc);
       hs[i] = fma(eend, hs[i], acc);
+    }
+    if (a.df && c0 + kSsdL < T) {
+      // DF-SSD: the state carried into the next chunk is the density-field readout of
+      // this one's (thread p: state row p, column p of hs)
+      __syncthreads();
+      if (tid < P)
+        df_row(
+            N, [&](int n) { return hs[n * P + tid]; }, [&](int n, double v) { hs[n * P + tid] = v; }, nullptr,
+            nullptr, nullptr);
     }
   }
   __syncthreads();

@@ -41,7 +41,7 @@ EXPORTS = [
     "dfssm_model_decode", "dfssm_model_decode_launches", "dfssm_last_error", "dfssm_version",
     "dfssm_model_decode_q8", "dfssm_quantize_rows_int8", "dfssm_phase_timers",
     "dfssm_prefill_workspace_bytes", "dfssm_prefill_workspace_layout", "dfssm_layer_prefill",
-    "dfssm_model_prefill",
+    "dfssm_model_prefill", "dfssm_df_field_words", "dfssm_df_encode", "dfssm_df_decode",
 ]
 
 
@@ -54,7 +54,7 @@ class DfssmError(RuntimeError):
 class CDims(C.Structure):
     _fields_ = [(n, C.c_int32) for n in
                 ("batch", "d_model", "d_inner", "nheads", "headdim", "d_state", "ngroups", "d_conv", "rank",
-                 "ssm_state_dtype")]
+                 "ssm_state_dtype", "df_chunk_codec")]
 
 
 class CProj(C.Structure):
@@ -120,6 +120,9 @@ def lib() -> C.CDLL:
                                       vp, vp, sz, vp]
     L.dfssm_model_prefill.argtypes = [C.POINTER(CDims), i, i, vp, C.POINTER(CLayerWeights),
                                       C.POINTER(CLayerState), vp, i, vp, vp, vp, vp, sz, vp]
+    L.dfssm_df_field_words.argtypes = [i]
+    L.dfssm_df_encode.argtypes = [vp, i, i, vp, vp, vp, vp, vp]
+    L.dfssm_df_decode.argtypes = [vp, vp, vp, i, i, vp, vp]
     L.dfssm_last_error.restype = C.c_char_p
     L.dfssm_version.restype = C.c_int
     for name in EXPORTS:
@@ -149,7 +152,7 @@ def _stream(stream) -> Optional[int]:
 
 def cdims(d) -> CDims:
     return CDims(d.batch, d.d_model, d.d_inner, d.nheads, d.headdim, d.d_state, d.ngroups, d.d_conv, d.rank,
-                 getattr(d, "ssm_state_dtype", 0))
+                 getattr(d, "ssm_state_dtype", 0), getattr(d, "df_chunk_codec", 0))
 
 
 # ------------------------------------------------------------------ host -> device
@@ -403,3 +406,28 @@ def model_prefill(m: DeviceModel, states: Sequence[DeviceState], tokens, tok_out
     _check(lib().dfssm_model_prefill(C.byref(cd), n, m.vocab, _ptr(m.embed), cw, cs, _ptr(m.normf_w),
                                      int(tokens.shape[1]), _ptr(tokens), _ptr(tok_out), _ptr(logits), _ptr(ws),
                                      ws.numel(), _stream(stream)))
+
+
+# ------------------------------------------------------------------ density-field state codec
+
+def df_field_words(d_state: int) -> int:
+    """32-bit words of one state row's density field (K x K cells, K^2 >= 4 d_state)."""
+    n = int(lib().dfssm_df_field_words(C.c_int(d_state)))
+    if n < 0:
+        _check(n)
+    return n
+
+
+def df_encode(rows, cells, lo, span, rows_out=None, stream=None) -> None:
+    """rows fp32 [R, n] (device) -> cells int32 [R, df_field_words(n)], lo, span fp32 [R];
+    rows_out (fp32 [R, n], may be rows itself) receives the readout."""
+    R, n = rows.shape
+    _check(lib().dfssm_df_encode(_ptr(rows), C.c_int(R), C.c_int(n), _ptr(cells), _ptr(lo), _ptr(span),
+                                 _ptr(rows_out) if rows_out is not None else None, _stream(stream)))
+
+
+def df_decode(cells, lo, span, rows, stream=None) -> None:
+    """Readout of fields written by df_encode into rows fp32 [R, n]."""
+    R, n = rows.shape
+    _check(lib().dfssm_df_decode(_ptr(cells), _ptr(lo), _ptr(span), C.c_int(R), C.c_int(n), _ptr(rows),
+                                 _stream(stream)))

@@ -45,6 +45,7 @@ class Dims:
     d_conv: int = 4
     rank: int = 0
     ssm_state_dtype: int = 0      # SSM state storage: 0 fp32, 1 fp16
+    df_chunk_codec: int = 0       # prompt pass: density-field codec between scan chunks
 
     @property
     def in_rows(self) -> int:

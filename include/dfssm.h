@@ -80,6 +80,12 @@ typedef struct dfssm_dims {
    * fp16; halves the state stream).  fp16 state runs the multi-launch path at
    * every batch size: the batch-1 token kernel holds fp32 state. */
   int32_t ssm_state_dtype;
+  /* Prompt pass only: 1 passes the SSM state carried from each 64-token chunk of the
+   * scan to the next through the density-field codec (DF-SSD; "Density Field State
+   * Space Models", Section 3.4 and Appendix D; see dfssm_df_encode); 0 (the default)
+   * carries it exactly.  The state after the last chunk is stored as computed.
+   * Decode steps ignore it. */
+  int32_t df_chunk_codec;
 } dfssm_dims;
 
 /* One DF-SSM projection (Eq. 3 with a per-row scaffold scale):
@@ -334,6 +340,33 @@ DFSSM_API const char* dfssm_last_error(void);
 
 /* ABI version (major * 100 + minor). */
 DFSSM_API int dfssm_version(void);
+
+/* ---- density-field state codec ("Density Field State Space Models", Section 3.4;
+ * Appendix D: K = 23 at d_state 128) ----------------------------------------------
+ * A state row of n = d_state values is held as a K x K binary field, K the least
+ * integer with K^2 >= 4 n: four cells per value (raster order; spare cells 0).  The
+ * row's mean mu and population standard deviation sigma (fp64, summed left to right)
+ * give lo = mu - 3 sigma and span = 6 sigma, kept as fp32; value i's 8-bit code is
+ * q = rint(255 clip((h - lo) / span, 0, 1)) (128 if span == 0); a first-order
+ * sigma-delta with a signed 8-bit error e (0 at the row's first cell, carried along
+ * the row) sets cell = [e + q >= 128], e <- e + q - 255 cell; the readout is
+ * lo + span * (ones among the value's four cells) / 4, rounded to fp32.
+ *
+ * dfssm_df_field_words: 32-bit words of one row's field (cell c is bit c % 32 of word
+ * c / 32), or a negative code for d_state < 1. */
+DFSSM_API int dfssm_df_field_words(int d_state);
+
+/* rows: fp32 [n_rows][d_state] (device).  cells: [n_rows][dfssm_df_field_words]
+ * words; lo, span: fp32 [n_rows] (device, written).  rows_out: fp32 [n_rows][d_state]
+ * readout (may be NULL, may equal rows).  Enqueued on `stream`; 16-byte alignment is
+ * not required.  Errors: DFSSM_ERR_INVALID_ARG (null pointer, n_rows < 0,
+ * d_state < 1), DFSSM_ERR_CUDA. */
+DFSSM_API int dfssm_df_encode(const float* rows, int n_rows, int d_state, uint32_t* cells, float* lo,
+                              float* span, float* rows_out, void* stream);
+
+/* Readout of fields written by dfssm_df_encode into rows: fp32 [n_rows][d_state]. */
+DFSSM_API int dfssm_df_decode(const uint32_t* cells, const float* lo, const float* span, int n_rows,
+                              int d_state, float* rows, void* stream);
 
 #ifdef __cplusplus
 }

@@ -23,7 +23,7 @@ def _declared():
 def test_library_builds_and_loads():
     build.build()
     L = F.lib()
-    assert L.dfssm_version() == 200
+    assert L.dfssm_version() == 210
 
 
 def test_phase_timers_absent_from_the_product_build():
