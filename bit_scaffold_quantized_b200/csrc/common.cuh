@@ -240,6 +240,22 @@ DFSSM_DEV void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* ba
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
+// Transaction bytes without an arrival (a second part of a phase's copies announced
+// after the arrival that armed it, or before it).
+DFSSM_DEV void mbar_expect_tx_only(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream still runs: it
+// may read only data that no earlier kernel of the sequence writes (weights) before
+// pdl_wait(), which returns once every earlier kernel has completed and its writes
+// are visible (at once for an ordinary launch); pdl_release() lets the next kernel
+// start its own setup.
+DFSSM_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+DFSSM_DEV void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Generic-proxy writes of this thread to shared memory become visible to later
 // bulk copies (async proxy) that read them.
 DFSSM_DEV void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

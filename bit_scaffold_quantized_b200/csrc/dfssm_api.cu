@@ -57,6 +57,45 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
     if (e_ != cudaSuccess) return fail(DFSSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e_)); \
   } while (0)
 
+// Kernels of the multi-launch chain are launched with programmatic stream
+// serialization: each may start while the kernel before it still runs, does its setup
+// and reads only weights until pdl_wait() (common.cuh), so the launch and the setup
+// overlap the previous kernel's tail.  DFSSM_PDL=0 at compile time turns it off.
+#ifndef DFSSM_PDL
+#define DFSSM_PDL 1
+#endif
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chain(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         unsigned cluster_z, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[2];
+  unsigned n = 0;
+  if (DFSSM_PDL) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_z > 0) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = 1;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = cluster_z;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+#define CHAIN_LAUNCH(what, ...) \
+  do { \
+    cudaError_t e_ = launch_chain(__VA_ARGS__); \
+    if (e_ != cudaSuccess) return fail(DFSSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+
 constexpr size_t kNone = ~size_t(0);
 constexpr int kHeadBlocks = 592;  // 4 per SM on a 148-SM B200
 
@@ -224,22 +263,20 @@ int launch_prologue(int K, int rank, int batch, const float* src, const uint16_t
   if (batch >= kPrologueRowMinBatch) {
     const int g = (K + 4 * kPrologueRowThreads - 1) / (4 * kPrologueRowThreads);
     switch (g) {
-      case 1: k_prologue_row<MODE, 1><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
-      case 2: k_prologue_row<MODE, 2><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
-      case 3: k_prologue_row<MODE, 3><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
-      default: k_prologue_row<MODE, 4><<<batch, kPrologueRowThreads, 0, st>>>(a); break;
+      case 1: CHAIN_LAUNCH("k_prologue_row", k_prologue_row<MODE, 1>, dim3(batch), dim3(kPrologueRowThreads), 0, st, 0, a); break;
+      case 2: CHAIN_LAUNCH("k_prologue_row", k_prologue_row<MODE, 2>, dim3(batch), dim3(kPrologueRowThreads), 0, st, 0, a); break;
+      case 3: CHAIN_LAUNCH("k_prologue_row", k_prologue_row<MODE, 3>, dim3(batch), dim3(kPrologueRowThreads), 0, st, 0, a); break;
+      default: CHAIN_LAUNCH("k_prologue_row", k_prologue_row<MODE, 4>, dim3(batch), dim3(kPrologueRowThreads), 0, st, 0, a); break;
     }
-    CHECK_LAUNCH("k_prologue_row");
     return DFSSM_OK;
   }
   const int v = (K / kPrologueCQ + kPrologueClThreads - 1) / kPrologueClThreads;
   switch (v) {
-    case 1: k_prologue_cl<MODE, 1><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
-    case 2: k_prologue_cl<MODE, 2><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
-    case 3: k_prologue_cl<MODE, 3><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
-    default: k_prologue_cl<MODE, 4><<<dim3(kPrologueCQ, batch), kPrologueClThreads, 0, st>>>(a); break;
+    case 1: CHAIN_LAUNCH("k_prologue_cl", k_prologue_cl<MODE, 1>, dim3(kPrologueCQ, batch), dim3(kPrologueClThreads), 0, st, 0, a); break;
+    case 2: CHAIN_LAUNCH("k_prologue_cl", k_prologue_cl<MODE, 2>, dim3(kPrologueCQ, batch), dim3(kPrologueClThreads), 0, st, 0, a); break;
+    case 3: CHAIN_LAUNCH("k_prologue_cl", k_prologue_cl<MODE, 3>, dim3(kPrologueCQ, batch), dim3(kPrologueClThreads), 0, st, 0, a); break;
+    default: CHAIN_LAUNCH("k_prologue_cl", k_prologue_cl<MODE, 4>, dim3(kPrologueCQ, batch), dim3(kPrologueClThreads), 0, st, 0, a); break;
   }
-  CHECK_LAUNCH("k_prologue_cl");
   return DFSSM_OK;
 }
 
@@ -312,8 +349,7 @@ int launch_proj_bt(const ProjArgs& a, cudaStream_t st) {
   const int wave = std::max(1, occ_blocks * sm_count() / gy);
   const int gx = std::max(1, std::min((ntiles + kProjWarps - 1) / kProjWarps, wave));
   dim3 grid(gx, gy);
-  k_proj<EPI, BT><<<grid, kProjThreads, smem, st>>>(a);
-  CHECK_LAUNCH("k_proj");
+  CHAIN_LAUNCH("k_proj", k_proj<EPI, BT>, grid, dim3(kProjThreads), smem, st, 0, a);
   return DFSSM_OK;
 }
 
@@ -391,20 +427,8 @@ int launch_proj_tc_bg(const ProjArgs& a, cudaStream_t st) {
   if (int rc = proj_tc_maps(a, BG, &tb, &tp)) return rc;
   const int mt = (a.rows + kTcM - 1) / kTcM, gb = (a.batch + BG - 1) / BG;
   const int ks = proj_tc_split(mt * gb, a.K / kTileCols);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 1;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = unsigned(ks);
-  cfg.gridDim = dim3(mt, gb, ks);
-  cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = size_t(smem);
-  cfg.stream = st;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k_proj_tc<EPI, BG>, a, tb, tp);
-  if (e != cudaSuccess) return fail(DFSSM_ERR_CUDA, "k_proj_tc launch: %s", cudaGetErrorString(e));
+  CHAIN_LAUNCH("k_proj_tc", k_proj_tc<EPI, BG>, dim3(mt, gb, ks), dim3(kTcThreads), size_t(smem), st, unsigned(ks),
+               a, tb, tp);
   return DFSSM_OK;
 }
 
@@ -442,8 +466,7 @@ int launch_head_tc(const HeadArgs& h, cudaStream_t st, int* nparts) {
   const int tiles = (h.vocab + 15) / 16;
   int gy = std::max(1, occ_blocks * sm_count() / gx);
   gy = std::min(gy, std::min(kHeadBlocks, (tiles + kHeadWarps - 1) / kHeadWarps));
-  k_lmhead_tc<NB, Q8><<<dim3(gx, gy), kHeadWarps * 32, smem, st>>>(h);
-  CHECK_LAUNCH("k_lmhead_tc");
+  CHAIN_LAUNCH("k_lmhead_tc", k_lmhead_tc<NB, Q8>, dim3(gx, gy), dim3(kHeadWarps * 32), smem, st, 0, h);
   *nparts = gy;
   return DFSSM_OK;
 }
@@ -456,8 +479,8 @@ int launch_head_q(const HeadArgs& h, cudaStream_t st, int* nparts) {
   }
   const size_t smem = size_t(4) * kHeadBatch * h.D;
   cudaFuncSetAttribute(k_lmhead<Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  k_lmhead<Q8><<<dim3(kHeadBlocks, (h.batch + kHeadBatch - 1) / kHeadBatch), kHeadWarps * 32, smem, st>>>(h);
-  CHECK_LAUNCH("k_lmhead");
+  CHAIN_LAUNCH("k_lmhead", k_lmhead<Q8>, dim3(kHeadBlocks, (h.batch + kHeadBatch - 1) / kHeadBatch),
+               dim3(kHeadWarps * 32), smem, st, 0, h);
   *nparts = kHeadBlocks;
   return DFSSM_OK;
 }
@@ -477,8 +500,7 @@ int launch_ssm_stream(const SsmArgs& sa, int smem, cudaStream_t st) {
   // every block's items fit its step-size table
   const int grid = std::max((items + kSsmStreamMaxItems - 1) / kSsmStreamMaxItems,
                             std::max(1, std::min(items, occ_blocks * sm_count())));
-  k_ssm_stream<NCH, ST><<<grid, kSsmStreamThreads, smem, st>>>(sa);
-  CHECK_LAUNCH("k_ssm_stream");
+  CHAIN_LAUNCH("k_ssm_stream", k_ssm_stream<NCH, ST>, dim3(grid), dim3(kSsmStreamThreads), smem, st, 0, sa);
   return DFSSM_OK;
 }
 
@@ -495,9 +517,8 @@ int launch_ssm_t(const SsmArgs& sa, cudaStream_t st) {
     if (sa.N <= 128) return launch_ssm_stream<1, ST>(sa, smem, st);
     return launch_ssm_stream<2, ST>(sa, smem, st);
   }
-  if (sa.N <= 128) k_ssm<1, ST><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
-  else k_ssm<2, ST><<<dim3(sa.H, sa.batch), kSsmThreads, 0, st>>>(sa);
-  CHECK_LAUNCH("k_ssm");
+  if (sa.N <= 128) CHAIN_LAUNCH("k_ssm", k_ssm<1, ST>, dim3(sa.H, sa.batch), dim3(kSsmThreads), 0, st, 0, sa);
+  else CHAIN_LAUNCH("k_ssm", k_ssm<2, ST>, dim3(sa.H, sa.batch), dim3(kSsmThreads), 0, st, 0, sa);
   return DFSSM_OK;
 }
 
@@ -1028,8 +1049,8 @@ int model_decode(const dfssm_dims* d, int n_layer, int vocab, const EmbedRef& em
       return rc;
     return ok();
   }
-  k_embed<<<B, 256, 0, st>>>(emb.f16, emb.q, emb.s, tok_in, vocab, D, b.res, b.status);
-  CHECK_LAUNCH("k_embed");
+  CHAIN_LAUNCH("k_embed", k_embed, dim3(B), dim3(256), 0, st, 0, emb.f16, emb.q, emb.s, tok_in, vocab, D, b.res,
+               b.status);
   for (int l = 0; l < n_layer; ++l)
     if ((rc = layer_multikernel(d, &layers[l], &states[l], b.res, b, st))) return rc;
   float* part_val = reinterpret_cast<float*>(b.scratch);
@@ -1040,8 +1061,7 @@ int model_decode(const dfssm_dims* d, int n_layer, int vocab, const EmbedRef& em
   h.logits = logits; h.part_val = part_val; h.part_idx = part_idx;
   int nparts = kHeadBlocks;
   if ((rc = launch_head(h, st, &nparts))) return rc;
-  k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, nparts, tok_out);
-  CHECK_LAUNCH("k_argmax");
+  CHAIN_LAUNCH("k_argmax", k_argmax, dim3(B), dim3(256), 0, st, 0, part_val, part_idx, nparts, tok_out);
   return ok();
 }
 
@@ -1220,8 +1240,7 @@ int dfssm_model_prefill(const dfssm_dims* d, int n_layer, int vocab, const uint1
   h.embed = embed; h.logits = logits; h.part_val = part_val; h.part_idx = part_idx;
   int nparts = kHeadBlocks;
   if ((rc = launch_head(h, st, &nparts))) return rc;
-  k_argmax<<<B, 256, 0, st>>>(part_val, part_idx, nparts, tok_out);
-  CHECK_LAUNCH("k_argmax");
+  CHAIN_LAUNCH("k_argmax", k_argmax, dim3(B), dim3(256), 0, st, 0, part_val, part_idx, nparts, tok_out);
   return ok();
 }
 

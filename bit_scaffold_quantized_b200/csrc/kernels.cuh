@@ -150,6 +150,8 @@ __global__ void __cluster_dims__(kPrologueCQ, 1, 1) __launch_bounds__(kPrologueC
       av[rr][m] = (j < a.rank && c < nvq) ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K + k0) + c)
                                           : make_uint4(0, 0, 0, 0);
     }
+  pdl_wait();                              // the source row is the previous kernel's output
+  pdl_release();
   uint32_t h[V];
   float am = 0.f;
   if (MODE == 0) {
@@ -310,6 +312,8 @@ __global__ void __launch_bounds__(kPrologueRowThreads, 1) k_prologue_row(Prologu
       av[rr][m] = (j < a.rank && c < nvq) ? __ldg(reinterpret_cast<const uint4*>(a.A + size_t(j) * K) + c)
                                           : make_uint4(0, 0, 0, 0);
     }
+  pdl_wait();                              // the source row is the previous kernel's output
+  pdl_release();
   uint32_t h[G][4];
   float am = 0.f;
   if (MODE == 0) {
@@ -598,6 +602,8 @@ __global__ void __launch_bounds__(kProjThreads) k_proj(ProjArgs a) {
   int* T = part + kProjWarps * 16 * PS;                                           // [BT][kDigits]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b0 = blockIdx.y * BT;
+  pdl_wait();                              // digit planes and u come from the prologue
+  pdl_release();
   const int kgroups = K / kTileCols;
   const int ntiles = (a.rows + kTileRows - 1) / kTileRows;
 
@@ -877,6 +883,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = tmem_s;
+  // the first stages' sign words are weights: requested before the previous kernel
+  // (which writes the digit planes, u and the digit sums) has finished
+  const int pre = min(S, kpc);
+  if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tm_bits)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tm_planes)) : "memory");
+    for (int kb = 0; kb < pre; ++kb) {
+      mbar_expect_tx_only(&full[kb], BITS);
+      tma_load_2d(sbase + kb * STAGE + 2 * B_SLAB, &tm_bits, (kb0 + kb) * kTileWords, m0 / kTileRows, &full[kb]);
+    }
+  }
+  pdl_wait();
+  pdl_release();
   if (ks > 1) {
     // the cluster's barriers are initialised before any CTA sends (the matching
     // wait comes just before the sends); rbar expects every CTA's partials
@@ -886,15 +905,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tm_bits)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tm_planes)) : "memory");
       int issued = 0;
       for (int kb = 0; kb < kpc; ++kb) {
         const int st = kb % S, kg = kb0 + kb;
         if (kb >= S && !tc_wait(&empty[st], unsigned(kb / S - 1) & 1u, a.status, &fail)) break;
         const uint32_t sg = sbase + st * STAGE;
-        mbar_expect_tx(&full[st], BITS + 2 * B_SLAB);
-        tma_load_2d(sg + 2 * B_SLAB, &tm_bits, kg * kTileWords, m0 / kTileRows, &full[st]);
+        if (kb < pre) {          // sign words already requested: the planes complete the phase
+          mbar_expect_tx(&full[st], 2 * B_SLAB);
+        } else {
+          mbar_expect_tx(&full[st], BITS + 2 * B_SLAB);
+          tma_load_2d(sg + 2 * B_SLAB, &tm_bits, kg * kTileWords, m0 / kTileRows, &full[st]);
+        }
         tma_load_2d(sg, &tm_planes, kg * kTileCols, b0 * kDigits, &full[st]);
         tma_load_2d(sg + B_SLAB, &tm_planes, kg * kTileCols + 128, b0 * kDigits, &full[st]);
         issued = kb + 1;
@@ -1204,6 +1225,8 @@ __global__ void __launch_bounds__(kSsmThreads, 2) k_ssm(SsmArgs a) {
         hv[i][c] = (p < P && n4 < N4) ? ld_state4(sbase + size_t(p) * a.N + 4 * n4)
                                       : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+    pdl_wait();                            // B, C, x, z and dt come from the in_proj
+    pdl_release();
     double Bv[NCH][4], Cv[NCH][4];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
@@ -1334,20 +1357,34 @@ __global__ void __launch_bounds__(kSsmStreamThreads) k_ssm_stream(SsmArgs a) {
   int issued[kSsmBufs], landed[kSsmBufs];   // thread 0: copy phases per buffer
 #pragma unroll
   for (int j = 0; j < kSsmBufs; ++j) issued[j] = landed[j] = 0;
-  auto issue = [&](int item, int buf) {
+  // an item's copies: its state (written only by this kernel, so it may be requested
+  // before the previous kernel has finished), then B, C, x and z (the in_proj output)
+  auto issue_state = [&](int item, int buf) {
     ++issued[buf];
     const int bh = item / kSsmSplit, part = item % kSsmSplit, b = bh / H, h = bh % H, r0 = part * RP;
-    unsigned char* base = sbuf + buf * bufb;
     mbar_expect_tx(&bar[buf], unsigned(it.bytes));
-    bulk_g2s(base + it.st, static_cast<const ST*>(a.state) + ((size_t(b) * H + h) * P + r0) * N,
+    bulk_g2s(sbuf + buf * bufb + it.st, static_cast<const ST*>(a.state) + ((size_t(b) * H + h) * P + r0) * N,
              unsigned(sizeof(ST) * RP * N), &bar[buf]);
+  };
+  auto issue_inputs = [&](int item, int buf) {
+    const int bh = item / kSsmSplit, part = item % kSsmSplit, b = bh / H, h = bh % H, r0 = part * RP;
+    unsigned char* base = sbuf + buf * bufb;
     bulk_g2s(base + it.bc, a.xc + size_t(b) * a.conv_dim + a.E, unsigned(16 * N), &bar[buf]);
     bulk_g2s(base + it.x, a.xc + size_t(b) * a.conv_dim + size_t(h) * P + r0, unsigned(8 * RP), &bar[buf]);
     bulk_g2s(base + it.z, a.zx + size_t(b) * a.in_rows + size_t(h) * P + r0, unsigned(8 * RP), &bar[buf]);
   };
+  auto issue = [&](int item, int buf) {
+    issue_state(item, buf);
+    issue_inputs(item, buf);
+  };
   if (tid == 0)
     for (int j = 0; j < kSsmBufs; ++j)
-      if (int(blockIdx.x + j * gridDim.x) < nitems) issue(blockIdx.x + j * gridDim.x, j);
+      if (int(blockIdx.x + j * gridDim.x) < nitems) issue_state(blockIdx.x + j * gridDim.x, j);
+  pdl_wait();
+  pdl_release();
+  if (tid == 0)
+    for (int j = 0; j < kSsmBufs; ++j)
+      if (int(blockIdx.x + j * gridDim.x) < nitems) issue_inputs(blockIdx.x + j * gridDim.x, j);
   for (int k = tid; k < kSsmStreamMaxItems; k += kSsmStreamThreads) {
     const int item = int(blockIdx.x) + k * int(gridDim.x);
     if (item < nitems) {
@@ -1741,6 +1778,8 @@ __global__ void k_embed(const uint16_t* __restrict__ embed, const int8_t* __rest
                         const float* __restrict__ embed_s, const int32_t* __restrict__ tok,
                         int vocab, int D, float* __restrict__ res, unsigned* status) {
   const int b = blockIdx.x;
+  pdl_wait();
+  pdl_release();
   int t = tok[b];
   if (t < 0 || t >= vocab) {
     if (threadIdx.x == 0) atomicOr(status, 2u);
@@ -1803,6 +1842,8 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead(HeadArgs a) {
   __shared__ float wbest[kHeadWarps][kHeadBatch];
   __shared__ int wbesti[kHeadWarps][kHeadBatch];
   const int b0 = blockIdx.y * kHeadBatch;
+  pdl_wait();
+  pdl_release();
   const int nb = min(kHeadBatch, a.batch - b0);
   const int D = a.D;
   for (int bb = 0; bb < nb; ++bb) {
@@ -1894,6 +1935,8 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
   __shared__ float wbest[kHeadWarps][8 * NB];
   __shared__ int wbesti[kHeadWarps][8 * NB];
   const int D = a.D, XS = D / 2 + 2;                       // row stride in words (== 2 mod 32)
+  pdl_wait();
+  pdl_release();
   const int b0 = blockIdx.x * 8 * NB;
   const int nb = min(8 * NB, a.batch - b0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -2052,6 +2095,8 @@ __global__ void k_argmax(const float* __restrict__ part_val, const int* __restri
   __shared__ float sv[256];
   __shared__ int si[256];
   const int b = blockIdx.x;
+  pdl_wait();
+  pdl_release();
   float bv = -INFINITY;
   int bi = 0x7fffffff;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) {
