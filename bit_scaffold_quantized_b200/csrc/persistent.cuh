@@ -1158,9 +1158,12 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
       }
       PT(PH_WAIT_LIN);
       // own shared rows: LoRA stage 2, then conv + SiLU (B/C) or step size + decay (dt),
-      // each value sent to every CTA of the cluster
-      if (tid < w.ns * 16) {
-        const int i = tid;
+      // each value sent to every CTA of the cluster.  Row i runs on thread
+      // kPThreads - 1 - i: the last warps get no unit of the z/x scaffold MMA that
+      // follows (fewer units than warps), so the step-size rows' fp64 softplus / exp
+      // chain no longer delays a warp that holds one.
+      if (kPThreads - 1 - tid < w.ns * 16) {
+        const int i = kPThreads - 1 - tid;
         const int si = w.s0 + i / 16, r = i % 16;        // shared tile of the cluster, row in it
         double v = yin[shslot * 16 + i];
         if (R) v = fma(h2d(sp<uint16_t>(sm, PSM(in_sb))[shslot * 16 + i]), lo[shslot * 16 + i], v);
