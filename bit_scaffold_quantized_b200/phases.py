@@ -20,7 +20,7 @@ PHASES = ["gather residual", "wait AB copies", "prep x (whole vector)", "codes +
           "MMA shared tiles", "wait LoRA partials", "shared rows (send)", "MMA z/x tiles", "z/x epilogue",
           "wait shared rows", "SSM + publish g", "gather g", "wait CD copies", "prep xo (whole vector)",
           "codes + LoRA partials (send)", "MMA out tiles", "wait LoRA partials", "residual rows + publish",
-          "LM head (per token)", "prep x, repeated (code cached)", "MMA z/x, repeated (code cached)"]
+          "LM head (per token)"]
 N_LAYER_PHASES = 18      # the per-layer phases; the LM head is per token
 SLOTS = 32
 
