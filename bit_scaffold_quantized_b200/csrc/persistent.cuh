@@ -96,7 +96,7 @@ enum { EX_LIN = 0, EX_SH = 1, EX_LOUT = 2, EX_N = 3 };
 enum {
   PH_GATHER_R = 0, PH_WAIT_AB, PH_PREP_IN, PH_LORA_IN, PH_MMA_SH, PH_WAIT_LIN, PH_SHARED, PH_MMA_ZX, PH_ZX_EPI,
   PH_WAIT_SH, PH_SSM, PH_GATHER_G, PH_WAIT_CD, PH_PREP_OUT, PH_LORA_OUT, PH_MMA_OUT, PH_WAIT_LOUT, PH_RESID,
-  PH_HEAD, PH_N
+  PH_HEAD, PH_HEAD_STREAM, PH_HEAD_ARG, PH_N   // LM head: gather + norm, row stream, argmax exchange
 };
 
 struct PLayer {
@@ -1389,6 +1389,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         const double rs = 1.0 / sqrt(sum_partials(scratch32, G) / double(D) + kEpsD);
         for (int k = tid; k < D; k += kPThreads) xn[k] = float((double(xn[k]) * rs) * h2d(a.normf_w[k]));
         csync();
+        PT(PH_HEAD);
         // Every compute warp takes whole rows -- row `warp` of each 15-row group of a
         // chunk (one group per fp16 chunk, two per int8 chunk) -- waits on the chunk's
         // slot itself and releases it with its own arrival (the empty barriers count
@@ -1413,8 +1414,25 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
         float best = -INFINITY;
         int besti = 0x7fffffff;
         bool hok = true;
+        // int8 rows: lane 0 loads its rows' scales one chunk ahead, so the load's
+        // latency is not paid after every row's reduction
+        constexpr int RW = CR / kPWarps;             // rows per warp and chunk
+        float scn[RW];
+        auto load_scales = [&](int ci2) {
+          const int r02 = v0 + ci2 * CR, nr2 = min(CR, v1 - r02);
+#pragma unroll
+          for (int rsub = 0; rsub < RW; ++rsub) {
+            const int row = warp + kPWarps * rsub;
+            scn[rsub] = (q8 && lane == 0 && row < nr2) ? __ldg(a.embed_s + r02 + row) : 1.f;
+          }
+        };
+        if (q8 && head_chunks > 0) load_scales(0);
         for (int ci = 0; ci < head_chunks; ++ci) {
           const int b = ci % NH;
+          float sc[RW];
+#pragma unroll
+          for (int rsub = 0; rsub < RW; ++rsub) sc[rsub] = scn[rsub];
+          if (q8 && ci + 1 < head_chunks) load_scales(ci + 1);
           {   // every lane takes the slot's phase (bounded; lane 0 flags a timeout)
             long long spins = 0;
             while (!mbar_try_wait(full_h + b, unsigned(ci / NH) & 1u)) {
@@ -1429,7 +1447,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
           if (!hok) break;
           const int r0 = v0 + ci * CR, nr = min(CR, v1 - r0);
 #pragma unroll
-          for (int rsub = 0; rsub < CR / kPWarps; ++rsub) {
+          for (int rsub = 0; rsub < RW; ++rsub) {
             const int row = warp + kPWarps * rsub;
             if (row < nr) {
               const unsigned char* wrow = head_slot(b) + size_t(row) * head_row_bytes;
@@ -1457,7 +1475,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
               }
               float lg = warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
               if (lane == 0) {
-                if (q8) lg *= a.embed_s[r0 + row];
+                if (q8) lg *= sc[rsub];
                 if (a.logits) a.logits[r0 + row] = lg;
                 if (lg > best || (lg == best && r0 + row < besti)) {
                   best = lg;
@@ -1469,6 +1487,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
           __syncwarp();
           if (lane == 0) mbar_arrive(empty_h + b);      // this warp is done with the slot
         }
+        PT(PH_HEAD_STREAM);
         // best of each warp, then of the CTA
         if (lane == 0) {
           scratch32[2 * warp] = __float_as_uint(best);
@@ -1501,7 +1520,7 @@ __global__ void __launch_bounds__(kPBlock, 1) k_decode_persistent(const __grid_c
           }
         }
       }
-      PT(PH_HEAD);
+      PT(PH_HEAD_ARG);
     }
 #ifdef DFSSM_PHASE_TIMERS
     if (tid == 0 && a.phase) {

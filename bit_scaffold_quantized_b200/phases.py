@@ -1,6 +1,6 @@
 """Per-phase time breakdown of the batch-1 token kernel on the GPU.
 
-    python -m bit_scaffold_quantized_b200.phases [--tokens 64] [--warmup 8]
+    python -m bit_scaffold_quantized_b200.phases [--tokens 64] [--warmup 8] [--head fp16|int8]
 
 Decodes the 48-layer, d_model 2048 benchmark model (batch 1, greedy, CUDA graph per
 token) with the phase-timer build of the library (libdfssm_phases.so, built here
@@ -20,8 +20,9 @@ PHASES = ["gather residual", "wait AB copies", "prep x (whole vector)", "codes +
           "MMA shared tiles", "wait LoRA partials", "shared rows (send)", "MMA z/x tiles", "z/x epilogue",
           "wait shared rows", "SSM + publish g", "gather g", "wait CD copies", "prep xo (whole vector)",
           "codes + LoRA partials (send)", "MMA out tiles", "wait LoRA partials", "residual rows + publish",
-          "LM head (per token)"]
-N_LAYER_PHASES = 18      # the per-layer phases; the LM head is per token
+          "LM head: gather + final norm", "LM head: stream rows (thread 0's warp)",
+          "LM head: argmax exchange"]
+N_LAYER_PHASES = 18      # the per-layer phases; the LM-head phases after them are per token
 SLOTS = 32
 
 
@@ -29,6 +30,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--tokens", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--head", choices=["fp16", "int8"], default="fp16", help="LM-head format")
     ap.add_argument("--json", action="store_true")
     args = ap.parse_args()
     os.environ["DFSSM_VARIANT"] = "phases"
@@ -44,7 +46,7 @@ def main():
     L = F.lib()
     m, tok0 = S.model_workload("model_48x2048_v50280_b1_greedy512")
     d = m.dims
-    dm = F.DeviceModel.from_host(m)
+    dm = F.DeviceModel.from_host(m, head=args.head)
     states = [F.DeviceState.zeros(d) for _ in m.layers]
     call = F.ModelCall(dm, states)
     ws = F.workspace(d, len(m.layers), m.vocab)
@@ -79,23 +81,23 @@ def main():
     cyc = a[ctas, :len(PHASES)] / calls[:, None]             # cycles per token per CTA
     per = cyc.copy()
     per[:, :N_LAYER_PHASES] /= len(m.layers)                  # per layer, except the LM head
-    per[:, N_LAYER_PHASES + 1:] /= len(m.layers)
     us = per / mhz
     rows = []
     for i, name in enumerate(PHASES):
         rows.append({"phase": name, "us_mean": round(float(us[:, i].mean()), 3), "us_max": round(float(us[:, i].max()), 3)})
     layer_us = float(us[:, :N_LAYER_PHASES].sum(axis=1).mean())
-    out = {"tokens": args.tokens, "ctas": int(len(ctas)), "sm_mhz_assumed": mhz, "us_per_token_event": round(us_tok, 2),
+    out = {"tokens": args.tokens, "head": args.head, "ctas": int(len(ctas)), "sm_mhz_assumed": mhz, "us_per_token_event": round(us_tok, 2),
            "us_per_layer_phase_sum": round(layer_us, 3), "phases": rows}
     if args.json:
         print(json.dumps(out))
         return
     print(f"token (event-timed, timer build): {us_tok:.1f} us over {args.tokens} tokens; {len(ctas)} CTAs; "
           f"clock {mhz:.0f} MHz assumed")
-    print(f"{'phase':34s} {'us/layer mean':>14s} {'max over CTAs':>14s}")
+    print(f"{'phase':40s} {'us/layer mean':>14s} {'max over CTAs':>14s}")
     for r in rows:
-        print(f"{r['phase']:34s} {r['us_mean']:14.3f} {r['us_max']:14.3f}")
-    print(f"{'sum of layer phases':34s} {layer_us:14.3f}")
+        print(f"{r['phase']:40s} {r['us_mean']:14.3f} {r['us_max']:14.3f}")
+    print(f"{'sum of layer phases':40s} {layer_us:14.3f}")
+    print("(the LM-head rows are microseconds per token, not per layer)")
 
 
 if __name__ == "__main__":
