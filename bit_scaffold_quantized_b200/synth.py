@@ -188,6 +188,24 @@ def gen_model(rng: np.random.Generator, d: Dims, n_layer: int, vocab: int) -> Mo
     return Model(d, vocab, embed, normf_w, layers)
 
 
+def silent_model(rng: np.random.Generator, d: Dims, n_layer: int, vocab: int) -> Model:
+    """gen_model with three changes: every layer's out_proj scales (alpha and, with a
+    LoRA, sB) are zero; the embedding rows are signed permutations of one fp16 vector,
+    so every row has exactly the same norm and two rows are parallel only if equal;
+    the final-norm weight is the constant 1.5."""
+    m = gen_model(rng, d, n_layer, vocab)
+    u = _f16(rng.normal(0.0, 0.05, size=d.d_model))
+    rows = rng.permuted(np.tile(u, (vocab, 1)), axis=1)
+    signs = rng.integers(0, 2, size=(vocab, d.d_model), dtype=np.int8) * 2 - 1
+    m.embed = (rows * signs.astype(np.float16)).astype(np.float16)
+    m.normf_w = np.full(d.d_model, 1.5, dtype=np.float16)
+    for lw in m.layers:
+        lw.out.alpha[:] = 0
+        if lw.out.sB is not None:
+            lw.out.sB[:] = 0
+    return m
+
+
 def gen_tokens(rng: np.random.Generator, batch: int, vocab: int) -> np.ndarray:
     return rng.integers(0, vocab, size=batch, dtype=np.int64).astype(np.int32)
 

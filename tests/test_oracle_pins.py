@@ -806,6 +806,35 @@ def test_model_prefill_last_logits_track_token_steps():
         O.layer_prefill(np.zeros((2, 0, d.d_model), np.float32), m.layers[0], S.zero_state(d), d)
 
 
+def test_silent_layers_greedy_decode_repeats_the_token():
+    """Closed form over several greedy tokens through a layer stack.  With every
+    out_proj scaled to zero, each layer returns its input residual unchanged (the
+    residual add of Section 4.1), so the final residual is the token's embedding row.
+    With equal-norm rows and a constant final-norm weight c, Cauchy-Schwarz makes the
+    token's own row the strict argmax of the tied head, with logit
+    c |e|^2 / sqrt(|e|^2 / D + eps).  A dropped residual, a wrong row gathered or a
+    transposed head fails this; the layers' states must still move."""
+    d = S.LAYER_SMALL.with_batch(2)
+    rng = np.random.default_rng(47)
+    m = S.silent_model(rng, d, 3, 64)
+    assert len(np.unique(m.embed, axis=0)) == 64
+    norms = np.sum(m.embed.astype(np.float64) ** 2, axis=1)
+    assert np.all(norms == norms[0])
+    states = [O.State(*(lambda z: (z.conv, z.ssm))(S.zero_state(d))) for _ in m.layers]
+    toks = np.array([5, 41], dtype=np.int32)
+    e2 = float(norms[0])
+    own = 1.5 * e2 / math.sqrt(e2 / d.d_model + O.EPS)
+    for _ in range(5):
+        tr = O.model_step(toks, m, states)
+        assert np.array_equal(tr.res, m.embed[toks].astype(np.float32))
+        assert tr.tokens.tolist() == toks.tolist()
+        for b, t in enumerate(toks):
+            assert tr.logits[b, t] == pytest.approx(own, rel=1e-12)
+            assert np.max(np.delete(tr.logits[b], t)) < 0.5 * own
+        states = tr.states
+    assert all(np.max(np.abs(s.ssm)) > 0 for s in states)
+
+
 def test_ssd_scan_strong_decay_stays_finite():
     """A strongly decaying head over a 64-token chunk (cumulative log-decay near -10^3):
     the scan must stay finite and equal the token recurrence (the state forgets its

@@ -444,6 +444,39 @@ def test_model_decode_1p3b_parity():
     _teacher_forced(m, tok, 8, all_layers=True)
 
 
+def test_model_decode_silent_layers_repeat_token_1p3b():
+    """A property that holds at any size, checked at the benchmark's shape and in its
+    launch configuration (the single-launch token kernel) without running the oracle.
+    Every out_proj is scaled to zero, the embedding rows have equal norms and the
+    final-norm weight is a constant c.  The residual therefore stays the token's
+    embedding row through the 48 layers.  The tied head's argmax is the token itself,
+    with logit c |e|^2 / sqrt(|e|^2 / D + eps), so greedy decode repeats it.  The SSM
+    states still move."""
+    rng = np.random.default_rng(61)
+    d = S.LAYER_1P3B
+    m = S.silent_model(rng, d, S.N_LAYER_1P3B, S.VOCAB_1P3B)
+    assert F.launches_per_decode_step(d, len(m.layers), m.vocab) == 1
+    dm = F.DeviceModel.from_host(m)
+    states = [F.DeviceState.zeros(d) for _ in m.layers]
+    call = F.ModelCall(dm, states)
+    ws = F.workspace(d, len(m.layers), m.vocab)
+    L = F.workspace_layout(d, len(m.layers), m.vocab)
+    t0 = 31337
+    tok = torch.tensor([t0], dtype=torch.int32, device=DEV)
+    logits = torch.zeros((1, m.vocab), dtype=torch.float32, device=DEV)
+    e2 = float(np.sum(m.embed[t0].astype(np.float64) ** 2))
+    own = 1.5 * e2 / np.sqrt(e2 / d.d_model + O.EPS)
+    for _ in range(6):
+        call(tok, tok, ws, logits)
+        _sync()
+        assert int(to_np(F.ws_view(ws, L.status, torch.int32, (1,)))[0]) == 0
+        assert int(to_np(tok)[0]) == t0
+        gl = to_np(logits)[0]
+        assert gl[t0] == pytest.approx(own, rel=1e-5)
+        assert np.max(np.delete(gl, t0)) < 0.5 * own
+    assert all(float(np.max(np.abs(to_np(s.ssm)))) > 0 for s in states)
+
+
 def test_model_decode_1p3b_b16_parity():
     """The batched decode workload at its own shape ("Density Field State Space
     Models", Section 4.3, Table 2: batched decode): 48 layers, d_model 2048, batch 16,
