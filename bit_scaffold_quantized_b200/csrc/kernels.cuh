@@ -1978,9 +1978,16 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
     const uint4* r1 = Q8 ? reinterpret_cast<const uint4*>(a.embed_q + size_t(min(v1, a.vocab - 1)) * D) + t
                          : reinterpret_cast<const uint4*>(a.embed + size_t(min(v1, a.vocab - 1)) * D) + 2 * t;
     const bool ok0 = v0 < a.vocab, ok1 = v1 < a.vocab;
-    float acc[NB][4];
+    // acc: one 64-column chunk's tensor-core sums; tot: the chunks' sum, taken with
+    // round-to-nearest fp32 adds.  The tensor cores' own fp32 accumulation does not
+    // round to nearest, and chained over a whole row (~256 MMAs at d_model 2048) it
+    // biased logits toward zero by ~1.5e-5 relative; eight MMAs per chain keep that
+    // bias near the fp32 rounding of the sum.
+    float acc[NB][4], tot[NB][4];
 #pragma unroll
-    for (int n = 0; n < NB; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    for (int n = 0; n < NB; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[n][e] = tot[n][e] = 0.f;
     // rows g and g + 8, 64-column chunks in a 4-slot register ring, three chunks ahead
     uint4 ring[4][2 * kLV];
     auto fetch = [&](uint4 (&dst)[2 * kLV], int c) {
@@ -2028,8 +2035,19 @@ __global__ void __launch_bounds__(kHeadWarps * 32) k_lmhead_tc(HeadArgs a) {
             mma_f16_16816(acc[n], af, bl.x, bl.y);
           }
         }
+#pragma unroll
+        for (int n = 0; n < NB; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            tot[n][e] += acc[n][e];
+            acc[n][e] = 0.f;
+          }
       }
     }
+#pragma unroll
+    for (int n = 0; n < NB; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[n][e] = tot[n][e];
     if constexpr (Q8) {      // logit = row scale * (codes . x)
       const float s0 = ok0 ? a.embed_s[v0] : 0.f, s1 = ok1 ? a.embed_s[v1] : 0.f;
 #pragma unroll

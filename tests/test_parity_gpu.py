@@ -477,6 +477,41 @@ def test_model_decode_silent_layers_repeat_token_1p3b():
     assert all(float(np.max(np.abs(to_np(s.ssm)))) > 0 for s in states)
 
 
+@pytest.mark.parametrize("batch", [16, 64])
+def test_model_decode_silent_layers_repeat_tokens_48x2048_batched(batch):
+    """The silent-layers closed form at the batched decode workloads' full shape (48
+    layers, d_model 2048, vocab 50280) on the multi-launch path, no oracle run: every
+    batch row must repeat its own token, and every row's own-token logit is the same
+    c |e|^2 / sqrt(|e|^2 / D + eps) (all embedding rows have one norm)."""
+    rng = np.random.default_rng(62)
+    d = S.LAYER_1P3B.with_batch(batch)
+    m = S.silent_model(rng, d, S.N_LAYER_1P3B, S.VOCAB_1P3B)
+    assert F.launches_per_decode_step(d, len(m.layers), m.vocab) > 1
+    dm = F.DeviceModel.from_host(m)
+    states = [F.DeviceState.zeros(d) for _ in m.layers]
+    call = F.ModelCall(dm, states)
+    ws = F.workspace(d, len(m.layers), m.vocab)
+    L = F.workspace_layout(d, len(m.layers), m.vocab)
+    t0 = rng.choice(m.vocab, size=batch, replace=False).astype(np.int32)
+    tok_in = torch.from_numpy(t0).to(DEV)
+    tok_out = torch.zeros(batch, dtype=torch.int32, device=DEV)
+    logits = torch.zeros((batch, m.vocab), dtype=torch.float32, device=DEV)
+    e2 = float(np.sum(m.embed[0].astype(np.float64) ** 2))
+    own = 1.5 * e2 / np.sqrt(e2 / d.d_model + O.EPS)
+    rows = np.arange(batch)
+    for _ in range(3):
+        call(tok_in, tok_out, ws, logits)
+        _sync()
+        assert int(to_np(F.ws_view(ws, L.status, torch.int32, (1,)))[0]) == 0
+        assert np.array_equal(to_np(tok_out), t0)
+        gl = to_np(logits).copy()
+        np.testing.assert_allclose(gl[rows, t0], own, rtol=1e-5)
+        gl[rows, t0] = -np.inf
+        assert np.max(gl) < 0.5 * own
+        tok_in.copy_(tok_out)
+    assert all(float(np.max(np.abs(to_np(s.ssm)))) > 0 for s in states)
+
+
 def test_model_decode_1p3b_b16_parity():
     """The batched decode workload at its own shape ("Density Field State Space
     Models", Section 4.3, Table 2: batched decode): 48 layers, d_model 2048, batch 16,
