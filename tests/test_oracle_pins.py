@@ -835,6 +835,46 @@ def test_silent_layers_greedy_decode_repeats_the_token():
     assert all(np.max(np.abs(s.ssm)) > 0 for s in states)
 
 
+def test_batch_rows_are_independent():
+    """A batch is its rows run one at a time: each sequence keeps its own conv and SSM
+    state (Section 4.1), and activations are normalised and quantised per row
+    (Section 3.3).  Rows of different magnitudes and random states; a reduction over
+    the wrong axis or a per-tensor quantiser scale mixes rows and fails this.  BLAS
+    may sum a batch and a single row in different orders, so fp values agree to 1e-12
+    and tokens and integer codes exactly."""
+    d = S.LAYER_SMALL.with_batch(3)
+    rng = np.random.default_rng(53)
+    m = S.gen_model(rng, d, 2, 200)
+    toks = np.array([5, 17, 123], dtype=np.int32)
+    m.embed[17] = (m.embed[17].astype(np.float32) * 4).astype(np.float16)
+    z = S.zero_state(d)
+    states = [O.State(rng.normal(size=z.conv.shape).astype(z.conv.dtype),
+                      rng.normal(0, 0.5, size=z.ssm.shape).astype(z.ssm.dtype)) for _ in m.layers]
+    m1 = replace(m, dims=d.with_batch(1))
+    single = [[O.State(st.conv[b:b + 1].copy(), st.ssm[b:b + 1].copy()) for st in states] for b in range(3)]
+    tok = toks.copy()
+    tok1 = [toks[b:b + 1].copy() for b in range(3)]
+    for _ in range(3):
+        tr = O.model_step(tok, m, states)
+        for b in range(3):
+            t1 = O.model_step(tok1[b], m1, single[b])
+            assert tr.tokens[b] == t1.tokens[0]
+            scale = np.max(np.abs(t1.logits))
+            assert np.max(np.abs(tr.logits[b] - t1.logits[0])) <= 1e-12 * scale
+            for l in range(len(m.layers)):
+                np.testing.assert_allclose(tr.states[l].ssm[b], t1.states[l].ssm[0], rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(tr.states[l].conv[b], t1.states[l].conv[0], rtol=1e-12, atol=1e-12)
+            single[b] = t1.states
+            tok1[b] = t1.tokens
+        states = tr.states
+        tok = tr.tokens
+    x16 = (rng.normal(size=(3, 64)) * np.array([[0.01], [1.0], [30.0]])).astype(np.float16)
+    q, sx = O.quantize_act(x16)
+    for b in range(3):
+        q1, sx1 = O.quantize_act(x16[b:b + 1])
+        assert np.array_equal(q[b], q1[0]) and sx[b] == sx1[0]
+
+
 def test_ssd_scan_strong_decay_stays_finite():
     """A strongly decaying head over a 64-token chunk (cumulative log-decay near -10^3):
     the scan must stay finite and equal the token recurrence (the state forgets its
